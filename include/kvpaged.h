@@ -1,0 +1,228 @@
+/*
+ * kvpaged.h -- C ABI of the paged KV-cache decode library (B200, sm_100a).
+ *
+ * Pages cited by title and section:
+ *   [KV-04] "04. 注意力与 KV 缓存" (inference series)
+ *   [HB-07] "07｜KV Cache、FlashAttention与PagedAttention的内部过程"
+ *           (AI engineering handbook, chapter 07, questions Q025-Q028)
+ *   [CN-06] "06 KV Cache、Prefix Cache、PagedAttention 与 vLLM" (course notes)
+ *   [KV-03] "03. KV Cache：用显存换计算" (llm-inference series)
+ *
+ * Conventions for every entry point:
+ *   - Returns an int status: KV_OK (0) or a negative KV_ERR_* code. No C++
+ *     exception crosses the ABI. On error nothing is launched and host state
+ *     is unchanged unless stated otherwise.
+ *   - Device pointers are owned by the caller (e.g. PyTorch tensors) and must
+ *     be 16-byte aligned. The library never allocates device memory; kernels
+ *     needing scratch take a caller-provided workspace.
+ *   - Host handles (kv_pool_t, kv_prefix_t) are owned by the library and
+ *     released with their _destroy call. They are not thread-safe.
+ *   - Launches are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream). A launch failure is reported as KV_ERR_CUDA.
+ *   - `err_flag` (nullable) is a device int that kernels OR KV_DEV_ERR_* bits
+ *     into when they meet bad data (out-of-range page id or slot, bad length,
+ *     a bounded wait that gave up). Kernels never trap; the caller reads the
+ *     flag when it wants to know.
+ *
+ * Physical layout (the pages leave it open, [HB-07] Q025: "kernels may use a
+ * different memory layout"): per layer, K and V pools of shape
+ *   [num_pages][H_kv][page_size][Dh]
+ * of the storage dtype, so one (page, head) chunk of page_size x Dh values is
+ * contiguous. Block tables are int32 [B][max_blocks] (row b lists the
+ * physical pages of sequence b in logical order). seq_lens are int32 [B] and
+ * count the token appended in this step. Slots are int64: page * page_size +
+ * offset. Query head h uses KV head h / (H_q / H_kv).
+ */
+#ifndef KVPAGED_H
+#define KVPAGED_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define KV_OK 0
+#define KV_ERR_ARG (-1)          /* bad argument, shape or alignment */
+#define KV_ERR_OOM (-2)          /* pool has fewer free pages than asked */
+#define KV_ERR_BAD_ID (-3)       /* page id out of range, or not held */
+#define KV_ERR_DOUBLE_FREE (-4)  /* free of a page more times than it is held */
+#define KV_ERR_SHARED_TAIL (-5)  /* append into a partial page another sequence holds */
+#define KV_ERR_CUDA (-6)         /* a CUDA launch or query failed */
+#define KV_ERR_WORKSPACE (-7)    /* workspace missing or too small */
+#define KV_ERR_UNSUPPORTED (-8)  /* shape outside the compiled kernel set */
+
+/* ---- storage dtypes ----------------------------------------------------- */
+#define KV_DTYPE_F32 0
+#define KV_DTYPE_BF16 1
+#define KV_DTYPE_F16 2
+
+/* ---- device error bits (OR-ed into *err_flag) --------------------------- */
+#define KV_DEV_ERR_PAGE_RANGE 1  /* a block-table entry outside [0, num_pages); that page is skipped */
+#define KV_DEV_ERR_SEQ_LEN 2     /* seq_len < 0 or > max_blocks * page_size; the row is zeroed */
+#define KV_DEV_ERR_SLOT 4        /* kv_append slot >= num_pages * page_size; that row is skipped */
+#define KV_DEV_ERR_TIMEOUT 8     /* a bounded pipeline wait gave up; outputs of that CTA are invalid */
+
+const char* kv_status_string(int status);
+int kv_version(void);
+
+/* =========================================================================
+ * Page pool -- [HB-07] Q028 (fixed-size blocks in a physical pool, allocated
+ * on demand, returned when a request ends); [CN-06] 6.5 (the allocation flow
+ * and copy-on-write with reference counts for shared blocks); [KV-04]
+ * "深入：引擎怎样找状态" (a page still used by another request is never
+ * reclaimed).
+ * The free list is FIFO: it starts as `init_free_order` (a permutation of
+ * 0..num_pages-1; NULL = ascending), alloc pops from the head, and a page whose
+ * count drops to 0 is pushed to the tail.
+ * ======================================================================= */
+typedef struct kv_pool kv_pool_t;
+
+/* Create a pool of num_pages pages of page_size tokens. KV_ERR_ARG if sizes
+ * are not positive or init_free_order is not a permutation. */
+int kv_pool_create(int32_t num_pages, int32_t page_size, const int32_t* init_free_order, kv_pool_t** out);
+int kv_pool_destroy(kv_pool_t* pool);
+
+/* Allocate n pages (refcount 1 each) into out_ids[n], all-or-nothing:
+ * KV_ERR_OOM leaves the pool unchanged. A page that a prefix index still
+ * lists as reusable is dropped from that index when it is handed out. */
+int kv_pool_alloc(kv_pool_t* pool, int32_t n, int32_t* out_ids);
+
+/* Drop one reference per listed id (an id may repeat). All-or-nothing:
+ * KV_ERR_BAD_ID for an id out of range, KV_ERR_DOUBLE_FREE if an id is
+ * listed more times than it is held. */
+int kv_pool_free(kv_pool_t* pool, int32_t n, const int32_t* ids);
+
+/* Add one reference per listed id (sharing, e.g. after a prefix hit). A page
+ * with count 0 may be revived only while a prefix index lists it (it leaves
+ * the free list); otherwise KV_ERR_BAD_ID. All-or-nothing. */
+int kv_pool_incref(kv_pool_t* pool, int32_t n, const int32_t* ids);
+int kv_pool_refcount(const kv_pool_t* pool, int32_t id, int32_t* out);
+int kv_pool_num_free(const kv_pool_t* pool, int32_t* out);
+int kv_pool_page_size(const kv_pool_t* pool, int32_t* out);
+
+/* Block accounting for one sequence of `len` tokens: pages = ceil(len / P),
+ * slots = pages * P, wasted = slots - len ([CN-06] 6.5: 35 @ 16 -> 3, 48, 13). */
+int kv_blocks_for_len(int32_t len, int32_t page_size, int32_t* pages, int32_t* slots, int32_t* wasted);
+
+/* KV bytes = 2 * L * B * T * H_kv * Dh * bytes_per_elem ([HB-07] Q026;
+ * [CN-06] 6.3). */
+int kv_cache_bytes(int64_t L, int64_t B, int64_t T, int64_t H_kv, int64_t Dh, int64_t bytes_per_elem, int64_t* out);
+
+/* Slot of logical position `pos` through one block-table row:
+ * table_row[pos / P] * P + pos % P ([HB-07] Q028, block-size-4 table).
+ * KV_ERR_ARG if pos / P >= n_blocks; KV_ERR_BAD_ID if the entry is negative. */
+int kv_slot_for_pos(const int32_t* table_row, int32_t n_blocks, int32_t page_size, int64_t pos, int64_t* out);
+
+/* Slots of `n` consecutive positions start..start+n-1 of one sequence
+ * (e.g. to write a prefill or a prefix with kv_append). Same errors. */
+int kv_slots_for_range(const int32_t* table_row, int32_t n_blocks, int32_t page_size, int64_t start, int64_t n,
+                       int64_t* out_slots);
+
+/* One decode step's host bookkeeping for B sequences (host arrays):
+ * for each b, the new token goes to position seq_lens[b]; when
+ * seq_lens[b] % P == 0 a page is allocated first and written to
+ * block_tables[b][seq_lens[b] / P] ([HB-07] Q028: positions 10 and 11 fill
+ * block 19, position 12 is the first that needs a new block).
+ * slot_mapping[b] receives the slot and seq_lens[b] is incremented.
+ * Pages are allocated together in order of b, all-or-nothing (KV_ERR_OOM).
+ * KV_ERR_SHARED_TAIL if the partial tail page is held by more than one
+ * sequence (it needs copy-on-write first, [HB-07] Q028 table step 6);
+ * KV_ERR_ARG if a table row is full. On error nothing is changed. */
+int kv_append_slots(kv_pool_t* pool, int32_t B, int32_t* block_tables, int32_t max_blocks, int32_t* seq_lens,
+                    int64_t* slot_mapping);
+
+/* =========================================================================
+ * Prefix index -- [CN-06] 6.4: full cached blocks are keyed by a chained
+ * hash of the parent block's key and this block's tokens; the first block
+ * that differs stops the match; whether partial blocks are reused is left to
+ * the implementation (here: never). [HB-07] Q028: the key must also carry the
+ * identity (model, adapter, template...) -> `salt`. [KV-04] prefix demo: a
+ * difference early in the prompt invalidates every later block even where
+ * tokens agree again.
+ * Key of block i: h_0 = salt, h_{i+1} = FNV-1a-64(h_i as 8 little-endian
+ * bytes, then the block's P tokens as 4 little-endian bytes each). A hit is
+ * confirmed by comparing the stored tokens and the parent entry, so results
+ * never depend on hash collisions.
+ * A registered page whose refcount reaches 0 stays matchable while it sits in
+ * the free list (kv_pool_incref revives it); when kv_pool_alloc hands it out
+ * again its entry and every entry registered below it are dropped.
+ * Registering a prefix block that is already registered keeps the first page.
+ * ======================================================================= */
+typedef struct kv_prefix kv_prefix_t;
+
+int kv_prefix_index_create(int32_t page_size, uint64_t salt, kv_prefix_t** out);
+int kv_prefix_index_destroy(kv_prefix_t* index);
+
+/* Register the full pages of a sequence: tokens[0..n) live in page_ids[i]
+ * for block i (only the first n / P blocks are registered). Binds the index
+ * to `pool` on first use (one pool per index). KV_ERR_BAD_ID if a page is not
+ * currently allocated; KV_ERR_ARG if a page is already registered for a
+ * different prefix, or the pool's page size differs. All-or-nothing. */
+int kv_prefix_register(kv_prefix_t* index, kv_pool_t* pool, const int32_t* tokens, int32_t n, const int32_t* page_ids);
+
+/* Number of leading FULL pages of tokens[0..n) already cached
+ * (*out_num_pages), and their ids in out_page_ids (nullable; room for n / P).
+ * page_size must equal the index's. Read-only: the caller takes references
+ * with kv_pool_incref before using the pages. */
+int kv_prefix_match(const kv_prefix_t* index, const int32_t* tokens, int32_t n, int32_t page_size,
+                    int32_t* out_page_ids, int32_t* out_num_pages);
+
+/* Number of registered pages. */
+int kv_prefix_num_entries(const kv_prefix_t* index, int32_t* out);
+
+/* =========================================================================
+ * Device kernels
+ * ======================================================================= */
+
+/* KV append -- [HB-07] Q025 (each layer appends the new token's K/V to its
+ * own cache before attending); [CN-06] 6.1-6.2; [KV-03] lifecycle "填充".
+ * For every b in [0, B) with slot_mapping[b] >= 0 and every head h:
+ *   k_pages[slot / P][h][slot % P][:] = k_new[b][h][:], same for V.
+ * k_new, v_new: [B][H_kv][Dh] contiguous, same dtype as the pools.
+ * slot_mapping: device int64 [B]; -1 skips the row. A slot >= num_pages * P
+ * sets KV_DEV_ERR_SLOT and the row is skipped. B may be any size (a prefill
+ * writes many tokens in one call). Rows must not share a slot. */
+int kv_append(void* k_pages, void* v_pages, const void* k_new, const void* v_new, const int64_t* slot_mapping,
+              int32_t B, int32_t H_kv, int32_t Dh, int32_t page_size, int32_t num_pages, int32_t dtype,
+              int* err_flag, void* stream);
+
+/* Paged decode attention -- one new query per sequence:
+ *   out[b][h][:] = softmax(scale * q[b][h] . K_t) V_t  over t < seq_lens[b]
+ * with K_t, V_t of KV head h / (H_q / H_kv) found through block_tables
+ * ([KV-04] / [KV-03] attention formula; [HB-07] Q028 block-table walk).
+ * Each CTA walks its pages and folds them with the online (m, l, u) merge of
+ * [HB-07] Q027; the result equals the full softmax up to rounding order.
+ *   out: fp32 [B][H_q][Dh].   q: [B][H_q][Dh] of `dtype` (same as K/V).
+ *   block_tables: int32 [B][max_blocks]; seq_lens: int32 [B] (0 -> zeros).
+ *   Supported: Dh in {64, 128}; page_size in {16, 32}; H_q % H_kv == 0 with
+ *   H_q / H_kv <= 32; dtype F32/BF16/F16. Else KV_ERR_UNSUPPORTED/KV_ERR_ARG.
+ *   num_splits: 1 = single pass; >1 = split each sequence's pages into that
+ *   many contiguous ranges (split-KV) merged by a second combine kernel;
+ *   0 = choose automatically from B, H_kv, max_blocks and the SM count.
+ *   workspace / ws_bytes: device scratch for split partials, at least
+ *   paged_decode_workspace_bytes(...) for the same arguments (NULL/0 is fine
+ *   when no split is used); KV_ERR_WORKSPACE if too small. */
+int paged_decode_attention(float* out, const void* q, const void* k_pages, const void* v_pages,
+                           const int32_t* block_tables, int32_t max_blocks, const int32_t* seq_lens, int32_t B,
+                           int32_t H_q, int32_t H_kv, int32_t Dh, int32_t page_size, int32_t num_pages, float scale,
+                           int32_t dtype, int32_t num_splits, void* workspace, size_t ws_bytes, int* err_flag,
+                           void* stream);
+
+/* The split count paged_decode_attention will use for these arguments
+ * (resolves num_splits = 0 on the current device). */
+int paged_decode_num_splits(int32_t B, int32_t H_kv, int32_t max_blocks, int32_t page_size, int32_t num_splits,
+                            int32_t* out);
+
+/* Workspace bytes needed by paged_decode_attention for the same arguments
+ * (0 when no split is used). */
+int paged_decode_workspace_bytes(int32_t B, int32_t H_q, int32_t H_kv, int32_t Dh, int32_t max_blocks,
+                                 int32_t page_size, int32_t num_splits, size_t* out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVPAGED_H */

@@ -189,21 +189,22 @@ def kv_cache_bytes_ragged(L: int, lengths: Sequence[int], H_kv: int, Dh: int, by
 
 
 def scatter_to_pages(pool: np.ndarray, table_row: Sequence[int], rows: np.ndarray, start: int = 0) -> None:
-    """Write logical rows [n, H_kv, Dh] at positions start.. into pool [pages, H_kv, P, Dh] (in place)."""
+    """Write logical rows [n, H_kv, Dh] at positions start.. into pool [pages, H_kv, P, Dh] (in place).
+
+    Position t goes to page table_row[t // P], offset t % P (vectorised over t).
+    """
     P = pool.shape[2]
-    for i in range(rows.shape[0]):
-        blk, off = logical_block(start + i, P)
-        pool[int(table_row[blk]), :, off, :] = rows[i]
+    t = np.arange(start, start + rows.shape[0])
+    pages = np.asarray(table_row, dtype=np.int64)[t // P]
+    pool[pages, :, t % P, :] = rows
 
 
 def gather_from_pages(pool: np.ndarray, table_row: Sequence[int], n: int) -> np.ndarray:
     """Logical rows [n, H_kv, Dh] of one sequence read back through its block-table row."""
     P = pool.shape[2]
-    out = np.empty((n,) + (pool.shape[1], pool.shape[3]), dtype=pool.dtype)
-    for t in range(n):
-        blk, off = logical_block(t, P)
-        out[t] = pool[int(table_row[blk]), :, off, :]
-    return out
+    t = np.arange(n)
+    pages = np.asarray(table_row, dtype=np.int64)[t // P]
+    return pool[pages, :, t % P, :]
 
 
 # --------------------------------------------------------------------------

@@ -1,0 +1,56 @@
+// Template dispatch for the decode kernels: maps the runtime shape (Dh, page
+// size, heads per warp GW, consumer warps NW) onto a compiled instance, sets
+// its shared-memory limit once per device, and launches it.
+#pragma once
+
+#include <atomic>
+
+#include "decode_kernel.cuh"
+
+namespace kvp {
+
+template <int DT, int DH, int P, int GW, int NW>
+cudaError_t launch_decode_inst(const DecodeParams& p, dim3 grid, cudaStream_t st) {
+    using C = DecodeCfg<DT, DH, P, GW, NW>;
+    static std::atomic<uint64_t> configured{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(configured.load(std::memory_order_acquire) & bit)) {
+        e = cudaFuncSetAttribute(paged_decode_kernel<DT, DH, P, GW, NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::kSmem);
+        if (e != cudaSuccess) return e;
+        configured.fetch_or(bit, std::memory_order_acq_rel);
+    }
+    paged_decode_kernel<DT, DH, P, GW, NW><<<grid, C::kThreads, C::kSmem, st>>>(p);
+    return cudaGetLastError();
+}
+
+template <int DT, int DH, int P>
+cudaError_t launch_decode_gw(const DecodeParams& p, int GW, int NW, dim3 grid, cudaStream_t st) {
+    if (NW == 4) {
+        if (GW == 4) return launch_decode_inst<DT, DH, P, 4, 4>(p, grid, st);
+        if (GW == 2) return launch_decode_inst<DT, DH, P, 2, 4>(p, grid, st);
+        return launch_decode_inst<DT, DH, P, 1, 4>(p, grid, st);
+    }
+    if (GW == 4) return launch_decode_inst<DT, DH, P, 4, 8>(p, grid, st);
+    if (GW == 2) return launch_decode_inst<DT, DH, P, 2, 8>(p, grid, st);
+    return launch_decode_inst<DT, DH, P, 1, 8>(p, grid, st);
+}
+
+template <int DT>
+cudaError_t launch_decode_dt(const DecodeParams& p, int DH, int P, int GW, int NW, dim3 grid, cudaStream_t st) {
+    if (DH == 128) {
+        return P == 16 ? launch_decode_gw<DT, 128, 16>(p, GW, NW, grid, st)
+                       : launch_decode_gw<DT, 128, 32>(p, GW, NW, grid, st);
+    }
+    return P == 16 ? launch_decode_gw<DT, 64, 16>(p, GW, NW, grid, st) : launch_decode_gw<DT, 64, 32>(p, GW, NW, grid, st);
+}
+
+// Defined in decode_f32.cu / decode_bf16.cu / decode_f16.cu.
+cudaError_t launch_decode_f32(const DecodeParams& p, int DH, int P, int GW, int NW, dim3 grid, cudaStream_t st);
+cudaError_t launch_decode_bf16(const DecodeParams& p, int DH, int P, int GW, int NW, dim3 grid, cudaStream_t st);
+cudaError_t launch_decode_f16(const DecodeParams& p, int DH, int P, int GW, int NW, dim3 grid, cudaStream_t st);
+
+}  // namespace kvp

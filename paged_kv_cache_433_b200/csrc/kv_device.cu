@@ -1,0 +1,242 @@
+// Device entry points of the C ABI: kv_append and paged_decode_attention
+// (argument checks, split-KV planning, launches). The kernels themselves are
+// in decode_kernel.cuh; see include/kvpaged.h for the contract.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+
+#include "decode_launch.cuh"
+#include "kvpaged.h"
+
+namespace kvp {
+
+// New token's K/V rows -> their slots ("07｜KV Cache、FlashAttention与
+// PagedAttention的内部过程", Q025: the new K/V are appended to the layer's
+// cache before the query attends). One thread moves 16 bytes; the first
+// `rows * vpr` threads copy K, the next ones V.
+__global__ void __launch_bounds__(256) kv_append_kernel(uint4* __restrict__ k_pages, uint4* __restrict__ v_pages,
+                                                        const uint4* __restrict__ k_new,
+                                                        const uint4* __restrict__ v_new,
+                                                        const int64_t* __restrict__ slots, int64_t rows, int32_t H_kv,
+                                                        int32_t vpr, int32_t P, int64_t num_slots, int* err) {
+    int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    const int64_t per = rows * vpr;
+    if (i >= 2 * per) return;
+    const bool is_v = i >= per;
+    if (is_v) i -= per;
+    const int64_t row = i / vpr;
+    const int32_t c = static_cast<int32_t>(i - row * vpr);
+    const int64_t b = row / H_kv;
+    const int32_t h = static_cast<int32_t>(row - b * H_kv);
+    const int64_t slot = slots[b];
+    if (slot < 0) return;
+    if (slot >= num_slots) {
+        if (!is_v && h == 0 && c == 0 && err) atomicOr(err, KV_DEV_ERR_SLOT);
+        return;
+    }
+    const int64_t page = slot / P, off = slot - page * P;
+    const int64_t dst = ((page * H_kv + h) * P + off) * vpr + c;
+    if (is_v)
+        v_pages[dst] = v_new[i];
+    else
+        k_pages[dst] = k_new[i];
+}
+
+namespace {
+
+int elem_bytes(int32_t dtype) {
+    switch (dtype) {
+        case KV_DTYPE_F32: return 4;
+        case KV_DTYPE_BF16: return 2;
+        case KV_DTYPE_F16: return 2;
+        default: return 0;
+    }
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int sm_count() {
+    static std::atomic<int> cached[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    int v = cached[dev & 63].load(std::memory_order_relaxed);
+    if (v > 0) return v;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    cached[dev & 63].store(v, std::memory_order_relaxed);
+    return v;
+}
+
+// Heads per consumer warp and consumer warps per CTA for a GQA group of g.
+bool plan_group(int32_t g, int* GW, int* HS, int* NW, int* WP) {
+    int gw = (g % 4 == 0) ? 4 : (g % 2 == 0) ? 2 : 1;
+    int hs = g / gw;
+    if (hs > 8) return false;
+    int nw = hs <= 4 ? 4 : 8;
+    *GW = gw;
+    *HS = hs;
+    *NW = nw;
+    *WP = nw / hs;
+    return true;
+}
+
+// Split count. Explicit requests are honoured (capped at max_blocks). For
+// num_splits == 0 the page walk is split only when (sequence, KV head) CTAs
+// alone cannot fill the GPU: aim for about four CTAs per SM while keeping at
+// least 8 pages in every split.
+int resolve_splits(int32_t B, int32_t H_kv, int32_t max_blocks, int32_t num_splits, int32_t* S_out, int32_t* C_out) {
+    int32_t S = num_splits;
+    if (S <= 0) {
+        int sms = sm_count();
+        if (sms <= 0) return KV_ERR_CUDA;
+        const int64_t ctas = static_cast<int64_t>(B) * H_kv;
+        const int64_t target = 4LL * sms;
+        if (ctas >= target) {
+            S = 1;
+        } else {
+            S = static_cast<int32_t>((target + ctas - 1) / ctas);
+            const int32_t cap = max_blocks / 8 > 1 ? max_blocks / 8 : 1;
+            if (S > cap) S = cap;
+        }
+    }
+    if (S > max_blocks) S = max_blocks;
+    if (S < 1) S = 1;
+    const int32_t C = (max_blocks + S - 1) / S;
+    S = (max_blocks + C - 1) / C;
+    *S_out = S;
+    *C_out = C;
+    return KV_OK;
+}
+
+size_t workspace_for(int32_t B, int32_t H_q, int32_t Dh, int32_t S) {
+    if (S <= 1) return 0;
+    const size_t rows = static_cast<size_t>(B) * H_q * S;
+    return rows * Dh * sizeof(float) + rows * sizeof(float2);
+}
+
+int check_shape(int32_t H_q, int32_t H_kv, int32_t Dh, int32_t page_size, int32_t dtype) {
+    if (H_q <= 0 || H_kv <= 0 || H_q % H_kv != 0) return KV_ERR_ARG;
+    if (elem_bytes(dtype) == 0) return KV_ERR_ARG;
+    if (Dh != 64 && Dh != 128) return KV_ERR_UNSUPPORTED;
+    if (page_size != 16 && page_size != 32) return KV_ERR_UNSUPPORTED;
+    int a, b, c, d;
+    if (!plan_group(H_q / H_kv, &a, &b, &c, &d)) return KV_ERR_UNSUPPORTED;
+    return KV_OK;
+}
+
+}  // namespace
+}  // namespace kvp
+
+using namespace kvp;
+
+extern "C" {
+
+int kv_append(void* k_pages, void* v_pages, const void* k_new, const void* v_new, const int64_t* slot_mapping,
+              int32_t B, int32_t H_kv, int32_t Dh, int32_t page_size, int32_t num_pages, int32_t dtype, int* err_flag,
+              void* stream) {
+    const int eb = elem_bytes(dtype);
+    if (B < 0 || H_kv <= 0 || Dh <= 0 || page_size <= 0 || num_pages <= 0 || eb == 0) return KV_ERR_ARG;
+    if ((static_cast<int64_t>(Dh) * eb) % 16 != 0) return KV_ERR_UNSUPPORTED;
+    if (B == 0) return KV_OK;
+    if (!k_pages || !v_pages || !k_new || !v_new || !slot_mapping) return KV_ERR_ARG;
+    if (!aligned16(k_pages) || !aligned16(v_pages) || !aligned16(k_new) || !aligned16(v_new)) return KV_ERR_ARG;
+    const int32_t vpr = Dh * eb / 16;
+    const int64_t rows = static_cast<int64_t>(B) * H_kv;
+    const int64_t threads = 2 * rows * vpr;
+    const int64_t blocks = (threads + 255) / 256;
+    if (blocks > 0x7fffffffLL) return KV_ERR_UNSUPPORTED;
+    kv_append_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint4*>(k_pages), static_cast<uint4*>(v_pages), static_cast<const uint4*>(k_new),
+        static_cast<const uint4*>(v_new), slot_mapping, rows, H_kv, vpr, page_size,
+        static_cast<int64_t>(num_pages) * page_size, err_flag);
+    return cudaGetLastError() == cudaSuccess ? KV_OK : KV_ERR_CUDA;
+}
+
+int paged_decode_num_splits(int32_t B, int32_t H_kv, int32_t max_blocks, int32_t page_size, int32_t num_splits,
+                            int32_t* out) {
+    if (!out || B < 0 || H_kv <= 0 || max_blocks <= 0 || page_size <= 0 || num_splits < 0) return KV_ERR_ARG;
+    int32_t S, C;
+    int rc = resolve_splits(B, H_kv, max_blocks, num_splits, &S, &C);
+    if (rc == KV_OK) *out = S;
+    return rc;
+}
+
+int paged_decode_workspace_bytes(int32_t B, int32_t H_q, int32_t H_kv, int32_t Dh, int32_t max_blocks,
+                                 int32_t page_size, int32_t num_splits, size_t* out) {
+    if (!out || B < 0 || H_q <= 0 || H_kv <= 0 || Dh <= 0 || max_blocks <= 0 || page_size <= 0 || num_splits < 0)
+        return KV_ERR_ARG;
+    int32_t S, C;
+    int rc = resolve_splits(B, H_kv, max_blocks, num_splits, &S, &C);
+    if (rc != KV_OK) return rc;
+    *out = workspace_for(B, H_q, Dh, S);
+    return KV_OK;
+}
+
+int paged_decode_attention(float* out, const void* q, const void* k_pages, const void* v_pages,
+                           const int32_t* block_tables, int32_t max_blocks, const int32_t* seq_lens, int32_t B,
+                           int32_t H_q, int32_t H_kv, int32_t Dh, int32_t page_size, int32_t num_pages, float scale,
+                           int32_t dtype, int32_t num_splits, void* workspace, size_t ws_bytes, int* err_flag,
+                           void* stream) {
+    int rc = check_shape(H_q, H_kv, Dh, page_size, dtype);
+    if (rc != KV_OK) return rc;
+    if (B < 0 || max_blocks <= 0 || num_pages <= 0 || num_splits < 0) return KV_ERR_ARG;
+    if (B == 0) return KV_OK;
+    if (B > 65535 || H_kv > 65535) return KV_ERR_UNSUPPORTED;
+    if (!out || !q || !k_pages || !v_pages || !block_tables || !seq_lens) return KV_ERR_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages)) return KV_ERR_ARG;
+    int GW, HS, NW, WP;
+    plan_group(H_q / H_kv, &GW, &HS, &NW, &WP);
+    int32_t S, C;
+    rc = resolve_splits(B, H_kv, max_blocks, num_splits, &S, &C);
+    if (rc != KV_OK) return rc;
+
+    DecodeParams p{};
+    p.out = out;
+    p.q = q;
+    p.k_pages = k_pages;
+    p.v_pages = v_pages;
+    p.block_tables = block_tables;
+    p.seq_lens = seq_lens;
+    p.err = err_flag;
+    p.max_blocks = max_blocks;
+    p.B = B;
+    p.H_q = H_q;
+    p.H_kv = H_kv;
+    p.num_pages = num_pages;
+    p.g = H_q / H_kv;
+    p.HS = HS;
+    p.WP = WP;
+    p.num_splits = S;
+    p.pages_per_split = C;
+    p.scale_log2 = scale * kLog2e;
+    if (S > 1) {
+        const size_t need = workspace_for(B, H_q, Dh, S);
+        if (!workspace || ws_bytes < need || !aligned16(workspace)) return KV_ERR_WORKSPACE;
+        const size_t rows = static_cast<size_t>(B) * H_q * S;
+        p.part_u = static_cast<float*>(workspace);
+        p.part_ml = reinterpret_cast<float2*>(static_cast<char*>(workspace) + rows * Dh * sizeof(float));
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    dim3 grid(static_cast<unsigned>(S), static_cast<unsigned>(H_kv), static_cast<unsigned>(B));
+    cudaError_t e;
+    switch (dtype) {
+        case KV_DTYPE_F32: e = launch_decode_f32(p, Dh, page_size, GW, NW, grid, st); break;
+        case KV_DTYPE_BF16: e = launch_decode_bf16(p, Dh, page_size, GW, NW, grid, st); break;
+        default: e = launch_decode_f16(p, Dh, page_size, GW, NW, grid, st); break;
+    }
+    if (e != cudaSuccess) return KV_ERR_CUDA;
+    if (S > 1) {
+        const int64_t items = static_cast<int64_t>(B) * H_q;
+        const unsigned blocks = static_cast<unsigned>((items + 3) / 4);
+        if (Dh == 128)
+            paged_combine_kernel<128><<<blocks, 128, 0, st>>>(out, p.part_u, p.part_ml, seq_lens, B, H_q, S, C,
+                                                              page_size, max_blocks);
+        else
+            paged_combine_kernel<64><<<blocks, 128, 0, st>>>(out, p.part_u, p.part_ml, seq_lens, B, H_q, S, C,
+                                                             page_size, max_blocks);
+        if (cudaGetLastError() != cudaSuccess) return KV_ERR_CUDA;
+    }
+    return KV_OK;
+}
+
+}  // extern "C"
