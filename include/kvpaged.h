@@ -64,6 +64,7 @@ extern "C" {
 #define KV_DEV_ERR_SEQ_LEN 2     /* seq_len < 0 or > max_blocks * page_size; the row is zeroed */
 #define KV_DEV_ERR_SLOT 4        /* kv_append slot >= num_pages * page_size; that row is skipped */
 #define KV_DEV_ERR_TIMEOUT 8     /* a bounded pipeline wait gave up; outputs of that CTA are invalid */
+#define KV_DEV_ERR_PIPELINE 16   /* a pipeline stage held another page than expected; outputs invalid */
 
 const char* kv_status_string(int status);
 int kv_version(void);

@@ -122,17 +122,23 @@ struct DecodeCfg {
     static constexpr int kChunk = P * kRowB;         // bytes of one (page, head) chunk
     static constexpr int kStage = 2 * kChunk;        // K + V
     static constexpr int kStageBudget = (NW <= 4) ? 96 * 1024 : 160 * 1024;
-    static constexpr int kNS0 = kStageBudget / kStage;
-    static constexpr int kNS = kNS0 > 16 ? 16 : (kNS0 < 2 ? 2 : kNS0);
+    // Stage i % NS of page i is consumed by page-warp i % WP. NS must be a
+    // multiple of WP (<= 4 when NW == 4, 1 when NW == 8): then every stage is
+    // always drained by the same warp, which waits on each of its phases in
+    // order, so a parity wait can never match a phase two fills old.
+    static constexpr int kWPMax = (NW <= 4) ? 4 : 1;
+    static constexpr int kNS0 = (kStageBudget / kStage) / kWPMax * kWPMax;
+    static constexpr int kNS = kNS0 > 16 ? 16 : (kNS0 < kWPMax ? kWPMax : (kNS0 < 2 ? 2 : kNS0));
     static constexpr int kThreads = 32 * (NW + 1);
     // shared memory layout (bytes)
     static constexpr int kOffBars = kNS * kStage;                      // full[NS], empty[NS] (8 B each)
-    static constexpr int kOffValid = kOffBars + 16 * kNS;              // int[NS]
+    static constexpr int kOffValid = kOffBars + 16 * kNS;              // int[NS]: page index held, -1 = skipped
     static constexpr int kOffPbuf = kOffValid + 4 * kNS;               // NW x (4 x kN + GW) floats
     static constexpr int kPbufFloats = 4 * kN + GW;
     static constexpr int kOffMerge = ((kOffPbuf + 4 * NW * kPbufFloats) + 15) / 16 * 16;  // NW x GW x (DH + 2)
     static constexpr int kSmem = kOffMerge + 4 * NW * GW * (DH + 2);
     static_assert(kNch % 8 == 0, "row must be a multiple of 128 bytes");
+    static_assert(kNS % kWPMax == 0, "stage ring must be a multiple of the page-warps");
     static_assert(P % 4 == 0, "page size must be a multiple of 4");
 };
 
@@ -229,14 +235,14 @@ __global__ void __launch_bounds__(32 * (NW + 1)) paged_decode_kernel(const Decod
                     } else {
                         const uint32_t dst = sbase + s * C::kStage;
                         if (pg >= 0 && pg < p.num_pages) {
-                            stage_valid[s] = 1;
+                            stage_valid[s] = i;
                             const int64_t off = ((int64_t)pg * p.H_kv + kvh) * (int64_t)C::kChunk;
                             mbar_arrive_expect_tx(full_bar + 8 * s, C::kStage);
                             bulk_g2s(dst, kbase + off, C::kChunk, full_bar + 8 * s);
                             bulk_g2s(dst + C::kChunk, vbase + off, C::kChunk, full_bar + 8 * s);
                         } else {
                             raise_err(p.err, KV_DEV_ERR_PAGE_RANGE);
-                            stage_valid[s] = 0;
+                            stage_valid[s] = -1 - i;
                             mbar_arrive(full_bar + 8 * s);
                         }
                         ++issued;
@@ -310,7 +316,13 @@ __global__ void __launch_bounds__(32 * (NW + 1)) paged_decode_kernel(const Decod
                 ok = false;
             }
             if (!__all_sync(0xffffffffu, ok)) break;
-            const bool valid = stage_valid[s] != 0;
+            // The stage must hold page i (a page the producer skipped is tagged -1 - i).
+            const int tag = stage_valid[s];
+            if (tag != i && tag != -1 - i) {
+                if (lane == 0) raise_err(p.err, KV_DEV_ERR_PIPELINE);
+                break;
+            }
+            const bool valid = tag == i;
             const int pos0 = (first + i) * P;
             const int nvalid = valid ? min(P, len - pos0) : 0;
             const uint32_t sK = sbase + s * C::kStage;

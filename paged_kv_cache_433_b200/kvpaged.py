@@ -35,6 +35,7 @@ KV_DEV_ERR_PAGE_RANGE = 1
 KV_DEV_ERR_SEQ_LEN = 2
 KV_DEV_ERR_SLOT = 4
 KV_DEV_ERR_TIMEOUT = 8
+KV_DEV_ERR_PIPELINE = 16
 
 # (name, restype, argtypes) of every exported function.
 _i32, _i64, _u64, _vp, _f32, _sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_void_p, ctypes.c_float, ctypes.c_size_t
