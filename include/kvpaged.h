@@ -212,6 +212,19 @@ int paged_decode_attention(float* out, const void* q, const void* k_pages, const
                            int32_t dtype, int32_t num_splits, void* workspace, size_t ws_bytes, int* err_flag,
                            void* stream);
 
+/* Which decode kernel paged_decode_attention uses (process-wide; default AUTO):
+ *   KV_DECODE_KERNEL_AUTO  tensor cores (warp MMA on TMA-staged swizzled tiles)
+ *                          for bf16/fp16 K/V with H_q / H_kv <= 64, CUDA cores
+ *                          (packed f32x2 FMA) for fp32 K/V;
+ *   KV_DECODE_KERNEL_SIMT  CUDA cores for every dtype (H_q / H_kv <= 32);
+ *   KV_DECODE_KERNEL_MMA   same as AUTO (fp32 K/V still use CUDA cores).
+ * Both kernels compute the same function; this exists to compare them.
+ * KV_ERR_ARG for an unknown kind. */
+#define KV_DECODE_KERNEL_AUTO 0
+#define KV_DECODE_KERNEL_SIMT 1
+#define KV_DECODE_KERNEL_MMA 2
+int paged_decode_set_kernel(int32_t kind);
+
 /* The split count paged_decode_attention will use for these arguments
  * (resolves num_splits = 0 on the current device). */
 int paged_decode_num_splits(int32_t B, int32_t H_kv, int32_t max_blocks, int32_t page_size, int32_t num_splits,

@@ -173,7 +173,9 @@ __device__ __forceinline__ void group_reduce(float (&v)[N], int lane) {
 }
 
 template <int DT, int DH, int P, int GW, int NW>
-__global__ void __launch_bounds__(32 * (NW + 1)) paged_decode_kernel(const DecodeParams p) {
+// Two CTAs of NW = 4 consumers per SM: 10 warps spread over 4 sub-partitions
+// put 3 warps on some, so registers are capped at 16384 / (3 * 32) = 168.
+__global__ void __launch_bounds__(32 * (NW + 1), (NW <= 4) ? 2 : 1) paged_decode_kernel(const DecodeParams p) {
     using C = DecodeCfg<DT, DH, P, GW, NW>;
     extern __shared__ __align__(128) unsigned char smem[];
 

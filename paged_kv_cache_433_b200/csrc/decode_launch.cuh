@@ -21,6 +21,9 @@ cudaError_t launch_decode_inst(const DecodeParams& p, dim3 grid, cudaStream_t st
         e = cudaFuncSetAttribute(paged_decode_kernel<DT, DH, P, GW, NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::kSmem);
         if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(paged_decode_kernel<DT, DH, P, GW, NW>,
+                                 cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        if (e != cudaSuccess) return e;
         configured.fetch_or(bit, std::memory_order_acq_rel);
     }
     paged_decode_kernel<DT, DH, P, GW, NW><<<grid, C::kThreads, C::kSmem, st>>>(p);
@@ -52,5 +55,49 @@ cudaError_t launch_decode_dt(const DecodeParams& p, int DH, int P, int GW, int N
 cudaError_t launch_decode_f32(const DecodeParams& p, int DH, int P, int GW, int NW, dim3 grid, cudaStream_t st);
 cudaError_t launch_decode_bf16(const DecodeParams& p, int DH, int P, int GW, int NW, dim3 grid, cudaStream_t st);
 cudaError_t launch_decode_f16(const DecodeParams& p, int DH, int P, int GW, int NW, dim3 grid, cudaStream_t st);
+
+}  // namespace kvp
+
+// ---- tensor-core variant (bf16 / fp16) ------------------------------------
+#include "decode_mma.cuh"
+
+namespace kvp {
+
+template <int DT, int DH, int P>
+cudaError_t launch_mma_inst(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, dim3 grid,
+                            cudaStream_t st) {
+    constexpr int NW = 4;
+    using C = MmaCfg<DH, P, NW>;
+    static std::atomic<uint64_t> configured{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(configured.load(std::memory_order_acquire) & bit)) {
+        e = cudaFuncSetAttribute(paged_decode_mma_kernel<DT, DH, P, NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::kSmem);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(paged_decode_mma_kernel<DT, DH, P, NW>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 100);
+        if (e != cudaSuccess) return e;
+        configured.fetch_or(bit, std::memory_order_acq_rel);
+    }
+    paged_decode_mma_kernel<DT, DH, P, NW><<<grid, C::kThreads, C::kSmem, st>>>(p, tk, tv);
+    return cudaGetLastError();
+}
+
+template <int DT>
+cudaError_t launch_mma_dt(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int DH, int P, dim3 grid,
+                          cudaStream_t st) {
+    if (DH == 128)
+        return P == 16 ? launch_mma_inst<DT, 128, 16>(p, tk, tv, grid, st) : launch_mma_inst<DT, 128, 32>(p, tk, tv, grid, st);
+    return P == 16 ? launch_mma_inst<DT, 64, 16>(p, tk, tv, grid, st) : launch_mma_inst<DT, 64, 32>(p, tk, tv, grid, st);
+}
+
+// Defined in decode_mma_bf16.cu / decode_mma_f16.cu.
+cudaError_t launch_mma_bf16(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int DH, int P, dim3 grid,
+                            cudaStream_t st);
+cudaError_t launch_mma_f16(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int DH, int P, dim3 grid,
+                           cudaStream_t st);
 
 }  // namespace kvp

@@ -1,0 +1,364 @@
+// Paged decode attention on the tensor cores (bf16 / fp16 K/V), sm_100a.
+//
+// Same contract and the same online (m, l, u) merge as decode_kernel.cuh
+// ("07｜KV Cache、FlashAttention与PagedAttention的内部过程", Q027; attention
+// formula of "04. 注意力与 KV 缓存" / "03. KV Cache：用显存换计算"), with the
+// two small contractions of every page done by warp-level MMA so each
+// (page, head) chunk costs ~100 instructions instead of ~800 on the CUDA
+// cores:
+//   S[16 x P]  = Q[16 heads x Dh] . K_page^T      (m16n8k16, k over Dh)
+//   O[16 x Dh] += P[16 x P] . V_page               (m16n8k16, k over tokens)
+// The GQA group is the M dimension (rows >= g are zero padding), so the S
+// accumulator fragment is, element for element, the A fragment of the second
+// product: probabilities never leave registers.
+//
+// Data movement: the producer warp issues 2-D TMA tile loads (no multicast)
+// of each (page, head) chunk of K and V, Dh/64 boxes of P rows x 128 bytes
+// with 128-byte swizzle, into a ring of NS stages; ldmatrix then reads rows
+// of 8 tokens without bank conflicts. Row max uses 2 shuffles; the output
+// rescale is lazy: the reference max of a row moves only when a score exceeds
+// it by more than 2^8 (exact: o = u / l for any common reference).
+// Masked tail tokens (t >= len) get p = 0 and their V rows are zeroed in
+// shared memory first, so stale values (even NaN) in unused slots never reach
+// the output.
+#pragma once
+
+#include <cuda.h>
+
+#include "decode_kernel.cuh"
+
+namespace kvp {
+
+template <int DH, int P, int NW>
+struct MmaCfg {
+    static constexpr int kBoxes = DH / 64;         // 128-byte boxes per token row
+    static constexpr int kBoxB = P * 128;          // bytes per box (P rows)
+    static constexpr int kChunk = kBoxes * kBoxB;  // one (page, head) chunk = P x Dh x 2 bytes
+    static constexpr int kStage = 2 * kChunk;      // K + V
+    static constexpr int kKSteps = DH / 16;        // QK k-steps
+    static constexpr int kNT = P / 8;              // token n-tiles of S
+    static constexpr int kPK = P / 16;             // PV k-steps
+    static constexpr int kOT = DH / 8;             // dim n-tiles of O
+    static constexpr int kStageBudget = 96 * 1024;
+    // Stage i % NS is drained by page-warp i % WP (WP divides NW): NS must be
+    // a multiple of NW so each stage always goes to the same warp.
+    static constexpr int kNS0 = (kStageBudget / kStage) / NW * NW;
+    static constexpr int kNS = kNS0 > 16 ? 16 : (kNS0 < NW ? NW : kNS0);
+    static constexpr int kMergeB = NW * 16 * (DH + 2) * 4;  // per-warp (m, l, O) rows, aliased on the stages
+    static constexpr int kRing = kNS * kStage;
+    static constexpr int kOffBars = kRing > kMergeB ? kRing : kMergeB;
+    static constexpr int kOffTag = kOffBars + 16 * kNS;
+    static constexpr int kSmem = 1024 + kOffTag + 4 * kNS;  // + slack to align the ring to 1024 bytes
+    static constexpr int kThreads = 32 * (NW + 1);
+    static_assert(DH % 64 == 0 && P % 16 == 0, "shape");
+    static_assert(kNS % NW == 0, "stage ring must be a multiple of the page-warps");
+};
+
+template <int DT, int DH, int P, int NW>
+__global__ void __launch_bounds__(32 * (NW + 1), 2)
+    paged_decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
+                            const __grid_constant__ CUtensorMap tmap_v) {
+    using C = MmaCfg<DH, P, NW>;
+    constexpr bool kBF16 = DT == KV_DTYPE_BF16;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+
+    const int split = blockIdx.x;
+    const int kvh = blockIdx.y;
+    const int b = blockIdx.z;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const bool split_mode = p.num_splits > 1;
+
+    int len = p.seq_lens[b];
+    if (len < 0 || len > p.max_blocks * P) {
+        if (threadIdx.x == 0 && split == 0) raise_err(p.err, KV_DEV_ERR_SEQ_LEN);
+        len = 0;
+    }
+    const int n_pages = (len + P - 1) / P;
+    const int first = split_mode ? split * p.pages_per_split : 0;
+    const int n_local = split_mode ? min(p.pages_per_split, n_pages - first) : n_pages;
+    if (n_local <= 0) {
+        if (!split_mode) {
+            for (int e = threadIdx.x; e < p.g * DH; e += blockDim.x)
+                p.out[((int64_t)b * p.H_q + (int64_t)kvh * p.g) * DH + e] = 0.f;
+        }
+        return;
+    }
+
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;
+    unsigned char* smem = smem_raw + (sbase - raw);
+    const uint32_t full_bar = sbase + C::kOffBars;
+    const uint32_t empty_bar = full_bar + 8 * C::kNS;
+    volatile int* stage_tag = reinterpret_cast<volatile int*>(smem + C::kOffTag);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kNS; ++s) {
+            mbar_init(full_bar + 8 * s, 1);
+            mbar_init(empty_bar + 8 * s, p.HS);
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tmap(&tmap_k);
+            prefetch_tmap(&tmap_v);
+        }
+        const int32_t* row = p.block_tables + (int64_t)b * p.max_blocks + first;
+        bool ok = true;
+        int issued = 0;
+        for (int base = 0; base < n_local && ok; base += 32) {
+            const int my = (base + lane < n_local) ? row[base + lane] : 0;
+            const int cnt = min(32, n_local - base);
+            for (int k = 0; k < cnt; ++k) {
+                const int pg = __shfl_sync(0xffffffffu, my, k);
+                const int i = base + k;
+                if (lane == 0) {
+                    const int s = i % C::kNS;
+                    if (i >= C::kNS && !mbar_wait_bounded(empty_bar + 8 * s, ((i / C::kNS) - 1) & 1, kWaitLimitNs)) {
+                        raise_err(p.err, KV_DEV_ERR_TIMEOUT);
+                        ok = false;
+                    } else {
+                        const uint32_t dst = sbase + s * C::kStage;
+                        if (pg >= 0 && pg < p.num_pages) {
+                            stage_tag[s] = i;
+                            const int32_t y = (pg * p.H_kv + kvh) * P;  // first row of the chunk
+                            mbar_arrive_expect_tx(full_bar + 8 * s, C::kStage);
+#pragma unroll
+                            for (int bx = 0; bx < C::kBoxes; ++bx) {
+                                tma_load_2d(dst + bx * C::kBoxB, &tmap_k, bx * 64, y, full_bar + 8 * s);
+                                tma_load_2d(dst + C::kChunk + bx * C::kBoxB, &tmap_v, bx * 64, y, full_bar + 8 * s);
+                            }
+                        } else {
+                            raise_err(p.err, KV_DEV_ERR_PAGE_RANGE);
+                            stage_tag[s] = -1 - i;
+                            mbar_arrive(full_bar + 8 * s);
+                        }
+                        ++issued;
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+            }
+        }
+        if (lane == 0) {
+            for (int i = max(0, issued - C::kNS); i < issued; ++i)
+                if (!mbar_wait_bounded(full_bar + 8 * (i % C::kNS), (i / C::kNS) & 1, kWaitLimitNs))
+                    raise_err(p.err, KV_DEV_ERR_TIMEOUT);
+        }
+        return;
+    }
+
+    // -------------------------------------------------------------- consumers
+    const int cw = warp - 1;
+    const int hs = cw % p.HS;  // 16-row head slice
+    const int wp = cw / p.HS;
+    const bool active = wp < p.WP;
+    const int quad = lane & 3;   // column pair within a fragment
+    const int r0 = lane >> 2;    // fragment rows r0 and r0 + 8
+    const int rows = min(16, p.g - hs * 16);  // real heads in this slice
+    const int hbase = kvh * p.g + hs * 16;    // query head of row 0
+
+    // Q as the A operand of S = Q K^T: rows = heads, k = dims (pairs of elements per register).
+    uint32_t qa[C::kKSteps][4];
+    {
+        const uint32_t* q32 = static_cast<const uint32_t*>(p.q);
+        const int64_t row0 = (int64_t)b * p.H_q + hbase;
+#pragma unroll
+        for (int kk = 0; kk < C::kKSteps; ++kk) {
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                const int r = r0 + 8 * rr;
+#pragma unroll
+                for (int ch = 0; ch < 2; ++ch) {
+                    const int d = kk * 16 + ch * 8 + 2 * quad;
+                    qa[kk][rr + 2 * ch] = (r < rows) ? q32[((row0 + r) * DH + d) >> 1] : 0u;
+                }
+            }
+        }
+    }
+
+    float o[C::kOT][4];
+#pragma unroll
+    for (int n = 0; n < C::kOT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    float m_ref[2] = {-INFINITY, -INFINITY};  // reference max (log2 units) of rows r0, r0 + 8
+    float l_part[2] = {0.f, 0.f};             // this lane's share of the row sums
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+
+    if (active) {
+        for (int i = wp; i < n_local; i += p.WP) {
+            const int s = i % C::kNS;
+            if (!mbar_wait_bounded(full_bar + 8 * s, (i / C::kNS) & 1, kWaitLimitNs)) {
+                raise_err(p.err, KV_DEV_ERR_TIMEOUT);
+                ok = false;
+            }
+            if (!__all_sync(0xffffffffu, ok)) break;
+            const int tag = stage_tag[s];
+            if (tag != i && tag != -1 - i) {
+                if (lane == 0) raise_err(p.err, KV_DEV_ERR_PIPELINE);
+                break;
+            }
+            const uint32_t sK = sbase + s * C::kStage;
+            const uint32_t sV = sK + C::kChunk;
+            if (tag == i) {
+                const int nvalid = min(P, len - (first + i) * P);
+
+                // ---- S = Q K^T (fp32 accumulators; rows = heads, cols = tokens)
+                float sc[C::kNT][4];
+#pragma unroll
+                for (int n = 0; n < C::kNT; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
+                const int mi = lane >> 3, rr8 = lane & 7;
+#pragma unroll
+                for (int kk = 0; kk < C::kKSteps; ++kk) {
+                    const int c = kk * 2 + (mi & 1);  // 16-byte chunk of the row (8 dims)
+                    const uint32_t boxb = sK + (c >> 3) * C::kBoxB;
+#pragma unroll
+                    for (int np = 0; np < C::kNT / 2; ++np) {
+                        const int t = np * 16 + (mi >> 1) * 8 + rr8;
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4(boxb + t * 128 + (((c & 7) ^ (t & 7)) << 4), b0, b1, b2, b3);
+                        mma_16816<kBF16>(sc[2 * np], qa[kk], b0, b1);
+                        mma_16816<kBF16>(sc[2 * np + 1], qa[kk], b2, b3);
+                    }
+                }
+
+                // ---- scale, mask, row max (4 lanes of a quad share a row)
+                float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+                for (int n = 0; n < C::kNT; ++n)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int t = n * 8 + 2 * quad + (e & 1);
+                        const float v = (t < nvalid) ? sc[n][e] * sl2 : -INFINITY;
+                        sc[n][e] = v;
+                        mx[e >> 1] = fmaxf(mx[e >> 1], v);
+                    }
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
+                    mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+                }
+                // lazy reference update: only when a row's max grows by more than 2^8
+                const bool grow = (mx[0] > m_ref[0] + 8.f) || (mx[1] > m_ref[1] + 8.f);
+                if (__any_sync(0xffffffffu, grow)) {
+                    float a[2];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const float mn = fmaxf(m_ref[h], mx[h]);
+                        a[h] = (mn == m_ref[h]) ? 1.f : exp2f(m_ref[h] - mn);
+                        m_ref[h] = mn;
+                        l_part[h] *= a[h];
+                    }
+#pragma unroll
+                    for (int n = 0; n < C::kOT; ++n) {
+                        o[n][0] *= a[0];
+                        o[n][1] *= a[0];
+                        o[n][2] *= a[1];
+                        o[n][3] *= a[1];
+                    }
+                }
+                // ---- probabilities straight into the A fragments of P V
+                uint32_t pa[C::kPK][4];
+#pragma unroll
+                for (int n = 0; n < C::kNT; ++n) {
+                    float pv[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float mr = m_ref[e >> 1];
+                        pv[e] = (sc[n][e] == -INFINITY) ? 0.f : exp2f(sc[n][e] - mr);
+                        l_part[e >> 1] += pv[e];
+                    }
+                    pa[n >> 1][(n & 1) * 2 + 0] = pack2<kBF16>(pv[0], pv[1]);
+                    pa[n >> 1][(n & 1) * 2 + 1] = pack2<kBF16>(pv[2], pv[3]);
+                }
+                // ---- tail page: zero V rows past the length (they may hold stale data)
+                if (nvalid < P) {
+                    for (int idx = lane; idx < (P - nvalid) * C::kBoxes * 8; idx += 32) {
+                        const int t = nvalid + idx / (C::kBoxes * 8);
+                        const int rem = idx % (C::kBoxes * 8);
+                        sts128_zero(sV + (rem >> 3) * C::kBoxB + t * 128 + ((rem & 7) << 4));
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+                // ---- O += P V (k = tokens, n = dims)
+#pragma unroll
+                for (int ks = 0; ks < C::kPK; ++ks) {
+                    const int t = ks * 16 + (mi & 1) * 8 + rr8;
+#pragma unroll
+                    for (int op = 0; op < C::kOT / 2; ++op) {
+                        const int c = op * 2 + (mi >> 1);
+                        uint32_t v0, v1, v2, v3;
+                        ldsm_x4_trans(sV + (c >> 3) * C::kBoxB + t * 128 + (((c & 7) ^ (t & 7)) << 4), v0, v1, v2, v3);
+                        mma_16816<kBF16>(o[2 * op], pa[ks], v0, v1);
+                        mma_16816<kBF16>(o[2 * op + 1], pa[ks], v2, v3);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty_bar + 8 * s);
+        }
+    }
+
+    // ---- finalize: row sums over the quad, then merge page-warps in shared memory
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        l_part[h] += __shfl_xor_sync(0xffffffffu, l_part[h], 1);
+        l_part[h] += __shfl_xor_sync(0xffffffffu, l_part[h], 2);
+    }
+    named_bar_sync(1, 32 * NW);  // every consumer is done with the stages (merge rows alias them)
+    float* merge = reinterpret_cast<float*>(smem);  // [NW][16][DH + 2]
+    if (active) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int r = r0 + 8 * h;
+            if (r < rows) {
+                float* dst = merge + (cw * 16 + r) * (DH + 2);
+#pragma unroll
+                for (int n = 0; n < C::kOT; ++n) {
+                    dst[n * 8 + 2 * quad] = o[n][2 * h];
+                    dst[n * 8 + 2 * quad + 1] = o[n][2 * h + 1];
+                }
+                if (quad == 0) {
+                    dst[DH] = m_ref[h];
+                    dst[DH + 1] = l_part[h];
+                }
+            }
+        }
+    }
+    named_bar_sync(1, 32 * NW);
+
+    const int tid = threadIdx.x - 32;
+    for (int e = tid; e < p.g * DH; e += 32 * NW) {
+        const int hh = e / DH;
+        const int d = e % DH;
+        const int slice = hh >> 4, r = hh & 15;
+        float mstar = -INFINITY;
+        for (int w = 0; w < p.WP; ++w) mstar = fmaxf(mstar, merge[((w * p.HS + slice) * 16 + r) * (DH + 2) + DH]);
+        float L = 0.f, U = 0.f;
+        if (mstar != -INFINITY) {
+            for (int w = 0; w < p.WP; ++w) {
+                const float* src = merge + ((w * p.HS + slice) * 16 + r) * (DH + 2);
+                const float mw = src[DH];
+                if (mw == -INFINITY) continue;
+                const float sw = exp2f(mw - mstar);
+                L += sw * src[DH + 1];
+                U += sw * src[d];
+            }
+        }
+        const int64_t hq = (int64_t)b * p.H_q + (int64_t)kvh * p.g + hh;
+        if (!split_mode) {
+            p.out[hq * DH + d] = (L > 0.f) ? U / L : 0.f;
+        } else {
+            const int64_t ps = hq * p.num_splits + split;
+            p.part_u[ps * DH + d] = U;
+            if (d == 0) p.part_ml[ps] = make_float2(mstar, L);
+        }
+    }
+}
+
+}  // namespace kvp

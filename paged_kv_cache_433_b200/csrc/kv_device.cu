@@ -1,6 +1,8 @@
 // Device entry points of the C ABI: kv_append and paged_decode_attention
 // (argument checks, split-KV planning, launches). The kernels themselves are
 // in decode_kernel.cuh; see include/kvpaged.h for the contract.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -108,6 +110,46 @@ int resolve_splits(int32_t B, int32_t H_kv, int32_t max_blocks, int32_t num_spli
     return KV_OK;
 }
 
+std::atomic<int> g_kernel_kind{KV_DECODE_KERNEL_AUTO};
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::atomic<bool> tried{false};
+    if (!tried.load(std::memory_order_acquire)) {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+        tried.store(true, std::memory_order_release);
+    }
+    return fn;
+}
+
+// A K or V pool [num_pages][H_kv][P][Dh] seen as a 2-D tensor of
+// num_pages * H_kv * P rows of Dh 16-bit elements; boxes of P rows x 64
+// elements (128 bytes) with 128-byte swizzle.
+bool make_pool_map(CUtensorMap* m, const void* base, int32_t dtype, int64_t rows, int32_t Dh, int32_t P) {
+    auto enc = tensor_map_encoder();
+    if (!enc || rows >= (1LL << 32)) return false;
+    cuuint64_t gdim[2] = {static_cast<cuuint64_t>(Dh), static_cast<cuuint64_t>(rows)};
+    cuuint64_t gstride[1] = {static_cast<cuuint64_t>(Dh) * 2};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(P)};
+    cuuint32_t estride[2] = {1, 1};
+    CUresult r = enc(m, dtype == KV_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                     const_cast<void*>(base), gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Tensor cores for 16-bit K/V when the GQA group fits 4 slices of 16 rows.
+bool use_mma(int32_t dtype, int32_t g) {
+    const int kind = g_kernel_kind.load(std::memory_order_relaxed);
+    if (dtype == KV_DTYPE_F32 || kind == KV_DECODE_KERNEL_SIMT) return false;
+    return g <= 64;
+}
+
 size_t workspace_for(int32_t B, int32_t H_q, int32_t Dh, int32_t S) {
     if (S <= 1) return 0;
     const size_t rows = static_cast<size_t>(B) * H_q * S;
@@ -120,7 +162,7 @@ int check_shape(int32_t H_q, int32_t H_kv, int32_t Dh, int32_t page_size, int32_
     if (Dh != 64 && Dh != 128) return KV_ERR_UNSUPPORTED;
     if (page_size != 16 && page_size != 32) return KV_ERR_UNSUPPORTED;
     int a, b, c, d;
-    if (!plan_group(H_q / H_kv, &a, &b, &c, &d)) return KV_ERR_UNSUPPORTED;
+    if (!use_mma(dtype, H_q / H_kv) && !plan_group(H_q / H_kv, &a, &b, &c, &d)) return KV_ERR_UNSUPPORTED;
     return KV_OK;
 }
 
@@ -150,6 +192,12 @@ int kv_append(void* k_pages, void* v_pages, const void* k_new, const void* v_new
         static_cast<const uint4*>(v_new), slot_mapping, rows, H_kv, vpr, page_size,
         static_cast<int64_t>(num_pages) * page_size, err_flag);
     return cudaGetLastError() == cudaSuccess ? KV_OK : KV_ERR_CUDA;
+}
+
+int paged_decode_set_kernel(int32_t kind) {
+    if (kind != KV_DECODE_KERNEL_AUTO && kind != KV_DECODE_KERNEL_SIMT && kind != KV_DECODE_KERNEL_MMA) return KV_ERR_ARG;
+    g_kernel_kind.store(kind, std::memory_order_relaxed);
+    return KV_OK;
 }
 
 int paged_decode_num_splits(int32_t B, int32_t H_kv, int32_t max_blocks, int32_t page_size, int32_t num_splits,
@@ -184,8 +232,17 @@ int paged_decode_attention(float* out, const void* q, const void* k_pages, const
     if (B > 65535 || H_kv > 65535) return KV_ERR_UNSUPPORTED;
     if (!out || !q || !k_pages || !v_pages || !block_tables || !seq_lens) return KV_ERR_ARG;
     if (!aligned16(out) || !aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages)) return KV_ERR_ARG;
-    int GW, HS, NW, WP;
-    plan_group(H_q / H_kv, &GW, &HS, &NW, &WP);
+    const int32_t g = H_q / H_kv;
+    // TMA row coordinates are int32: very large pools stay on the CUDA-core kernel.
+    const bool mma = use_mma(dtype, g) && static_cast<int64_t>(num_pages) * H_kv * page_size < (1LL << 31);
+    int GW = 0, HS, NW, WP;
+    if (mma) {
+        HS = (g + 15) / 16;
+        NW = 4;
+        WP = NW / HS;
+    } else {
+        plan_group(g, &GW, &HS, &NW, &WP);
+    }
     int32_t S, C;
     rc = resolve_splits(B, H_kv, max_blocks, num_splits, &S, &C);
     if (rc != KV_OK) return rc;
@@ -219,10 +276,20 @@ int paged_decode_attention(float* out, const void* q, const void* k_pages, const
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     dim3 grid(static_cast<unsigned>(S), static_cast<unsigned>(H_kv), static_cast<unsigned>(B));
     cudaError_t e;
-    switch (dtype) {
-        case KV_DTYPE_F32: e = launch_decode_f32(p, Dh, page_size, GW, NW, grid, st); break;
-        case KV_DTYPE_BF16: e = launch_decode_bf16(p, Dh, page_size, GW, NW, grid, st); break;
-        default: e = launch_decode_f16(p, Dh, page_size, GW, NW, grid, st); break;
+    if (mma) {
+        CUtensorMap tk, tv;
+        const int64_t rows = static_cast<int64_t>(num_pages) * H_kv * page_size;
+        if (!make_pool_map(&tk, k_pages, dtype, rows, Dh, page_size) ||
+            !make_pool_map(&tv, v_pages, dtype, rows, Dh, page_size))
+            return KV_ERR_CUDA;
+        e = dtype == KV_DTYPE_BF16 ? launch_mma_bf16(p, tk, tv, Dh, page_size, grid, st)
+                                   : launch_mma_f16(p, tk, tv, Dh, page_size, grid, st);
+    } else {
+        switch (dtype) {
+            case KV_DTYPE_F32: e = launch_decode_f32(p, Dh, page_size, GW, NW, grid, st); break;
+            case KV_DTYPE_BF16: e = launch_decode_bf16(p, Dh, page_size, GW, NW, grid, st); break;
+            default: e = launch_decode_f16(p, Dh, page_size, GW, NW, grid, st); break;
+        }
     }
     if (e != cudaSuccess) return KV_ERR_CUDA;
     if (S > 1) {

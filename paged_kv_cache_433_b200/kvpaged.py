@@ -67,6 +67,7 @@ SIGNATURES = [
     ("kv_append", ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
     ("paged_decode_attention", ctypes.c_int,
      [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _i32, _vp, _sz, _vp, _vp]),
+    ("paged_decode_set_kernel", ctypes.c_int, [_i32]),
     ("paged_decode_num_splits", ctypes.c_int, [_i32, _i32, _i32, _i32, _i32, _pi32]),
     ("paged_decode_workspace_bytes", ctypes.c_int, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, _psz]),
 ]
@@ -279,6 +280,13 @@ def kv_append(k_pages, v_pages, k_new, v_new, slot_mapping, page_size: int, err_
                          _dev(v_new, "v_new", k_pages.dtype), _dev(slot_mapping, "slot_mapping", torch.int64), B, H_kv, Dh,
                          page_size, num_pages, dt, _dev(err_flag, "err_flag", torch.int32), _stream(stream))
     _check("kv_append", rc)
+
+
+KV_DECODE_KERNEL_AUTO, KV_DECODE_KERNEL_SIMT, KV_DECODE_KERNEL_MMA = 0, 1, 2
+
+
+def paged_decode_set_kernel(kind: int) -> None:
+    _check("paged_decode_set_kernel", lib().paged_decode_set_kernel(kind))
 
 
 def paged_decode_num_splits(B: int, H_kv: int, max_blocks: int, page_size: int, num_splits: int = 0) -> int:

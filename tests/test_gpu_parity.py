@@ -28,6 +28,14 @@ def _built():
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
 
 
+@pytest.fixture(params=["mma", "simt"])
+def kernel(request):
+    """Run the test with the tensor-core kernel (default for 16-bit K/V) and with the CUDA-core kernel."""
+    K.paged_decode_set_kernel(K.KV_DECODE_KERNEL_MMA if request.param == "mma" else K.KV_DECODE_KERNEL_SIMT)
+    yield request.param
+    K.paged_decode_set_kernel(K.KV_DECODE_KERNEL_AUTO)
+
+
 # ---------------------------------------------------------------- tiny (fp32)
 @pytest.mark.parametrize("splits", [1, 2, 0])
 def test_tiny_fp32_against_oracle_and_full_causal(splits):
@@ -52,7 +60,7 @@ def test_tiny_fp32_against_oracle_and_full_causal(splits):
 
 # ---------------------------------------------------------------- Llama-3.1-8B-shaped layer (bf16)
 @pytest.mark.parametrize("splits", [1, 3, 0])
-def test_llama8b_reduced_batch(splits):
+def test_llama8b_reduced_batch(splits, kernel):
     cfg = W.LLAMA8B
     lens = W.cached_lengths(cfg)[:8]
     st = build_cache(cfg, lens)
@@ -63,7 +71,7 @@ def test_llama8b_reduced_batch(splits):
 
 
 @pytest.mark.parametrize("splits", [0, 1])
-def test_llama8b_full_size(splits):
+def test_llama8b_full_size(splits, kernel):
     """The full workload (B=64, lengths U[512, 4096]) in the launch configuration the benchmark times."""
     cfg = W.LLAMA8B
     st = build_cache(cfg, W.cached_lengths(cfg))
@@ -74,7 +82,7 @@ def test_llama8b_full_size(splits):
 
 # ---------------------------------------------------------------- 32K context (fp16, split-KV)
 @pytest.mark.parametrize("layer,splits", [(0, 0), (31, 0), (0, 1), (0, 7)])
-def test_long_context_layer(layer, splits):
+def test_long_context_layer(layer, splits, kernel):
     cfg = W.LONG32K
     st = build_cache(cfg, W.cached_lengths(cfg), layer=layer)
     if splits == 0:
@@ -85,7 +93,7 @@ def test_long_context_layer(layer, splits):
 
 
 # ---------------------------------------------------------------- shared prefix (bf16)
-def test_shared_prefix_batch():
+def test_shared_prefix_batch(kernel):
     cfg = W.SHARED_PREFIX
     P = cfg.page_size
     wl = W.prefix_workload(cfg)
@@ -160,7 +168,7 @@ def test_shared_prefix_batch():
 
 # ---------------------------------------------------------------- mixed continuous batching
 @pytest.mark.parametrize("H_kv,P", W.MIXED_POINTS)
-def test_mixed_sweep_with_churn(H_kv, P):
+def test_mixed_sweep_with_churn(H_kv, P, kernel):
     base = W.mixed_config(H_kv, P)
     B = 24
     lens = W.cached_lengths(base)[:B]
@@ -189,7 +197,7 @@ EDGE_SHAPES = [
 
 @pytest.mark.parametrize("dtype,Dh,P,H_q,H_kv", EDGE_SHAPES)
 @pytest.mark.parametrize("splits", [1, 2, 0])
-def test_edge_lengths_and_shapes(dtype, Dh, P, H_q, H_kv, splits):
+def test_edge_lengths_and_shapes(dtype, Dh, P, H_q, H_kv, splits, kernel):
     cfg = W.DecodeConfig(f"edge-{dtype}-{Dh}-{P}-{H_q}-{H_kv}", dtype, B=6, H_q=H_q, H_kv=H_kv, Dh=Dh, page_size=P, seed=9)
     # after the append: 1, P-1, P, P+1, 3P+5 tokens, and one sequence filling its table exactly
     lens = [0, P - 2, P - 1, P, 3 * P + 4, 4 * P - 1]
@@ -206,7 +214,7 @@ def test_edge_lengths_and_shapes(dtype, Dh, P, H_q, H_kv, splits):
         assert np.array_equal(out[0, h], v0[h // g].astype(np.float32))
 
 
-def test_zero_length_rows_are_zero():
+def test_zero_length_rows_are_zero(kernel):
     cfg = W.DecodeConfig("zero", "bf16", B=3, H_q=8, H_kv=2, Dh=128, page_size=16, seed=12)
     P = cfg.page_size
     k_pages = torch.full((4, 2, P, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
@@ -224,7 +232,7 @@ def test_zero_length_rows_are_zero():
         assert torch.count_nonzero(out).item() == 0 and int(err.item()) == 0
 
 
-def test_page_permutation_invariance_bitwise():
+def test_page_permutation_invariance_bitwise(kernel):
     """Same logical content behind two different physical page orders -> bit-identical output."""
     cfg = W.LLAMA8B
     lens = W.cached_lengths(cfg)[:6]
@@ -239,7 +247,7 @@ def test_page_permutation_invariance_bitwise():
 
 
 # ---------------------------------------------------------------- device error flags (host-checked, no faults)
-def test_device_error_flags():
+def test_device_error_flags(kernel):
     P, Dh = 16, 128
     k_pages = torch.zeros((4, 2, P, Dh), dtype=torch.bfloat16, device="cuda")
     v_pages = torch.zeros_like(k_pages)

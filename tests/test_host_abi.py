@@ -351,8 +351,15 @@ def test_device_entry_argument_checks_without_gpu():
     args[11] = 24
     assert L.paged_decode_attention(*args) == K.KV_ERR_UNSUPPORTED  # page size 24
     args[11] = 16
-    args[8], args[9] = 33, 1
-    assert L.paged_decode_attention(*args) == K.KV_ERR_UNSUPPORTED  # GQA group of 33
+    args[8], args[9] = 65, 1
+    assert L.paged_decode_attention(*args) == K.KV_ERR_UNSUPPORTED  # GQA group of 65 (tensor-core limit 64)
+    args[8] = 33
+    K.paged_decode_set_kernel(K.KV_DECODE_KERNEL_SIMT)
+    try:
+        assert L.paged_decode_attention(*args) == K.KV_ERR_UNSUPPORTED  # CUDA-core limit 32
+    finally:
+        K.paged_decode_set_kernel(K.KV_DECODE_KERNEL_AUTO)
+    assert L.paged_decode_set_kernel(7) == K.KV_ERR_ARG
     args[8], args[9] = 32, 7
     assert L.paged_decode_attention(*args) == K.KV_ERR_ARG  # H_q % H_kv != 0
     args[9] = 8
