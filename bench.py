@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="config 3: launch the 32 layers without a CUDA graph")
+    ap.add_argument("--kernel", choices=["auto", "simt", "mma"], default="auto",
+                    help="decode kernel: tensor cores (auto/mma, 16-bit K/V) or CUDA cores (simt)")
     return ap.parse_args()
 
 
@@ -586,6 +588,10 @@ def main():
         print(json.dumps(run_reference(args)), flush=True)
         return 0
     world, rank, local = setup_dist(args)
+    from paged_kv_cache_433_b200 import kvpaged as K
+
+    K.paged_decode_set_kernel({"auto": K.KV_DECODE_KERNEL_AUTO, "simt": K.KV_DECODE_KERNEL_SIMT,
+                               "mma": K.KV_DECODE_KERNEL_MMA}[args.kernel])
     if args.config == 2:
         res = run_layer_bench(args, world, rank, local)
     else:
