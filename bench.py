@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="config 3: launch the 32 layers without a CUDA graph")
+    ap.add_argument("--page-order", choices=["shuffled", "sequential"], default="shuffled",
+                    help="physical page order of the pool's free list (the workloads use shuffled pages)")
     ap.add_argument("--kernel", choices=["auto", "simt", "mma"], default="auto",
                     help="decode kernel: tensor cores (auto/mma, 16-bit K/V) or CUDA cores (simt)")
     return ap.parse_args()
@@ -117,7 +119,7 @@ class ClockSampler:
 class Workload:
     """Device-resident inputs of every step, built through the library's own calls."""
 
-    def __init__(self, cfg, lens, n_steps, rank, splits, layers=1):
+    def __init__(self, cfg, lens, n_steps, rank, splits, layers=1, sequential=False):
         import torch
 
         from paged_kv_cache_433_b200 import kvpaged as K
@@ -133,7 +135,8 @@ class Workload:
         self.dt = dt
         self.max_blocks = max(-(-(int(L) + n_steps) // P) for L in lens) + 1
         self.num_pages = int(sum(-(-(int(L) + n_steps) // P) for L in lens)) + 8
-        order = W.page_order(self.num_pages, cfg.seed + 1000 * rank)
+        order = (np.arange(self.num_pages, dtype=np.int32) if sequential
+                 else W.page_order(self.num_pages, cfg.seed + 1000 * rank))
         self.pool = K.KvPool(self.num_pages, P, order)
         self.tab = np.full((B, self.max_blocks), -1, np.int32)
         for b in range(B):
@@ -235,7 +238,7 @@ def run_layer_bench(args, world, rank, local):
     lens = W.cached_lengths(cfg)
     e2e_steps = 0 if args.no_e2e else steps
     n_steps = warm + steps + (warm + e2e_steps if e2e_steps else 0)
-    wl = Workload(cfg, lens, n_steps, rank, args.splits)
+    wl = Workload(cfg, lens, n_steps, rank, args.splits, sequential=args.page_order == "sequential")
     B, P = wl.B, cfg.page_size
     dev = torch.device("cuda")
 
@@ -304,7 +307,7 @@ def run_layer_bench(args, world, rank, local):
         "ms_per_step": elapsed_ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": cfg.dtype, "data": "synthetic (seeded N(0,1) K/V, q; lengths U[512,4096])",
         "config": {"workload": cfg.name, "B": B, "H_q": cfg.H_q, "H_kv": cfg.H_kv, "Dh": cfg.Dh, "page_size": P,
-                   "layers": 1, "num_splits": S, "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+                   "layers": 1, "num_splits": S, "page_order": args.page_order, "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
                    "l2": "inputs larger than L2 (K/V working set %.0f MB > 126 MB L2); no flush" % (mean_bytes / 1e6)},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS hbm_gbs)" if peak_kind == "measured" else "fallback",
@@ -396,7 +399,7 @@ def run_long_bench(args, world, rank, local):
     L = cfg.layers
     lens = W.cached_lengths(cfg)
     T1 = warm + steps
-    wl = Workload(cfg, lens, T1 + 1, rank, args.splits, layers=L)
+    wl = Workload(cfg, lens, T1 + 1, rank, args.splits, layers=L, sequential=args.page_order == "sequential")
     B, P = wl.B, cfg.page_size
     dev = torch.device("cuda")
     slot_list, lens_list = [], []

@@ -496,17 +496,25 @@ __global__ void __launch_bounds__(32 * (NW + 1), (NW <= 4) ? 2 : 1) paged_decode
 
 // Merge split partials (the same (m, l, u) rule over the splits of one row):
 // m* = max_s m_s, o = sum_s 2^{m_s - m*} u_s / sum_s 2^{m_s - m*} l_s.
-// One warp per (sequence, query head).
+// One CTA of kCombineWarps warps per (sequence, query head). Every warp finds
+// m* over all splits; warp w then accumulates splits w, w + kCombineWarps, ...
+// eight at a time (loads of a batch are independent, so their latencies
+// overlap), and the warps' sums -- all relative to the same m* -- are added
+// in shared memory.
+constexpr int kCombineWarps = 4;
+
 template <int DH>
-__global__ void __launch_bounds__(128) paged_combine_kernel(float* __restrict__ out, const float* __restrict__ part_u,
-                                                            const float2* __restrict__ part_ml,
-                                                            const int32_t* __restrict__ seq_lens, int32_t B,
-                                                            int32_t H_q, int32_t S, int32_t pages_per_split,
-                                                            int32_t P, int32_t max_blocks) {
+__global__ void __launch_bounds__(32 * kCombineWarps) paged_combine_kernel(
+    float* __restrict__ out, const float* __restrict__ part_u, const float2* __restrict__ part_ml,
+    const int32_t* __restrict__ seq_lens, int32_t B, int32_t H_q, int32_t S, int32_t pages_per_split, int32_t P,
+    int32_t max_blocks) {
     constexpr int kD = DH / 32;  // dims per lane
-    const int item = blockIdx.x * 4 + (threadIdx.x >> 5);
+    constexpr int kBatch = 8;
+    __shared__ float red_u[kCombineWarps][DH];
+    __shared__ float red_l[kCombineWarps];
+    const int item = blockIdx.x;
+    const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    if (item >= B * H_q) return;
     const int b = item / H_q;
     int len = seq_lens[b];
     if (len < 0 || len > max_blocks * P) len = 0;
@@ -523,24 +531,50 @@ __global__ void __launch_bounds__(128) paged_combine_kernel(float* __restrict__ 
     for (int i = 0; i < kD; ++i) acc[i] = 0.f;
     float L = 0.f;
     if (mstar != -INFINITY) {
-        for (int s = 0; s < ns; ++s) {
-            const float2 st = ml[s];
-            const float w = (st.x == -INFINITY) ? 0.f : exp2f(st.x - mstar);
-            L += w * st.y;
-            const float* src = pu + (int64_t)s * DH + lane * kD;
-            if constexpr (kD == 4) {
-                const float4 v = *reinterpret_cast<const float4*>(src);
-                acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
-            } else {
+        for (int s0 = warp; s0 < ns; s0 += kCombineWarps * kBatch) {
+            float2 st[kBatch];
+            float v[kBatch][kD];
 #pragma unroll
-                for (int i = 0; i < kD; ++i) acc[i] += w * src[i];
+            for (int j = 0; j < kBatch; ++j) {
+                const int s = s0 + j * kCombineWarps;
+                if (s < ns) {
+                    st[j] = ml[s];
+                    const float* src = pu + (int64_t)s * DH + lane * kD;
+                    if constexpr (kD == 4) {
+                        const float4 x = *reinterpret_cast<const float4*>(src);
+                        v[j][0] = x.x; v[j][1] = x.y; v[j][2] = x.z; v[j][3] = x.w;
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < kD; ++i) v[j][i] = src[i];
+                    }
+                } else {
+                    st[j] = make_float2(-INFINITY, 0.f);
+#pragma unroll
+                    for (int i = 0; i < kD; ++i) v[j][i] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) {
+                const float w = (st[j].x == -INFINITY) ? 0.f : exp2f(st[j].x - mstar);
+                L += w * st[j].y;
+#pragma unroll
+                for (int i = 0; i < kD; ++i) acc[i] += w * v[j][i];
             }
         }
     }
-    const float inv = (L > 0.f) ? 1.f / L : 0.f;
-    float* dst = out + (int64_t)item * DH + lane * kD;
 #pragma unroll
-    for (int i = 0; i < kD; ++i) dst[i] = acc[i] * inv;
+    for (int i = 0; i < kD; ++i) red_u[warp][lane * kD + i] = acc[i];
+    if (lane == 0) red_l[warp] = L;
+    __syncthreads();
+    for (int d = threadIdx.x; d < DH; d += blockDim.x) {
+        float U = 0.f, Lt = 0.f;
+#pragma unroll
+        for (int w = 0; w < kCombineWarps; ++w) {
+            U += red_u[w][d];
+            Lt += red_l[w];
+        }
+        out[(int64_t)item * DH + d] = (Lt > 0.f) ? U / Lt : 0.f;
+    }
 }
 
 }  // namespace kvp

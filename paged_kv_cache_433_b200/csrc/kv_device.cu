@@ -293,14 +293,13 @@ int paged_decode_attention(float* out, const void* q, const void* k_pages, const
     }
     if (e != cudaSuccess) return KV_ERR_CUDA;
     if (S > 1) {
-        const int64_t items = static_cast<int64_t>(B) * H_q;
-        const unsigned blocks = static_cast<unsigned>((items + 3) / 4);
+        const unsigned blocks = static_cast<unsigned>(static_cast<int64_t>(B) * H_q);
         if (Dh == 128)
-            paged_combine_kernel<128><<<blocks, 128, 0, st>>>(out, p.part_u, p.part_ml, seq_lens, B, H_q, S, C,
-                                                              page_size, max_blocks);
+            paged_combine_kernel<128><<<blocks, 32 * kCombineWarps, 0, st>>>(out, p.part_u, p.part_ml, seq_lens, B, H_q,
+                                                                              S, C, page_size, max_blocks);
         else
-            paged_combine_kernel<64><<<blocks, 128, 0, st>>>(out, p.part_u, p.part_ml, seq_lens, B, H_q, S, C,
-                                                             page_size, max_blocks);
+            paged_combine_kernel<64><<<blocks, 32 * kCombineWarps, 0, st>>>(out, p.part_u, p.part_ml, seq_lens, B, H_q,
+                                                                             S, C, page_size, max_blocks);
         if (cudaGetLastError() != cudaSuccess) return KV_ERR_CUDA;
     }
     return KV_OK;
