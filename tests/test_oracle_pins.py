@@ -338,3 +338,23 @@ def test_cached_free_page_is_matchable_until_reallocated():
     assert got == [3] and ix.match(toks) == pages
     got = pool.alloc(1)  # hands out block 2 -> its prefix entry is dropped
     assert got == [2] and ix.match(toks) == pages[:2]
+
+
+def test_merge_of_summarised_blocks_equals_full_softmax():
+    """Merging per-block (m, l, u) summaries (the split combine rule) == online merge == full softmax."""
+    gd = golden("online_merge_two_blocks.json")
+    b1, b2 = ((b["scores"], np.array(b["values"])) for b in gd["blocks"])
+    m, l, u = R.merge_states(R.block_state(*b1), R.block_state(*b2))
+    assert m == 3.0 and abs(l - gd["l"]) <= 5e-7 and abs(u[0] - gd["u"]) <= 5e-7
+    rng = np.random.default_rng(3)
+    s = rng.standard_normal(40) * 3
+    v = rng.standard_normal((40, 5))
+    cuts = [0, 7, 8, 23, 40]
+    states = [R.block_state(s[a:b], v[a:b]) for a, b in zip(cuts[:-1], cuts[1:])]
+    acc = states[0]
+    for st in states[1:]:
+        acc = R.merge_states(acc, st)
+    full = R.softmax_weighted_sum(s, v)
+    assert np.allclose(acc[2] / acc[1], full, atol=1e-12)
+    _, _, _, o = R.online_softmax([(s[a:b], v[a:b]) for a, b in zip(cuts[:-1], cuts[1:])])
+    assert np.allclose(o, full, atol=1e-12)
