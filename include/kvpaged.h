@@ -235,6 +235,29 @@ int paged_decode_num_splits(int32_t B, int32_t H_kv, int32_t max_blocks, int32_t
 int paged_decode_workspace_bytes(int32_t B, int32_t H_q, int32_t H_kv, int32_t Dh, int32_t max_blocks,
                                  int32_t page_size, int32_t num_splits, size_t* out);
 
+/* Same computation as paged_decode_attention, for callers that cannot
+ * allocate device memory -- for example a plug-in whose host framework owns
+ * every device allocation and passes in only input and output tensors, or a
+ * latency-critical path that must not allocate. Instead of a workspace, the
+ * split partials use a fixed array of KV_NOALLOC_SCRATCH_BYTES in the
+ * library's own device memory (held on every GPU that loads the library until
+ * the process exits). No allocation of any kind happens in the call.
+ * The pages describe nothing of this kind: it has no counterpart there.
+ *   - The first call on a device looks up that array's device address
+ *     (cudaGetSymbolAddress, which may load the module): make it before any
+ *     stream capture on that device.
+ *   - All calls share the array and it keeps the last call's contents; calls
+ *     whose kernels may overlap on the GPU (unordered streams) race on it.
+ *   - KV_ERR_WORKSPACE when the partials for these arguments
+ *     (paged_decode_workspace_bytes) exceed KV_NOALLOC_SCRATCH_BYTES; use
+ *     fewer splits or the workspace entry point then.
+ * Other arguments, errors and results: as paged_decode_attention. */
+#define KV_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
+int paged_decode_attention_noalloc(float* out, const void* q, const void* k_pages, const void* v_pages,
+                                   const int32_t* block_tables, int32_t max_blocks, const int32_t* seq_lens, int32_t B,
+                                   int32_t H_q, int32_t H_kv, int32_t Dh, int32_t page_size, int32_t num_pages,
+                                   float scale, int32_t dtype, int32_t num_splits, int* err_flag, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
