@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="config 3: launch the 32 layers without a CUDA graph")
+    ap.add_argument("--page-size", type=int, choices=[16, 32], default=None,
+                    help="override the workload's page size (the 8B-shaped workload uses 16)")
     ap.add_argument("--page-order", choices=["shuffled", "sequential"], default="shuffled",
                     help="physical page order of the pool's free list (the workloads use shuffled pages)")
     ap.add_argument("--kernel", choices=["auto", "simt", "mma"], default="auto",
@@ -175,7 +177,7 @@ class Workload:
         cfg = self.cfg
         nb = self.K.paged_decode_workspace_bytes(self.B, cfg.H_q, cfg.H_kv, cfg.Dh, self.max_blocks, cfg.page_size,
                                                  self.splits)
-        return self.torch.empty(max(nb, 16), dtype=self.torch.uint8, device="cuda")
+        return self.torch.zeros(max(nb, 16), dtype=self.torch.uint8, device="cuda")
 
     def step_bytes(self, lens_after):
         """Algorithmic bytes of one decode launch (one layer): K/V rows actually attended,
@@ -233,6 +235,10 @@ def run_layer_bench(args, world, rank, local):
     from paged_kv_cache_433_b200 import workloads as W
 
     cfg = W.LLAMA8B
+    if args.page_size is not None and args.page_size != cfg.page_size:
+        import dataclasses
+
+        cfg = dataclasses.replace(cfg, page_size=args.page_size, name=cfg.name.replace("-P16", f"-P{args.page_size}"))
     steps = args.steps if args.steps is not None else cfg.timed_steps
     warm = args.warmup if args.warmup is not None else cfg.warmup_steps
     lens = W.cached_lengths(cfg)

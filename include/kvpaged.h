@@ -205,7 +205,8 @@ int kv_append(void* k_pages, void* v_pages, const void* k_new, const void* v_new
  *   0 = choose automatically from B, H_kv, max_blocks and the SM count.
  *   workspace / ws_bytes: device scratch for split partials, at least
  *   paged_decode_workspace_bytes(...) for the same arguments (NULL/0 is fine
- *   when no split is used); KV_ERR_WORKSPACE if too small. */
+ *   when no split is used); KV_ERR_WORKSPACE if too small. Calls sharing one
+ *   workspace must be ordered on the GPU (e.g. one stream). */
 int paged_decode_attention(float* out, const void* q, const void* k_pages, const void* v_pages,
                            const int32_t* block_tables, int32_t max_blocks, const int32_t* seq_lens, int32_t B,
                            int32_t H_q, int32_t H_kv, int32_t Dh, int32_t page_size, int32_t num_pages, float scale,

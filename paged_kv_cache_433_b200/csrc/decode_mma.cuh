@@ -27,6 +27,13 @@
 
 #include "decode_kernel.cuh"
 
+#ifndef KVP_PRODUCER_SINGLE_LANE
+#define KVP_PRODUCER_SINGLE_LANE 0
+#endif
+#ifndef KVP_MMA_STAGE_BUDGET
+#define KVP_MMA_STAGE_BUDGET (96 * 1024)
+#endif
+
 namespace kvp {
 
 template <int DH, int P, int NW>
@@ -39,7 +46,7 @@ struct MmaCfg {
     static constexpr int kNT = P / 8;              // token n-tiles of S
     static constexpr int kPK = P / 16;             // PV k-steps
     static constexpr int kOT = DH / 8;             // dim n-tiles of O
-    static constexpr int kStageBudget = 96 * 1024;
+    static constexpr int kStageBudget = KVP_MMA_STAGE_BUDGET;
     // Stage i % NS is drained by page-warp i % WP (WP divides NW): NS must be
     // a multiple of NW so each stage always goes to the same warp.
     static constexpr int kNS0 = (kStageBudget / kStage) / NW * NW;
@@ -110,6 +117,7 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
         const int32_t* row = p.block_tables + (int64_t)b * p.max_blocks + first;
         bool ok = true;
         int issued = 0;
+#if KVP_PRODUCER_SINGLE_LANE
         for (int base = 0; base < n_local && ok; base += 32) {
             const int my = (base + lane < n_local) ? row[base + lane] : 0;
             const int cnt = min(32, n_local - base);
@@ -144,6 +152,52 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
                 if (!ok) break;
             }
         }
+#else
+        // A group of kGrp pages per step: lane l < kGrp claims the stage of
+        // page base + l (bounded wait on its empty barrier, tag, expect_tx),
+        // then every lane issues one TMA box: box l % kBPP of page l / kBPP.
+        constexpr int kBPP = 2 * C::kBoxes;  // boxes per page (K and V)
+        constexpr int kGrp0 = 32 / kBPP;
+        constexpr int kGrpMax = kGrp0 < C::kNS ? kGrp0 : C::kNS;
+        constexpr int kGrp = kGrpMax >= 16 ? 16 : kGrpMax >= 8 ? 8 : kGrpMax >= 4 ? 4 : kGrpMax >= 2 ? 2 : 1;
+        static_assert(32 % kGrp == 0, "page groups must tile the 32-entry table window");
+        int tab = 0;  // block-table entry of page (base & ~31) + lane
+        for (int base = 0; base < n_local; base += kGrp) {
+            if ((base & 31) == 0) tab = (base + lane < n_local) ? row[base + lane] : 0;
+            const int cnt = min(kGrp, n_local - base);
+            const int pg = __shfl_sync(0xffffffffu, tab, ((base & 31) + lane) & 31);
+            bool valid = false;
+            if (lane < cnt) {
+                const int i = base + lane;
+                const int s = i % C::kNS;
+                if (i >= C::kNS && !mbar_wait_bounded(empty_bar + 8 * s, ((i / C::kNS) - 1) & 1, kWaitLimitNs)) {
+                    raise_err(p.err, KV_DEV_ERR_TIMEOUT);
+                    ok = false;
+                } else if (pg >= 0 && pg < p.num_pages) {
+                    valid = true;
+                    stage_tag[s] = i;
+                    mbar_arrive_expect_tx(full_bar + 8 * s, C::kStage);
+                } else {
+                    raise_err(p.err, KV_DEV_ERR_PAGE_RANGE);
+                    stage_tag[s] = -1 - i;
+                    mbar_arrive(full_bar + 8 * s);
+                }
+            }
+            if (!__all_sync(0xffffffffu, ok)) break;
+            const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+            const int pl = lane / kBPP, bx = lane % kBPP;
+            const int pgl = __shfl_sync(0xffffffffu, pg, pl);
+            if (pl < cnt && ((vmask >> pl) & 1u)) {
+                const int s = (base + pl) % C::kNS;
+                const bool is_v = bx >= C::kBoxes;
+                const int bb = is_v ? bx - C::kBoxes : bx;
+                const uint32_t dst = sbase + s * C::kStage + (is_v ? C::kChunk : 0) + bb * C::kBoxB;
+                tma_load_2d(dst, is_v ? static_cast<const void*>(&tmap_v) : static_cast<const void*>(&tmap_k), bb * 64,
+                            (pgl * p.H_kv + kvh) * P, full_bar + 8 * s);
+            }
+            issued = base + cnt;
+        }
+#endif
         if (lane == 0) {
             for (int i = max(0, issued - C::kNS); i < issued; ++i)
                 if (!mbar_wait_bounded(full_bar + 8 * (i % C::kNS), (i / C::kNS) & 1, kWaitLimitNs))

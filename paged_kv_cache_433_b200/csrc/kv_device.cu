@@ -83,21 +83,24 @@ bool plan_group(int32_t g, int* GW, int* HS, int* NW, int* WP) {
 }
 
 // Split count. Explicit requests are honoured (capped at max_blocks). For
-// num_splits == 0 the page walk is split only when (sequence, KV head) CTAs
-// alone cannot fill the GPU: aim for about four CTAs per SM while keeping at
-// least 8 pages in every split.
+// num_splits == 0, with `slots` = 2 CTAs per SM resident:
+//  * B == 1 (every row has the same length): one full wave, S = slots / H_kv;
+//  * otherwise (lengths unknown on the host and usually unequal): about six
+//    CTAs per slot so late short CTAs even out long ones, S = ceil(6 slots /
+//    (B H_kv)), with at least 16 pages per split; S = 1 once rows alone are
+//    that many.
 int resolve_splits(int32_t B, int32_t H_kv, int32_t max_blocks, int32_t num_splits, int32_t* S_out, int32_t* C_out) {
     int32_t S = num_splits;
     if (S <= 0) {
         int sms = sm_count();
         if (sms <= 0) return KV_ERR_CUDA;
-        const int64_t ctas = static_cast<int64_t>(B) * H_kv;
-        const int64_t target = 4LL * sms;
-        if (ctas >= target) {
-            S = 1;
+        const int64_t rows = static_cast<int64_t>(B) * H_kv;
+        const int64_t slots = 2LL * sms;
+        if (B == 1) {
+            S = static_cast<int32_t>(slots / rows > 1 ? slots / rows : 1);
         } else {
-            S = static_cast<int32_t>((target + ctas - 1) / ctas);
-            const int32_t cap = max_blocks / 8 > 1 ? max_blocks / 8 : 1;
+            S = static_cast<int32_t>((6 * slots + rows - 1) / rows);
+            const int32_t cap = max_blocks / 16 > 1 ? max_blocks / 16 : 1;
             if (S > cap) S = cap;
         }
     }

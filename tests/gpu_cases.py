@@ -162,7 +162,7 @@ def append_and_decode(st: Step, layer: int = 0, step: int = 0, num_splits: int =
                 torch.from_numpy(slots).cuda(), P, err_flag=err)
     out = torch.empty((B, cfg.H_q, cfg.Dh), dtype=torch.float32, device="cuda")
     ws_bytes = K.paged_decode_workspace_bytes(B, cfg.H_q, cfg.H_kv, cfg.Dh, st.max_blocks, P, num_splits)
-    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
     K.paged_decode_attention(out, to_device(q, cfg.dtype), st.k_pages, st.v_pages, torch.from_numpy(st.tab).cuda(),
                              torch.from_numpy(lens32).cuda(), cfg.scale, num_splits=num_splits, workspace=ws,
                              err_flag=err)

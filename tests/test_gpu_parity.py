@@ -157,7 +157,7 @@ def test_shared_prefix_batch(kernel):
     K.kv_append(k_pages, v_pages, to_device(k_new, cfg.dtype), to_device(v_new, cfg.dtype), torch.from_numpy(slots).cuda(), P,
                 err_flag=err)
     out = torch.empty((B, cfg.H_q, cfg.Dh), dtype=torch.float32, device="cuda")
-    ws = torch.empty(max(16, K.paged_decode_workspace_bytes(B, cfg.H_q, cfg.H_kv, cfg.Dh, max_blocks, P)), dtype=torch.uint8,
+    ws = torch.zeros(max(16, K.paged_decode_workspace_bytes(B, cfg.H_q, cfg.H_kv, cfg.Dh, max_blocks, P)), dtype=torch.uint8,
                      device="cuda")
     K.paged_decode_attention(out, to_device(q, cfg.dtype), k_pages, v_pages, torch.from_numpy(tab).cuda(),
                              torch.from_numpy(lens32).cuda(), cfg.scale, workspace=ws, err_flag=err)
@@ -224,7 +224,7 @@ def test_zero_length_rows_are_zero(kernel):
     q = to_device(W.queries(cfg, 0, 0), "bf16")
     for splits in (1, 2):
         out = torch.full((3, 8, 128), 7.0, device="cuda")
-        ws = torch.empty(1 << 16, dtype=torch.uint8, device="cuda")
+        ws = torch.zeros(1 << 16, dtype=torch.uint8, device="cuda")
         err = torch.zeros(1, dtype=torch.int32, device="cuda")
         K.paged_decode_attention(out, q, k_pages, v_pages, tab, lens, cfg.scale, num_splits=splits, workspace=ws,
                                  err_flag=err)

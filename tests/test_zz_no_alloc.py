@@ -33,7 +33,7 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
     need = K.paged_decode_workspace_bytes(cfg.B, cfg.H_q, cfg.H_kv, cfg.Dh, st.max_blocks, P, 0)
     assert S > 1 and 0 < need <= K.KV_NOALLOC_SCRATCH_BYTES
     tab = torch.from_numpy(st.tab).cuda()
-    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
     atol, rtol = TOL[cfg.dtype]
     for step in range(2):
         lens32 = st.lens.astype(np.int32).copy()
