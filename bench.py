@@ -33,6 +33,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "paged decode attention seq-steps/s; achieved HBM GB/s and % of B200 peak"
+PROFILE_DECODE = os.path.join(ROOT, "profiles", "paged_decode_mma_kernel__llama8b_layer_bf16_B64.md")
 UNIT = "seq-steps/s"
 FALLBACK_HBM_GBS = 6650.0
 
@@ -53,6 +54,9 @@ def parse():
                     help="override the workload's page size (the 8B-shaped workload uses 16)")
     ap.add_argument("--page-order", choices=["shuffled", "sequential"], default="shuffled",
                     help="physical page order of the pool's free list (the workloads use shuffled pages)")
+    ap.add_argument("--append", choices=["fused", "separate"], default="fused",
+                    help="append the new token inside the decode launch (paged_decode_attention_append) "
+                         "or with kv_append before paged_decode_attention")
     ap.add_argument("--kernel", choices=["auto", "simt", "mma"], default="auto",
                     help="decode kernel: tensor cores (auto/mma, 16-bit K/V) or CUDA cores (simt)")
     return ap.parse_args()
@@ -66,6 +70,34 @@ def peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def decode_kernel_digest():
+    """Digest of the tensor-core decode kernel's sources (a profile is valid only for these)."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for name in ("decode_mma.cuh", "decode_kernel.cuh", "ptx.cuh"):
+        with open(os.path.join(ROOT, "paged_kv_cache_433_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic_ratio():
+    """DRAM bytes / algorithmic bytes of the decode kernel from the committed ncu summary, or None
+    when that capture was not taken from the current kernel sources."""
+    import re
+
+    try:
+        with open(PROFILE_DECODE, encoding="utf-8") as f:
+            text = f.read()
+    except OSError:
+        return None
+    dg = re.search(r"source digest:\s*`?([0-9a-f]{16})", text)
+    ratio = re.search(r"traffic / algorithmic bytes:\s*([0-9.]+)", text)
+    if not dg or not ratio or dg.group(1) != decode_kernel_digest():
+        return None
+    return float(ratio.group(1))
 
 
 # ---------------------------------------------------------------------------- clocks
@@ -190,6 +222,25 @@ class Workload:
         return kv + q + out + tables
 
 
+def hot_path(K, args, cfg, kp, vp, kn, vn, slots, q, tab, lens, out, ws, err, stream, ev=None):
+    """One layer's step on the device: append the new token, then decode (fused into one launch by default).
+    `ev` = (start, end) events recorded around the timed kernel call."""
+    P = cfg.page_size
+    if args.append == "fused":
+        if ev is not None:
+            ev[0].record(stream)
+        K.paged_decode_attention_append(out, q, kn, vn, kp, vp, tab, lens, cfg.scale, num_splits=args.splits,
+                                        workspace=ws, err_flag=err, stream=stream)
+    else:
+        K.kv_append(kp, vp, kn, vn, slots, P, err_flag=err, stream=stream)
+        if ev is not None:
+            ev[0].record(stream)
+        K.paged_decode_attention(out, q, kp, vp, tab, lens, cfg.scale, num_splits=args.splits, workspace=ws,
+                                 err_flag=err, stream=stream)
+    if ev is not None:
+        ev[1].record(stream)
+
+
 def setup_dist(args):
     import torch
 
@@ -216,15 +267,22 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """Max of a per-rank float over the process group (device tensor for NCCL, host tensor for gloo)."""
     import torch
 
     if world == 1:
         return x
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cpu" if dist.get_backend() == "gloo" else "cuda"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_value(seqs_per_rank, steps, world, elapsed_ms_max):
+    """Whole-job seq-steps/s: every rank decodes its own batch (weak scaling); time = slowest rank."""
+    return seqs_per_rank * steps * world / (elapsed_ms_max / 1e3)
 
 
 # ---------------------------------------------------------------------------- our arm: config 2
@@ -268,10 +326,9 @@ def run_layer_bench(args, world, rank, local):
     stream = torch.cuda.current_stream()
     kp, vp = wl.k_pages[0], wl.v_pages[0]
 
-    def step(i):
-        K.kv_append(kp, vp, kn_dev[i], vn_dev[i], slots_dev[i], P, err_flag=err, stream=stream)
-        K.paged_decode_attention(out, q_dev[i], kp, vp, tab_dev, lens_dev[i], cfg.scale, num_splits=args.splits,
-                                 workspace=ws, err_flag=err, stream=stream)
+    def step(i, ev=None):
+        hot_path(K, args, cfg, kp, vp, kn_dev[i], vn_dev[i], slots_dev[i], q_dev[i], tab_dev, lens_dev[i], out, ws, err,
+                 stream, ev)
 
     for i in range(warm):
         step(i)
@@ -283,31 +340,30 @@ def run_layer_bench(args, world, rank, local):
     torch.cuda.synchronize()
     start.record(stream)
     for n, i in enumerate(range(warm, T1)):
-        K.kv_append(kp, vp, kn_dev[i], vn_dev[i], slots_dev[i], P, err_flag=err, stream=stream)
-        ev[n][0].record(stream)
-        K.paged_decode_attention(out, q_dev[i], kp, vp, tab_dev, lens_dev[i], cfg.scale, num_splits=args.splits,
-                                 workspace=ws, err_flag=err, stream=stream)
-        ev[n][1].record(stream)
+        step(i, ev[n])
     end.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     clocks = clk.stop()
     elapsed_ms = max_over_ranks(start.elapsed_time(end), world)
     dec_ms = [a.elapsed_time(b) for a, b in ev]
-    bytes_per_launch = [wl.step_bytes(lens_list[i]) for i in range(warm, T1)]
+    append_bytes = 2 * 2 * B * cfg.H_kv * cfg.Dh * cfg.elem_bytes if args.append == "fused" else 0
+    bytes_per_launch = [wl.step_bytes(lens_list[i]) + append_bytes for i in range(warm, T1)]
     if int(err.item()) != 0:
         raise RuntimeError(f"device error flag {int(err.item())}")
 
     # ---- end-to-end: same calls, inputs from pinned host memory, output read back each step
     e2e = None
     if e2e_steps:
-        e2e = run_e2e(wl, cfg, warm, e2e_steps, args.splits, world)
+        e2e = run_e2e(wl, cfg, warm, e2e_steps, args, world)
 
-    value = B * steps * world / (elapsed_ms / 1e3)
+    value = replica_value(B, steps, world, elapsed_ms)
     peak, peak_kind = peaks()
     mean_bytes = float(np.mean(bytes_per_launch))
     mean_dec_s = float(np.mean(dec_ms)) / 1e3
     achieved = mean_bytes / mean_dec_s / 1e9
+    ratio = measured_traffic_ratio() if args.kernel != "simt" and P == 16 else None
+    traffic = ratio * mean_bytes if ratio is not None else None
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps, "warmup": warm,
         "ms_per_step": elapsed_ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -317,16 +373,18 @@ def run_layer_bench(args, world, rank, local):
                    "l2": "inputs larger than L2 (K/V working set %.0f MB > 126 MB L2); no flush" % (mean_bytes / 1e6)},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS hbm_gbs)" if peak_kind == "measured" else "fallback",
-                     "traffic": None, "kernel": "paged_decode_attention" + (" (split + combine)" if S > 1 else " (single pass)"),
+                     "traffic": traffic,
+                     "traffic_source": ("ncu dram bytes of the decode kernel (profiles/" + os.path.basename(PROFILE_DECODE)
+                                        + "), scaled to this run's algorithmic bytes") if traffic else None, "kernel": "paged_decode_attention" + (" (split + combine)" if S > 1 else " (single pass)"),
                      "bytes_per_launch": mean_bytes, "launch_us": mean_dec_s * 1e6},
-        "gpu_launches": steps * (3 if S > 1 else 2),
+        "gpu_launches": steps * ((2 if S > 1 else 1) + (args.append == "separate")),
         "e2e": e2e,
         "clocks": clocks,
     }
     return res
 
 
-def run_e2e(wl, cfg, warm, steps, splits, world):
+def run_e2e(wl, cfg, warm, steps, args, world):
     """Each step: host bookkeeping, H2D of slots/lens/q/k_new/v_new (+ table rows when a page was added),
     kv_append + paged_decode_attention, D2H of the fp32 output, wait for it."""
     import torch
@@ -370,9 +428,8 @@ def run_e2e(wl, cfg, warm, steps, splits, world):
         d_kn.copy_(host_kn[i], non_blocking=True)
         d_vn.copy_(host_vn[i], non_blocking=True)
         nb += s.nbytes + l.nbytes + cfg.elem_bytes * (host_q[i].numel() + 2 * host_kn[i].numel())
-        K.kv_append(wl.k_pages[0], wl.v_pages[0], d_kn, d_vn, d_slots, P, err_flag=err, stream=stream)
-        K.paged_decode_attention(d_out, d_q, wl.k_pages[0], wl.v_pages[0], d_tab, d_lens, cfg.scale, num_splits=splits,
-                                 workspace=ws, err_flag=err, stream=stream)
+        hot_path(K, args, cfg, wl.k_pages[0], wl.v_pages[0], d_kn, d_vn, d_slots, d_q, d_tab, d_lens, d_out, ws, err,
+                 stream)
         host_out.copy_(d_out, non_blocking=True)
         stream.synchronize()
         return nb
@@ -388,7 +445,7 @@ def run_e2e(wl, cfg, warm, steps, splits, world):
     end.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(start.elapsed_time(end), world)
-    return {"value": B * steps * world / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d_total[0] / steps,
+    return {"value": replica_value(B, steps, world, ms), "unit": UNIT, "h2d_bytes_per_step": h2d_total[0] / steps,
             "d2h_bytes_per_step": host_out.numel() * 4, "ms_per_step": ms / steps}
 
 
@@ -430,11 +487,8 @@ def run_long_bench(args, world, rank, local):
 
     def layers_pass(stream):
         for layer in range(L):
-            K.kv_append(wl.k_pages[layer], wl.v_pages[layer], cur["kn"][layer], cur["vn"][layer], cur["slots"], P,
-                        err_flag=err, stream=stream)
-            K.paged_decode_attention(out[layer], cur["q"][layer], wl.k_pages[layer], wl.v_pages[layer], tab_dev,
-                                     cur["lens"], cfg.scale, num_splits=args.splits, workspace=ws, err_flag=err,
-                                     stream=stream)
+            hot_path(K, args, cfg, wl.k_pages[layer], wl.v_pages[layer], cur["kn"][layer], cur["vn"][layer], cur["slots"],
+                     cur["q"][layer], tab_dev, cur["lens"], out[layer], ws, err, stream)
 
     def stage(i, stream):
         with torch.cuda.stream(stream):
@@ -479,7 +533,7 @@ def run_long_bench(args, world, rank, local):
     if int(err.item()) != 0:
         raise RuntimeError(f"device error flag {int(err.item())}")
     bytes_step = [L * wl.step_bytes(lens_list[i]) for i in range(warm, T1)]
-    value = B * steps * world / (elapsed_ms / 1e3)
+    value = replica_value(B, steps, world, elapsed_ms)
     peak, peak_kind = peaks()
     achieved = float(np.mean(bytes_step)) / (float(np.mean(pass_ms)) / 1e3) / 1e9
     return {
@@ -491,9 +545,10 @@ def run_long_bench(args, world, rank, local):
                    "l2": "inputs larger than L2 (4 GiB cache); no flush"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} copy bandwidth", "traffic": None,
-                     "kernel": "32 x (kv_append + paged_decode_attention split + combine) per step",
+                     "kernel": ("32 x (paged_decode_attention_append + combine) per step" if args.append == "fused"
+                                else "32 x (kv_append + paged_decode_attention + combine) per step"),
                      "bytes_per_step": float(np.mean(bytes_step)), "pass_us": float(np.mean(pass_ms)) * 1e3},
-        "gpu_launches": steps * L * (3 if S > 1 else 2),
+        "gpu_launches": steps * L * ((2 if S > 1 else 1) + (args.append == "separate")),
         "e2e": None,
         "clocks": clocks,
     }

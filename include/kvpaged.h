@@ -213,6 +213,22 @@ int paged_decode_attention(float* out, const void* q, const void* k_pages, const
                            int32_t dtype, int32_t num_splits, void* workspace, size_t ws_bytes, int* err_flag,
                            void* stream);
 
+/* kv_append and paged_decode_attention in one launch. The new token of each
+ * sequence is at position seq_lens[b] - 1 (seq_lens counts it, as for
+ * paged_decode_attention); its K and V rows k_new[b][h][:], v_new[b][h][:]
+ * ([B][H_kv][Dh], pool dtype) are written to slot
+ * block_tables[b][(len-1)/P] * P + (len-1) % P of k_pages / v_pages by the
+ * CTA that reads that page, before it reads it; then attention proceeds as in
+ * paged_decode_attention ([HB-07] Q025: append, then q_new @ K_all^T). The
+ * slot's page must already be in the block table (kv_append_slots allocates
+ * it). Same arguments, errors and workspace otherwise; KV_ERR_ARG if k_new or
+ * v_new is NULL or not 16-byte aligned. */
+int paged_decode_attention_append(float* out, const void* q, const void* k_new, const void* v_new, void* k_pages,
+                                  void* v_pages, const int32_t* block_tables, int32_t max_blocks,
+                                  const int32_t* seq_lens, int32_t B, int32_t H_q, int32_t H_kv, int32_t Dh,
+                                  int32_t page_size, int32_t num_pages, float scale, int32_t dtype, int32_t num_splits,
+                                  void* workspace, size_t ws_bytes, int* err_flag, void* stream);
+
 /* Which decode kernel paged_decode_attention uses (process-wide; default AUTO):
  *   KV_DECODE_KERNEL_AUTO  tensor cores (warp MMA on TMA-staged swizzled tiles)
  *                          for bf16/fp16 K/V with H_q / H_kv <= 64, CUDA cores

@@ -57,6 +57,8 @@ struct DecodeParams {
     const void* v_pages;
     const int32_t* block_tables;  // [B][max_blocks]
     const int32_t* seq_lens;      // [B]
+    const void* k_new;          // nullable: fused append of the token at position len - 1, [B][H_kv][Dh]
+    const void* v_new;
     float* part_u;              // split: [B][H_q][S][Dh]
     float2* part_ml;            // split: [B][H_q][S] (m in log2 units, l)
     int* err;
@@ -102,6 +104,35 @@ struct Fmt<KV_DTYPE_F16> {
 
 __device__ __forceinline__ void raise_err(int* err, int bit) {
     if (err) atomicOr(err, bit);
+}
+
+// Fused append ("07｜KV Cache、FlashAttention与PagedAttention的内部过程", Q025:
+// the new token's K/V join the layer's cache before the query attends). The
+// CTA whose page range ends at the sequence's last page writes the new
+// token's K and V rows for its KV head into position len - 1 (slot
+// table[(len-1)/P] * P + (len-1) % P), before its producer loads that page.
+// Each lane fences its stores against the async proxy and the warp syncs, so
+// the bulk / TMA reads issued afterwards see them. Called by one whole warp.
+__device__ __forceinline__ void append_new_token(const DecodeParams& p, int b, int kvh, int len, int P,
+                                                 int row_bytes, int lane) {
+    const int pos = len - 1;
+    const int32_t page = p.block_tables[(int64_t)b * p.max_blocks + pos / P];
+    if (page >= 0 && page < p.num_pages) {
+        const int nch = row_bytes / 16;
+        const int64_t dst_row = ((int64_t)page * p.H_kv + kvh) * P + pos % P;
+        const int64_t src_row = (int64_t)b * p.H_kv + kvh;
+        for (int c = lane; c < 2 * nch; c += 32) {
+            const bool is_v = c >= nch;
+            const int cc = is_v ? c - nch : c;
+            const uint4* src = static_cast<const uint4*>(is_v ? p.v_new : p.k_new) + src_row * nch + cc;
+            uint4* dst = static_cast<uint4*>(const_cast<void*>(is_v ? p.v_pages : p.k_pages)) + dst_row * nch + cc;
+            *dst = *src;
+        }
+        fence_proxy_async_global();
+    } else if (lane == 0) {
+        raise_err(p.err, KV_DEV_ERR_PAGE_RANGE);
+    }
+    __syncwarp();
 }
 
 template <int DT, int DH, int P, int GW, int NW>
@@ -186,6 +217,8 @@ __global__ void __launch_bounds__(32 * (NW + 1), (NW <= 4) ? 2 : 1) paged_decode
     const int lane = threadIdx.x & 31;
     const bool split_mode = p.num_splits > 1;
 
+    grid_dependency_wait();  // inputs may come from the previous kernel in the stream
+    if (threadIdx.x == 0) grid_launch_dependents();
     int len = p.seq_lens[b];
     if (len < 0 || len > p.max_blocks * P) {
         if (threadIdx.x == 0 && split == 0) raise_err(p.err, KV_DEV_ERR_SEQ_LEN);
@@ -218,6 +251,7 @@ __global__ void __launch_bounds__(32 * (NW + 1), (NW <= 4) ? 2 : 1) paged_decode
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
+        if (p.k_new != nullptr && first + n_local == n_pages) append_new_token(p, b, kvh, len, P, C::kRowB, lane);
         const int32_t* row = p.block_tables + (int64_t)b * p.max_blocks + first;
         const char* kbase = static_cast<const char*>(p.k_pages);
         const char* vbase = static_cast<const char*>(p.v_pages);
@@ -491,89 +525,6 @@ __global__ void __launch_bounds__(32 * (NW + 1), (NW <= 4) ? 2 : 1) paged_decode
             p.part_u[ps * DH + d] = U;
             if (d == 0) p.part_ml[ps] = make_float2(mstar, L);
         }
-    }
-}
-
-// Merge split partials (the same (m, l, u) rule over the splits of one row):
-// m* = max_s m_s, o = sum_s 2^{m_s - m*} u_s / sum_s 2^{m_s - m*} l_s.
-// One CTA of kCombineWarps warps per (sequence, query head). Every warp finds
-// m* over all splits; warp w then accumulates splits w, w + kCombineWarps, ...
-// eight at a time (loads of a batch are independent, so their latencies
-// overlap), and the warps' sums -- all relative to the same m* -- are added
-// in shared memory.
-constexpr int kCombineWarps = 4;
-
-template <int DH>
-__global__ void __launch_bounds__(32 * kCombineWarps) paged_combine_kernel(
-    float* __restrict__ out, const float* __restrict__ part_u, const float2* __restrict__ part_ml,
-    const int32_t* __restrict__ seq_lens, int32_t B, int32_t H_q, int32_t S, int32_t pages_per_split, int32_t P,
-    int32_t max_blocks) {
-    constexpr int kD = DH / 32;  // dims per lane
-    constexpr int kBatch = 8;
-    __shared__ float red_u[kCombineWarps][DH];
-    __shared__ float red_l[kCombineWarps];
-    const int item = blockIdx.x;
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int b = item / H_q;
-    int len = seq_lens[b];
-    if (len < 0 || len > max_blocks * P) len = 0;
-    const int n_pages = (len + P - 1) / P;
-    const int ns = min(S, (n_pages + pages_per_split - 1) / pages_per_split);
-    const float2* ml = part_ml + (int64_t)item * S;
-    const float* pu = part_u + (int64_t)item * S * DH;
-    float mstar = -INFINITY;
-    for (int s = lane; s < ns; s += 32) mstar = fmaxf(mstar, ml[s].x);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mstar = fmaxf(mstar, __shfl_xor_sync(0xffffffffu, mstar, o));
-    float acc[kD];
-#pragma unroll
-    for (int i = 0; i < kD; ++i) acc[i] = 0.f;
-    float L = 0.f;
-    if (mstar != -INFINITY) {
-        for (int s0 = warp; s0 < ns; s0 += kCombineWarps * kBatch) {
-            float2 st[kBatch];
-            float v[kBatch][kD];
-#pragma unroll
-            for (int j = 0; j < kBatch; ++j) {
-                const int s = s0 + j * kCombineWarps;
-                if (s < ns) {
-                    st[j] = ml[s];
-                    const float* src = pu + (int64_t)s * DH + lane * kD;
-                    if constexpr (kD == 4) {
-                        const float4 x = *reinterpret_cast<const float4*>(src);
-                        v[j][0] = x.x; v[j][1] = x.y; v[j][2] = x.z; v[j][3] = x.w;
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < kD; ++i) v[j][i] = src[i];
-                    }
-                } else {
-                    st[j] = make_float2(-INFINITY, 0.f);
-#pragma unroll
-                    for (int i = 0; i < kD; ++i) v[j][i] = 0.f;
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < kBatch; ++j) {
-                const float w = (st[j].x == -INFINITY) ? 0.f : exp2f(st[j].x - mstar);
-                L += w * st[j].y;
-#pragma unroll
-                for (int i = 0; i < kD; ++i) acc[i] += w * v[j][i];
-            }
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < kD; ++i) red_u[warp][lane * kD + i] = acc[i];
-    if (lane == 0) red_l[warp] = L;
-    __syncthreads();
-    for (int d = threadIdx.x; d < DH; d += blockDim.x) {
-        float U = 0.f, Lt = 0.f;
-#pragma unroll
-        for (int w = 0; w < kCombineWarps; ++w) {
-            U += red_u[w][d];
-            Lt += red_l[w];
-        }
-        out[(int64_t)item * DH + d] = (Lt > 0.f) ? U / Lt : 0.f;
     }
 }
 

@@ -4,10 +4,29 @@
 #pragma once
 
 #include <atomic>
+#include <utility>
 
 #include "decode_kernel.cuh"
 
 namespace kvp {
+
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel in the stream finishes; every kernel of this
+// library starts with griddepcontrol.wait, so nothing is read early.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 template <int DT, int DH, int P, int GW, int NW>
 cudaError_t launch_decode_inst(const DecodeParams& p, dim3 grid, cudaStream_t st) {
@@ -26,8 +45,7 @@ cudaError_t launch_decode_inst(const DecodeParams& p, dim3 grid, cudaStream_t st
         if (e != cudaSuccess) return e;
         configured.fetch_or(bit, std::memory_order_acq_rel);
     }
-    paged_decode_kernel<DT, DH, P, GW, NW><<<grid, C::kThreads, C::kSmem, st>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(paged_decode_kernel<DT, DH, P, GW, NW>, grid, dim3(C::kThreads), C::kSmem, st, p);
 }
 
 template <int DT, int DH, int P>
@@ -82,8 +100,7 @@ cudaError_t launch_mma_inst(const DecodeParams& p, const CUtensorMap& tk, const 
         if (e != cudaSuccess) return e;
         configured.fetch_or(bit, std::memory_order_acq_rel);
     }
-    paged_decode_mma_kernel<DT, DH, P, NW><<<grid, C::kThreads, C::kSmem, st>>>(p, tk, tv);
-    return cudaGetLastError();
+    return launch_pdl(paged_decode_mma_kernel<DT, DH, P, NW>, grid, dim3(C::kThreads), C::kSmem, st, p, tk, tv);
 }
 
 template <int DT>

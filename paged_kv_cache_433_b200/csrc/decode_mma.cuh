@@ -76,13 +76,23 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
     const int lane = threadIdx.x & 31;
     const bool split_mode = p.num_splits > 1;
 
+    if (threadIdx.x == 0) {
+        prefetch_tmap(&tmap_k);
+        prefetch_tmap(&tmap_v);
+    }
+    grid_dependency_wait();  // inputs may come from the previous kernel in the stream
+    if (threadIdx.x == 0) grid_launch_dependents();
+    // The producer's first 32 block-table entries do not depend on the length:
+    // load them alongside it.
+    const int first = split_mode ? split * p.pages_per_split : 0;
+    int tab0 = 0;
+    if (warp == 0 && first + lane < p.max_blocks) tab0 = p.block_tables[(int64_t)b * p.max_blocks + first + lane];
     int len = p.seq_lens[b];
     if (len < 0 || len > p.max_blocks * P) {
         if (threadIdx.x == 0 && split == 0) raise_err(p.err, KV_DEV_ERR_SEQ_LEN);
         len = 0;
     }
     const int n_pages = (len + P - 1) / P;
-    const int first = split_mode ? split * p.pages_per_split : 0;
     const int n_local = split_mode ? min(p.pages_per_split, n_pages - first) : n_pages;
     if (n_local <= 0) {
         if (!split_mode) {
@@ -110,10 +120,7 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            prefetch_tmap(&tmap_k);
-            prefetch_tmap(&tmap_v);
-        }
+        if (p.k_new != nullptr && first + n_local == n_pages) append_new_token(p, b, kvh, len, P, DH * 2, lane);
         const int32_t* row = p.block_tables + (int64_t)b * p.max_blocks + first;
         bool ok = true;
         int issued = 0;
@@ -163,7 +170,7 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
         static_assert(32 % kGrp == 0, "page groups must tile the 32-entry table window");
         int tab = 0;  // block-table entry of page (base & ~31) + lane
         for (int base = 0; base < n_local; base += kGrp) {
-            if ((base & 31) == 0) tab = (base + lane < n_local) ? row[base + lane] : 0;
+            if ((base & 31) == 0) tab = base == 0 ? tab0 : ((base + lane < n_local) ? row[base + lane] : 0);
             const int cnt = min(kGrp, n_local - base);
             const int pg = __shfl_sync(0xffffffffu, tab, ((base & 31) + lane) & 31);
             bool valid = false;

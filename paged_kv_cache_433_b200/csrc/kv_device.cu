@@ -8,6 +8,7 @@
 #include <atomic>
 #include <cstdint>
 
+#include "combine_kernel.cuh"
 #include "decode_launch.cuh"
 #include "kvpaged.h"
 
@@ -22,6 +23,8 @@ __global__ void __launch_bounds__(256) kv_append_kernel(uint4* __restrict__ k_pa
                                                         const uint4* __restrict__ v_new,
                                                         const int64_t* __restrict__ slots, int64_t rows, int32_t H_kv,
                                                         int32_t vpr, int32_t P, int64_t num_slots, int* err) {
+    grid_dependency_wait();
+    if (threadIdx.x == 0) grid_launch_dependents();
     int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     const int64_t per = rows * vpr;
     if (i >= 2 * per) return;
@@ -190,11 +193,12 @@ int kv_append(void* k_pages, void* v_pages, const void* k_new, const void* v_new
     const int64_t threads = 2 * rows * vpr;
     const int64_t blocks = (threads + 255) / 256;
     if (blocks > 0x7fffffffLL) return KV_ERR_UNSUPPORTED;
-    kv_append_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<uint4*>(k_pages), static_cast<uint4*>(v_pages), static_cast<const uint4*>(k_new),
-        static_cast<const uint4*>(v_new), slot_mapping, rows, H_kv, vpr, page_size,
-        static_cast<int64_t>(num_pages) * page_size, err_flag);
-    return cudaGetLastError() == cudaSuccess ? KV_OK : KV_ERR_CUDA;
+    cudaError_t e = launch_pdl(kv_append_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
+                               static_cast<cudaStream_t>(stream), static_cast<uint4*>(k_pages),
+                               static_cast<uint4*>(v_pages), static_cast<const uint4*>(k_new),
+                               static_cast<const uint4*>(v_new), slot_mapping, rows, H_kv, vpr, page_size,
+                               static_cast<int64_t>(num_pages) * page_size, err_flag);
+    return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;
 }
 
 int paged_decode_set_kernel(int32_t kind) {
@@ -223,11 +227,15 @@ int paged_decode_workspace_bytes(int32_t B, int32_t H_q, int32_t H_kv, int32_t D
     return KV_OK;
 }
 
-int paged_decode_attention(float* out, const void* q, const void* k_pages, const void* v_pages,
-                           const int32_t* block_tables, int32_t max_blocks, const int32_t* seq_lens, int32_t B,
-                           int32_t H_q, int32_t H_kv, int32_t Dh, int32_t page_size, int32_t num_pages, float scale,
-                           int32_t dtype, int32_t num_splits, void* workspace, size_t ws_bytes, int* err_flag,
-                           void* stream) {
+}  // extern "C"
+
+namespace kvp {
+namespace {
+
+int decode_impl(float* out, const void* q, const void* k_new, const void* v_new, const void* k_pages,
+                const void* v_pages, const int32_t* block_tables, int32_t max_blocks, const int32_t* seq_lens, int32_t B,
+                int32_t H_q, int32_t H_kv, int32_t Dh, int32_t page_size, int32_t num_pages, float scale, int32_t dtype,
+                int32_t num_splits, void* workspace, size_t ws_bytes, int* err_flag, void* stream) {
     int rc = check_shape(H_q, H_kv, Dh, page_size, dtype);
     if (rc != KV_OK) return rc;
     if (B < 0 || max_blocks <= 0 || num_pages <= 0 || num_splits < 0) return KV_ERR_ARG;
@@ -253,6 +261,8 @@ int paged_decode_attention(float* out, const void* q, const void* k_pages, const
     DecodeParams p{};
     p.out = out;
     p.q = q;
+    p.k_new = k_new;
+    p.v_new = v_new;
     p.k_pages = k_pages;
     p.v_pages = v_pages;
     p.block_tables = block_tables;
@@ -296,16 +306,51 @@ int paged_decode_attention(float* out, const void* q, const void* k_pages, const
     }
     if (e != cudaSuccess) return KV_ERR_CUDA;
     if (S > 1) {
-        const unsigned blocks = static_cast<unsigned>(static_cast<int64_t>(B) * H_q);
+        // one warp per row when a single round of 8 loads per lane covers the splits, else 8 warps per row
+        const int64_t rows = static_cast<int64_t>(B) * H_q;
+        const bool narrow = S <= 8;
+        const int64_t rows_per_cta = narrow ? kCombineWarps : 1;
+        const dim3 blocks(static_cast<unsigned>((rows + rows_per_cta - 1) / rows_per_cta));
+        const dim3 threads(32 * kCombineWarps);
+        const float2* ml = p.part_ml;
+        const float* pu = p.part_u;
         if (Dh == 128)
-            paged_combine_kernel<128><<<blocks, 32 * kCombineWarps, 0, st>>>(out, p.part_u, p.part_ml, seq_lens, B, H_q,
-                                                                              S, C, page_size, max_blocks);
+            e = narrow ? launch_pdl(paged_combine_kernel<128, 1>, blocks, threads, 0, st, out, pu, ml, seq_lens, B, H_q,
+                                    S, C, page_size, max_blocks)
+                       : launch_pdl(paged_combine_kernel<128, kCombineWarps>, blocks, threads, 0, st, out, pu, ml,
+                                    seq_lens, B, H_q, S, C, page_size, max_blocks);
         else
-            paged_combine_kernel<64><<<blocks, 32 * kCombineWarps, 0, st>>>(out, p.part_u, p.part_ml, seq_lens, B, H_q,
-                                                                             S, C, page_size, max_blocks);
-        if (cudaGetLastError() != cudaSuccess) return KV_ERR_CUDA;
+            e = narrow ? launch_pdl(paged_combine_kernel<64, 1>, blocks, threads, 0, st, out, pu, ml, seq_lens, B, H_q, S,
+                                    C, page_size, max_blocks)
+                       : launch_pdl(paged_combine_kernel<64, kCombineWarps>, blocks, threads, 0, st, out, pu, ml,
+                                    seq_lens, B, H_q, S, C, page_size, max_blocks);
+        if (e != cudaSuccess) return KV_ERR_CUDA;
     }
     return KV_OK;
+}
+
+}  // namespace
+}  // namespace kvp
+
+extern "C" {
+
+int paged_decode_attention(float* out, const void* q, const void* k_pages, const void* v_pages,
+                           const int32_t* block_tables, int32_t max_blocks, const int32_t* seq_lens, int32_t B,
+                           int32_t H_q, int32_t H_kv, int32_t Dh, int32_t page_size, int32_t num_pages, float scale,
+                           int32_t dtype, int32_t num_splits, void* workspace, size_t ws_bytes, int* err_flag,
+                           void* stream) {
+    return decode_impl(out, q, nullptr, nullptr, k_pages, v_pages, block_tables, max_blocks, seq_lens, B, H_q, H_kv, Dh,
+                       page_size, num_pages, scale, dtype, num_splits, workspace, ws_bytes, err_flag, stream);
+}
+
+int paged_decode_attention_append(float* out, const void* q, const void* k_new, const void* v_new, void* k_pages,
+                                  void* v_pages, const int32_t* block_tables, int32_t max_blocks,
+                                  const int32_t* seq_lens, int32_t B, int32_t H_q, int32_t H_kv, int32_t Dh,
+                                  int32_t page_size, int32_t num_pages, float scale, int32_t dtype, int32_t num_splits,
+                                  void* workspace, size_t ws_bytes, int* err_flag, void* stream) {
+    if (B > 0 && (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new))) return KV_ERR_ARG;
+    return decode_impl(out, q, k_new, v_new, k_pages, v_pages, block_tables, max_blocks, seq_lens, B, H_q, H_kv, Dh,
+                       page_size, num_pages, scale, dtype, num_splits, workspace, ws_bytes, err_flag, stream);
 }
 
 }  // extern "C"

@@ -67,6 +67,9 @@ SIGNATURES = [
     ("kv_append", ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
     ("paged_decode_attention", ctypes.c_int,
      [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _i32, _vp, _sz, _vp, _vp]),
+    ("paged_decode_attention_append", ctypes.c_int,
+     [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _i32, _vp, _sz, _vp,
+      _vp]),
     ("paged_decode_attention_noalloc", ctypes.c_int,
      [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _i32, _vp, _vp]),
     ("paged_decode_set_kernel", ctypes.c_int, [_i32]),
@@ -326,6 +329,31 @@ def paged_decode_attention(out, q, k_pages, v_pages, block_tables, seq_lens, sca
         _dev(seq_lens, "seq_lens", torch.int32), B, H_q, H_kv, Dh, P, num_pages, float(scale), dt, num_splits, ws_ptr,
         ws_bytes, _dev(err_flag, "err_flag", torch.int32), _stream(stream))
     _check("paged_decode_attention", rc)
+
+
+def paged_decode_attention_append(out, q, k_new, v_new, k_pages, v_pages, block_tables, seq_lens, scale: float,
+                                  num_splits: int = 0, workspace=None, err_flag=None, stream=None) -> None:
+    """kv_append of the token at position seq_lens[b] - 1 and paged_decode_attention in one launch.
+    k_new / v_new [B, H_kv, Dh] in the pools' dtype; other arguments as paged_decode_attention."""
+    import torch
+
+    B, H_q, Dh = q.shape
+    num_pages, H_kv, P, Dh2 = k_pages.shape
+    assert Dh2 == Dh and v_pages.shape == k_pages.shape and tuple(out.shape) == (B, H_q, Dh)
+    assert tuple(k_new.shape) == (B, H_kv, Dh) and v_new.shape == k_new.shape
+    assert block_tables.shape[0] == B and tuple(seq_lens.shape) == (B,)
+    dt = _torch_dtype_code(k_pages)
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr = _dev(workspace, "workspace")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib().paged_decode_attention_append(
+        _dev(out, "out", torch.float32), _dev(q, "q", k_pages.dtype), _dev(k_new, "k_new", k_pages.dtype),
+        _dev(v_new, "v_new", k_pages.dtype), _dev(k_pages, "k_pages"), _dev(v_pages, "v_pages", k_pages.dtype),
+        _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1], _dev(seq_lens, "seq_lens", torch.int32), B,
+        H_q, H_kv, Dh, P, num_pages, float(scale), dt, num_splits, ws_ptr, ws_bytes, _dev(err_flag, "err_flag", torch.int32),
+        _stream(stream))
+    _check("paged_decode_attention_append", rc)
 
 
 KV_NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024

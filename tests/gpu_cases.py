@@ -131,8 +131,11 @@ def build_cache(cfg: W.DecodeConfig, lens: Sequence[int], layer: int = 0, slack_
 
 
 def append_and_decode(st: Step, layer: int = 0, step: int = 0, num_splits: int = 0, check_pools: bool = True,
-                      sample: Optional[Sequence[int]] = None):
-    """New token append + decode on both sides. Returns (gpu_out fp32 np, ref fp64 np, err_flag)."""
+                      sample: Optional[Sequence[int]] = None, fused: bool = False):
+    """New token append + decode on both sides. Returns (gpu_out fp32 np, ref fp64 np, err_flag).
+
+    fused=True appends through paged_decode_attention_append (one launch) instead of
+    kv_append followed by paged_decode_attention."""
     cfg = st.cfg
     P = cfg.page_size
     B = len(st.lens)
@@ -158,14 +161,20 @@ def append_and_decode(st: Step, layer: int = 0, step: int = 0, num_splits: int =
 
     # product side
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    K.kv_append(st.k_pages, st.v_pages, to_device(k_new, cfg.dtype), to_device(v_new, cfg.dtype),
-                torch.from_numpy(slots).cuda(), P, err_flag=err)
     out = torch.empty((B, cfg.H_q, cfg.Dh), dtype=torch.float32, device="cuda")
     ws_bytes = K.paged_decode_workspace_bytes(B, cfg.H_q, cfg.H_kv, cfg.Dh, st.max_blocks, P, num_splits)
     ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
-    K.paged_decode_attention(out, to_device(q, cfg.dtype), st.k_pages, st.v_pages, torch.from_numpy(st.tab).cuda(),
-                             torch.from_numpy(lens32).cuda(), cfg.scale, num_splits=num_splits, workspace=ws,
-                             err_flag=err)
+    if fused:
+        K.paged_decode_attention_append(out, to_device(q, cfg.dtype), to_device(k_new, cfg.dtype),
+                                        to_device(v_new, cfg.dtype), st.k_pages, st.v_pages,
+                                        torch.from_numpy(st.tab).cuda(), torch.from_numpy(lens32).cuda(), cfg.scale,
+                                        num_splits=num_splits, workspace=ws, err_flag=err)
+    else:
+        K.kv_append(st.k_pages, st.v_pages, to_device(k_new, cfg.dtype), to_device(v_new, cfg.dtype),
+                    torch.from_numpy(slots).cuda(), P, err_flag=err)
+        K.paged_decode_attention(out, to_device(q, cfg.dtype), st.k_pages, st.v_pages, torch.from_numpy(st.tab).cuda(),
+                                 torch.from_numpy(lens32).cuda(), cfg.scale, num_splits=num_splits, workspace=ws,
+                                 err_flag=err)
     torch.cuda.synchronize()
     st.lens = st.lens + 1
     if check_pools:

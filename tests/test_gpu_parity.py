@@ -186,6 +186,29 @@ def test_mixed_sweep_with_churn(H_kv, P, kernel):
         check_close(out, ref, base.dtype, f"mixed Hkv={H_kv} P={P} step {step}")
 
 
+# ---------------------------------------------------------------- fused append + decode
+FUSED_CASES = [("tiny", 1), ("tiny", 2), ("8b", 0), ("8b", 1), ("32k", 0), ("edge", 1), ("edge", 3)]
+
+
+@pytest.mark.parametrize("case,splits", FUSED_CASES)
+def test_fused_append_decode(case, splits, kernel):
+    """paged_decode_attention_append == kv_append + paged_decode_attention: same pool bytes, same oracle match."""
+    if case == "tiny":
+        cfg, lens = W.TINY, W.cached_lengths(W.TINY)
+    elif case == "8b":
+        cfg, lens = W.LLAMA8B, W.cached_lengths(W.LLAMA8B)[:12]
+    elif case == "32k":
+        cfg, lens = W.LONG32K, W.cached_lengths(W.LONG32K)
+    else:
+        cfg = W.DecodeConfig("edge-fused", "fp16", B=6, H_q=12, H_kv=4, Dh=64, page_size=32, seed=13)
+        lens = [0, 30, 31, 32, 100, 127]
+    st = build_cache(cfg, lens)
+    for step in range(2):
+        out, ref, err = append_and_decode(st, step=step, num_splits=splits, fused=True, check_pools=True)
+        assert err == 0
+        check_close(out, ref, cfg.dtype, f"fused {case} step {step}")
+
+
 # ---------------------------------------------------------------- edge cases
 EDGE_SHAPES = [
     # dtype, Dh, P, H_q, H_kv
