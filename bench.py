@@ -44,12 +44,16 @@ def parse():
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", type=int, choices=[2, 3], default=2)
+    ap.add_argument("--config", type=int, choices=[2, 3, 4, 5], default=2,
+                    help="2: 8B-shaped layer (default); 3: 32K context x 32 layers; 4: shared-prefix batch; "
+                         "5: mixed continuous-batching sweep")
     ap.add_argument("--splits", type=int, default=0, help="num_splits passed to paged_decode_attention (0 = auto)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="config 3: launch the 32 layers without a CUDA graph")
+    ap.add_argument("--mixed-point", type=str, default=None,
+                    help="config 5: run one point only, 'H_kv,page_size' (e.g. 1,16)")
     ap.add_argument("--page-size", type=int, choices=[16, 32], default=None,
                     help="override the workload's page size (the 8B-shaped workload uses 16)")
     ap.add_argument("--page-order", choices=["shuffled", "sequential"], default="shuffled",
@@ -554,6 +558,211 @@ def run_long_bench(args, world, rank, local):
     }
 
 
+# ---------------------------------------------------------------------------- our arm: configs 4 and 5
+class PagedState:
+    """A batch on the device built through the library: pool, block table, pools filled by kv_append."""
+
+    def __init__(self, cfg, lens, max_blocks, num_pages, seed, dev="cuda"):
+        import torch
+
+        from paged_kv_cache_433_b200 import kvpaged as K
+        from paged_kv_cache_433_b200 import workloads as W
+
+        self.K, self.torch, self.cfg = K, torch, cfg
+        self.P = cfg.page_size
+        self.B = len(lens)
+        self.max_blocks = max_blocks
+        self.num_pages = num_pages
+        self.dt = {"bf16": torch.bfloat16, "fp16": torch.float16, "fp32": torch.float32}[cfg.dtype]
+        self.pool = K.KvPool(num_pages, self.P, W.page_order(num_pages, seed))
+        self.tab = np.full((self.B, max_blocks), -1, np.int32)
+        self.lens = np.asarray(lens, np.int32).copy()
+        shape = (num_pages, cfg.H_kv, self.P, cfg.Dh)
+        self.k_pages = torch.zeros(shape, dtype=self.dt, device=dev)
+        self.v_pages = torch.zeros(shape, dtype=self.dt, device=dev)
+        self.gen = torch.Generator(device=dev)
+        self.gen.manual_seed(seed)
+
+    def fill(self, b, start, n):
+        """Write n synthetic tokens at positions start.. of row b (the row's pages must exist)."""
+        if n <= 0:
+            return
+        cfg, torch = self.cfg, self.torch
+        slots = self.torch.from_numpy(self.K.kv_slots_for_range(self.tab[b], self.P, start, n)).cuda()
+        kr = torch.randn((n, cfg.H_kv, cfg.Dh), generator=self.gen, device="cuda").to(self.dt)
+        vr = torch.randn((n, cfg.H_kv, cfg.Dh), generator=self.gen, device="cuda").to(self.dt)
+        self.K.kv_append(self.k_pages, self.v_pages, kr, vr, slots, self.P)
+
+    def admit(self, b, n_tokens):
+        k = -(-int(n_tokens) // self.P)
+        self.tab[b, :] = -1
+        self.tab[b, :k] = self.pool.alloc(k)
+        self.lens[b] = n_tokens
+        self.fill(b, 0, int(n_tokens))
+
+    def release(self, b):
+        held = self.tab[b][self.tab[b] >= 0]
+        self.pool.free(held)
+        self.tab[b, :] = -1
+        self.lens[b] = 0
+
+    def step_bytes(self, lens_after, fused=True):
+        cfg = self.cfg
+        kv = int(np.sum(lens_after)) * cfg.H_kv * cfg.Dh * 2 * cfg.elem_bytes
+        q = self.B * cfg.H_q * cfg.Dh * cfg.elem_bytes
+        out = self.B * cfg.H_q * cfg.Dh * 4
+        tables = int(np.sum(-(-np.asarray(lens_after) // self.P))) * 4 + self.B * 4
+        app = 2 * 2 * self.B * cfg.H_kv * cfg.Dh * cfg.elem_bytes if fused else 0
+        return kv + q + out + tables + app
+
+
+def time_steps(args, st, steps, warm, before_step=None):
+    """Run warm + steps decode steps on `st`; each step: optional untimed host work (before_step),
+    bookkeeping + uploads (untimed), then the timed append + decode call. Returns per-step (ms, bytes)."""
+    import torch
+
+    K, cfg = st.K, st.cfg
+    dev = torch.device("cuda")
+    stream = torch.cuda.current_stream()
+    out = torch.empty((st.B, cfg.H_q, cfg.Dh), dtype=torch.float32, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    nb = K.paged_decode_workspace_bytes(st.B, cfg.H_q, cfg.H_kv, cfg.Dh, st.max_blocks, st.P, args.splits)
+    ws = torch.zeros(max(nb, 16), dtype=torch.uint8, device=dev)
+    res = []
+    S = K.paged_decode_num_splits(st.B, cfg.H_kv, st.max_blocks, st.P, args.splits)
+    st.launches_per_step = (2 if S > 1 else 1) + (args.append == "separate")
+    for i in range(warm + steps):
+        if before_step is not None:
+            before_step(i)
+        slots = st.pool.append_slots(st.tab, st.lens)
+        d_slots = torch.from_numpy(slots).to(dev)
+        d_lens = torch.from_numpy(st.lens.copy()).to(dev)
+        d_tab = torch.from_numpy(st.tab).to(dev)
+        q = torch.randn((st.B, cfg.H_q, cfg.Dh), generator=st.gen, device=dev).to(st.dt)
+        kn = torch.randn((st.B, cfg.H_kv, cfg.Dh), generator=st.gen, device=dev).to(st.dt)
+        vn = torch.randn((st.B, cfg.H_kv, cfg.Dh), generator=st.gen, device=dev).to(st.dt)
+        ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+        torch.cuda.synchronize()
+        hot_path(K, args, cfg, st.k_pages, st.v_pages, kn, vn, d_slots, q, d_tab, d_lens, out, ws, err, stream, ev)
+        torch.cuda.synchronize()
+        if i >= warm:
+            res.append((ev[0].elapsed_time(ev[1]), st.step_bytes(st.lens, args.append == "fused")))
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error flag {int(err.item())}")
+    return res
+
+
+def run_prefix_bench(args, world, rank, local):
+    """Shared-prefix batch: 32 sequences reuse one 4096-token prefix (256 refcounted pages) through the
+    chained-hash prefix index, then append + decode. Logical bytes count the prefix once per sequence."""
+    from paged_kv_cache_433_b200 import kvpaged as K
+    from paged_kv_cache_433_b200 import workloads as W
+
+    cfg = W.SHARED_PREFIX
+    steps = args.steps if args.steps is not None else cfg.timed_steps
+    warm = args.warmup if args.warmup is not None else cfg.warmup_steps
+    P = cfg.page_size
+    wl = W.prefix_workload(cfg)
+    lens = W.cached_lengths(cfg)
+    n_steps = steps + warm
+    max_blocks = max(-(-(int(L) + n_steps) // P) for L in lens) + 1
+    num_pages = W.PREFIX_LEN // P + int(sum(-(-(int(L) + n_steps - W.PREFIX_LEN) // P) + 1 for L in lens)) + 8
+    st = PagedState(cfg, np.zeros(cfg.B, np.int32), max_blocks, num_pages, cfg.seed + 1000 * rank)
+    ix = K.KvPrefixIndex(P, salt=0x5EED)
+    hits = 0
+    for b in range(cfg.B):
+        toks = wl.tokens(b)
+        hit = ix.match(toks)
+        st.pool.incref(hit)
+        own = st.pool.alloc(-(-len(toks) // P) - len(hit))
+        row = np.concatenate([hit, own]).astype(np.int32)
+        st.tab[b, :row.size] = row
+        st.lens[b] = len(toks)
+        ix.register(st.pool, toks, row)
+        st.fill(b, len(hit) * P, len(toks) - len(hit) * P)
+        hits += len(hit)
+    res = time_steps(args, st, steps, warm)
+    ms = float(np.sum([r[0] for r in res]))
+    logical = float(np.mean([r[1] for r in res]))
+    unique = (W.PREFIX_LEN + float(np.sum(st.lens - W.PREFIX_LEN))) * cfg.H_kv * cfg.Dh * 2 * cfg.elem_bytes
+    peak, _ = peaks()
+    per_ms = ms / steps
+    achieved = logical / (per_ms / 1e3) / 1e9
+    return {
+        "metric": METRIC, "value": replica_value(cfg.B, steps, world, max_over_ranks(ms, world)), "unit": UNIT,
+        "n_gpus": world, "steps": steps, "warmup": warm, "ms_per_step": per_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic (seeded token ids; N(0,1) K/V, q)",
+        "config": {"workload": cfg.name, "B": cfg.B, "prefix_tokens": W.PREFIX_LEN, "prefix_pages_shared": hits // max(cfg.B - 1, 1),
+                   "H_q": cfg.H_q, "H_kv": cfg.H_kv, "Dh": cfg.Dh, "page_size": P,
+                   "l2": "prefix pages (~17 MB) stay L2-resident; logical bytes count them per sequence; no flush"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None, "bytes": "logical (prefix read per sequence)", "logical_bytes_per_launch": logical,
+                     "unique_kv_bytes": unique, "launch_us": per_ms * 1e3},
+        "gpu_launches": steps * st.launches_per_step, "e2e": None, "clocks": None,
+    }
+
+
+def run_mixed_bench(args, world, rank, local):
+    """Mixed continuous-batching sweep: B=256, log-normal lengths, H_kv in {1, 8, 32}, P in {16, 32}; before
+    every step each sequence exits with probability 1/32 and a new one is admitted in its row (pages freed /
+    allocated on the host, its K/V written outside the timed region); the timed part is append + decode."""
+    from paged_kv_cache_433_b200 import workloads as W
+
+    steps = args.steps if args.steps is not None else 20
+    warm = args.warmup if args.warmup is not None else 3
+    points = []
+    tot_ms = tot_seq = tot_bytes = 0.0
+    launches = 0
+    pts = W.MIXED_POINTS
+    if args.mixed_point:
+        h, p = (int(x) for x in args.mixed_point.split(","))
+        pts = [(h, p)]
+    for H_kv, P in pts:
+        cfg = W.mixed_config(H_kv, P)
+        lens = W.cached_lengths(cfg)
+        events = W.churn_events(cfg, warm + steps)
+        max_blocks = -(-(16384 + warm + steps + 1) // P) + 1
+        num_pages = int(sum(-(-(int(L) + warm + steps) // P) for L in lens)) * 3 // 2 + 4 * max_blocks
+        st = PagedState(cfg, lens, max_blocks, num_pages, cfg.seed * 100 + H_kv + P + 1000 * rank)
+        for b in range(cfg.B):
+            st.admit(b, int(lens[b]))
+
+        def churn(i, st=st, events=events):
+            ev = events[i]
+            for b, L in zip(ev.exits, ev.new_lengths):
+                st.release(int(b))
+                st.admit(int(b), int(L))
+
+        res = time_steps(args, st, steps, warm, before_step=churn)
+        ms = float(np.sum([r[0] for r in res]))
+        byts = float(np.sum([r[1] for r in res]))
+        peak, _ = peaks()
+        points.append({"H_kv": H_kv, "page_size": P, "seq_steps_per_s": cfg.B * steps / (ms / 1e3),
+                       "GBps": byts / (ms / 1e3) / 1e9, "frac": byts / (ms / 1e3) / 1e9 / peak,
+                       "us_per_step": ms / steps * 1e3, "mean_len": float(np.mean(st.lens))})
+        tot_ms += ms
+        tot_seq += cfg.B * steps
+        launches += steps * st.launches_per_step
+        tot_bytes += byts
+        del st
+        import torch
+
+        torch.cuda.empty_cache()
+    peak, _ = peaks()
+    achieved = tot_bytes / (tot_ms / 1e3) / 1e9
+    return {
+        "metric": METRIC, "value": tot_seq * world / (max_over_ranks(tot_ms, world) / 1e3), "unit": UNIT,
+        "n_gpus": world, "steps": steps, "warmup": warm, "ms_per_step": tot_ms / (steps * len(points)),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded log-normal lengths, churn 1/32 per step; N(0,1) K/V, q)",
+        "config": {"workload": "mixed-bf16-B256-lognormal1024-sweep", "B": 256, "H_q": 32, "Dh": 128,
+                   "points": "H_kv x page_size = {1,8,32} x {16,32}", "l2": "inputs larger than L2; no flush"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None},
+        "sweep": points, "gpu_launches": launches, "e2e": None, "clocks": None,
+    }
+
+
 # ---------------------------------------------------------------------------- CPU oracle (baseline / reference arm)
 class OracleSample:
     """Host copy of the 8B-shaped decode workload for the fp64 oracle (seeded synthetic inputs)."""
@@ -656,11 +865,9 @@ def main():
 
     K.paged_decode_set_kernel({"auto": K.KV_DECODE_KERNEL_AUTO, "simt": K.KV_DECODE_KERNEL_SIMT,
                                "mma": K.KV_DECODE_KERNEL_MMA}[args.kernel])
-    if args.config == 2:
-        res = run_layer_bench(args, world, rank, local)
-    else:
-        res = run_long_bench(args, world, rank, local)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    run = {2: run_layer_bench, 3: run_long_bench, 4: run_prefix_bench, 5: run_mixed_bench}[args.config]
+    res = run(args, world, rank, local)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config == 2:
         res["cpu_baseline"] = cpu_baseline()
     if world > 1:
         import torch.distributed as dist

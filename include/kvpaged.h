@@ -135,6 +135,22 @@ int kv_slots_for_range(const int32_t* table_row, int32_t n_blocks, int32_t page_
 int kv_append_slots(kv_pool_t* pool, int32_t B, int32_t* block_tables, int32_t max_blocks, int32_t* seq_lens,
                     int64_t* slot_mapping);
 
+/* Copy-on-write of shared partial tail pages ([HB-07] Q028: a partial last
+ * block shared by two sequences must be copied, or kept apart, before either
+ * writes to it -- table step 6; [CN-06] 6.5: shared blocks are read-only and
+ * copied on write, with reference counts). Sequences are taken in order of
+ * b; when the page that sequence b's next token goes to (position
+ * seq_lens[b], with seq_lens[b] % P != 0) still has refcount > 1, a fresh
+ * page replaces it in block_tables[b], one reference to the old page is
+ * dropped, and the pair is reported in src_pages[k], dst_pages[k] for
+ * k < *n_copies (host arrays with room for B entries). The last holder keeps
+ * the original. Fresh pages are allocated together, all-or-nothing
+ * (KV_ERR_OOM leaves everything unchanged); KV_ERR_BAD_ID for a tail entry
+ * out of range; KV_ERR_ARG for a full table row. The caller copies the page
+ * contents with kv_copy_pages before the next append. */
+int kv_pool_cow_tails(kv_pool_t* pool, int32_t B, int32_t* block_tables, int32_t max_blocks, const int32_t* seq_lens,
+                      int32_t* src_pages, int32_t* dst_pages, int32_t* n_copies);
+
 /* =========================================================================
  * Prefix index -- [CN-06] 6.4: full cached blocks are keyed by a chained
  * hash of the parent block's key and this block's tokens; the first block
@@ -189,6 +205,15 @@ int kv_prefix_num_entries(const kv_prefix_t* index, int32_t* out);
 int kv_append(void* k_pages, void* v_pages, const void* k_new, const void* v_new, const int64_t* slot_mapping,
               int32_t B, int32_t H_kv, int32_t Dh, int32_t page_size, int32_t num_pages, int32_t dtype,
               int* err_flag, void* stream);
+
+/* Copy whole pages of both pools: for i < n, page src_pages[i] -> page
+ * dst_pages[i] (all H_kv heads and page_size slots; src/dst are device int32
+ * arrays), e.g. after kv_pool_cow_tails. A page id outside [0, num_pages)
+ * sets KV_DEV_ERR_PAGE_RANGE and that pair is skipped. Destinations must be
+ * distinct and must not be sources. */
+int kv_copy_pages(void* k_pages, void* v_pages, const int32_t* src_pages, const int32_t* dst_pages, int32_t n,
+                  int32_t H_kv, int32_t Dh, int32_t page_size, int32_t num_pages, int32_t dtype, int* err_flag,
+                  void* stream);
 
 /* Paged decode attention -- one new query per sequence:
  *   out[b][h][:] = softmax(scale * q[b][h] . K_t) V_t  over t < seq_lens[b]

@@ -132,6 +132,43 @@ class PoolModel:
         return slots
 
 
+    # -- copy-on-write of shared partial tails ([HB-07] Q028 step 6; [CN-06] 6.5) ----
+    def cow_tails(self, tables: List[List[int]], max_blocks: int, lens: List[int]) -> List[Tuple[int, int]]:
+        """Give a sequence whose next append lands in a partial page that is
+        still shared a private copy of that page.
+
+        Sequences are taken in order; sequence b gets a copy when its tail
+        page (lens[b] % P != 0) has refcount > 1 at that moment: a fresh page
+        replaces the tail in its table row, one reference to the old page is
+        dropped, and (old, new) is reported -- the caller copies the contents.
+        The last holder keeps the original. All fresh pages are allocated
+        together, all-or-nothing (a first pass counts them).
+        """
+        P = self.page_size
+        sim = {}
+        marked = []
+        for b, L in enumerate(lens):
+            if L < 0 or L // P >= max_blocks:
+                raise PoolError(ARG)
+            if L % P != 0:
+                t = int(tables[b][L // P])
+                if not (0 <= t < self.num_pages):
+                    raise PoolError(BAD_ID)
+                r = sim.get(t, self.ref[t])
+                if r > 1:
+                    marked.append(b)
+                    sim[t] = r - 1
+        fresh = self.alloc(len(marked))
+        pairs = []
+        for b, new in zip(marked, fresh):
+            L = lens[b]
+            old = int(tables[b][L // P])
+            tables[b][L // P] = new
+            self.free_pages([old])
+            pairs.append((old, new))
+        return pairs
+
+
 class PrefixModel:
     """Brute-force prefix index: full token prefix (with salt) -> block id."""
 

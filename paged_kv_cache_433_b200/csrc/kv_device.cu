@@ -48,6 +48,31 @@ __global__ void __launch_bounds__(256) kv_append_kernel(uint4* __restrict__ k_pa
         k_pages[dst] = k_new[i];
 }
 
+// Whole-page copy for copy-on-write: pair i copies page src[i] to dst[i] in
+// both pools (all H_kv heads, all P slots). One thread moves 16 bytes;
+// threads run over (pair, K/V, 16-byte word).
+__global__ void __launch_bounds__(256) kv_copy_pages_kernel(uint4* __restrict__ k_pages, uint4* __restrict__ v_pages,
+                                                            const int32_t* __restrict__ src,
+                                                            const int32_t* __restrict__ dst, int32_t n,
+                                                            int64_t words_per_page, int32_t num_pages, int* err) {
+    grid_dependency_wait();
+    if (threadIdx.x == 0) grid_launch_dependents();
+    const int64_t total = 2 * (int64_t)n * words_per_page;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t pair_w = i % (n * words_per_page);
+        const bool is_v = i >= n * words_per_page;
+        const int32_t k = static_cast<int32_t>(pair_w / words_per_page);
+        const int64_t w = pair_w - (int64_t)k * words_per_page;
+        const int32_t s = src[k], d = dst[k];
+        if (s < 0 || s >= num_pages || d < 0 || d >= num_pages) {
+            if (w == 0 && !is_v && err) atomicOr(err, KV_DEV_ERR_PAGE_RANGE);
+            continue;
+        }
+        uint4* base = is_v ? v_pages : k_pages;
+        base[(int64_t)d * words_per_page + w] = base[(int64_t)s * words_per_page + w];
+    }
+}
+
 namespace {
 
 int elem_bytes(int32_t dtype) {
@@ -198,6 +223,25 @@ int kv_append(void* k_pages, void* v_pages, const void* k_new, const void* v_new
                                static_cast<uint4*>(v_pages), static_cast<const uint4*>(k_new),
                                static_cast<const uint4*>(v_new), slot_mapping, rows, H_kv, vpr, page_size,
                                static_cast<int64_t>(num_pages) * page_size, err_flag);
+    return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;
+}
+
+int kv_copy_pages(void* k_pages, void* v_pages, const int32_t* src_pages, const int32_t* dst_pages, int32_t n,
+                  int32_t H_kv, int32_t Dh, int32_t page_size, int32_t num_pages, int32_t dtype, int* err_flag,
+                  void* stream) {
+    const int eb = elem_bytes(dtype);
+    if (n < 0 || H_kv <= 0 || Dh <= 0 || page_size <= 0 || num_pages <= 0 || eb == 0) return KV_ERR_ARG;
+    const int64_t page_bytes = static_cast<int64_t>(H_kv) * page_size * Dh * eb;
+    if (page_bytes % 16 != 0) return KV_ERR_UNSUPPORTED;
+    if (n == 0) return KV_OK;
+    if (!k_pages || !v_pages || !src_pages || !dst_pages || !aligned16(k_pages) || !aligned16(v_pages)) return KV_ERR_ARG;
+    const int64_t words = page_bytes / 16;
+    const int64_t total = 2 * static_cast<int64_t>(n) * words;
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > 65535LL * 16) blocks = 65535LL * 16;
+    cudaError_t e = launch_pdl(kv_copy_pages_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
+                               static_cast<cudaStream_t>(stream), static_cast<uint4*>(k_pages),
+                               static_cast<uint4*>(v_pages), src_pages, dst_pages, n, words, num_pages, err_flag);
     return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;
 }
 

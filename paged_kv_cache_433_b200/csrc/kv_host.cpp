@@ -328,6 +328,44 @@ int kv_append_slots(kv_pool_t* pool, int32_t B, int32_t* block_tables, int32_t m
     return KV_OK;
 }
 
+int kv_pool_cow_tails(kv_pool_t* pool, int32_t B, int32_t* block_tables, int32_t max_blocks, const int32_t* seq_lens,
+                      int32_t* src_pages, int32_t* dst_pages, int32_t* n_copies) {
+    if (!pool || !n_copies || B < 0 || max_blocks <= 0 ||
+        (B > 0 && (!block_tables || !seq_lens || !src_pages || !dst_pages)))
+        return KV_ERR_ARG;
+    const int32_t P = pool->page_size;
+    // First pass: which sequences copy (in order, while the tail is still shared).
+    std::unordered_map<int32_t, int32_t> sim;
+    std::vector<int32_t> marked;
+    for (int32_t b = 0; b < B; ++b) {
+        const int32_t L = seq_lens[b];
+        if (L < 0 || L / P >= max_blocks) return KV_ERR_ARG;
+        if (L % P == 0) continue;
+        const int32_t t = block_tables[static_cast<int64_t>(b) * max_blocks + L / P];
+        if (!pool->valid(t)) return KV_ERR_BAD_ID;
+        auto it = sim.find(t);
+        const int32_t r = it == sim.end() ? pool->ref[t] : it->second;
+        if (r > 1) {
+            marked.push_back(b);
+            sim[t] = r - 1;
+        }
+    }
+    std::vector<int32_t> fresh(marked.size());
+    int rc = kv_pool_alloc(pool, static_cast<int32_t>(marked.size()), fresh.data());
+    if (rc != KV_OK) return rc;
+    for (size_t k = 0; k < marked.size(); ++k) {
+        const int32_t b = marked[k];
+        int32_t& slot = block_tables[static_cast<int64_t>(b) * max_blocks + seq_lens[b] / P];
+        const int32_t old = slot;
+        slot = fresh[k];
+        if (--pool->ref[old] == 0) pool->push_tail(old);
+        src_pages[k] = old;
+        dst_pages[k] = fresh[k];
+    }
+    *n_copies = static_cast<int32_t>(marked.size());
+    return KV_OK;
+}
+
 int kv_prefix_index_create(int32_t page_size, uint64_t salt, kv_prefix_t** out) {
     if (!out || page_size <= 0) return KV_ERR_ARG;
     kv_prefix* ix = new (std::nothrow) kv_prefix();

@@ -59,6 +59,8 @@ SIGNATURES = [
     ("kv_slot_for_pos", ctypes.c_int, [_vp, _i32, _i32, _i64, _pi64]),
     ("kv_slots_for_range", ctypes.c_int, [_vp, _i32, _i32, _i64, _i64, _vp]),
     ("kv_append_slots", ctypes.c_int, [_vp, _i32, _vp, _i32, _vp, _vp]),
+    ("kv_pool_cow_tails", ctypes.c_int, [_vp, _i32, _vp, _i32, _vp, _vp, _vp, _pi32]),
+    ("kv_copy_pages", ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
     ("kv_prefix_index_create", ctypes.c_int, [_i32, _u64, _pvp]),
     ("kv_prefix_index_destroy", ctypes.c_int, [_vp]),
     ("kv_prefix_register", ctypes.c_int, [_vp, _vp, _vp, _i32, _vp]),
@@ -203,6 +205,19 @@ class KvPool:
         return slots
 
 
+    def cow_tails(self, block_tables: np.ndarray, seq_lens: np.ndarray):
+        """kv_pool_cow_tails on host arrays (table updated in place); returns (src, dst) int32 arrays."""
+        assert block_tables.dtype == np.int32 and block_tables.flags.c_contiguous
+        lens = _np_i32(seq_lens)
+        B = lens.size
+        src = np.empty(max(B, 1), dtype=np.int32)
+        dst = np.empty(max(B, 1), dtype=np.int32)
+        n = ctypes.c_int32()
+        _check("kv_pool_cow_tails", lib().kv_pool_cow_tails(self._h, B, _p(block_tables), block_tables.shape[1], _p(lens),
+                                                             _p(src), _p(dst), n))
+        return src[: n.value].copy(), dst[: n.value].copy()
+
+
 class KvPrefixIndex:
     """Chained-hash prefix index over full pages (kv_prefix_*)."""
 
@@ -292,6 +307,20 @@ KV_DECODE_KERNEL_AUTO, KV_DECODE_KERNEL_SIMT, KV_DECODE_KERNEL_MMA = 0, 1, 2
 
 def paged_decode_set_kernel(kind: int) -> None:
     _check("paged_decode_set_kernel", lib().paged_decode_set_kernel(kind))
+
+
+def kv_copy_pages(k_pages, v_pages, src_pages, dst_pages, err_flag=None, stream=None) -> None:
+    """Copy whole pages src_pages[i] -> dst_pages[i] of both pools (int32 device tensors)."""
+    import torch
+
+    num_pages, H_kv, P, Dh = k_pages.shape
+    n = src_pages.numel()
+    assert dst_pages.numel() == n and v_pages.shape == k_pages.shape
+    rc = lib().kv_copy_pages(_dev(k_pages, "k_pages"), _dev(v_pages, "v_pages", k_pages.dtype),
+                             _dev(src_pages, "src_pages", torch.int32) if n else None,
+                             _dev(dst_pages, "dst_pages", torch.int32) if n else None, n, H_kv, Dh, P, num_pages,
+                             _torch_dtype_code(k_pages), _dev(err_flag, "err_flag", torch.int32), _stream(stream))
+    _check("kv_copy_pages", rc)
 
 
 def paged_decode_num_splits(B: int, H_kv: int, max_blocks: int, page_size: int, num_splits: int = 0) -> int:

@@ -317,3 +317,49 @@ def test_workspace_too_small_is_refused():
         K.paged_decode_attention(out, q, k_pages, k_pages, tab, lens, 0.1, num_splits=4,
                                  workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
     assert e.value.name == "WORKSPACE"
+
+
+# ---------------------------------------------------------------- copy-on-write (beam fork)
+@pytest.mark.parametrize("dtype,P", [("bf16", 16), ("fp16", 32), ("fp32", 16)])
+def test_beam_fork_copy_on_write(dtype, P, kernel):
+    """Fork sequences that share every page (beam search), give each one a
+    private copy of the shared partial tail (kv_pool_cow_tails + kv_copy_pages),
+    then append different tokens and decode: pools bit-exact, outputs within
+    tolerance of the oracle, and the forks diverge only at the new token."""
+    cfg = W.DecodeConfig(f"fork-{dtype}-{P}", dtype, B=4, H_q=8, H_kv=2, Dh=128 if dtype != "fp32" else 64,
+                         page_size=P, seed=21)
+    lens = [37, 70]  # parents; rows 2 and 3 fork them
+    st = build_cache(cfg, lens + [0, 0], slack_pages=8)
+    for child, parent in ((2, 0), (3, 1)):
+        ids = [int(x) for x in st.tab[parent] if x >= 0]
+        st.pool.incref(ids)
+        st.mpool.incref(ids)
+        st.tab[child] = st.tab[parent]
+        st.mtab[child] = list(st.mtab[parent])
+    st.lens = np.array(lens + lens, dtype=np.int64)
+    src, dst = st.pool.cow_tails(st.tab, st.lens.astype(np.int32))
+    pairs = st.mpool.cow_tails(st.mtab, st.max_blocks, [int(x) for x in st.lens])
+    assert list(zip(src.tolist(), dst.tolist())) == pairs and len(pairs) == 2 and st.tab.tolist() == st.mtab
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    K.kv_copy_pages(st.k_pages, st.v_pages, torch.from_numpy(src).cuda(), torch.from_numpy(dst).cuda(), err_flag=err)
+    for s_, d_ in pairs:
+        st.kp[d_] = st.kp[s_]
+        st.vp[d_] = st.vp[s_]
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    out, ref, err2 = append_and_decode(st, num_splits=0, check_pools=True)
+    assert err2 == 0
+    check_close(out, ref, dtype, "beam fork")
+    assert not np.allclose(out[0], out[2])  # same history, different new token
+
+
+def test_copy_pages_refuses_bad_ids():
+    k_pages = torch.zeros((4, 2, 16, 128), dtype=torch.bfloat16, device="cuda")
+    v_pages = torch.zeros_like(k_pages)
+    k_pages[1] = 1.0
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    K.kv_copy_pages(k_pages, v_pages, torch.tensor([1, 9], dtype=torch.int32, device="cuda"),
+                    torch.tensor([2, 3], dtype=torch.int32, device="cuda"), err_flag=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & K.KV_DEV_ERR_PAGE_RANGE
+    assert torch.equal(k_pages[2], k_pages[1]) and torch.count_nonzero(k_pages[3]).item() == 0

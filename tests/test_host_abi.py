@@ -370,3 +370,54 @@ def test_device_entry_argument_checks_without_gpu():
     assert L.kv_append(None, None, None, None, None, 0, 8, 128, 16, 10, 1, None, None) == K.KV_OK
     assert L.kv_append(None, None, None, None, None, 3, 8, 128, 16, 10, 1, None, None) == K.KV_ERR_ARG
     assert L.kv_append(None, None, None, None, None, 3, 8, 128, 16, 10, 9, None, None) == K.KV_ERR_ARG
+
+
+# ------------------------------------------------------------------ copy-on-write vs model
+@pytest.mark.parametrize("seed", range(4))
+def test_cow_tails_matches_model(seed):
+    rng = np.random.default_rng(500 + seed)
+    P, n, max_blocks = 4, 64, 8
+    order = rng.permutation(n).astype(np.int32)
+    pool, model = K.KvPool(n, P, order), PoolModel(n, P, order)
+    B = 6
+    tab = np.full((B, max_blocks), -1, np.int32)
+    mtab = [[-1] * max_blocks for _ in range(B)]
+    lens = np.zeros(B, np.int32)
+    for b in range(B):
+        if b > 0 and rng.random() < 0.5:  # fork of an earlier sequence
+            src = int(rng.integers(0, b))
+            ids = [int(x) for x in tab[src] if x >= 0]
+            pool.incref(ids)
+            model.incref(ids)
+            tab[b] = tab[src]
+            mtab[b] = list(mtab[src])
+            lens[b] = lens[src]
+        else:
+            L = int(rng.integers(1, max_blocks * P - 1))
+            k = -(-L // P)
+            ids = pool.alloc(k)
+            assert list(ids) == model.alloc(k)
+            tab[b, :k] = ids
+            mtab[b][:k] = list(ids)
+            lens[b] = L
+    src, dst = pool.cow_tails(tab, lens)
+    pairs = model.cow_tails(mtab, max_blocks, [int(x) for x in lens])
+    assert list(zip(src.tolist(), dst.tolist())) == pairs
+    assert tab.tolist() == mtab
+    for p in range(n):
+        assert pool.refcount(p) == model.refcount(p)
+    assert pool.num_free() == model.num_free()
+    # afterwards every append goes to a private page
+    pool.append_slots(tab, lens.copy())
+
+
+def test_cow_tails_oom_leaves_everything_unchanged():
+    pool = K.KvPool(2, 4)
+    a = pool.alloc(2)
+    pool.incref(a[1:])
+    tab = np.array([[a[0], a[1]], [a[0], a[1]]], np.int32)
+    pool.incref(a[:1])
+    before = tab.copy()
+    with pytest.raises(K.KvError) as e:
+        pool.cow_tails(tab, np.array([6, 6], np.int32))
+    assert e.value.name == "OOM" and np.array_equal(tab, before) and pool.refcount(a[1]) == 2

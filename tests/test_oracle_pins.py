@@ -358,3 +358,39 @@ def test_merge_of_summarised_blocks_equals_full_softmax():
     assert np.allclose(acc[2] / acc[1], full, atol=1e-12)
     _, _, _, o = R.online_softmax([(s[a:b], v[a:b]) for a, b in zip(cuts[:-1], cuts[1:])])
     assert np.allclose(o, full, atol=1e-12)
+
+
+def test_copy_on_write_of_a_shared_partial_tail():
+    """[HB-07] Q028 table step 6: A and B share an unfilled last block; before
+    they append different tokens one of them needs its own copy."""
+    P = 4
+    pool = PoolModel(16, P, list(range(16)))
+    a = pool.alloc(3)  # 10 tokens: blocks 0, 1 full, block 2 holds positions 8, 9
+    pool.incref(a)  # B is a fork of A (beam): shares all three blocks
+    tabs = [a + [-1], list(a) + [-1]]
+    lens = [10, 10]
+    with pytest.raises(PoolError) as e:
+        pool.append_slots([list(r) for r in tabs], 4, list(lens))
+    assert e.value.kind == "SHARED_TAIL"
+    pairs = pool.cow_tails(tabs, 4, lens)
+    assert pairs == [(a[2], 3)]  # A copies, B (last holder) keeps the original
+    assert tabs[0][:3] == [a[0], a[1], 3] and tabs[1][:3] == a
+    assert pool.refcount(a[2]) == 1 and pool.refcount(3) == 1 and pool.refcount(a[0]) == 2
+    slots = pool.append_slots(tabs, 4, lens)
+    assert slots == [3 * P + 2, a[2] * P + 2]  # different physical slots, same logical position 10
+    # full shared blocks are never copied; nothing to do once tails are private
+    assert pool.cow_tails(tabs, 4, lens) == []
+
+
+def test_copy_on_write_keeps_outside_holders():
+    P = 4
+    pool = PoolModel(16, P)
+    a = pool.alloc(1)
+    pool.incref(a)
+    pool.incref(a)  # three holders; two of them append this step
+    tabs = [[a[0], -1], [a[0], -1]]
+    pairs = pool.cow_tails(tabs, 2, [2, 2])
+    assert len(pairs) == 2 and pool.refcount(a[0]) == 1  # the third holder keeps the original
+    with pytest.raises(PoolError) as e:
+        PoolModel(1, P).cow_tails([[0]], 1, [4])  # full table row
+    assert e.value.kind == "ARG"
