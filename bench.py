@@ -226,6 +226,12 @@ class Workload:
         return kv + q + out + tables
 
 
+def launches_per_call(S, args):
+    """Library kernels per append+decode call: plan + decode + combine for a device-planned launch (S == 0),
+    decode (+ combine when split) otherwise, plus kv_append when it is not fused."""
+    return (3 if S == 0 else (2 if S > 1 else 1)) + (args.append == "separate")
+
+
 def hot_path(K, args, cfg, kp, vp, kn, vn, slots, q, tab, lens, out, ws, err, stream, ev=None):
     """One layer's step on the device: append the new token, then decode (fused into one launch by default).
     `ev` = (start, end) events recorded around the timed kernel call."""
@@ -381,7 +387,7 @@ def run_layer_bench(args, world, rank, local):
                      "traffic_source": ("ncu dram bytes of the decode kernel (profiles/" + os.path.basename(PROFILE_DECODE)
                                         + "), scaled to this run's algorithmic bytes") if traffic else None, "kernel": "paged_decode_attention" + (" (split + combine)" if S > 1 else " (single pass)"),
                      "bytes_per_launch": mean_bytes, "launch_us": mean_dec_s * 1e6},
-        "gpu_launches": steps * ((2 if S > 1 else 1) + (args.append == "separate")),
+        "gpu_launches": steps * launches_per_call(S, args),
         "e2e": e2e,
         "clocks": clocks,
     }
@@ -552,7 +558,7 @@ def run_long_bench(args, world, rank, local):
                      "kernel": ("32 x (paged_decode_attention_append + combine) per step" if args.append == "fused"
                                 else "32 x (kv_append + paged_decode_attention + combine) per step"),
                      "bytes_per_step": float(np.mean(bytes_step)), "pass_us": float(np.mean(pass_ms)) * 1e3},
-        "gpu_launches": steps * L * ((2 if S > 1 else 1) + (args.append == "separate")),
+        "gpu_launches": steps * L * launches_per_call(S, args),
         "e2e": None,
         "clocks": clocks,
     }
@@ -630,7 +636,7 @@ def time_steps(args, st, steps, warm, before_step=None):
     ws = torch.zeros(max(nb, 16), dtype=torch.uint8, device=dev)
     res = []
     S = K.paged_decode_num_splits(st.B, cfg.H_kv, st.max_blocks, st.P, args.splits)
-    st.launches_per_step = (2 if S > 1 else 1) + (args.append == "separate")
+    st.launches_per_step = launches_per_call(S, args)
     for i in range(warm + steps):
         if before_step is not None:
             before_step(i)

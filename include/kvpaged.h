@@ -227,7 +227,13 @@ int kv_copy_pages(void* k_pages, void* v_pages, const int32_t* src_pages, const 
  *   H_q / H_kv <= 32; dtype F32/BF16/F16. Else KV_ERR_UNSUPPORTED/KV_ERR_ARG.
  *   num_splits: 1 = single pass; >1 = split each sequence's pages into that
  *   many contiguous ranges (split-KV) merged by a second combine kernel;
- *   0 = choose automatically from B, H_kv, max_blocks and the SM count.
+ *   0 = choose automatically from B, H_kv, max_blocks and the SM count;
+ *   for bf16/fp16 K/V on the tensor-core kernel with more (sequence, KV
+ *   head) rows than 4 x the SM count (and B <= 8192), a planned launch is
+ *   used instead: a one-CTA plan kernel reads seq_lens and cuts every row
+ *   into chunks of C pages chosen from the actual lengths (full chunks at
+ *   the front of the grid, short tail chunks at the back), then the decode
+ *   and combine kernels follow that plan (three launches).
  *   workspace / ws_bytes: device scratch for split partials, at least
  *   paged_decode_workspace_bytes(...) for the same arguments (NULL/0 is fine
  *   when no split is used); KV_ERR_WORKSPACE if too small. Calls sharing one
@@ -268,7 +274,10 @@ int paged_decode_attention_append(float* out, const void* q, const void* k_new, 
 int paged_decode_set_kernel(int32_t kind);
 
 /* The split count paged_decode_attention will use for these arguments
- * (resolves num_splits = 0 on the current device). */
+ * (resolves num_splits = 0 on the current device). 0 means the launch is
+ * planned on the device (see paged_decode_attention) -- which holds for
+ * bf16/fp16 K/V on the tensor-core kernel; fp32 K/V and the CUDA-core kernel
+ * use the grid rule's split count even then. */
 int paged_decode_num_splits(int32_t B, int32_t H_kv, int32_t max_blocks, int32_t page_size, int32_t num_splits,
                             int32_t* out);
 

@@ -20,12 +20,17 @@ namespace kvp {
 // and (WPR > 1) a shared-memory sum over the row's warps, all relative to the
 // same m*.
 constexpr int kCombineWarps = 8;
+constexpr int kPlanHdrCombine = 4;  // first S_b entry of a plan
 
+// Planned launches (plan != nullptr, WPR == 1 only): the row's chunk size and
+// first item come from the plan; rows with one chunk were written by the
+// decode kernel and are skipped, empty rows are zeroed here; partial s of
+// (b, query head h) sits at item t0 + s, row h of that item's [g][Dh] block.
 template <int DH, int WPR>
 __global__ void __launch_bounds__(32 * kCombineWarps) paged_combine_kernel(
     float* __restrict__ out, const float* __restrict__ part_u, const float2* __restrict__ part_ml,
     const int32_t* __restrict__ seq_lens, int32_t B, int32_t H_q, int32_t S, int32_t pages_per_split, int32_t P,
-    int32_t max_blocks) {
+    int32_t max_blocks, const int32_t* __restrict__ plan, int32_t H_kv) {
     constexpr int kD = DH / 32;  // dims per lane
     constexpr int kPer = 8;      // splits per warp per round
     constexpr int kRound = WPR * kPer;
@@ -38,16 +43,30 @@ __global__ void __launch_bounds__(32 * kCombineWarps) paged_combine_kernel(
     const int64_t item = (int64_t)blockIdx.x * kRows + warp / WPR;
     grid_dependency_wait();  // the decode kernel's partials
     if (threadIdx.x == 0) grid_launch_dependents();
-    const bool live = item < (int64_t)B * H_q;
+    bool live = item < (int64_t)B * H_q;
     int ns = 0;
+    int64_t base = item * S, stride = 1;
     if (live) {
-        int len = seq_lens[item / H_q];
+        const int b = static_cast<int>(item / H_q);
+        int len = seq_lens[b];
         if (len < 0 || len > max_blocks * P) len = 0;
         const int n_pages = (len + P - 1) / P;
-        ns = min(S, (n_pages + pages_per_split - 1) / pages_per_split);
+        if (plan != nullptr) {
+            const int C = plan[0];
+            const int items_b = (n_pages + C - 1) / C;
+            const int g = H_q / H_kv;
+            const int hq = static_cast<int>(item % H_q);
+            if (items_b == 1) live = false;  // the decode kernel wrote this row
+            ns = items_b > 1 ? items_b : 0;
+            const int64_t t0 = (int64_t)H_kv * plan[kPlanHdrCombine + b] + (int64_t)(hq / g) * items_b;
+            base = t0 * g + hq % g;
+            stride = g;
+        } else {
+            ns = min(S, (n_pages + pages_per_split - 1) / pages_per_split);
+        }
     }
-    const float2* ml = part_ml + item * S;
-    const float* pu = part_u + item * S * DH + lane * kD;
+    const float2* ml = part_ml + base;
+    const float* pu = part_u + base * DH + lane * kD;
 
     float acc[kD];
 #pragma unroll
@@ -61,8 +80,8 @@ __global__ void __launch_bounds__(32 * kCombineWarps) paged_combine_kernel(
         for (int j = 0; j < kPer; ++j) {
             const int s = r0 + rw + j * WPR;
             if (s < ns) {
-                st[j] = ml[s];
-                const float* src = pu + (int64_t)s * DH;
+                st[j] = ml[s * stride];
+                const float* src = pu + (int64_t)s * stride * DH;
                 if constexpr (kD == 4) {
                     const float4 x = *reinterpret_cast<const float4*>(src);
                     v[j][0] = x.x; v[j][1] = x.y; v[j][2] = x.z; v[j][3] = x.w;
@@ -77,7 +96,7 @@ __global__ void __launch_bounds__(32 * kCombineWarps) paged_combine_kernel(
             }
         }
         if (r0 == 0) {
-            for (int s = lane; s < ns; s += 32) mstar = fmaxf(mstar, ml[s].x);
+            for (int s = lane; s < ns; s += 32) mstar = fmaxf(mstar, ml[s * stride].x);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) mstar = fmaxf(mstar, __shfl_xor_sync(0xffffffffu, mstar, o));
         }

@@ -59,8 +59,10 @@ struct DecodeParams {
     const int32_t* seq_lens;      // [B]
     const void* k_new;          // nullable: fused append of the token at position len - 1, [B][H_kv][Dh]
     const void* v_new;
-    float* part_u;              // split: [B][H_q][S][Dh]
-    float2* part_ml;            // split: [B][H_q][S] (m in log2 units, l)
+    float* part_u;              // split: [B][H_q][S][Dh]; planned: [item][g][Dh]
+    float2* part_ml;            // split: [B][H_q][S]; planned: [item][g] (m in log2 units, l)
+    const int4* items;          // planned launch: {b, kvh, chunk, item} per CTA (nullable)
+    const int32_t* plan;        // planned launch: [0] pages per chunk, [4 + b] item prefix
     int* err;
     int32_t max_blocks, B, H_q, H_kv, num_pages;
     int32_t g, HS, WP;          // GQA group, head slices, page-warps

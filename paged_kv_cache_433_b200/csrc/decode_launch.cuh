@@ -81,7 +81,7 @@ cudaError_t launch_decode_f16(const DecodeParams& p, int DH, int P, int GW, int 
 
 namespace kvp {
 
-template <int DT, int DH, int P>
+template <int DT, int DH, int P, bool LO>
 cudaError_t launch_mma_inst(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, dim3 grid,
                             cudaStream_t st) {
     constexpr int NW = 4;
@@ -92,23 +92,33 @@ cudaError_t launch_mma_inst(const DecodeParams& p, const CUtensorMap& tk, const 
     if (e != cudaSuccess) return e;
     const uint64_t bit = 1ull << (dev & 63);
     if (!(configured.load(std::memory_order_acquire) & bit)) {
-        e = cudaFuncSetAttribute(paged_decode_mma_kernel<DT, DH, P, NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(paged_decode_mma_kernel<DT, DH, P, NW, LO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::kSmem);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(paged_decode_mma_kernel<DT, DH, P, NW>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 100);
+        e = cudaFuncSetAttribute(paged_decode_mma_kernel<DT, DH, P, NW, LO>,
+                                 cudaFuncAttributePreferredSharedMemoryCarveout, 100);
         if (e != cudaSuccess) return e;
         configured.fetch_or(bit, std::memory_order_acq_rel);
     }
-    return launch_pdl(paged_decode_mma_kernel<DT, DH, P, NW>, grid, dim3(C::kThreads), C::kSmem, st, p, tk, tv);
+    return launch_pdl(paged_decode_mma_kernel<DT, DH, P, NW, LO>, grid, dim3(C::kThreads), C::kSmem, st, p, tk, tv);
+}
+
+// Groups of at most 8 heads take the instance that carries the probability
+// residual in the MMA's padding rows.
+template <int DT, int DH, int P>
+cudaError_t launch_mma_group(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, dim3 grid,
+                             cudaStream_t st) {
+    return p.g <= 8 ? launch_mma_inst<DT, DH, P, true>(p, tk, tv, grid, st)
+                    : launch_mma_inst<DT, DH, P, false>(p, tk, tv, grid, st);
 }
 
 template <int DT>
 cudaError_t launch_mma_dt(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int DH, int P, dim3 grid,
                           cudaStream_t st) {
     if (DH == 128)
-        return P == 16 ? launch_mma_inst<DT, 128, 16>(p, tk, tv, grid, st) : launch_mma_inst<DT, 128, 32>(p, tk, tv, grid, st);
-    return P == 16 ? launch_mma_inst<DT, 64, 16>(p, tk, tv, grid, st) : launch_mma_inst<DT, 64, 32>(p, tk, tv, grid, st);
+        return P == 16 ? launch_mma_group<DT, 128, 16>(p, tk, tv, grid, st)
+                       : launch_mma_group<DT, 128, 32>(p, tk, tv, grid, st);
+    return P == 16 ? launch_mma_group<DT, 64, 16>(p, tk, tv, grid, st) : launch_mma_group<DT, 64, 32>(p, tk, tv, grid, st);
 }
 
 // Defined in decode_mma_bf16.cu / decode_mma_f16.cu.

@@ -7,7 +7,8 @@
 // (page, head) chunk costs ~100 instructions instead of ~800 on the CUDA
 // cores:
 //   S[16 x P]  = Q[16 heads x Dh] . K_page^T      (m16n8k16, k over Dh)
-//   O[16 x Dh] += P[16 x P] . V_page               (m16n8k16, k over tokens)
+//   O[16 x Dh] += P[16 x P] . V_page               (m16n8k16, k over tokens;
+//                                                   P as a 16-bit pair + residual)
 // The GQA group is the M dimension (rows >= g are zero padding), so the S
 // accumulator fragment is, element for element, the A fragment of the second
 // product: probabilities never leave registers.
@@ -61,7 +62,9 @@ struct MmaCfg {
     static_assert(kNS % NW == 0, "stage ring must be a multiple of the page-warps");
 };
 
-template <int DT, int DH, int P, int NW>
+// LO: the GQA group has at most 8 heads (one head slice, rows 8..15 are
+// padding), so each row's probability residual rides in row r + 8.
+template <int DT, int DH, int P, int NW, bool LO>
 __global__ void __launch_bounds__(32 * (NW + 1), 2)
     paged_decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                             const __grid_constant__ CUtensorMap tmap_v) {
@@ -69,31 +72,46 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
     constexpr bool kBF16 = DT == KV_DTYPE_BF16;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
 
-    const int split = blockIdx.x;
-    const int kvh = blockIdx.y;
-    const int b = blockIdx.z;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const bool split_mode = p.num_splits > 1;
-
     if (threadIdx.x == 0) {
         prefetch_tmap(&tmap_k);
         prefetch_tmap(&tmap_v);
     }
-    grid_dependency_wait();  // inputs may come from the previous kernel in the stream
+    grid_dependency_wait();  // inputs (and a plan) may come from the previous kernel in the stream
     if (threadIdx.x == 0) grid_launch_dependents();
+
+    // Work of this CTA: (split, kvh, b) from the grid, or a planned chunk.
+    int split, kvh, b, item = 0, chunk_pages;
+    if (p.items != nullptr) {
+        const int4 it = p.items[blockIdx.x];
+        if (it.x < 0) return;
+        b = it.x;
+        kvh = it.y;
+        split = it.z;
+        item = it.w;
+        chunk_pages = p.plan[0];
+    } else {
+        split = blockIdx.x;
+        kvh = blockIdx.y;
+        b = blockIdx.z;
+        chunk_pages = p.pages_per_split;
+    }
+    const bool chunked = p.items != nullptr || p.num_splits > 1;
     // The producer's first 32 block-table entries do not depend on the length:
     // load them alongside it.
-    const int first = split_mode ? split * p.pages_per_split : 0;
+    const int first = chunked ? split * chunk_pages : 0;
     int tab0 = 0;
     if (warp == 0 && first + lane < p.max_blocks) tab0 = p.block_tables[(int64_t)b * p.max_blocks + first + lane];
     int len = p.seq_lens[b];
     if (len < 0 || len > p.max_blocks * P) {
-        if (threadIdx.x == 0 && split == 0) raise_err(p.err, KV_DEV_ERR_SEQ_LEN);
+        if (threadIdx.x == 0 && split == 0 && p.items == nullptr) raise_err(p.err, KV_DEV_ERR_SEQ_LEN);
         len = 0;
     }
     const int n_pages = (len + P - 1) / P;
-    const int n_local = split_mode ? min(p.pages_per_split, n_pages - first) : n_pages;
+    const int n_local = chunked ? min(chunk_pages, n_pages - first) : n_pages;
+    // Partials are needed when the row has more than one chunk.
+    const bool split_mode = p.items != nullptr ? n_pages > chunk_pages : p.num_splits > 1;
     if (n_local <= 0) {
         if (!split_mode) {
             for (int e = threadIdx.x; e < p.g * DH; e += blockDim.x)
@@ -221,6 +239,7 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
     const int quad = lane & 3;   // column pair within a fragment
     const int r0 = lane >> 2;    // fragment rows r0 and r0 + 8
     const int rows = min(16, p.g - hs * 16);  // real heads in this slice
+    constexpr bool lo_rows = LO;               // padding rows 8..15 carry the P residual
     const int hbase = kvh * p.g + hs * 16;    // query head of row 0
 
     // Q as the A operand of S = Q K^T: rows = heads, k = dims (pairs of elements per register).
@@ -304,7 +323,7 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
                     mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
                 }
                 // lazy reference update: only when a row's max grows by more than 2^8
-                const bool grow = (mx[0] > m_ref[0] + 8.f) || (mx[1] > m_ref[1] + 8.f);
+                const bool grow = (mx[0] > m_ref[0] + 8.f) || (!lo_rows && mx[1] > m_ref[1] + 8.f);
                 if (__any_sync(0xffffffffu, grow)) {
                     float a[2];
 #pragma unroll
@@ -314,6 +333,7 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
                         m_ref[h] = mn;
                         l_part[h] *= a[h];
                     }
+                    if constexpr (lo_rows) a[1] = a[0];  // rows r0 + 8 hold row r0's residual sums
 #pragma unroll
                     for (int n = 0; n < C::kOT; ++n) {
                         o[n][0] *= a[0];
@@ -322,19 +342,29 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
                         o[n][3] *= a[1];
                     }
                 }
-                // ---- probabilities straight into the A fragments of P V
-                uint32_t pa[C::kPK][4];
+                // ---- probabilities straight into the A fragments of P V, as a
+                // 16-bit pair plus its residual: one rounding of p to bf16
+                // (2^-9 relative) alone can move a short row's output by
+                // 2^-9 * max|v|, beyond the accuracy this kernel keeps. With
+                // at most 8 real heads the residual of row r rides in padding
+                // row r + 8 of the same MMA (summed at the end); otherwise it
+                // takes a second MMA.
+                uint32_t pa[C::kPK][4], pr[C::kPK][4];
 #pragma unroll
                 for (int n = 0; n < C::kNT; ++n) {
                     float pv[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
+                    for (int e = 0; e < (lo_rows ? 2 : 4); ++e) {
                         const float mr = m_ref[e >> 1];
                         pv[e] = (sc[n][e] == -INFINITY) ? 0.f : exp2f(sc[n][e] - mr);
                         l_part[e >> 1] += pv[e];
                     }
-                    pa[n >> 1][(n & 1) * 2 + 0] = pack2<kBF16>(pv[0], pv[1]);
-                    pa[n >> 1][(n & 1) * 2 + 1] = pack2<kBF16>(pv[2], pv[3]);
+                    if constexpr (lo_rows) {
+                        pack2_split<kBF16>(pv[0], pv[1], pa[n >> 1][(n & 1) * 2 + 0], pa[n >> 1][(n & 1) * 2 + 1]);
+                    } else {
+                        pack2_split<kBF16>(pv[0], pv[1], pa[n >> 1][(n & 1) * 2 + 0], pr[n >> 1][(n & 1) * 2 + 0]);
+                        pack2_split<kBF16>(pv[2], pv[3], pa[n >> 1][(n & 1) * 2 + 1], pr[n >> 1][(n & 1) * 2 + 1]);
+                    }
                 }
                 // ---- tail page: zero V rows past the length (they may hold stale data)
                 if (nvalid < P) {
@@ -357,6 +387,10 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
                         ldsm_x4_trans(sV + (c >> 3) * C::kBoxB + t * 128 + (((c & 7) ^ (t & 7)) << 4), v0, v1, v2, v3);
                         mma_16816<kBF16>(o[2 * op], pa[ks], v0, v1);
                         mma_16816<kBF16>(o[2 * op + 1], pa[ks], v2, v3);
+                        if constexpr (!lo_rows) {
+                            mma_16816<kBF16>(o[2 * op], pr[ks], v0, v1);
+                            mma_16816<kBF16>(o[2 * op + 1], pr[ks], v2, v3);
+                        }
                     }
                 }
             }
@@ -381,8 +415,8 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
                 float* dst = merge + (cw * 16 + r) * (DH + 2);
 #pragma unroll
                 for (int n = 0; n < C::kOT; ++n) {
-                    dst[n * 8 + 2 * quad] = o[n][2 * h];
-                    dst[n * 8 + 2 * quad + 1] = o[n][2 * h + 1];
+                    dst[n * 8 + 2 * quad] = o[n][2 * h] + (lo_rows ? o[n][2] : 0.f);
+                    dst[n * 8 + 2 * quad + 1] = o[n][2 * h + 1] + (lo_rows ? o[n][3] : 0.f);
                 }
                 if (quad == 0) {
                     dst[DH] = m_ref[h];
@@ -415,7 +449,7 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
         if (!split_mode) {
             p.out[hq * DH + d] = (L > 0.f) ? U / L : 0.f;
         } else {
-            const int64_t ps = hq * p.num_splits + split;
+            const int64_t ps = p.items != nullptr ? (int64_t)item * p.g + hh : hq * p.num_splits + split;
             p.part_u[ps * DH + d] = U;
             if (d == 0) p.part_ml[ps] = make_float2(mstar, L);
         }

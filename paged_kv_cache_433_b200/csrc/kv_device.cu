@@ -5,12 +5,14 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 
 #include "combine_kernel.cuh"
 #include "decode_launch.cuh"
 #include "kvpaged.h"
+#include "plan_kernel.cuh"
 
 namespace kvp {
 
@@ -187,6 +189,44 @@ size_t workspace_for(int32_t B, int32_t H_q, int32_t Dh, int32_t S) {
     return rows * Dh * sizeof(float) + rows * sizeof(float2);
 }
 
+// Planned launches (tensor-core kernel, num_splits == 0, B > 1): the grid is
+// an upper bound on the plan's chunk count -- 4 chunks per resident slot plus
+// one tail chunk per row.
+int64_t planned_grid(int32_t B, int32_t H_kv) {
+    const int sms = sm_count();
+    if (sms <= 0) return -1;
+    return 4LL * 2 * sms + static_cast<int64_t>(B) * H_kv;
+}
+
+struct PlannedLayout {
+    size_t plan_off, items_off, u_off, ml_off, total;
+};
+
+PlannedLayout planned_layout(int32_t B, int32_t H_q, int32_t H_kv, int32_t Dh, int64_t grid) {
+    auto r16 = [](size_t x) { return (x + 15) / 16 * 16; };
+    const size_t g = static_cast<size_t>(H_q / H_kv);
+    PlannedLayout L{};
+    L.plan_off = 0;
+    L.items_off = r16(sizeof(int32_t) * (kPlanHdr + static_cast<size_t>(B) + 1));
+    L.u_off = L.items_off + r16(sizeof(int4) * static_cast<size_t>(grid));
+    L.ml_off = L.u_off + r16(sizeof(float) * static_cast<size_t>(grid) * g * Dh);
+    L.total = L.ml_off + r16(sizeof(float2) * static_cast<size_t>(grid) * g);
+    return L;
+}
+
+// Automatic split choice between the two launch forms. With no more
+// (sequence, KV head) rows than two waves of resident CTAs, the grid rule
+// splits every row into equal ranges of the longest possible row and keeps
+// up (measured on the 8B-shaped B=64 layer and the shared-prefix batch);
+// beyond that it cannot split rows at all (S = 1), and in a skewed batch a
+// few long rows end the launch alone -- there the plan, which chunks rows by
+// their actual lengths on the device, is used.
+bool planned_ok(bool mma, int32_t B, int32_t H_q, int32_t H_kv, int32_t num_splits) {
+    const int sms = sm_count();
+    return mma && num_splits == 0 && B > 1 && B <= kPlanThreads * kPlanRowsPerThread && (H_q / H_kv) <= 64 &&
+           sms > 0 && static_cast<int64_t>(B) * H_kv > 4LL * sms;
+}
+
 int check_shape(int32_t H_q, int32_t H_kv, int32_t Dh, int32_t page_size, int32_t dtype) {
     if (H_q <= 0 || H_kv <= 0 || H_q % H_kv != 0) return KV_ERR_ARG;
     if (elem_bytes(dtype) == 0) return KV_ERR_ARG;
@@ -256,7 +296,7 @@ int paged_decode_num_splits(int32_t B, int32_t H_kv, int32_t max_blocks, int32_t
     if (!out || B < 0 || H_kv <= 0 || max_blocks <= 0 || page_size <= 0 || num_splits < 0) return KV_ERR_ARG;
     int32_t S, C;
     int rc = resolve_splits(B, H_kv, max_blocks, num_splits, &S, &C);
-    if (rc == KV_OK) *out = S;
+    if (rc == KV_OK) *out = planned_ok(true, B, /*H_q=*/H_kv, H_kv, num_splits) ? 0 : S;
     return rc;
 }
 
@@ -267,7 +307,14 @@ int paged_decode_workspace_bytes(int32_t B, int32_t H_q, int32_t H_kv, int32_t D
     int32_t S, C;
     int rc = resolve_splits(B, H_kv, max_blocks, num_splits, &S, &C);
     if (rc != KV_OK) return rc;
-    *out = workspace_for(B, H_q, Dh, S);
+    size_t need = workspace_for(B, H_q, Dh, S);
+    if (planned_ok(true, B, H_q, H_kv, num_splits)) {
+        const int64_t grid = planned_grid(B, H_kv);
+        if (grid < 0) return KV_ERR_CUDA;
+        const size_t pl = planned_layout(B, H_q, H_kv, Dh, grid).total;
+        if (pl > need) need = pl;
+    }
+    *out = need;
     return KV_OK;
 }
 
@@ -301,6 +348,7 @@ int decode_impl(float* out, const void* q, const void* k_new, const void* v_new,
     int32_t S, C;
     rc = resolve_splits(B, H_kv, max_blocks, num_splits, &S, &C);
     if (rc != KV_OK) return rc;
+    const bool planned = planned_ok(mma, B, H_q, H_kv, num_splits);
 
     DecodeParams p{};
     p.out = out;
@@ -323,16 +371,41 @@ int decode_impl(float* out, const void* q, const void* k_new, const void* v_new,
     p.num_splits = S;
     p.pages_per_split = C;
     p.scale_log2 = scale * kLog2e;
-    if (S > 1) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    dim3 grid(static_cast<unsigned>(S), static_cast<unsigned>(H_kv), static_cast<unsigned>(B));
+    cudaError_t e;
+    int64_t pgrid = 0;
+    if (planned) {
+        pgrid = planned_grid(B, H_kv);
+        if (pgrid < 0) return KV_ERR_CUDA;
+        if (pgrid > 0x7fffffffLL) return KV_ERR_UNSUPPORTED;
+        const PlannedLayout L = planned_layout(B, H_q, H_kv, Dh, pgrid);
+        if (!workspace || ws_bytes < L.total || !aligned16(workspace)) return KV_ERR_WORKSPACE;
+        char* w = static_cast<char*>(workspace);
+        int32_t* plan = reinterpret_cast<int32_t*>(w + L.plan_off);
+        int4* items = reinterpret_cast<int4*>(w + L.items_off);
+        p.plan = plan;
+        p.items = items;
+        p.part_u = reinterpret_cast<float*>(w + L.u_off);
+        p.part_ml = reinterpret_cast<float2*>(w + L.ml_off);
+        p.num_splits = 0;
+        // chunk floor: a chunk's partial (g x (Dh + 2) fp32) at most ~6 % of its K/V bytes
+        const int64_t chunk_bytes_per_page = 2LL * page_size * Dh * elem_bytes(dtype);
+        const int64_t partial_bytes = static_cast<int64_t>(H_q / H_kv) * (Dh + 2) * 4;
+        const int32_t c_floor = static_cast<int32_t>(std::max<int64_t>(8, (16 * partial_bytes + chunk_bytes_per_page - 1) /
+                                                                                chunk_bytes_per_page));
+        e = launch_pdl(paged_plan_kernel, dim3(1), dim3(kPlanThreads), 0, st, seq_lens, B, H_kv, page_size, max_blocks,
+                       static_cast<int32_t>(2 * sm_count()), static_cast<int32_t>(pgrid), c_floor, plan, items,
+                       err_flag);
+        if (e != cudaSuccess) return KV_ERR_CUDA;
+        grid = dim3(static_cast<unsigned>(pgrid), 1, 1);
+    } else if (S > 1) {
         const size_t need = workspace_for(B, H_q, Dh, S);
         if (!workspace || ws_bytes < need || !aligned16(workspace)) return KV_ERR_WORKSPACE;
         const size_t rows = static_cast<size_t>(B) * H_q * S;
         p.part_u = static_cast<float*>(workspace);
         p.part_ml = reinterpret_cast<float2*>(static_cast<char*>(workspace) + rows * Dh * sizeof(float));
     }
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    dim3 grid(static_cast<unsigned>(S), static_cast<unsigned>(H_kv), static_cast<unsigned>(B));
-    cudaError_t e;
     if (mma) {
         CUtensorMap tk, tv;
         const int64_t rows = static_cast<int64_t>(num_pages) * H_kv * page_size;
@@ -349,10 +422,12 @@ int decode_impl(float* out, const void* q, const void* k_new, const void* v_new,
         }
     }
     if (e != cudaSuccess) return KV_ERR_CUDA;
-    if (S > 1) {
-        // one warp per row when a single round of 8 loads per lane covers the splits, else 8 warps per row
+    if (planned || S > 1) {
+        // one warp per row when a single round of 8 loads per lane covers the splits (and for
+        // planned launches, where rows have different chunk counts), else 8 warps per row
         const int64_t rows = static_cast<int64_t>(B) * H_q;
-        const bool narrow = S <= 8;
+        const bool narrow = planned || S <= 8;
+        const int32_t* plan = planned ? p.plan : nullptr;
         const int64_t rows_per_cta = narrow ? kCombineWarps : 1;
         const dim3 blocks(static_cast<unsigned>((rows + rows_per_cta - 1) / rows_per_cta));
         const dim3 threads(32 * kCombineWarps);
@@ -360,14 +435,14 @@ int decode_impl(float* out, const void* q, const void* k_new, const void* v_new,
         const float* pu = p.part_u;
         if (Dh == 128)
             e = narrow ? launch_pdl(paged_combine_kernel<128, 1>, blocks, threads, 0, st, out, pu, ml, seq_lens, B, H_q,
-                                    S, C, page_size, max_blocks)
+                                    S, C, page_size, max_blocks, plan, H_kv)
                        : launch_pdl(paged_combine_kernel<128, kCombineWarps>, blocks, threads, 0, st, out, pu, ml,
-                                    seq_lens, B, H_q, S, C, page_size, max_blocks);
+                                    seq_lens, B, H_q, S, C, page_size, max_blocks, plan, H_kv);
         else
             e = narrow ? launch_pdl(paged_combine_kernel<64, 1>, blocks, threads, 0, st, out, pu, ml, seq_lens, B, H_q, S,
-                                    C, page_size, max_blocks)
+                                    C, page_size, max_blocks, plan, H_kv)
                        : launch_pdl(paged_combine_kernel<64, kCombineWarps>, blocks, threads, 0, st, out, pu, ml,
-                                    seq_lens, B, H_q, S, C, page_size, max_blocks);
+                                    seq_lens, B, H_q, S, C, page_size, max_blocks, plan, H_kv);
         if (e != cudaSuccess) return KV_ERR_CUDA;
     }
     return KV_OK;

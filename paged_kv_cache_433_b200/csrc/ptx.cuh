@@ -158,6 +158,25 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     return r;
 }
 
+// Two fp32 values as a rounded 16-bit pair `hi` plus the rounded residual
+// pair `lo` (x - float(hi), exact in fp32): hi + lo carries x to ~2^-16
+// relative, so a product summed over both pairs loses almost nothing to the
+// 16-bit operand format.
+template <bool IS_BF16>
+__device__ __forceinline__ void pack2_split(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+    hi = pack2<IS_BF16>(x0, x1);
+    float h0, h1;
+    if constexpr (IS_BF16) {
+        h0 = __uint_as_float(hi << 16);
+        h1 = __uint_as_float(hi & 0xffff0000u);
+    } else {
+        asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
+            : "=f"(h0), "=f"(h1)
+            : "r"(hi));
+    }
+    lo = pack2<IS_BF16>(x0 - h0, x1 - h1);
+}
+
 __device__ __forceinline__ void sts128_zero(uint32_t addr) {
     asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
 }

@@ -156,6 +156,25 @@ def lognormal_lengths(n: int, g: np.random.Generator) -> np.ndarray:
     return np.clip(np.rint(x), 16, 16384).astype(np.int64)
 
 
+def ragged_lengths(B: int, page_size: int, seed: int, uniform: bool = False) -> np.ndarray:
+    """Cached lengths for a many-row batch with the ragged cases a chunked
+    launch meets: log-normal body (median 96 tokens, sigma 1), empty rows,
+    rows that end exactly on a page boundary after the append, rows of 8, 16,
+    65 and 130 whole pages after the append, and one long row (60 pages).
+    uniform=True: every row 37 pages + 3 tokens after the append."""
+    P = page_size
+    if uniform:
+        return np.full(B, 37 * P + 2, dtype=np.int64)
+    g = generator(seed, S_LENGTHS, B, P)
+    x = np.clip(np.rint(np.exp(np.log(96.0) + g.standard_normal(B))), 0, 40 * P).astype(np.int64)
+    x[0::17] = 0
+    x[1::23] = P - 1
+    for i, pages in enumerate((8, 16, 65, 130)):
+        x[5 + i::31] = pages * P - 1
+    x[B // 2] = 60 * P - 7
+    return x
+
+
 @dataclass
 class ChurnEvent:
     """One step of the mixed sweep: which batch slots exit and their new lengths."""

@@ -215,6 +215,8 @@ EDGE_SHAPES = [
     ("bf16", 128, 16, 32, 8), ("fp16", 128, 32, 32, 8), ("bf16", 64, 16, 8, 8), ("fp16", 64, 32, 12, 4),
     ("fp32", 128, 16, 4, 2), ("fp32", 64, 32, 6, 6), ("bf16", 128, 16, 32, 1), ("bf16", 128, 32, 16, 2),
     ("fp16", 128, 16, 7, 1), ("bf16", 64, 16, 20, 4),
+    # head slices of 9..16 rows (residual in a second MMA) and a 16 + 4 split
+    ("bf16", 128, 16, 24, 2), ("fp16", 64, 16, 40, 2),
 ]
 
 
@@ -245,14 +247,71 @@ def test_zero_length_rows_are_zero(kernel):
     tab = torch.full((3, 2), -1, dtype=torch.int32, device="cuda")
     lens = torch.zeros(3, dtype=torch.int32, device="cuda")
     q = to_device(W.queries(cfg, 0, 0), "bf16")
-    for splits in (1, 2):
+    for splits in (1, 2, 0):
         out = torch.full((3, 8, 128), 7.0, device="cuda")
-        ws = torch.zeros(1 << 16, dtype=torch.uint8, device="cuda")
+        ws = torch.zeros(max(1 << 16, K.paged_decode_workspace_bytes(3, 8, 2, 128, 2, 16, 0)), dtype=torch.uint8,
+                         device="cuda")
         err = torch.zeros(1, dtype=torch.int32, device="cuda")
         K.paged_decode_attention(out, q, k_pages, v_pages, tab, lens, cfg.scale, num_splits=splits, workspace=ws,
                                  err_flag=err)
         torch.cuda.synchronize()
         assert torch.count_nonzero(out).item() == 0 and int(err.item()) == 0
+
+
+# ---------------------------------------------------------------- planned launches
+def _planned_B(H_kv: int, extra: int) -> int:
+    """Rows past the automatic planned-launch threshold (4 x SM count) on this GPU."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    return (4 * sms) // H_kv + extra
+
+
+PLANNED_SHAPES = [
+    # dtype, Dh, P, H_q, H_kv, extra rows
+    ("bf16", 128, 16, 32, 8, 20), ("fp16", 64, 32, 16, 4, 9), ("bf16", 128, 16, 64, 1, 5), ("fp16", 128, 32, 8, 8, 3),
+]
+
+
+@pytest.mark.parametrize("dtype,Dh,P,H_q,H_kv,extra", PLANNED_SHAPES)
+@pytest.mark.parametrize("uniform", [False, True])
+@pytest.mark.parametrize("fused", [False, True])
+def test_planned_launch(dtype, Dh, P, H_q, H_kv, extra, uniform, fused):
+    """num_splits = 0 with many rows: the device plan chunks rows by their actual lengths."""
+    B = _planned_B(H_kv, extra)
+    cfg = W.DecodeConfig(f"planned-{dtype}-{Dh}-{P}-{H_q}-{H_kv}-B{B}", dtype, B=B, H_q=H_q, H_kv=H_kv, Dh=Dh,
+                         page_size=P, seed=21)
+    st = build_cache(cfg, W.ragged_lengths(B, P, cfg.seed, uniform), slack_pages=B)  # room for a second step
+    assert K.paged_decode_num_splits(B, H_kv, st.max_blocks, P, 0) == 0
+    for step in range(2):
+        out, ref, err = append_and_decode(st, step=step, num_splits=0, fused=fused, check_pools=(step == 1))
+        assert err == 0
+        check_close(out, ref, dtype, f"{cfg.name} step {step}")
+
+
+def test_planned_launch_zero_length_rows():
+    """Planned launch with empty rows (seq_len 0): those rows are zeros, the rest match the oracle."""
+    cfg = W.DecodeConfig("planned-zero", "bf16", B=_planned_B(2, 4), H_q=8, H_kv=2, Dh=128, page_size=16, seed=22)
+    st = build_cache(cfg, W.ragged_lengths(cfg.B, cfg.page_size, cfg.seed))
+    out, ref, err = append_and_decode(st, num_splits=0)
+    assert err == 0
+    check_close(out, ref, cfg.dtype, "planned before zeroing")
+    lens = st.lens.astype(np.int32).copy()
+    lens[1::3] = 0
+    q = to_device(W.queries(cfg, 0, 0), cfg.dtype)
+    ws = torch.zeros(K.paged_decode_workspace_bytes(cfg.B, cfg.H_q, cfg.H_kv, cfg.Dh, st.max_blocks, 16, 0),
+                     dtype=torch.uint8, device="cuda")
+    for lens_case in (lens, np.zeros_like(lens)):
+        got = torch.full((cfg.B, cfg.H_q, cfg.Dh), 7.0, device="cuda")
+        errt = torch.zeros(1, dtype=torch.int32, device="cuda")
+        K.paged_decode_attention(got, q, st.k_pages, st.v_pages, torch.from_numpy(st.tab).cuda(),
+                                 torch.from_numpy(lens_case).cuda(), cfg.scale, num_splits=0, workspace=ws,
+                                 err_flag=errt)
+        torch.cuda.synchronize()
+        g = got.cpu().numpy()
+        assert int(errt.item()) == 0
+        zero = lens_case == 0
+        assert np.count_nonzero(g[zero]) == 0
+        if (~zero).any():
+            check_close(g[~zero], ref[~zero], cfg.dtype, "planned with empty rows")
 
 
 def test_page_permutation_invariance_bitwise(kernel):
