@@ -17,5 +17,7 @@ Modules:
   reference   attention definitions, online-softmax merge, slot and block
               arithmetic, KV-bytes formula, fp64 paged decode (C, OpenMP)
   pool_model  refcounted FIFO page pool and brute-force prefix index
+  rope        rotary position embedding of q / k ahead of the KV append
+              ([CN-06] 6.1), exact and at stored precision
 """
-from . import reference, pool_model  # noqa: F401
+from . import reference, pool_model, rope  # noqa: F401
