@@ -44,9 +44,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", type=int, choices=[2, 3, 4, 5], default=2,
+    ap.add_argument("--config", type=int, choices=[2, 3, 4, 5, 6], default=2,
                     help="2: 8B-shaped layer (default); 3: 32K context x 32 layers; 4: shared-prefix batch; "
-                         "5: mixed continuous-batching sweep")
+                         "5: mixed continuous-batching sweep; 6: rotary embedding + append of a prefill chunk")
     ap.add_argument("--splits", type=int, default=0, help="num_splits passed to paged_decode_attention (0 = auto)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -61,6 +61,7 @@ def parse():
     ap.add_argument("--append", choices=["fused", "separate"], default="fused",
                     help="append the new token inside the decode launch (paged_decode_attention_append) "
                          "or with kv_append before paged_decode_attention")
+    ap.add_argument("--tokens", type=int, default=8192, help="config 6: tokens in the prefill chunk")
     ap.add_argument("--kernel", choices=["auto", "simt", "mma"], default="auto",
                     help="decode kernel: tensor cores (auto/mma, 16-bit K/V) or CUDA cores (simt)")
     return ap.parse_args()
@@ -859,6 +860,83 @@ def run_reference(args):
     }
 
 
+def run_rope_bench(args, world, rank, local):
+    """kv_rope_append on a prefill chunk of the 8B-shaped layer: 8192 tokens rotate q (into a separate
+    buffer) and k by their positions and append k, v into shuffled pages. HBM-bound streaming kernel."""
+    import torch
+
+    from paged_kv_cache_433_b200 import kvpaged as K
+    from paged_kv_cache_433_b200 import workloads as W
+
+    cfg = W.LLAMA8B
+    T, max_pos, P = args.tokens, 65536, cfg.page_size
+    steps = args.steps if args.steps is not None else 50
+    warm = args.warmup if args.warmup is not None else 5
+    dev = torch.device("cuda", local)
+    dt = torch.bfloat16
+    num_pages = T // P + 8
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(cfg.seed + 6000 + rank)
+    k_pages = torch.zeros((num_pages, cfg.H_kv, P, cfg.Dh), dtype=dt, device=dev)
+    v_pages = torch.zeros_like(k_pages)
+    q = torch.randn((T, cfg.H_q, cfg.Dh), generator=gen, device=dev).to(dt)
+    q_out = torch.empty_like(q)
+    kn = torch.randn((T, cfg.H_kv, cfg.Dh), generator=gen, device=dev).to(dt)
+    vn = torch.randn((T, cfg.H_kv, cfg.Dh), generator=gen, device=dev).to(dt)
+    order = torch.from_numpy(W.page_order(num_pages, cfg.seed + 6000)).to(dev).long()
+    assert T + 4096 <= max_pos
+    pos = torch.arange(T, dtype=torch.int32, device=dev) + 4096  # a chunk after a 4096-token prefix
+    slots = (order[(pos.long() - 4096) // P] * P + (pos.long() - 4096) % P).contiguous()
+    # cos / sin table of the usual rotary embedding (base 500000), fp32 [max_pos, Dh]
+    k = torch.arange(cfg.Dh // 2, dtype=torch.float64, device=dev)
+    ang = torch.arange(max_pos, dtype=torch.float64, device=dev)[:, None] * (500000.0 ** (-2.0 * k / cfg.Dh))[None, :]
+    table = torch.cat([torch.cos(ang), torch.sin(ang)], dim=1).float().contiguous()
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def call():
+        K.kv_rope_append(k_pages, v_pages, kn, vn, slots, pos, table, P, style="half", q=q, q_out=q_out, err_flag=err,
+                         stream=stream)
+
+    for _ in range(warm):
+        call()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local, enabled=not args.no_clocks)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error flag {int(err.item())}")
+    eb = 2
+    bytes_per = (2 * T * cfg.H_q * cfg.Dh * eb            # q read, q_out written
+                 + 2 * 2 * T * cfg.H_kv * cfg.Dh * eb     # k, v read and written
+                 + T * (8 + 4) + T * cfg.Dh * 4)          # slots, positions, one cos/sin row per token
+    peak, src = peaks()
+    per_ms = ms / steps
+    achieved = bytes_per / (per_ms / 1e3) / 1e9
+    return {
+        "metric": "kv_rope_append tokens/s; achieved HBM GB/s", "value": T * steps * world / (ms / 1e3),
+        "unit": "tokens/s", "n_gpus": world, "steps": steps, "warmup": warm, "ms_per_step": per_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": f"synthetic (N(0,1) q, k, v; positions 4096..{4095 + T}; shuffled pages)",
+        "config": {"workload": f"rope-append-prefill-chunk-T{T}-{cfg.name}", "tokens": T, "H_q": cfg.H_q,
+                   "H_kv": cfg.H_kv, "Dh": cfg.Dh, "page_size": P, "style": "half", "max_pos": max_pos,
+                   "l2": f"{bytes_per / 1e6:.0f} MB moved per launch > 126 MB L2; no flush"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_source": src, "traffic": None, "kernel": "kv_rope_append_kernel<bf16>",
+                     "bytes_per_launch": bytes_per, "launch_us": per_ms * 1e3},
+        "gpu_launches": steps, "e2e": None, "clocks": clocks,
+    }
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -871,7 +949,7 @@ def main():
 
     K.paged_decode_set_kernel({"auto": K.KV_DECODE_KERNEL_AUTO, "simt": K.KV_DECODE_KERNEL_SIMT,
                                "mma": K.KV_DECODE_KERNEL_MMA}[args.kernel])
-    run = {2: run_layer_bench, 3: run_long_bench, 4: run_prefix_bench, 5: run_mixed_bench}[args.config]
+    run = {2: run_layer_bench, 3: run_long_bench, 4: run_prefix_bench, 5: run_mixed_bench, 6: run_rope_bench}[args.config]
     res = run(args, world, rank, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config == 2:
         res["cpu_baseline"] = cpu_baseline()

@@ -65,6 +65,7 @@ extern "C" {
 #define KV_DEV_ERR_SLOT 4        /* kv_append slot >= num_pages * page_size; that row is skipped */
 #define KV_DEV_ERR_TIMEOUT 8     /* a bounded pipeline wait gave up; outputs of that CTA are invalid */
 #define KV_DEV_ERR_PIPELINE 16   /* a pipeline stage held another page than expected; outputs invalid */
+#define KV_DEV_ERR_POSITION 32   /* kv_rope_append position outside [0, max_pos); that token is skipped */
 
 const char* kv_status_string(int status);
 int kv_version(void);
@@ -205,6 +206,35 @@ int kv_prefix_num_entries(const kv_prefix_t* index, int32_t* out);
 int kv_append(void* k_pages, void* v_pages, const void* k_new, const void* v_new, const int64_t* slot_mapping,
               int32_t B, int32_t H_kv, int32_t Dh, int32_t page_size, int32_t num_pages, int32_t dtype,
               int* err_flag, void* stream);
+
+/* Rotary position embedding fused with the KV append -- [CN-06] 6.1 (for a
+ * new token: rotate q and k by its position, append k and v, then attend).
+ * The pages name the rotation without defining it; this is the usual rotary
+ * embedding. For token b at position pos = positions[b] and pair k of a row
+ * (k = 0 .. Dh/2 - 1), with c = cos_sin[pos][k], s = cos_sin[pos][Dh/2 + k]:
+ *   x_i' = x_i c - x_j s,   x_j' = x_j c + x_i s,
+ * where (i, j) = (k, k + Dh/2) for KV_ROPE_HALF (split halves, Llama-family
+ * layout) or (2k, 2k + 1) for KV_ROPE_INTERLEAVED. Every product and sum is
+ * rounded to fp32 on its own (no fused multiply-add), then x' is rounded to
+ * the storage dtype with round-to-nearest-even: results are bit-reproducible.
+ * Writes, per token: the rotated k_new rows to k_pages and the v_new rows
+ * (unrotated) to v_pages at slot_mapping[b] (as kv_append: -1 skips the
+ * cache write; a slot past the pool sets KV_DEV_ERR_SLOT); and, when q is not
+ * NULL, the rotated q rows to q_out (q_out may equal q; in-place is safe).
+ *   q, q_out: [B][H_q][Dh] (both NULL, or both set with H_q > 0).
+ *   k_new, v_new: [B][H_kv][Dh]; all of the pools' dtype.
+ *   positions: device int32 [B]; outside [0, max_pos) sets
+ *   KV_DEV_ERR_POSITION and nothing is written for that token.
+ *   cos_sin: device fp32 [max_pos][Dh] (cos then sin per row), owned by the
+ *   caller (typically cos / sin of pos * base^(-2k/Dh), computed once).
+ *   Dh * sizeof(dtype) must be a multiple of 32 (KV_ERR_UNSUPPORTED); all
+ *   row pointers 16-byte aligned (KV_ERR_ARG). */
+#define KV_ROPE_HALF 0
+#define KV_ROPE_INTERLEAVED 1
+int kv_rope_append(void* k_pages, void* v_pages, void* q_out, const void* q, const void* k_new, const void* v_new,
+                   const int64_t* slot_mapping, const int32_t* positions, const float* cos_sin, int32_t max_pos,
+                   int32_t rope_style, int32_t B, int32_t H_q, int32_t H_kv, int32_t Dh, int32_t page_size,
+                   int32_t num_pages, int32_t dtype, int* err_flag, void* stream);
 
 /* Copy whole pages of both pools: for i < n, page src_pages[i] -> page
  * dst_pages[i] (all H_kv heads and page_size slots; src/dst are device int32

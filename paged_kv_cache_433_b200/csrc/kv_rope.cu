@@ -1,0 +1,231 @@
+// Rotary position embedding fused with the KV append ("06 KV Cache、Prefix
+// Cache、PagedAttention 与 vLLM", 6.1: a new token's q and k are rotated by
+// its position before k and v are appended and q attends).
+//
+// One thread owns one pair of 16-byte vectors of a row: for the split-halves
+// pairing the vector at element e (< Dh/2) and the one at e + Dh/2, for the
+// interleaved pairing two adjacent vectors. Both cover the same run of pair
+// indices k, so the thread loads those cos / sin entries of the token's table
+// row as float4s. Rows are, per token: H_q query heads (rotated into q_out),
+// H_kv key heads (rotated into the K page slot) and H_kv value heads (copied
+// into the V page slot). The rotation is done in fp32 with every product and
+// sum rounded on its own (__fmul_rn / __fadd_rn / __fsub_rn, which the
+// compiler never contracts into an FMA), then rounded to the storage dtype
+// with round-to-nearest-even: the stored bits are fully determined.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+
+#include "decode_launch.cuh"
+#include "kvpaged.h"
+
+namespace kvp {
+namespace {
+
+template <int DT>
+struct RopeVec;
+
+template <>
+struct RopeVec<KV_DTYPE_BF16> {
+    static constexpr int kN = 8;
+    __device__ static void load(const uint4& v, float* x) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            x[2 * i] = __uint_as_float(w[i] << 16);
+            x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+    __device__ static uint4 store(const float* x) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const __nv_bfloat16 lo = __float2bfloat16_rn(x[2 * i]);
+            const __nv_bfloat16 hi = __float2bfloat16_rn(x[2 * i + 1]);
+            w[i] = static_cast<uint32_t>(__bfloat16_as_ushort(lo)) | (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
+        }
+        return make_uint4(w[0], w[1], w[2], w[3]);
+    }
+};
+
+template <>
+struct RopeVec<KV_DTYPE_F16> {
+    static constexpr int kN = 8;
+    __device__ static void load(const uint4& v, float* x) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            x[2 * i] = __half2float(__ushort_as_half(static_cast<unsigned short>(w[i] & 0xffffu)));
+            x[2 * i + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(w[i] >> 16)));
+        }
+    }
+    __device__ static uint4 store(const float* x) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const __half lo = __float2half_rn(x[2 * i]);
+            const __half hi = __float2half_rn(x[2 * i + 1]);
+            w[i] = static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
+        }
+        return make_uint4(w[0], w[1], w[2], w[3]);
+    }
+};
+
+template <>
+struct RopeVec<KV_DTYPE_F32> {
+    static constexpr int kN = 4;
+    __device__ static void load(const uint4& v, float* x) {
+        x[0] = __uint_as_float(v.x);
+        x[1] = __uint_as_float(v.y);
+        x[2] = __uint_as_float(v.z);
+        x[3] = __uint_as_float(v.w);
+    }
+    __device__ static uint4 store(const float* x) {
+        return make_uint4(__float_as_uint(x[0]), __float_as_uint(x[1]), __float_as_uint(x[2]), __float_as_uint(x[3]));
+    }
+};
+
+// x_i' = x_i c - x_j s, x_j' = x_j c + x_i s, each operation rounded to fp32.
+__device__ __forceinline__ void rotate_pair(float& xi, float& xj, float c, float s) {
+    const float a = __fsub_rn(__fmul_rn(xi, c), __fmul_rn(xj, s));
+    const float b = __fadd_rn(__fmul_rn(xj, c), __fmul_rn(xi, s));
+    xi = a;
+    xj = b;
+}
+
+template <int DT>
+__global__ void __launch_bounds__(256) kv_rope_append_kernel(
+    uint4* __restrict__ k_pages, uint4* __restrict__ v_pages, uint4* q_out, const uint4* q,
+    const uint4* __restrict__ k_new, const uint4* __restrict__ v_new, const int64_t* __restrict__ slots,
+    const int32_t* __restrict__ positions, const float* __restrict__ cos_sin, int32_t max_pos, int32_t style, int64_t B,
+    int32_t H_q, int32_t H_kv, int32_t Dh, int32_t P, int64_t num_slots, int* err) {
+    using V = RopeVec<DT>;
+    constexpr int N = V::kN;  // elements per 16-byte vector
+    grid_dependency_wait();
+    if (threadIdx.x == 0) grid_launch_dependents();
+    const int32_t vpr = Dh / N;          // vectors per row
+    const int32_t upr = vpr / 2;         // units (vector pairs) per row
+    const int32_t q_rows = q_out != nullptr ? H_q : 0;
+    const int32_t units = (q_rows + 2 * H_kv) * upr;  // per token
+    const int64_t total = B * units;
+    for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total; t += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t b = total < (1LL << 31) ? static_cast<int64_t>(static_cast<uint32_t>(t) / static_cast<uint32_t>(units))
+                                              : t / units;
+        const int32_t rem = static_cast<int32_t>(t - b * units);
+        const int32_t r = rem / upr, u = rem - r * upr;
+        const int32_t pos = positions[b];
+        if (pos < 0 || pos >= max_pos) {
+            if (rem == 0 && err) atomicOr(err, KV_DEV_ERR_POSITION);
+            continue;
+        }
+        const int64_t slot = r < q_rows ? 0 : slots[b];
+        // source row and destination row (16-byte units)
+        const uint4* src;
+        uint4* dst;
+        bool rotate = true;
+        if (r < q_rows) {
+            src = q + (b * H_q + r) * vpr;
+            dst = q_out + (b * H_q + r) * vpr;
+        } else {
+            if (slot < 0) continue;
+            const bool is_v = r >= q_rows + H_kv;
+            const int32_t h = r - q_rows - (is_v ? H_kv : 0);
+            if (slot >= num_slots) {
+                if (h == 0 && u == 0 && !is_v && err) atomicOr(err, KV_DEV_ERR_SLOT);
+                continue;
+            }
+            const int64_t page = slot / P, off = slot - page * P;
+            src = (is_v ? v_new : k_new) + (b * H_kv + h) * vpr;
+            dst = (is_v ? v_pages : k_pages) + ((page * H_kv + h) * P + off) * vpr;
+            rotate = !is_v;
+        }
+        // the two vectors of this unit and the first pair index they hold
+        const int32_t va = style == KV_ROPE_HALF ? u : 2 * u;
+        const int32_t vb = style == KV_ROPE_HALF ? u + upr : 2 * u + 1;
+        const uint4 a = src[va], bv = src[vb];
+        if (!rotate) {
+            dst[va] = a;
+            dst[vb] = bv;
+            continue;
+        }
+        float xa[N], xb[N];
+        V::load(a, xa);
+        V::load(bv, xb);
+        const float* crow = cos_sin + (int64_t)pos * Dh;
+        const int32_t k0 = u * N;  // pairs k0 .. k0 + N - 1
+        float c[N], s[N];
+#pragma unroll
+        for (int i = 0; i < N; i += 4) {
+            const float4 cc = *reinterpret_cast<const float4*>(crow + k0 + i);
+            const float4 ss = *reinterpret_cast<const float4*>(crow + Dh / 2 + k0 + i);
+            c[i] = cc.x, c[i + 1] = cc.y, c[i + 2] = cc.z, c[i + 3] = cc.w;
+            s[i] = ss.x, s[i + 1] = ss.y, s[i + 2] = ss.z, s[i + 3] = ss.w;
+        }
+        if (style == KV_ROPE_HALF) {
+            // pair k0 + i = (element i of a, element i of b)
+#pragma unroll
+            for (int i = 0; i < N; ++i) rotate_pair(xa[i], xb[i], c[i], s[i]);
+        } else {
+            // a holds pairs k0 .. k0 + N/2 - 1, b the next N/2, as (2i, 2i + 1)
+#pragma unroll
+            for (int i = 0; i < N / 2; ++i) {
+                rotate_pair(xa[2 * i], xa[2 * i + 1], c[i], s[i]);
+                rotate_pair(xb[2 * i], xb[2 * i + 1], c[N / 2 + i], s[N / 2 + i]);
+            }
+        }
+        dst[va] = V::store(xa);
+        dst[vb] = V::store(xb);
+    }
+}
+
+int elem_size(int32_t dtype) {
+    return dtype == KV_DTYPE_F32 ? 4 : (dtype == KV_DTYPE_BF16 || dtype == KV_DTYPE_F16) ? 2 : 0;
+}
+
+bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+}  // namespace kvp
+
+using namespace kvp;
+
+extern "C" int kv_rope_append(void* k_pages, void* v_pages, void* q_out, const void* q, const void* k_new,
+                              const void* v_new, const int64_t* slot_mapping, const int32_t* positions,
+                              const float* cos_sin, int32_t max_pos, int32_t rope_style, int32_t B, int32_t H_q,
+                              int32_t H_kv, int32_t Dh, int32_t page_size, int32_t num_pages, int32_t dtype,
+                              int* err_flag, void* stream) {
+    const int eb = elem_size(dtype);
+    if (B < 0 || H_kv <= 0 || Dh <= 0 || page_size <= 0 || num_pages <= 0 || eb == 0 || max_pos <= 0) return KV_ERR_ARG;
+    if (rope_style != KV_ROPE_HALF && rope_style != KV_ROPE_INTERLEAVED) return KV_ERR_ARG;
+    if ((q == nullptr) != (q_out == nullptr) || (q != nullptr && H_q <= 0)) return KV_ERR_ARG;
+    if ((static_cast<int64_t>(Dh) * eb) % 32 != 0) return KV_ERR_UNSUPPORTED;  // whole vector pairs per row
+    if (B == 0) return KV_OK;
+    if (!k_pages || !v_pages || !k_new || !v_new || !slot_mapping || !positions || !cos_sin) return KV_ERR_ARG;
+    if (!al16(k_pages) || !al16(v_pages) || !al16(k_new) || !al16(v_new) || !al16(cos_sin)) return KV_ERR_ARG;
+    if (q != nullptr && (!al16(q) || !al16(q_out))) return KV_ERR_ARG;
+    const int32_t vpr = Dh * eb / 16;
+    const int64_t rows = (q != nullptr ? H_q : 0) + 2LL * H_kv;
+    const int64_t units = static_cast<int64_t>(B) * rows * (vpr / 2);
+    const int threads = 256;
+    const int64_t blocks = std::min<int64_t>((units + threads - 1) / threads, 148LL * 64);  // grid-stride beyond
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t num_slots = static_cast<int64_t>(num_pages) * page_size;
+    cudaError_t e;
+    auto args = [&](auto kernel) {
+        return launch_pdl(kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, st, static_cast<uint4*>(k_pages),
+                          static_cast<uint4*>(v_pages), static_cast<uint4*>(q_out), static_cast<const uint4*>(q),
+                          static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), slot_mapping, positions,
+                          cos_sin, max_pos, rope_style, static_cast<int64_t>(B), H_q, H_kv, Dh, page_size, num_slots,
+                          err_flag);
+    };
+    if (dtype == KV_DTYPE_BF16)
+        e = args(kv_rope_append_kernel<KV_DTYPE_BF16>);
+    else if (dtype == KV_DTYPE_F16)
+        e = args(kv_rope_append_kernel<KV_DTYPE_F16>);
+    else
+        e = args(kv_rope_append_kernel<KV_DTYPE_F32>);
+    return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;
+}

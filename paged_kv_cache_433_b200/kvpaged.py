@@ -36,6 +36,7 @@ KV_DEV_ERR_SEQ_LEN = 2
 KV_DEV_ERR_SLOT = 4
 KV_DEV_ERR_TIMEOUT = 8
 KV_DEV_ERR_PIPELINE = 16
+KV_DEV_ERR_POSITION = 32
 
 # (name, restype, argtypes) of every exported function.
 _i32, _i64, _u64, _vp, _f32, _sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_void_p, ctypes.c_float, ctypes.c_size_t
@@ -67,6 +68,8 @@ SIGNATURES = [
     ("kv_prefix_match", ctypes.c_int, [_vp, _vp, _i32, _i32, _vp, _pi32]),
     ("kv_prefix_num_entries", ctypes.c_int, [_vp, _pi32]),
     ("kv_append", ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
+    ("kv_rope_append", ctypes.c_int,
+     [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
     ("paged_decode_attention", ctypes.c_int,
      [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _i32, _vp, _sz, _vp, _vp]),
     ("paged_decode_attention_append", ctypes.c_int,
@@ -300,6 +303,37 @@ def kv_append(k_pages, v_pages, k_new, v_new, slot_mapping, page_size: int, err_
                          _dev(v_new, "v_new", k_pages.dtype), _dev(slot_mapping, "slot_mapping", torch.int64), B, H_kv, Dh,
                          page_size, num_pages, dt, _dev(err_flag, "err_flag", torch.int32), _stream(stream))
     _check("kv_append", rc)
+
+
+KV_ROPE_HALF, KV_ROPE_INTERLEAVED = 0, 1
+ROPE_STYLE = {"half": KV_ROPE_HALF, "interleaved": KV_ROPE_INTERLEAVED}
+
+
+def kv_rope_append(k_pages, v_pages, k_new, v_new, slot_mapping, positions, cos_sin, page_size: int,
+                   style: str = "half", q=None, q_out=None, err_flag=None, stream=None) -> None:
+    """Rotate k_new (and q, into q_out; q_out may be q) by `positions`, then append.
+
+    k/v_pages [num_pages, H_kv, P, Dh]; k/v_new [B, H_kv, Dh]; q/q_out [B, H_q, Dh];
+    slot_mapping int64 [B]; positions int32 [B]; cos_sin fp32 [max_pos, Dh] (all device)."""
+    import torch
+
+    num_pages, H_kv, P, Dh = k_pages.shape
+    assert P == page_size and v_pages.shape == k_pages.shape
+    B = k_new.shape[0]
+    assert tuple(k_new.shape) == (B, H_kv, Dh) and v_new.shape == k_new.shape
+    assert cos_sin.dim() == 2 and cos_sin.shape[1] == Dh
+    H_q = 0
+    if q is not None:
+        assert q_out is not None and q.shape == q_out.shape and q.shape[0] == B and q.shape[2] == Dh
+        H_q = q.shape[1]
+    dt = _torch_dtype_code(k_pages)
+    rc = lib().kv_rope_append(_dev(k_pages, "k_pages"), _dev(v_pages, "v_pages", k_pages.dtype),
+                              _dev(q_out, "q_out", k_pages.dtype), _dev(q, "q", k_pages.dtype),
+                              _dev(k_new, "k_new", k_pages.dtype), _dev(v_new, "v_new", k_pages.dtype),
+                              _dev(slot_mapping, "slot_mapping", torch.int64), _dev(positions, "positions", torch.int32),
+                              _dev(cos_sin, "cos_sin", torch.float32), cos_sin.shape[0], ROPE_STYLE[style], B, H_q, H_kv,
+                              Dh, page_size, num_pages, dt, _dev(err_flag, "err_flag", torch.int32), _stream(stream))
+    _check("kv_rope_append", rc)
 
 
 KV_DECODE_KERNEL_AUTO, KV_DECODE_KERNEL_SIMT, KV_DECODE_KERNEL_MMA = 0, 1, 2
