@@ -19,5 +19,7 @@ Modules:
   pool_model  refcounted FIFO page pool and brute-force prefix index
   rope        rotary position embedding of q / k ahead of the KV append
               ([CN-06] 6.1), exact and at stored precision
+  fp8         E4M3 K/V cache: format, quantising append, fp64 decode over
+              the read values
 """
-from . import reference, pool_model, rope  # noqa: F401
+from . import reference, pool_model, rope, fp8  # noqa: F401
