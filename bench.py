@@ -44,9 +44,10 @@ def parse():
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", type=int, choices=[2, 3, 4, 5, 6], default=2,
+    ap.add_argument("--config", type=int, choices=[2, 3, 4, 5, 6, 7], default=2,
                     help="2: 8B-shaped layer (default); 3: 32K context x 32 layers; 4: shared-prefix batch; "
-                         "5: mixed continuous-batching sweep; 6: rotary embedding + append of a prefill chunk")
+                         "5: mixed continuous-batching sweep; 6: rotary embedding + append of a prefill chunk; "
+                         "7: the 8B-shaped layer with an E4M3 K/V cache")
     ap.add_argument("--splits", type=int, default=0, help="num_splits passed to paged_decode_attention (0 = auto)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -158,7 +159,7 @@ class ClockSampler:
 class Workload:
     """Device-resident inputs of every step, built through the library's own calls."""
 
-    def __init__(self, cfg, lens, n_steps, rank, splits, layers=1, sequential=False):
+    def __init__(self, cfg, lens, n_steps, rank, splits, layers=1, sequential=False, fp8=False):
         import torch
 
         from paged_kv_cache_433_b200 import kvpaged as K
@@ -187,18 +188,25 @@ class Workload:
         gen = torch.Generator(device=dev)
         gen.manual_seed(cfg.seed * 7919 + rank)
         shape = (self.num_pages, cfg.H_kv, P, cfg.Dh)
+        self.fp8 = fp8
+        # E4M3 pools: per-head scales that map N(0,1) values up to 4.5 onto the E4M3 range
+        self.k_scale = torch.full((cfg.H_kv,), 4.5 / 448, dtype=torch.float32, device=dev)
+        self.v_scale = self.k_scale.clone()
         self.k_pages, self.v_pages = [], []
         slots = np.concatenate([K.kv_slots_for_range(self.tab[b], P, 0, int(lens[b])) for b in range(B)])
         slots_dev = torch.from_numpy(slots).to(dev)
         for _ in range(layers):
-            kp = torch.zeros(shape, dtype=dt, device=dev)
-            vp = torch.zeros(shape, dtype=dt, device=dev)
+            kp = torch.zeros(shape, dtype=torch.uint8 if fp8 else dt, device=dev)
+            vp = torch.zeros_like(kp)
             chunk = 1 << 20
             for s0 in range(0, slots.size, chunk):
                 n = min(chunk, slots.size - s0)
                 kr = torch.randn((n, cfg.H_kv, cfg.Dh), generator=gen, device=dev).to(dt)
                 vr = torch.randn((n, cfg.H_kv, cfg.Dh), generator=gen, device=dev).to(dt)
-                K.kv_append(kp, vp, kr, vr, slots_dev[s0:s0 + n], P)
+                if fp8:
+                    K.kv_append_fp8(kp, vp, kr, vr, self.k_scale, self.v_scale, slots_dev[s0:s0 + n], P)
+                else:
+                    K.kv_append(kp, vp, kr, vr, slots_dev[s0:s0 + n], P)
             self.k_pages.append(kp)
             self.v_pages.append(vp)
         self.splits = splits
@@ -220,7 +228,7 @@ class Workload:
         """Algorithmic bytes of one decode launch (one layer): K/V rows actually attended,
         q, fp32 out, block-table entries and seq_lens."""
         cfg = self.cfg
-        kv = int(np.sum(lens_after)) * cfg.H_kv * cfg.Dh * 2 * cfg.elem_bytes
+        kv = int(np.sum(lens_after)) * cfg.H_kv * cfg.Dh * 2 * (1 if self.fp8 else cfg.elem_bytes)
         q = self.B * cfg.H_q * cfg.Dh * cfg.elem_bytes
         out = self.B * cfg.H_q * cfg.Dh * 4
         tables = int(np.sum(-(-lens_after // cfg.page_size))) * 4 + self.B * 4
@@ -393,6 +401,90 @@ def run_layer_bench(args, world, rank, local):
         "clocks": clocks,
     }
     return res
+
+
+def run_fp8_bench(args, world, rank, local):
+    """The 8B-shaped layer with an E4M3 K/V cache (per-head scales) and bf16 q: each step appends the new
+    token (kv_append_fp8, quantising) and decodes (paged_decode_attention_fp8). The roofline is the decode call."""
+    import torch
+
+    from paged_kv_cache_433_b200 import kvpaged as K
+    from paged_kv_cache_433_b200 import workloads as W
+
+    cfg = W.LLAMA8B
+    steps = args.steps if args.steps is not None else cfg.timed_steps
+    warm = args.warmup if args.warmup is not None else cfg.warmup_steps
+    lens = W.cached_lengths(cfg)
+    wl = Workload(cfg, lens, warm + steps, rank, args.splits, fp8=True)
+    B, P = wl.B, cfg.page_size
+    dev = torch.device("cuda")
+    T1 = warm + steps
+    slot_list, lens_list = [], []
+    for _ in range(T1):
+        sl, ln = wl.bookkeeping()
+        slot_list.append(sl)
+        lens_list.append(ln)
+    slots_dev = torch.from_numpy(np.stack(slot_list)).to(dev)
+    lens_dev = torch.from_numpy(np.stack(lens_list)).to(dev)
+    tab_dev = torch.from_numpy(wl.tab).to(dev)
+    q_dev = torch.randn((T1, B, cfg.H_q, cfg.Dh), generator=wl.gen, device=dev).to(wl.dt)
+    kn_dev = torch.randn((T1, B, cfg.H_kv, cfg.Dh), generator=wl.gen, device=dev).to(wl.dt)
+    vn_dev = torch.randn((T1, B, cfg.H_kv, cfg.Dh), generator=wl.gen, device=dev).to(wl.dt)
+    out = torch.empty((B, cfg.H_q, cfg.Dh), dtype=torch.float32, device=dev)
+    ws = wl.workspace()
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    S = K.paged_decode_num_splits(B, cfg.H_kv, wl.max_blocks, P, args.splits)
+    stream = torch.cuda.current_stream()
+    kp, vp = wl.k_pages[0], wl.v_pages[0]
+
+    def step(i, ev=None):
+        K.kv_append_fp8(kp, vp, kn_dev[i], vn_dev[i], wl.k_scale, wl.v_scale, slots_dev[i], P, err_flag=err,
+                        stream=stream)
+        if ev is not None:
+            ev[0].record(stream)
+        K.paged_decode_attention_fp8(out, q_dev[i], kp, vp, wl.k_scale, wl.v_scale, tab_dev, lens_dev[i], cfg.scale,
+                                     num_splits=args.splits, workspace=ws, err_flag=err, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for i in range(warm):
+        step(i)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk = ClockSampler(local, enabled=not args.no_clocks)
+    barrier(world)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for n, i in enumerate(range(warm, T1)):
+        step(i, ev[n])
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = clk.stop()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error flag {int(err.item())}")
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), world)
+    dec_ms = [a.elapsed_time(b) for a, b in ev]
+    mean_bytes = float(np.mean([wl.step_bytes(lens_list[i]) for i in range(warm, T1)]))
+    peak, peak_kind = peaks()
+    mean_dec_s = float(np.mean(dec_ms)) / 1e3
+    achieved = mean_bytes / mean_dec_s / 1e9
+    return {
+        "metric": METRIC, "value": replica_value(B, steps, world, elapsed_ms), "unit": UNIT, "n_gpus": world,
+        "steps": steps, "warmup": warm, "ms_per_step": elapsed_ms / steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3 K/V, bf16 q, f16 MMA",
+        "data": "synthetic (N(0,1) K/V quantised with scale 4.5/448 per head; bf16 q; lengths U[512,4096])",
+        "config": {"workload": cfg.name.replace("-bf16-", "-fp8kv-"), "B": B, "H_q": cfg.H_q, "H_kv": cfg.H_kv,
+                   "Dh": cfg.Dh, "page_size": P, "kv_dtype": "e4m3", "num_splits": S,
+                   "l2": "inputs larger than L2 (K/V working set %.0f MB > 126 MB L2); no flush" % (mean_bytes / 1e6)},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_source": peak_kind, "traffic": None,
+                     "kernel": "paged_decode_attention_fp8" + (" (split + combine)" if S > 1 else ""),
+                     "bytes_per_launch": mean_bytes, "launch_us": mean_dec_s * 1e6},
+        "gpu_launches": steps * (1 + (3 if S == 0 else (2 if S > 1 else 1))),
+        "e2e": None, "clocks": clocks,
+    }
 
 
 def run_e2e(wl, cfg, warm, steps, args, world):
@@ -615,7 +707,7 @@ class PagedState:
 
     def step_bytes(self, lens_after, fused=True):
         cfg = self.cfg
-        kv = int(np.sum(lens_after)) * cfg.H_kv * cfg.Dh * 2 * cfg.elem_bytes
+        kv = int(np.sum(lens_after)) * cfg.H_kv * cfg.Dh * 2 * (1 if self.fp8 else cfg.elem_bytes)
         q = self.B * cfg.H_q * cfg.Dh * cfg.elem_bytes
         out = self.B * cfg.H_q * cfg.Dh * 4
         tables = int(np.sum(-(-np.asarray(lens_after) // self.P))) * 4 + self.B * 4
@@ -949,7 +1041,8 @@ def main():
 
     K.paged_decode_set_kernel({"auto": K.KV_DECODE_KERNEL_AUTO, "simt": K.KV_DECODE_KERNEL_SIMT,
                                "mma": K.KV_DECODE_KERNEL_MMA}[args.kernel])
-    run = {2: run_layer_bench, 3: run_long_bench, 4: run_prefix_bench, 5: run_mixed_bench, 6: run_rope_bench}[args.config]
+    run = {2: run_layer_bench, 3: run_long_bench, 4: run_prefix_bench, 5: run_mixed_bench, 6: run_rope_bench,
+           7: run_fp8_bench}[args.config]
     res = run(args, world, rank, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config == 2:
         res["cpu_baseline"] = cpu_baseline()

@@ -58,6 +58,7 @@ extern "C" {
 #define KV_DTYPE_F32 0
 #define KV_DTYPE_BF16 1
 #define KV_DTYPE_F16 2
+#define KV_DTYPE_FP8_E4M3 3  /* K/V pools only: 8-bit E4M3 codes with per-KV-head scales */
 
 /* ---- device error bits (OR-ed into *err_flag) --------------------------- */
 #define KV_DEV_ERR_PAGE_RANGE 1  /* a block-table entry outside [0, num_pages); that page is skipped */
@@ -289,6 +290,39 @@ int paged_decode_attention_append(float* out, const void* q, const void* k_new, 
                                   const int32_t* seq_lens, int32_t B, int32_t H_q, int32_t H_kv, int32_t Dh,
                                   int32_t page_size, int32_t num_pages, float scale, int32_t dtype, int32_t num_splits,
                                   void* workspace, size_t ws_bytes, int* err_flag, void* stream);
+
+/* ---- FP8 (E4M3) K/V cache ---------------------------------------------
+ * "03. KV Cache：用显存换计算" (KV quantisation follow-up) and [CN-06]'s
+ * KV-size table name storing K / V in 8 bits without fixing a format. Here:
+ * pools of E4M3 codes (1 byte per element; same [num_pages][H_kv][P][Dh]
+ * layout) and one fp32 scale per KV head and pool, read value = E4M3 value *
+ * scale. The scales are the caller's (device fp32 [H_kv], e.g. calibrated as
+ * max|x| / 448); they must not change while codes written with them live.
+ * kv_copy_pages and kv_append (raw codes) accept KV_DTYPE_FP8_E4M3. */
+
+/* Quantising append: for each b with slot_mapping[b] >= 0 and head h,
+ *   k_pages[slot][h][:] = E4M3(k_new[b][h][:] / k_scale[h]), same for V,
+ * where x / scale is an IEEE fp32 division and E4M3() rounds to nearest even,
+ * saturating at +-448 (NaN stays NaN). k_new, v_new: [B][H_kv][Dh] of
+ * src_dtype (bf16, fp16 or fp32). Dh % 16 == 0 (else KV_ERR_UNSUPPORTED).
+ * Slots as kv_append (-1 skips; past the pool: KV_DEV_ERR_SLOT). */
+int kv_append_fp8(void* k_pages, void* v_pages, const void* k_new, const void* v_new, int32_t src_dtype,
+                  const float* k_scale, const float* v_scale, const int64_t* slot_mapping, int32_t B, int32_t H_kv,
+                  int32_t Dh, int32_t page_size, int32_t num_pages, int* err_flag, void* stream);
+
+/* Decode attention over E4M3 pools: as paged_decode_attention with
+ *   K_t = code_t * k_scale[kv head], V_t = code_t * v_scale[kv head],
+ * q of q_dtype (KV_DTYPE_BF16 or KV_DTYPE_F16; its values must lie within
+ * fp16's range, +-65504, as the products run on the tensor cores in fp16 --
+ * E4M3 values are exact in fp16). Tensor-core kernel only (H_q / H_kv <= 64,
+ * Dh in {64, 128}, page_size in {16, 32}); num_splits, workspace (same size
+ * as paged_decode_workspace_bytes), errors and output as
+ * paged_decode_attention. */
+int paged_decode_attention_fp8(float* out, const void* q, int32_t q_dtype, const void* k_pages, const void* v_pages,
+                               const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                               int32_t max_blocks, const int32_t* seq_lens, int32_t B, int32_t H_q, int32_t H_kv,
+                               int32_t Dh, int32_t page_size, int32_t num_pages, float scale, int32_t num_splits,
+                               void* workspace, size_t ws_bytes, int* err_flag, void* stream);
 
 /* Which decode kernel paged_decode_attention uses (process-wide; default AUTO):
  *   KV_DECODE_KERNEL_AUTO  tensor cores (warp MMA on TMA-staged swizzled tiles)

@@ -62,6 +62,8 @@ struct DecodeParams {
     float* part_u;              // split: [B][H_q][S][Dh]; planned: [item][g][Dh]
     float2* part_ml;            // split: [B][H_q][S]; planned: [item][g] (m in log2 units, l)
     const int4* items;          // planned launch: {b, kvh, chunk, item} per CTA (nullable)
+    const float* k_scale;       // E4M3 K/V: per-KV-head scales (read value = code * scale)
+    const float* v_scale;
     const int32_t* plan;        // planned launch: [0] pages per chunk, [4 + b] item prefix
     int* err;
     int32_t max_blocks, B, H_q, H_kv, num_pages;

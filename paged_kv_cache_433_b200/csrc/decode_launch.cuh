@@ -81,50 +81,53 @@ cudaError_t launch_decode_f16(const DecodeParams& p, int DH, int P, int GW, int 
 
 namespace kvp {
 
-template <int DT, int DH, int P, bool LO>
+template <int KT, int QT, int DH, int P, bool LO>
 cudaError_t launch_mma_inst(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, dim3 grid,
                             cudaStream_t st) {
     constexpr int NW = 4;
-    using C = MmaCfg<DH, P, NW>;
+    using C = MmaCfg<DH, P, NW, KT == KV_DTYPE_FP8_E4M3 ? 1 : 2>;
     static std::atomic<uint64_t> configured{0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     const uint64_t bit = 1ull << (dev & 63);
+    auto* kern = paged_decode_mma_kernel<KT, QT, DH, P, NW, LO>;
     if (!(configured.load(std::memory_order_acquire) & bit)) {
-        e = cudaFuncSetAttribute(paged_decode_mma_kernel<DT, DH, P, NW, LO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::kSmem);
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(paged_decode_mma_kernel<DT, DH, P, NW, LO>,
-                                 cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
         if (e != cudaSuccess) return e;
         configured.fetch_or(bit, std::memory_order_acq_rel);
     }
-    return launch_pdl(paged_decode_mma_kernel<DT, DH, P, NW, LO>, grid, dim3(C::kThreads), C::kSmem, st, p, tk, tv);
+    return launch_pdl(kern, grid, dim3(C::kThreads), C::kSmem, st, p, tk, tv);
 }
 
 // Groups of at most 8 heads take the instance that carries the probability
 // residual in the MMA's padding rows.
-template <int DT, int DH, int P>
+template <int KT, int QT, int DH, int P>
 cudaError_t launch_mma_group(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, dim3 grid,
                              cudaStream_t st) {
-    return p.g <= 8 ? launch_mma_inst<DT, DH, P, true>(p, tk, tv, grid, st)
-                    : launch_mma_inst<DT, DH, P, false>(p, tk, tv, grid, st);
+    return p.g <= 8 ? launch_mma_inst<KT, QT, DH, P, true>(p, tk, tv, grid, st)
+                    : launch_mma_inst<KT, QT, DH, P, false>(p, tk, tv, grid, st);
 }
 
-template <int DT>
+template <int KT, int QT>
 cudaError_t launch_mma_dt(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int DH, int P, dim3 grid,
                           cudaStream_t st) {
     if (DH == 128)
-        return P == 16 ? launch_mma_group<DT, 128, 16>(p, tk, tv, grid, st)
-                       : launch_mma_group<DT, 128, 32>(p, tk, tv, grid, st);
-    return P == 16 ? launch_mma_group<DT, 64, 16>(p, tk, tv, grid, st) : launch_mma_group<DT, 64, 32>(p, tk, tv, grid, st);
+        return P == 16 ? launch_mma_group<KT, QT, 128, 16>(p, tk, tv, grid, st)
+                       : launch_mma_group<KT, QT, 128, 32>(p, tk, tv, grid, st);
+    return P == 16 ? launch_mma_group<KT, QT, 64, 16>(p, tk, tv, grid, st)
+                   : launch_mma_group<KT, QT, 64, 32>(p, tk, tv, grid, st);
 }
 
-// Defined in decode_mma_bf16.cu / decode_mma_f16.cu.
+// Defined in decode_mma_bf16.cu / decode_mma_f16.cu / decode_mma_fp8.cu.
 cudaError_t launch_mma_bf16(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int DH, int P, dim3 grid,
                             cudaStream_t st);
 cudaError_t launch_mma_f16(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int DH, int P, dim3 grid,
                            cudaStream_t st);
+// E4M3 K/V with q of type q_dtype (bf16 or fp16).
+cudaError_t launch_mma_fp8(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int q_dtype, int DH,
+                           int P, dim3 grid, cudaStream_t st);
 
 }  // namespace kvp

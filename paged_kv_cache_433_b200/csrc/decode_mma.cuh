@@ -27,6 +27,7 @@
 #include <cuda.h>
 
 #include "decode_kernel.cuh"
+#include "fp8.cuh"
 
 #ifndef KVP_PRODUCER_SINGLE_LANE
 #define KVP_PRODUCER_SINGLE_LANE 0
@@ -37,16 +38,22 @@
 
 namespace kvp {
 
-template <int DH, int P, int NW>
+// EB: bytes per K/V element (2: bf16 / fp16; 1: E4M3). A token row of Dh
+// elements is loaded as boxes of at most 128 bytes (rows of 128 bytes use the
+// 128-byte swizzle, rows of 64 bytes -- E4M3 at Dh = 64 -- the 64-byte one).
+template <int DH, int P, int NW, int EB>
 struct MmaCfg {
-    static constexpr int kBoxes = DH / 64;         // 128-byte boxes per token row
-    static constexpr int kBoxB = P * 128;          // bytes per box (P rows)
-    static constexpr int kChunk = kBoxes * kBoxB;  // one (page, head) chunk = P x Dh x 2 bytes
-    static constexpr int kStage = 2 * kChunk;      // K + V
-    static constexpr int kKSteps = DH / 16;        // QK k-steps
-    static constexpr int kNT = P / 8;              // token n-tiles of S
-    static constexpr int kPK = P / 16;             // PV k-steps
-    static constexpr int kOT = DH / 8;             // dim n-tiles of O
+    static constexpr int kRowB = DH * EB;                        // bytes per token row
+    static constexpr int kBoxInner = kRowB < 128 ? kRowB : 128;  // bytes per box row
+    static constexpr int kBoxElems = kBoxInner / EB;
+    static constexpr int kBoxes = kRowB / kBoxInner;             // boxes per token row
+    static constexpr int kBoxB = P * kBoxInner;                  // bytes per box (P rows)
+    static constexpr int kChunk = P * kRowB;                     // one (page, head) chunk
+    static constexpr int kStage = 2 * kChunk;                    // K + V
+    static constexpr int kKSteps = DH / 16;                      // QK k-steps
+    static constexpr int kNT = P / 8;                            // token n-tiles of S
+    static constexpr int kPK = P / 16;                           // PV k-steps
+    static constexpr int kOT = DH / 8;                           // dim n-tiles of O
     static constexpr int kStageBudget = KVP_MMA_STAGE_BUDGET;
     // Stage i % NS is drained by page-warp i % WP (WP divides NW): NS must be
     // a multiple of NW so each stage always goes to the same warp.
@@ -59,17 +66,32 @@ struct MmaCfg {
     static constexpr int kSmem = 1024 + kOffTag + 4 * kNS;  // + slack to align the ring to 1024 bytes
     static constexpr int kThreads = 32 * (NW + 1);
     static_assert(DH % 64 == 0 && P % 16 == 0, "shape");
+    static_assert(kRowB % kBoxInner == 0 && (kBoxInner == 128 || kBoxInner == 64), "box rows");
     static_assert(kNS % NW == 0, "stage ring must be a multiple of the page-warps");
 };
 
-// LO: the GQA group has at most 8 heads (one head slice, rows 8..15 are
-// padding), so each row's probability residual rides in row r + 8.
-template <int DT, int DH, int P, int NW, bool LO>
+// Byte offset of 16-byte chunk c of row t in a box whose rows are kBoxInner
+// bytes, as the TMA swizzle placed it (128-byte: chunk ^ row % 8; 64-byte:
+// chunk ^ (row / 2) % 4).
+template <int kBoxInner>
+__device__ __forceinline__ uint32_t swz(int t, int c) {
+    if constexpr (kBoxInner == 128)
+        return t * 128 + (((c & 7) ^ (t & 7)) << 4);
+    else
+        return t * 64 + (((c & 3) ^ ((t >> 1) & 3)) << 4);
+}
+
+// KT: K/V storage type (bf16, fp16 or E4M3); QT: q's type (equal to KT for
+// 16-bit K/V; bf16 or fp16 for E4M3, whose products run in f16). LO: the GQA
+// group has at most 8 heads (one head slice, rows 8..15 are padding), so each
+// row's probability residual rides in row r + 8.
+template <int KT, int QT, int DH, int P, int NW, bool LO>
 __global__ void __launch_bounds__(32 * (NW + 1), 2)
     paged_decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                             const __grid_constant__ CUtensorMap tmap_v) {
-    using C = MmaCfg<DH, P, NW>;
-    constexpr bool kBF16 = DT == KV_DTYPE_BF16;
+    constexpr bool kFP8 = KT == KV_DTYPE_FP8_E4M3;
+    using C = MmaCfg<DH, P, NW, kFP8 ? 1 : 2>;
+    constexpr bool kBF16 = KT == KV_DTYPE_BF16;  // MMA operand type: bf16, else f16
     extern __shared__ __align__(1024) unsigned char smem_raw[];
 
     const int warp = threadIdx.x >> 5;
@@ -138,7 +160,9 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (p.k_new != nullptr && first + n_local == n_pages) append_new_token(p, b, kvh, len, P, DH * 2, lane);
+        if constexpr (!kFP8) {
+            if (p.k_new != nullptr && first + n_local == n_pages) append_new_token(p, b, kvh, len, P, DH * 2, lane);
+        }
         const int32_t* row = p.block_tables + (int64_t)b * p.max_blocks + first;
         bool ok = true;
         int issued = 0;
@@ -162,8 +186,9 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
                             mbar_arrive_expect_tx(full_bar + 8 * s, C::kStage);
 #pragma unroll
                             for (int bx = 0; bx < C::kBoxes; ++bx) {
-                                tma_load_2d(dst + bx * C::kBoxB, &tmap_k, bx * 64, y, full_bar + 8 * s);
-                                tma_load_2d(dst + C::kChunk + bx * C::kBoxB, &tmap_v, bx * 64, y, full_bar + 8 * s);
+                                tma_load_2d(dst + bx * C::kBoxB, &tmap_k, bx * C::kBoxElems, y, full_bar + 8 * s);
+                                tma_load_2d(dst + C::kChunk + bx * C::kBoxB, &tmap_v, bx * C::kBoxElems, y,
+                                            full_bar + 8 * s);
                             }
                         } else {
                             raise_err(p.err, KV_DEV_ERR_PAGE_RANGE);
@@ -217,8 +242,8 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
                 const bool is_v = bx >= C::kBoxes;
                 const int bb = is_v ? bx - C::kBoxes : bx;
                 const uint32_t dst = sbase + s * C::kStage + (is_v ? C::kChunk : 0) + bb * C::kBoxB;
-                tma_load_2d(dst, is_v ? static_cast<const void*>(&tmap_v) : static_cast<const void*>(&tmap_k), bb * 64,
-                            (pgl * p.H_kv + kvh) * P, full_bar + 8 * s);
+                tma_load_2d(dst, is_v ? static_cast<const void*>(&tmap_v) : static_cast<const void*>(&tmap_k),
+                            bb * C::kBoxElems, (pgl * p.H_kv + kvh) * P, full_bar + 8 * s);
             }
             issued = base + cnt;
         }
@@ -254,8 +279,13 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
                 const int r = r0 + 8 * rr;
 #pragma unroll
                 for (int ch = 0; ch < 2; ++ch) {
-                    const int d = kk * 16 + ch * 8 + 2 * quad;
-                    qa[kk][rr + 2 * ch] = (r < rows) ? q32[((row0 + r) * DH + d) >> 1] : 0u;
+                    // 16-bit K/V: k-step kk covers dims kk*16 .. +15 in ldmatrix order. E4M3: the
+                    // thread's K words hold dims quad*Dh/4 + 4*kk .. +3, so its q pairs follow them.
+                    const int d = kFP8 ? quad * (DH / 4) + 4 * kk + 2 * ch : kk * 16 + ch * 8 + 2 * quad;
+                    uint32_t v = (r < rows) ? q32[((row0 + r) * DH + d) >> 1] : 0u;
+                    if constexpr (kFP8 && QT == KV_DTYPE_BF16)  // bf16 q -> f16 operands (exact in f16's range)
+                        v = pack2_satfinite_f16(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+                    qa[kk][rr + 2 * ch] = v;
                 }
             }
         }
@@ -266,7 +296,7 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
     for (int n = 0; n < C::kOT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
     float m_ref[2] = {-INFINITY, -INFINITY};  // reference max (log2 units) of rows r0, r0 + 8
     float l_part[2] = {0.f, 0.f};             // this lane's share of the row sums
-    const float sl2 = p.scale_log2;
+    const float sl2 = kFP8 ? p.scale_log2 * p.k_scale[kvh] : p.scale_log2;
     bool ok = true;
 
     if (active) {
@@ -292,17 +322,34 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
 #pragma unroll
                 for (int n = 0; n < C::kNT; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
                 const int mi = lane >> 3, rr8 = lane & 7;
+                if constexpr (kFP8) {
+                    // token r0 of each n-tile: the thread's Dh/4 bytes of that row (E4M3 -> f16 pairs)
 #pragma unroll
-                for (int kk = 0; kk < C::kKSteps; ++kk) {
-                    const int c = kk * 2 + (mi & 1);  // 16-byte chunk of the row (8 dims)
-                    const uint32_t boxb = sK + (c >> 3) * C::kBoxB;
+                    for (int n = 0; n < C::kNT; ++n) {
+                        const int t = n * 8 + r0;
+                        uint32_t w[DH / 16];
 #pragma unroll
-                    for (int np = 0; np < C::kNT / 2; ++np) {
-                        const int t = np * 16 + (mi >> 1) * 8 + rr8;
-                        uint32_t b0, b1, b2, b3;
-                        ldsm_x4(boxb + t * 128 + (((c & 7) ^ (t & 7)) << 4), b0, b1, b2, b3);
-                        mma_16816<kBF16>(sc[2 * np], qa[kk], b0, b1);
-                        mma_16816<kBF16>(sc[2 * np + 1], qa[kk], b2, b3);
+                        for (int c = 0; c < DH / 64; ++c) {
+                            const uint4 x = lds128(sK + swz<C::kBoxInner>(t, quad * (DH / 64) + c));
+                            w[4 * c] = x.x, w[4 * c + 1] = x.y, w[4 * c + 2] = x.z, w[4 * c + 3] = x.w;
+                        }
+#pragma unroll
+                        for (int kk = 0; kk < C::kKSteps; ++kk)
+                            mma_16816<false>(sc[n], qa[kk], e4m3x2_to_f16x2(w[kk]), e4m3x2_to_f16x2(w[kk] >> 16));
+                    }
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < C::kKSteps; ++kk) {
+                        const int c = kk * 2 + (mi & 1);  // 16-byte chunk of the row (8 dims)
+                        const uint32_t boxb = sK + (c >> 3) * C::kBoxB;
+#pragma unroll
+                        for (int np = 0; np < C::kNT / 2; ++np) {
+                            const int t = np * 16 + (mi >> 1) * 8 + rr8;
+                            uint32_t b0, b1, b2, b3;
+                            ldsm_x4(boxb + t * 128 + (((c & 7) ^ (t & 7)) << 4), b0, b1, b2, b3);
+                            mma_16816<kBF16>(sc[2 * np], qa[kk], b0, b1);
+                            mma_16816<kBF16>(sc[2 * np + 1], qa[kk], b2, b3);
+                        }
                     }
                 }
 
@@ -368,15 +415,53 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
                 }
                 // ---- tail page: zero V rows past the length (they may hold stale data)
                 if (nvalid < P) {
-                    for (int idx = lane; idx < (P - nvalid) * C::kBoxes * 8; idx += 32) {
-                        const int t = nvalid + idx / (C::kBoxes * 8);
-                        const int rem = idx % (C::kBoxes * 8);
-                        sts128_zero(sV + (rem >> 3) * C::kBoxB + t * 128 + ((rem & 7) << 4));
+                    constexpr int kCPR = C::kBoxInner / 16;  // 16-byte chunks per box row
+                    for (int idx = lane; idx < (P - nvalid) * C::kBoxes * kCPR; idx += 32) {
+                        const int t = nvalid + idx / (C::kBoxes * kCPR);
+                        const int rem = idx % (C::kBoxes * kCPR);
+                        sts128_zero(sV + (rem / kCPR) * C::kBoxB + t * C::kBoxInner + ((rem % kCPR) << 4));
                     }
                     fence_proxy_async_smem();
                     __syncwarp();
                 }
                 // ---- O += P V (k = tokens, n = dims)
+                if constexpr (kFP8) {
+                    // Dim n-tile j, column r0 is dim r0 * Dh/8 + j: the thread reads its Dh/8 bytes of
+                    // tokens 2q, 2q + 1, 2q + 8, 2q + 9 and pairs the two tokens' bytes per dim.
+                    constexpr int kW = DH / 32;  // words per token row per thread
+#pragma unroll
+                    for (int ks = 0; ks < C::kPK; ++ks) {
+                        uint32_t wv[4][kW];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int t = ks * 16 + 2 * quad + (e & 1) + 8 * (e >> 1);
+                            if constexpr (DH == 128) {
+                                const uint4 x = lds128(sV + swz<C::kBoxInner>(t, r0));
+                                wv[e][0] = x.x, wv[e][1] = x.y, wv[e][2] = x.z, wv[e][3] = x.w;
+                            } else {
+                                const uint2 x = lds64(sV + swz<C::kBoxInner>(t, r0 >> 1) + (r0 & 1) * 8);
+                                wv[e][0] = x.x, wv[e][1] = x.y;
+                            }
+                        }
+#pragma unroll
+                        for (int m = 0; m < kW; ++m) {
+#pragma unroll
+                            for (int hh = 0; hh < 2; ++hh) {  // bytes 0-1 or 2-3 of word m
+                                const uint32_t sel = hh ? 0x7362u : 0x5140u;
+                                const uint32_t lo = byte_perm(wv[0][m], wv[1][m], sel);  // tokens 2q, 2q + 1
+                                const uint32_t hi = byte_perm(wv[2][m], wv[3][m], sel);  // tokens 2q + 8, 2q + 9
+#pragma unroll
+                                for (int e = 0; e < 2; ++e) {
+                                    const int j = 4 * m + 2 * hh + e;
+                                    const uint32_t b0 = e4m3x2_to_f16x2(lo >> (16 * e));
+                                    const uint32_t b1 = e4m3x2_to_f16x2(hi >> (16 * e));
+                                    mma_16816<false>(o[j], pa[ks], b0, b1);
+                                    if constexpr (!lo_rows) mma_16816<false>(o[j], pr[ks], b0, b1);
+                                }
+                            }
+                        }
+                    }
+                } else {
 #pragma unroll
                 for (int ks = 0; ks < C::kPK; ++ks) {
                     const int t = ks * 16 + (mi & 1) * 8 + rr8;
@@ -392,6 +477,7 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
                             mma_16816<kBF16>(o[2 * op + 1], pr[ks], v2, v3);
                         }
                     }
+                }
                 }
             }
             __syncwarp();
@@ -413,10 +499,14 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
             const int r = r0 + 8 * h;
             if (r < rows) {
                 float* dst = merge + (cw * 16 + r) * (DH + 2);
+                const float vs = kFP8 ? p.v_scale[kvh] : 1.f;
 #pragma unroll
                 for (int n = 0; n < C::kOT; ++n) {
-                    dst[n * 8 + 2 * quad] = o[n][2 * h] + (lo_rows ? o[n][2] : 0.f);
-                    dst[n * 8 + 2 * quad + 1] = o[n][2 * h + 1] + (lo_rows ? o[n][3] : 0.f);
+                    // column 2q (+1) of dim n-tile n: dim n*8 + 2q (+1); E4M3: dim (2q (+1)) * Dh/8 + n
+                    const int d0 = kFP8 ? (2 * quad) * (DH / 8) + n : n * 8 + 2 * quad;
+                    const int d1 = kFP8 ? (2 * quad + 1) * (DH / 8) + n : n * 8 + 2 * quad + 1;
+                    dst[d0] = (o[n][2 * h] + (lo_rows ? o[n][2] : 0.f)) * vs;
+                    dst[d1] = (o[n][2 * h + 1] + (lo_rows ? o[n][3] : 0.f)) * vs;
                 }
                 if (quad == 0) {
                     dst[DH] = m_ref[h];

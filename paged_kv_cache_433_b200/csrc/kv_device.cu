@@ -11,6 +11,7 @@
 
 #include "combine_kernel.cuh"
 #include "decode_launch.cuh"
+#include "fp8.cuh"
 #include "kvpaged.h"
 #include "plan_kernel.cuh"
 
@@ -75,6 +76,74 @@ __global__ void __launch_bounds__(256) kv_copy_pages_kernel(uint4* __restrict__ 
     }
 }
 
+// Quantising append for E4M3 pools: code = E4M3(x / scale[h]) with the
+// division in IEEE fp32 and round-to-nearest-even, saturating at +-448. One
+// thread converts 16 elements of one row (16 output bytes); the first half of
+// the threads serve K, the rest V.
+template <int SRC>
+__global__ void __launch_bounds__(256) kv_append_fp8_kernel(uint4* __restrict__ k_pages, uint4* __restrict__ v_pages,
+                                                            const void* __restrict__ k_new,
+                                                            const void* __restrict__ v_new,
+                                                            const float* __restrict__ k_scale,
+                                                            const float* __restrict__ v_scale,
+                                                            const int64_t* __restrict__ slots, int64_t B, int32_t H_kv,
+                                                            int32_t cpr, int32_t P, int64_t num_slots, int* err) {
+    grid_dependency_wait();
+    if (threadIdx.x == 0) grid_launch_dependents();
+    int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    const int64_t per = B * H_kv * cpr;
+    if (i >= 2 * per) return;
+    const bool is_v = i >= per;
+    if (is_v) i -= per;
+    const int64_t row = i / cpr;
+    const int32_t c = static_cast<int32_t>(i - row * cpr);
+    const int64_t b = row / H_kv;
+    const int32_t h = static_cast<int32_t>(row - b * H_kv);
+    const int64_t slot = slots[b];
+    if (slot < 0) return;
+    if (slot >= num_slots) {
+        if (!is_v && h == 0 && c == 0 && err) atomicOr(err, KV_DEV_ERR_SLOT);
+        return;
+    }
+    float x[16];
+    if constexpr (SRC == KV_DTYPE_F32) {
+        const float4* src = static_cast<const float4*>(is_v ? v_new : k_new) + i * 4;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float4 f = src[k];
+            x[4 * k] = f.x, x[4 * k + 1] = f.y, x[4 * k + 2] = f.z, x[4 * k + 3] = f.w;
+        }
+    } else {
+        const uint4* src = static_cast<const uint4*>(is_v ? v_new : k_new) + i * 2;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const uint4 u = src[k];
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if constexpr (SRC == KV_DTYPE_BF16) {
+                    x[8 * k + 2 * j] = __uint_as_float(w[j] << 16);
+                    x[8 * k + 2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+                } else {
+                    x[8 * k + 2 * j] = __half2float(__ushort_as_half(static_cast<unsigned short>(w[j] & 0xffffu)));
+                    x[8 * k + 2 * j + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(w[j] >> 16)));
+                }
+            }
+        }
+    }
+    const float sc = (is_v ? v_scale : k_scale)[h];
+    uint32_t out[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t lo = f32x2_to_e4m3x2(__fdiv_rn(x[4 * j], sc), __fdiv_rn(x[4 * j + 1], sc));
+        const uint32_t hi = f32x2_to_e4m3x2(__fdiv_rn(x[4 * j + 2], sc), __fdiv_rn(x[4 * j + 3], sc));
+        out[j] = lo | (hi << 16);
+    }
+    const int64_t page = slot / P, off = slot - page * P;
+    const int64_t dst = ((page * H_kv + h) * P + off) * cpr + c;
+    (is_v ? v_pages : k_pages)[dst] = make_uint4(out[0], out[1], out[2], out[3]);
+}
+
 namespace {
 
 int elem_bytes(int32_t dtype) {
@@ -82,6 +151,7 @@ int elem_bytes(int32_t dtype) {
         case KV_DTYPE_F32: return 4;
         case KV_DTYPE_BF16: return 2;
         case KV_DTYPE_F16: return 2;
+        case KV_DTYPE_FP8_E4M3: return 1;
         default: return 0;
     }
 }
@@ -161,25 +231,34 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // A K or V pool [num_pages][H_kv][P][Dh] seen as a 2-D tensor of
-// num_pages * H_kv * P rows of Dh 16-bit elements; boxes of P rows x 64
-// elements (128 bytes) with 128-byte swizzle.
+// num_pages * H_kv * P rows of Dh elements; boxes of P rows x 128 bytes with
+// the 128-byte swizzle (64 elements of 16 bits, or 128 E4M3 codes), or, for
+// E4M3 rows of 64 bytes, P rows x 64 bytes with the 64-byte swizzle.
 bool make_pool_map(CUtensorMap* m, const void* base, int32_t dtype, int64_t rows, int32_t Dh, int32_t P) {
     auto enc = tensor_map_encoder();
     if (!enc || rows >= (1LL << 32)) return false;
+    const int eb = elem_bytes(dtype);
+    const int row_bytes = Dh * eb;
+    const int box_bytes = row_bytes < 128 ? row_bytes : 128;
     cuuint64_t gdim[2] = {static_cast<cuuint64_t>(Dh), static_cast<cuuint64_t>(rows)};
-    cuuint64_t gstride[1] = {static_cast<cuuint64_t>(Dh) * 2};
-    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(P)};
+    cuuint64_t gstride[1] = {static_cast<cuuint64_t>(row_bytes)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(box_bytes / eb), static_cast<cuuint32_t>(P)};
     cuuint32_t estride[2] = {1, 1};
-    CUresult r = enc(m, dtype == KV_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
-                     const_cast<void*>(base), gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    const CUtensorMapDataType t = dtype == KV_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                  : dtype == KV_DTYPE_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                          : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    const CUtensorMapSwizzle sw = box_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    CUresult r = enc(m, t, 2, const_cast<void*>(base), gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
 // Tensor cores for 16-bit K/V when the GQA group fits 4 slices of 16 rows.
+// E4M3 K/V exist only on the tensor-core kernel.
 bool use_mma(int32_t dtype, int32_t g) {
     const int kind = g_kernel_kind.load(std::memory_order_relaxed);
-    if (dtype == KV_DTYPE_F32 || kind == KV_DECODE_KERNEL_SIMT) return false;
+    if (dtype == KV_DTYPE_F32) return false;
+    if (kind == KV_DECODE_KERNEL_SIMT && dtype != KV_DTYPE_FP8_E4M3) return false;
     return g <= 64;
 }
 
@@ -233,6 +312,7 @@ int check_shape(int32_t H_q, int32_t H_kv, int32_t Dh, int32_t page_size, int32_
     if (Dh != 64 && Dh != 128) return KV_ERR_UNSUPPORTED;
     if (page_size != 16 && page_size != 32) return KV_ERR_UNSUPPORTED;
     int a, b, c, d;
+    if (dtype == KV_DTYPE_FP8_E4M3) return use_mma(dtype, H_q / H_kv) ? KV_OK : KV_ERR_UNSUPPORTED;
     if (!use_mma(dtype, H_q / H_kv) && !plan_group(H_q / H_kv, &a, &b, &c, &d)) return KV_ERR_UNSUPPORTED;
     return KV_OK;
 }
@@ -323,12 +403,23 @@ int paged_decode_workspace_bytes(int32_t B, int32_t H_q, int32_t H_kv, int32_t D
 namespace kvp {
 namespace {
 
+// dtype: the K/V pools' type; q_dtype: q's (the same for 16-bit and fp32
+// K/V; bf16 or fp16 with E4M3 K/V, which also need k_scale / v_scale).
 int decode_impl(float* out, const void* q, const void* k_new, const void* v_new, const void* k_pages,
                 const void* v_pages, const int32_t* block_tables, int32_t max_blocks, const int32_t* seq_lens, int32_t B,
                 int32_t H_q, int32_t H_kv, int32_t Dh, int32_t page_size, int32_t num_pages, float scale, int32_t dtype,
-                int32_t num_splits, void* workspace, size_t ws_bytes, int* err_flag, void* stream) {
+                int32_t num_splits, void* workspace, size_t ws_bytes, int* err_flag, void* stream,
+                int32_t q_dtype = -1, const float* k_scale = nullptr, const float* v_scale = nullptr) {
     int rc = check_shape(H_q, H_kv, Dh, page_size, dtype);
     if (rc != KV_OK) return rc;
+    if (q_dtype < 0) q_dtype = dtype;
+    if (dtype == KV_DTYPE_FP8_E4M3) {
+        if (q_dtype != KV_DTYPE_BF16 && q_dtype != KV_DTYPE_F16) return KV_ERR_ARG;
+        if (k_new != nullptr || v_new != nullptr) return KV_ERR_UNSUPPORTED;  // quantising append: kv_append_fp8
+        if (B > 0 && (!k_scale || !v_scale)) return KV_ERR_ARG;
+    } else if (q_dtype != dtype) {
+        return KV_ERR_ARG;
+    }
     if (B < 0 || max_blocks <= 0 || num_pages <= 0 || num_splits < 0) return KV_ERR_ARG;
     if (B == 0) return KV_OK;
     if (B > 65535 || H_kv > 65535) return KV_ERR_UNSUPPORTED;
@@ -337,6 +428,7 @@ int decode_impl(float* out, const void* q, const void* k_new, const void* v_new,
     const int32_t g = H_q / H_kv;
     // TMA row coordinates are int32: very large pools stay on the CUDA-core kernel.
     const bool mma = use_mma(dtype, g) && static_cast<int64_t>(num_pages) * H_kv * page_size < (1LL << 31);
+    if (dtype == KV_DTYPE_FP8_E4M3 && !mma) return KV_ERR_UNSUPPORTED;
     int GW = 0, HS, NW, WP;
     if (mma) {
         HS = (g + 15) / 16;
@@ -371,6 +463,8 @@ int decode_impl(float* out, const void* q, const void* k_new, const void* v_new,
     p.num_splits = S;
     p.pages_per_split = C;
     p.scale_log2 = scale * kLog2e;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     dim3 grid(static_cast<unsigned>(S), static_cast<unsigned>(H_kv), static_cast<unsigned>(B));
     cudaError_t e;
@@ -412,8 +506,9 @@ int decode_impl(float* out, const void* q, const void* k_new, const void* v_new,
         if (!make_pool_map(&tk, k_pages, dtype, rows, Dh, page_size) ||
             !make_pool_map(&tv, v_pages, dtype, rows, Dh, page_size))
             return KV_ERR_CUDA;
-        e = dtype == KV_DTYPE_BF16 ? launch_mma_bf16(p, tk, tv, Dh, page_size, grid, st)
-                                   : launch_mma_f16(p, tk, tv, Dh, page_size, grid, st);
+        e = dtype == KV_DTYPE_BF16   ? launch_mma_bf16(p, tk, tv, Dh, page_size, grid, st)
+            : dtype == KV_DTYPE_F16 ? launch_mma_f16(p, tk, tv, Dh, page_size, grid, st)
+                                    : launch_mma_fp8(p, tk, tv, q_dtype, Dh, page_size, grid, st);
     } else {
         switch (dtype) {
             case KV_DTYPE_F32: e = launch_decode_f32(p, Dh, page_size, GW, NW, grid, st); break;
@@ -470,6 +565,40 @@ int paged_decode_attention_append(float* out, const void* q, const void* k_new, 
     if (B > 0 && (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new))) return KV_ERR_ARG;
     return decode_impl(out, q, k_new, v_new, k_pages, v_pages, block_tables, max_blocks, seq_lens, B, H_q, H_kv, Dh,
                        page_size, num_pages, scale, dtype, num_splits, workspace, ws_bytes, err_flag, stream);
+}
+
+int paged_decode_attention_fp8(float* out, const void* q, int32_t q_dtype, const void* k_pages, const void* v_pages,
+                               const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                               int32_t max_blocks, const int32_t* seq_lens, int32_t B, int32_t H_q, int32_t H_kv,
+                               int32_t Dh, int32_t page_size, int32_t num_pages, float scale, int32_t num_splits,
+                               void* workspace, size_t ws_bytes, int* err_flag, void* stream) {
+    return decode_impl(out, q, nullptr, nullptr, k_pages, v_pages, block_tables, max_blocks, seq_lens, B, H_q, H_kv, Dh,
+                       page_size, num_pages, scale, KV_DTYPE_FP8_E4M3, num_splits, workspace, ws_bytes, err_flag,
+                       stream, q_dtype, k_scale, v_scale);
+}
+
+int kv_append_fp8(void* k_pages, void* v_pages, const void* k_new, const void* v_new, int32_t src_dtype,
+                  const float* k_scale, const float* v_scale, const int64_t* slot_mapping, int32_t B, int32_t H_kv,
+                  int32_t Dh, int32_t page_size, int32_t num_pages, int* err_flag, void* stream) {
+    const int eb = elem_bytes(src_dtype);
+    if (B < 0 || H_kv <= 0 || Dh <= 0 || page_size <= 0 || num_pages <= 0 || eb == 0 || src_dtype == KV_DTYPE_FP8_E4M3)
+        return KV_ERR_ARG;
+    if (Dh % 16 != 0) return KV_ERR_UNSUPPORTED;
+    if (B == 0) return KV_OK;
+    if (!k_pages || !v_pages || !k_new || !v_new || !slot_mapping || !k_scale || !v_scale) return KV_ERR_ARG;
+    if (!aligned16(k_pages) || !aligned16(v_pages) || !aligned16(k_new) || !aligned16(v_new)) return KV_ERR_ARG;
+    const int32_t cpr = Dh / 16;  // 16-code groups per row
+    const int64_t threads = 2LL * B * H_kv * cpr;
+    int64_t blocks = (threads + 255) / 256;
+    if (blocks > 0x7fffffffLL) return KV_ERR_UNSUPPORTED;
+    auto* kern = src_dtype == KV_DTYPE_BF16  ? kv_append_fp8_kernel<KV_DTYPE_BF16>
+                 : src_dtype == KV_DTYPE_F16 ? kv_append_fp8_kernel<KV_DTYPE_F16>
+                                             : kv_append_fp8_kernel<KV_DTYPE_F32>;
+    cudaError_t e = launch_pdl(kern, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, static_cast<cudaStream_t>(stream),
+                               static_cast<uint4*>(k_pages), static_cast<uint4*>(v_pages), k_new, v_new, k_scale,
+                               v_scale, slot_mapping, static_cast<int64_t>(B), H_kv, cpr, page_size,
+                               static_cast<int64_t>(num_pages) * page_size, err_flag);
+    return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -28,7 +28,7 @@ KV_ERR_UNSUPPORTED = -8
 STATUS_NAMES = {0: "OK", -1: "ARG", -2: "OOM", -3: "BAD_ID", -4: "DOUBLE_FREE", -5: "SHARED_TAIL", -6: "CUDA",
                 -7: "WORKSPACE", -8: "UNSUPPORTED"}
 
-KV_DTYPE_F32, KV_DTYPE_BF16, KV_DTYPE_F16 = 0, 1, 2
+KV_DTYPE_F32, KV_DTYPE_BF16, KV_DTYPE_F16, KV_DTYPE_FP8_E4M3 = 0, 1, 2, 3
 DTYPE_CODE = {"fp32": 0, "bf16": 1, "fp16": 2}
 
 KV_DEV_ERR_PAGE_RANGE = 1
@@ -77,6 +77,10 @@ SIGNATURES = [
       _vp]),
     ("paged_decode_attention_noalloc", ctypes.c_int,
      [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _i32, _vp, _vp]),
+    ("kv_append_fp8", ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
+    ("paged_decode_attention_fp8", ctypes.c_int,
+     [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _sz, _vp,
+      _vp]),
     ("paged_decode_set_kernel", ctypes.c_int, [_i32]),
     ("paged_decode_num_splits", ctypes.c_int, [_i32, _i32, _i32, _i32, _i32, _pi32]),
     ("paged_decode_workspace_bytes", ctypes.c_int, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, _psz]),
@@ -264,7 +268,8 @@ class KvPrefixIndex:
 def _torch_dtype_code(t) -> int:
     import torch
 
-    m = {torch.float32: KV_DTYPE_F32, torch.bfloat16: KV_DTYPE_BF16, torch.float16: KV_DTYPE_F16}
+    m = {torch.float32: KV_DTYPE_F32, torch.bfloat16: KV_DTYPE_BF16, torch.float16: KV_DTYPE_F16,
+         torch.uint8: KV_DTYPE_FP8_E4M3}
     if t.dtype not in m:
         raise KvError("dtype", KV_ERR_ARG)
     return m[t.dtype]
@@ -334,6 +339,43 @@ def kv_rope_append(k_pages, v_pages, k_new, v_new, slot_mapping, positions, cos_
                               _dev(cos_sin, "cos_sin", torch.float32), cos_sin.shape[0], ROPE_STYLE[style], B, H_q, H_kv,
                               Dh, page_size, num_pages, dt, _dev(err_flag, "err_flag", torch.int32), _stream(stream))
     _check("kv_rope_append", rc)
+
+
+def kv_append_fp8(k_pages, v_pages, k_new, v_new, k_scale, v_scale, slot_mapping, page_size: int, err_flag=None,
+                  stream=None) -> None:
+    """Quantise k/v_new [B, H_kv, Dh] (bf16/fp16/fp32) to E4M3 with per-head fp32 scales [H_kv] and append them
+    into uint8 pools [num_pages, H_kv, P, Dh]."""
+    import torch
+
+    num_pages, H_kv, P, Dh = k_pages.shape
+    assert P == page_size and v_pages.shape == k_pages.shape and k_pages.dtype == torch.uint8
+    B = k_new.shape[0]
+    assert tuple(k_new.shape) == (B, H_kv, Dh) and v_new.shape == k_new.shape
+    rc = lib().kv_append_fp8(_dev(k_pages, "k_pages"), _dev(v_pages, "v_pages", torch.uint8), _dev(k_new, "k_new"),
+                             _dev(v_new, "v_new", k_new.dtype), _torch_dtype_code(k_new), _dev(k_scale, "k_scale", torch.float32),
+                             _dev(v_scale, "v_scale", torch.float32), _dev(slot_mapping, "slot_mapping", torch.int64), B,
+                             H_kv, Dh, page_size, num_pages, _dev(err_flag, "err_flag", torch.int32), _stream(stream))
+    _check("kv_append_fp8", rc)
+
+
+def paged_decode_attention_fp8(out, q, k_pages, v_pages, k_scale, v_scale, block_tables, seq_lens, scale: float,
+                               num_splits: int = 0, workspace=None, err_flag=None, stream=None) -> None:
+    """Decode over uint8 E4M3 pools [num_pages, H_kv, P, Dh] with per-head scales; q bf16/fp16 [B, H_q, Dh]."""
+    import torch
+
+    num_pages, H_kv, P, Dh = k_pages.shape
+    B, H_q, Dh2 = q.shape
+    assert Dh2 == Dh and v_pages.shape == k_pages.shape and k_pages.dtype == torch.uint8
+    assert tuple(out.shape) == (B, H_q, Dh) and out.dtype == torch.float32
+    max_blocks = block_tables.shape[1]
+    rc = lib().paged_decode_attention_fp8(
+        _dev(out, "out"), _dev(q, "q"), _torch_dtype_code(q), _dev(k_pages, "k_pages"), _dev(v_pages, "v_pages", torch.uint8),
+        _dev(k_scale, "k_scale", torch.float32), _dev(v_scale, "v_scale", torch.float32),
+        _dev(block_tables, "block_tables", torch.int32), max_blocks, _dev(seq_lens, "seq_lens", torch.int32), B, H_q,
+        H_kv, Dh, P, num_pages, float(scale), num_splits, _dev(workspace, "workspace"),
+        0 if workspace is None else workspace.numel() * workspace.element_size(), _dev(err_flag, "err_flag", torch.int32),
+        _stream(stream))
+    _check("paged_decode_attention_fp8", rc)
 
 
 KV_DECODE_KERNEL_AUTO, KV_DECODE_KERNEL_SIMT, KV_DECODE_KERNEL_MMA = 0, 1, 2
