@@ -85,13 +85,15 @@ template <int KT, int QT, int DH, int P, bool LO>
 cudaError_t launch_mma_inst(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, dim3 grid,
                             cudaStream_t st) {
     constexpr int NW = 4;
-    using C = MmaCfg<DH, P, NW, KT == KV_DTYPE_FP8_E4M3 ? 1 : 2>;
+    // E4M3 pages of 16 tokens are half the bytes of a 16-bit page: two of them share a stage
+    constexpr int PPS = (KT == KV_DTYPE_FP8_E4M3 && P == 16) ? 2 : 1;
+    using C = MmaCfg<DH, P, NW, KT == KV_DTYPE_FP8_E4M3 ? 1 : 2, PPS>;
     static std::atomic<uint64_t> configured{0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     const uint64_t bit = 1ull << (dev & 63);
-    auto* kern = paged_decode_mma_kernel<KT, QT, DH, P, NW, LO>;
+    auto* kern = paged_decode_mma_kernel<KT, QT, DH, P, NW, LO, PPS>;
     if (!(configured.load(std::memory_order_acquire) & bit)) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         if (e != cudaSuccess) return e;

@@ -29,9 +29,6 @@
 #include "decode_kernel.cuh"
 #include "fp8.cuh"
 
-#ifndef KVP_PRODUCER_SINGLE_LANE
-#define KVP_PRODUCER_SINGLE_LANE 0
-#endif
 #ifndef KVP_MMA_STAGE_BUDGET
 #define KVP_MMA_STAGE_BUDGET (96 * 1024)
 #endif
@@ -41,18 +38,22 @@ namespace kvp {
 // EB: bytes per K/V element (2: bf16 / fp16; 1: E4M3). A token row of Dh
 // elements is loaded as boxes of at most 128 bytes (rows of 128 bytes use the
 // 128-byte swizzle, rows of 64 bytes -- E4M3 at Dh = 64 -- the 64-byte one).
-template <int DH, int P, int NW, int EB>
+// PPS pages share one pipeline stage (tokens per stage TP = P * PPS): the
+// consumer then works on TP tokens per barrier round trip.
+template <int DH, int P, int NW, int EB, int PPS>
 struct MmaCfg {
+    static constexpr int kTP = P * PPS;                          // tokens per stage
     static constexpr int kRowB = DH * EB;                        // bytes per token row
     static constexpr int kBoxInner = kRowB < 128 ? kRowB : 128;  // bytes per box row
     static constexpr int kBoxElems = kBoxInner / EB;
     static constexpr int kBoxes = kRowB / kBoxInner;             // boxes per token row
-    static constexpr int kBoxB = P * kBoxInner;                  // bytes per box (P rows)
-    static constexpr int kChunk = P * kRowB;                     // one (page, head) chunk
+    static constexpr int kPageB = P * kBoxInner;                 // bytes of one page's box (P rows)
+    static constexpr int kBoxB = kTP * kBoxInner;                // bytes per box column of a stage
+    static constexpr int kChunk = kTP * kRowB;                   // K (or V) of one stage
     static constexpr int kStage = 2 * kChunk;                    // K + V
     static constexpr int kKSteps = DH / 16;                      // QK k-steps
-    static constexpr int kNT = P / 8;                            // token n-tiles of S
-    static constexpr int kPK = P / 16;                           // PV k-steps
+    static constexpr int kNT = kTP / 8;                          // token n-tiles of S
+    static constexpr int kPK = kTP / 16;                         // PV k-steps
     static constexpr int kOT = DH / 8;                           // dim n-tiles of O
     static constexpr int kStageBudget = KVP_MMA_STAGE_BUDGET;
     // Stage i % NS is drained by page-warp i % WP (WP divides NW): NS must be
@@ -85,12 +86,12 @@ __device__ __forceinline__ uint32_t swz(int t, int c) {
 // 16-bit K/V; bf16 or fp16 for E4M3, whose products run in f16). LO: the GQA
 // group has at most 8 heads (one head slice, rows 8..15 are padding), so each
 // row's probability residual rides in row r + 8.
-template <int KT, int QT, int DH, int P, int NW, bool LO>
+template <int KT, int QT, int DH, int P, int NW, bool LO, int PPS>
 __global__ void __launch_bounds__(32 * (NW + 1), 2)
     paged_decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                             const __grid_constant__ CUtensorMap tmap_v) {
     constexpr bool kFP8 = KT == KV_DTYPE_FP8_E4M3;
-    using C = MmaCfg<DH, P, NW, kFP8 ? 1 : 2>;
+    using C = MmaCfg<DH, P, NW, kFP8 ? 1 : 2, PPS>;
     constexpr bool kBF16 = KT == KV_DTYPE_BF16;  // MMA operand type: bf16, else f16
     extern __shared__ __align__(1024) unsigned char smem_raw[];
 
@@ -164,69 +165,41 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
             if (p.k_new != nullptr && first + n_local == n_pages) append_new_token(p, b, kvh, len, P, DH * 2, lane);
         }
         const int32_t* row = p.block_tables + (int64_t)b * p.max_blocks + first;
+        const int n_st = (n_local + PPS - 1) / PPS;  // stages of this CTA
         bool ok = true;
         int issued = 0;
-#if KVP_PRODUCER_SINGLE_LANE
-        for (int base = 0; base < n_local && ok; base += 32) {
-            const int my = (base + lane < n_local) ? row[base + lane] : 0;
-            const int cnt = min(32, n_local - base);
-            for (int k = 0; k < cnt; ++k) {
-                const int pg = __shfl_sync(0xffffffffu, my, k);
-                const int i = base + k;
-                if (lane == 0) {
-                    const int s = i % C::kNS;
-                    if (i >= C::kNS && !mbar_wait_bounded(empty_bar + 8 * s, ((i / C::kNS) - 1) & 1, kWaitLimitNs)) {
-                        raise_err(p.err, KV_DEV_ERR_TIMEOUT);
-                        ok = false;
-                    } else {
-                        const uint32_t dst = sbase + s * C::kStage;
-                        if (pg >= 0 && pg < p.num_pages) {
-                            stage_tag[s] = i;
-                            const int32_t y = (pg * p.H_kv + kvh) * P;  // first row of the chunk
-                            mbar_arrive_expect_tx(full_bar + 8 * s, C::kStage);
-#pragma unroll
-                            for (int bx = 0; bx < C::kBoxes; ++bx) {
-                                tma_load_2d(dst + bx * C::kBoxB, &tmap_k, bx * C::kBoxElems, y, full_bar + 8 * s);
-                                tma_load_2d(dst + C::kChunk + bx * C::kBoxB, &tmap_v, bx * C::kBoxElems, y,
-                                            full_bar + 8 * s);
-                            }
-                        } else {
-                            raise_err(p.err, KV_DEV_ERR_PAGE_RANGE);
-                            stage_tag[s] = -1 - i;
-                            mbar_arrive(full_bar + 8 * s);
-                        }
-                        ++issued;
-                    }
-                }
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
-            }
-        }
-#else
-        // A group of kGrp pages per step: lane l < kGrp claims the stage of
-        // page base + l (bounded wait on its empty barrier, tag, expect_tx),
-        // then every lane issues one TMA box: box l % kBPP of page l / kBPP.
-        constexpr int kBPP = 2 * C::kBoxes;  // boxes per page (K and V)
-        constexpr int kGrp0 = 32 / kBPP;
+        // A group of kGrp stages per step: lane l < kGrp claims stage base + l
+        // (bounded wait on its empty barrier, tag, expect_tx for its pages),
+        // then every lane issues one TMA box: box l % kBPS of stage l / kBPS.
+        constexpr int kBPS = PPS * 2 * C::kBoxes;  // boxes per stage (K and V of each page)
+        constexpr int kGrp0 = 32 / kBPS;
         constexpr int kGrpMax = kGrp0 < C::kNS ? kGrp0 : C::kNS;
         constexpr int kGrp = kGrpMax >= 16 ? 16 : kGrpMax >= 8 ? 8 : kGrpMax >= 4 ? 4 : kGrpMax >= 2 ? 2 : 1;
-        static_assert(32 % kGrp == 0, "page groups must tile the 32-entry table window");
-        int tab = 0;  // block-table entry of page (base & ~31) + lane
-        for (int base = 0; base < n_local; base += kGrp) {
-            if ((base & 31) == 0) tab = base == 0 ? tab0 : ((base + lane < n_local) ? row[base + lane] : 0);
-            const int cnt = min(kGrp, n_local - base);
-            const int pg = __shfl_sync(0xffffffffu, tab, ((base & 31) + lane) & 31);
+        static_assert(32 % (kGrp * PPS) == 0, "page groups must tile the 32-entry table window");
+        int tab = 0;  // block-table entry of page (first page of the group & ~31) + lane
+        for (int base = 0; base < n_st; base += kGrp) {
+            const int pbase = base * PPS;
+            if ((pbase & 31) == 0) tab = pbase == 0 ? tab0 : ((pbase + lane < n_local) ? row[pbase + lane] : 0);
+            const int cnt = min(kGrp, n_st - base);
+            int pg[PPS];
+#pragma unroll
+            for (int j = 0; j < PPS; ++j) pg[j] = __shfl_sync(0xffffffffu, tab, ((base + lane) * PPS + j) & 31);
             bool valid = false;
             if (lane < cnt) {
                 const int i = base + lane;
                 const int s = i % C::kNS;
+                const int np = min(PPS, n_local - i * PPS);  // pages in this stage
+                bool in_range = true;
+#pragma unroll
+                for (int j = 0; j < PPS; ++j)
+                    if (j < np) in_range = in_range && pg[j] >= 0 && pg[j] < p.num_pages;
                 if (i >= C::kNS && !mbar_wait_bounded(empty_bar + 8 * s, ((i / C::kNS) - 1) & 1, kWaitLimitNs)) {
                     raise_err(p.err, KV_DEV_ERR_TIMEOUT);
                     ok = false;
-                } else if (pg >= 0 && pg < p.num_pages) {
+                } else if (in_range) {
                     valid = true;
                     stage_tag[s] = i;
-                    mbar_arrive_expect_tx(full_bar + 8 * s, C::kStage);
+                    mbar_arrive_expect_tx(full_bar + 8 * s, np * 2 * C::kBoxes * C::kPageB);
                 } else {
                     raise_err(p.err, KV_DEV_ERR_PAGE_RANGE);
                     stage_tag[s] = -1 - i;
@@ -235,19 +208,21 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
             }
             if (!__all_sync(0xffffffffu, ok)) break;
             const unsigned vmask = __ballot_sync(0xffffffffu, valid);
-            const int pl = lane / kBPP, bx = lane % kBPP;
-            const int pgl = __shfl_sync(0xffffffffu, pg, pl);
-            if (pl < cnt && ((vmask >> pl) & 1u)) {
+            const int pl = lane / kBPS, bx = lane % kBPS;
+            const int j = bx / (2 * C::kBoxes);          // page of the stage
+            const bool is_v = ((bx / C::kBoxes) & 1) != 0;
+            const int bb = bx % C::kBoxes;               // box of the token row
+            const int page_idx = (base + pl) * PPS + j;  // page of this CTA's range
+            const int pgl = __shfl_sync(0xffffffffu, tab, page_idx & 31);
+            if (pl < cnt && ((vmask >> pl) & 1u) && page_idx < n_local) {
                 const int s = (base + pl) % C::kNS;
-                const bool is_v = bx >= C::kBoxes;
-                const int bb = is_v ? bx - C::kBoxes : bx;
-                const uint32_t dst = sbase + s * C::kStage + (is_v ? C::kChunk : 0) + bb * C::kBoxB;
+                const uint32_t dst =
+                    sbase + s * C::kStage + (is_v ? C::kChunk : 0) + bb * C::kBoxB + j * C::kPageB;
                 tma_load_2d(dst, is_v ? static_cast<const void*>(&tmap_v) : static_cast<const void*>(&tmap_k),
                             bb * C::kBoxElems, (pgl * p.H_kv + kvh) * P, full_bar + 8 * s);
             }
             issued = base + cnt;
         }
-#endif
         if (lane == 0) {
             for (int i = max(0, issued - C::kNS); i < issued; ++i)
                 if (!mbar_wait_bounded(full_bar + 8 * (i % C::kNS), (i / C::kNS) & 1, kWaitLimitNs))
@@ -300,7 +275,8 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
     bool ok = true;
 
     if (active) {
-        for (int i = wp; i < n_local; i += p.WP) {
+        const int n_st = (n_local + PPS - 1) / PPS;
+        for (int i = wp; i < n_st; i += p.WP) {
             const int s = i % C::kNS;
             if (!mbar_wait_bounded(full_bar + 8 * s, (i / C::kNS) & 1, kWaitLimitNs)) {
                 raise_err(p.err, KV_DEV_ERR_TIMEOUT);
@@ -315,7 +291,8 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
             const uint32_t sK = sbase + s * C::kStage;
             const uint32_t sV = sK + C::kChunk;
             if (tag == i) {
-                const int nvalid = min(P, len - (first + i) * P);
+                // tokens of this stage: its pages (the last stage of a range may hold fewer than PPS)
+                const int nvalid = min(min(PPS, n_local - i * PPS) * P, len - (first + i * PPS) * P);
 
                 // ---- S = Q K^T (fp32 accumulators; rows = heads, cols = tokens)
                 float sc[C::kNT][4];
@@ -414,9 +391,9 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
                     }
                 }
                 // ---- tail page: zero V rows past the length (they may hold stale data)
-                if (nvalid < P) {
+                if (nvalid < C::kTP) {
                     constexpr int kCPR = C::kBoxInner / 16;  // 16-byte chunks per box row
-                    for (int idx = lane; idx < (P - nvalid) * C::kBoxes * kCPR; idx += 32) {
+                    for (int idx = lane; idx < (C::kTP - nvalid) * C::kBoxes * kCPR; idx += 32) {
                         const int t = nvalid + idx / (C::kBoxes * kCPR);
                         const int rem = idx % (C::kBoxes * kCPR);
                         sts128_zero(sV + (rem / kCPR) * C::kBoxB + t * C::kBoxInner + ((rem % kCPR) << 4));
