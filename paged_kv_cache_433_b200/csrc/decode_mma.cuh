@@ -311,8 +311,11 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
                             w[4 * c] = x.x, w[4 * c + 1] = x.y, w[4 * c + 2] = x.z, w[4 * c + 3] = x.w;
                         }
 #pragma unroll
-                        for (int kk = 0; kk < C::kKSteps; ++kk)
-                            mma_16816<false>(sc[n], qa[kk], e4m3x2_to_f16x2(w[kk]), e4m3x2_to_f16x2(w[kk] >> 16));
+                        for (int kk = 0; kk < C::kKSteps; ++kk) {
+                            uint32_t b0, b1;
+                            e4m3x4_to_f16x2x2(w[kk], b0, b1);
+                            mma_16816<false>(sc[n], qa[kk], b0, b1);
+                        }
                     }
                 } else {
 #pragma unroll
@@ -425,15 +428,14 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
 #pragma unroll
                             for (int hh = 0; hh < 2; ++hh) {  // bytes 0-1 or 2-3 of word m
                                 const uint32_t sel = hh ? 0x7362u : 0x5140u;
-                                const uint32_t lo = byte_perm(wv[0][m], wv[1][m], sel);  // tokens 2q, 2q + 1
-                                const uint32_t hi = byte_perm(wv[2][m], wv[3][m], sel);  // tokens 2q + 8, 2q + 9
+                                uint32_t b0[2], b1[2];  // [dim n-tile 4m + 2hh + e]
+                                e4m3x4_to_f16x2x2(byte_perm(wv[0][m], wv[1][m], sel), b0[0], b0[1]);  // tokens 2q, 2q + 1
+                                e4m3x4_to_f16x2x2(byte_perm(wv[2][m], wv[3][m], sel), b1[0], b1[1]);  // tokens 2q + 8, + 9
 #pragma unroll
                                 for (int e = 0; e < 2; ++e) {
                                     const int j = 4 * m + 2 * hh + e;
-                                    const uint32_t b0 = e4m3x2_to_f16x2(lo >> (16 * e));
-                                    const uint32_t b1 = e4m3x2_to_f16x2(hi >> (16 * e));
-                                    mma_16816<false>(o[j], pa[ks], b0, b1);
-                                    if constexpr (!lo_rows) mma_16816<false>(o[j], pr[ks], b0, b1);
+                                    mma_16816<false>(o[j], pa[ks], b0[e], b1[e]);
+                                    if constexpr (!lo_rows) mma_16816<false>(o[j], pr[ks], b0[e], b1[e]);
                                 }
                             }
                         }

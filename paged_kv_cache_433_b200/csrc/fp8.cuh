@@ -7,12 +7,14 @@
 
 namespace kvp {
 
-// Two E4M3 codes (bits 0-7 and 8-15 of v) -> f16x2 (low code -> low half).
-// Exact: every E4M3 value is an f16 value.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t v) {
-    uint32_t r;
-    asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(r) : "r"(v));
-    return r;
+// Four E4M3 codes (bytes 0-3 of w) -> two f16x2 (lo: bytes 0-1, hi: bytes
+// 2-3; the lower code of a pair in the lower half). Exact: every E4M3 value
+// is an f16 value. The 32-bit register is split into halves without an
+// instruction.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
 }
 
 // Two fp32 values -> two E4M3 codes (lo in bits 0-7, hi in bits 8-15):
