@@ -173,7 +173,10 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
         // then every lane issues one TMA box: box l % kBPS of stage l / kBPS.
         constexpr int kBPS = PPS * 2 * C::kBoxes;  // boxes per stage (K and V of each page)
         constexpr int kGrp0 = 32 / kBPS;
-        constexpr int kGrpMax = kGrp0 < C::kNS ? kGrp0 : C::kNS;
+        // groups of at most 4 stages: a group is issued only once all of its
+        // stages are free, so large groups leave the ring partly idle (8B-shaped
+        // layer: 4 -> 0.85 of peak, 8 -> 0.82, 2 -> 0.80; E4M3: 0.62 / 0.59 / 0.57)
+        constexpr int kGrpMax = kGrp0 < 4 ? kGrp0 : 4;
         constexpr int kGrp = kGrpMax >= 16 ? 16 : kGrpMax >= 8 ? 8 : kGrpMax >= 4 ? 4 : kGrpMax >= 2 ? 2 : 1;
         static_assert(32 % (kGrp * PPS) == 0, "page groups must tile the 32-entry table window");
         int tab = 0;  // block-table entry of page (first page of the group & ~31) + lane
