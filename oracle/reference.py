@@ -278,3 +278,42 @@ def paged_decode(q: np.ndarray, k_pages: np.ndarray, v_pages: np.ndarray, block_
     if rc != 0:
         raise ValueError(f"oracle_paged_decode failed: {rc}")
     return out
+
+
+# --------------------------------------------------------------------------
+# Multi-token query over the paged cache (chunked prefill / prompt extension)
+# --------------------------------------------------------------------------
+
+
+def chunk_positions(q_start: Sequence[int], seq_lens: Sequence[int]) -> np.ndarray:
+    """Position of every query row: the chunk of sequence b is its last
+    n_b = q_start[b+1] - q_start[b] tokens, at positions seq_lens[b] - n_b ...
+    seq_lens[b] - 1 ([CN-06] 6.2: a prefill chunk is processed after the part
+    of the prompt already cached; 6.6 chunked prefill)."""
+    qs = np.asarray(q_start, dtype=np.int64)
+    sl = np.asarray(seq_lens, dtype=np.int64)
+    pos = np.empty(int(qs[-1]), dtype=np.int64)
+    for b in range(len(sl)):
+        n = int(qs[b + 1] - qs[b])
+        pos[qs[b]:qs[b + 1]] = sl[b] - n + np.arange(n)
+    return pos
+
+
+def paged_prefill(q: np.ndarray, q_start: Sequence[int], k_pages: np.ndarray, v_pages: np.ndarray,
+                  block_tables: np.ndarray, seq_lens: Sequence[int], scale: float, dtype: str) -> np.ndarray:
+    """fp64 causal attention of a chunk of query rows over the paged cache.
+
+    q [N, H_q, Dh] (N = q_start[-1] rows; rows q_start[b] .. q_start[b+1]-1
+    belong to sequence b). The query at position p attends to the keys at
+    positions 0 .. p (the causal rule of [KV-04] / [HB-07] Q025: a token sees
+    itself and everything before it), i.e. it is exactly a decode over a
+    sequence of length p + 1 that shares sequence b's block table. Each row is
+    computed that way by the fp64 decode above.
+    """
+    qs = np.asarray(q_start, dtype=np.int64)
+    B = len(seq_lens)
+    pos = chunk_positions(qs, seq_lens)
+    owner = np.repeat(np.arange(B), np.diff(qs))
+    tables = np.ascontiguousarray(np.asarray(block_tables, dtype=np.int32)[owner])
+    lens = (pos + 1).astype(np.int32)
+    return paged_decode(q, k_pages, v_pages, tables, lens, scale, dtype)
