@@ -291,6 +291,27 @@ int paged_decode_attention_append(float* out, const void* q, const void* k_new, 
                                   int32_t page_size, int32_t num_pages, float scale, int32_t dtype, int32_t num_splits,
                                   void* workspace, size_t ws_bytes, int* err_flag, void* stream);
 
+/* Multi-token query over the paged cache (chunked prefill / prompt
+ * extension) -- [CN-06] 6.2 and 6.6 (a prompt processed in chunks after the
+ * part already cached); causal rule of [KV-04] / [HB-07] Q025 (a token sees
+ * itself and every earlier position). The chunk's K/V must already be in the
+ * cache (kv_append / kv_rope_append of its rows). For sequence b its chunk is
+ * the last n_b = q_start[b+1] - q_start[b] of its seq_lens[b] tokens; chunk
+ * row i (q row q_start[b] + i) sits at position pos = seq_lens[b] - n_b + i
+ * and
+ *   out[row][h][:] = softmax(scale * q[row][h] . K_t) V_t over t <= pos.
+ *   q: [q_start[B]][H_q][Dh] of `dtype` (bf16 / fp16); out: fp32, same rows.
+ *   q_start: device int32 [B + 1], non-decreasing from 0; max_q_len >= every
+ *   n_b (it sizes the grid: rows past max_q_len are not computed).
+ *   n_b > seq_lens[b] sets KV_DEV_ERR_SEQ_LEN and zeroes those rows.
+ *   Tensor cores only: H_q / H_kv <= 64, Dh in {64, 128}, page_size in
+ *   {16, 32}; fp32 K/V -> KV_ERR_UNSUPPORTED. No workspace. */
+int paged_prefill_attention(float* out, const void* q, const int32_t* q_start, int32_t max_q_len,
+                            const void* k_pages, const void* v_pages, const int32_t* block_tables, int32_t max_blocks,
+                            const int32_t* seq_lens, int32_t B, int32_t H_q, int32_t H_kv, int32_t Dh,
+                            int32_t page_size, int32_t num_pages, float scale, int32_t dtype, int* err_flag,
+                            void* stream);
+
 /* ---- FP8 (E4M3) K/V cache ---------------------------------------------
  * "03. KV Cache：用显存换计算" (KV quantisation follow-up) and [CN-06]'s
  * KV-size table name storing K / V in 8 bits without fixing a format. Here:

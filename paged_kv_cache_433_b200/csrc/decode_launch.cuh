@@ -81,7 +81,7 @@ cudaError_t launch_decode_f16(const DecodeParams& p, int DH, int P, int GW, int 
 
 namespace kvp {
 
-template <int KT, int QT, int DH, int P, bool LO>
+template <int KT, int QT, int DH, int P, bool LO, bool QM = false>
 cudaError_t launch_mma_inst(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, dim3 grid,
                             cudaStream_t st) {
     constexpr int NW = 4;
@@ -93,7 +93,7 @@ cudaError_t launch_mma_inst(const DecodeParams& p, const CUtensorMap& tk, const 
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     const uint64_t bit = 1ull << (dev & 63);
-    auto* kern = paged_decode_mma_kernel<KT, QT, DH, P, NW, LO, PPS>;
+    auto* kern = paged_decode_mma_kernel<KT, QT, DH, P, NW, LO, PPS, QM>;
     if (!(configured.load(std::memory_order_acquire) & bit)) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         if (e != cudaSuccess) return e;
@@ -123,7 +123,22 @@ cudaError_t launch_mma_dt(const DecodeParams& p, const CUtensorMap& tk, const CU
                    : launch_mma_group<KT, QT, 64, 32>(p, tk, tv, grid, st);
 }
 
+// Multi-token query (chunk of new tokens per sequence, causal within it).
+template <int KT>
+cudaError_t launch_prefill_dt(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int DH, int P,
+                              dim3 grid, cudaStream_t st) {
+    if (DH == 128)
+        return P == 16 ? launch_mma_inst<KT, KT, 128, 16, false, true>(p, tk, tv, grid, st)
+                       : launch_mma_inst<KT, KT, 128, 32, false, true>(p, tk, tv, grid, st);
+    return P == 16 ? launch_mma_inst<KT, KT, 64, 16, false, true>(p, tk, tv, grid, st)
+                   : launch_mma_inst<KT, KT, 64, 32, false, true>(p, tk, tv, grid, st);
+}
+
 // Defined in decode_mma_bf16.cu / decode_mma_f16.cu / decode_mma_fp8.cu.
+cudaError_t launch_prefill_bf16(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int DH, int P,
+                                dim3 grid, cudaStream_t st);
+cudaError_t launch_prefill_f16(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int DH, int P,
+                               dim3 grid, cudaStream_t st);
 cudaError_t launch_mma_bf16(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int DH, int P, dim3 grid,
                             cudaStream_t st);
 cudaError_t launch_mma_f16(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int DH, int P, dim3 grid,

@@ -85,8 +85,11 @@ __device__ __forceinline__ uint32_t swz(int t, int c) {
 // KT: K/V storage type (bf16, fp16 or E4M3); QT: q's type (equal to KT for
 // 16-bit K/V; bf16 or fp16 for E4M3, whose products run in f16). LO: the GQA
 // group has at most 8 heads (one head slice, rows 8..15 are padding), so each
-// row's probability residual rides in row r + 8.
-template <int KT, int QT, int DH, int P, int NW, bool LO, int PPS>
+// row's probability residual rides in row r + 8. QM: multi-token query (a
+// chunk of new tokens per sequence): the MMA rows are (token, head) pairs of
+// q_tile chunk tokens, and row i of the chunk sees keys up to its own
+// position (causal within the chunk).
+template <int KT, int QT, int DH, int P, int NW, bool LO, int PPS, bool QM>
 __global__ void __launch_bounds__(32 * (NW + 1), 2)
     paged_decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                             const __grid_constant__ CUtensorMap tmap_v) {
@@ -104,9 +107,21 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
     grid_dependency_wait();  // inputs (and a plan) may come from the previous kernel in the stream
     if (threadIdx.x == 0) grid_launch_dependents();
 
-    // Work of this CTA: (split, kvh, b) from the grid, or a planned chunk.
+    // Work of this CTA: (split, kvh, b) from the grid, or a planned chunk; for a
+    // multi-token query (tile, kvh, b) with the tile's chunk tokens t0 .. t0 + nt - 1.
     int split, kvh, b, item = 0, chunk_pages;
-    if (p.items != nullptr) {
+    int qs0 = 0, n_q = 1, t0 = 0, nt = 1;
+    if constexpr (QM) {
+        split = 0;
+        kvh = blockIdx.y;
+        b = blockIdx.z;
+        chunk_pages = 0;
+        qs0 = p.q_start[b];
+        n_q = p.q_start[b + 1] - qs0;
+        t0 = blockIdx.x * p.q_tile;
+        if (t0 >= n_q) return;
+        nt = min(p.q_tile, n_q - t0);
+    } else if (p.items != nullptr) {
         const int4 it = p.items[blockIdx.x];
         if (it.x < 0) return;
         b = it.x;
@@ -120,23 +135,30 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
         b = blockIdx.z;
         chunk_pages = p.pages_per_split;
     }
-    const bool chunked = p.items != nullptr || p.num_splits > 1;
+    const bool chunked = !QM && (p.items != nullptr || p.num_splits > 1);
     // The producer's first 32 block-table entries do not depend on the length:
     // load them alongside it.
     const int first = chunked ? split * chunk_pages : 0;
     int tab0 = 0;
     if (warp == 0 && first + lane < p.max_blocks) tab0 = p.block_tables[(int64_t)b * p.max_blocks + first + lane];
     int len = p.seq_lens[b];
-    if (len < 0 || len > p.max_blocks * P) {
-        if (threadIdx.x == 0 && split == 0 && p.items == nullptr) raise_err(p.err, KV_DEV_ERR_SEQ_LEN);
+    if (len < 0 || len > p.max_blocks * P || (QM && n_q > len)) {
+        if (threadIdx.x == 0 && split == 0 && p.items == nullptr && t0 == 0) raise_err(p.err, KV_DEV_ERR_SEQ_LEN);
         len = 0;
     }
-    const int n_pages = (len + P - 1) / P;
+    // keys of this CTA: the whole sequence, or (multi-token) up to the tile's last position
+    const int key_end = QM ? (len > 0 ? len - n_q + t0 + nt : 0) : len;
+    const int n_pages = (key_end + P - 1) / P;
     const int n_local = chunked ? min(chunk_pages, n_pages - first) : n_pages;
     // Partials are needed when the row has more than one chunk.
     const bool split_mode = p.items != nullptr ? n_pages > chunk_pages : p.num_splits > 1;
     if (n_local <= 0) {
-        if (!split_mode) {
+        if constexpr (QM) {
+            for (int e = threadIdx.x; e < nt * p.g * DH; e += blockDim.x) {
+                const int rr = e / DH;
+                p.out[((int64_t)(qs0 + t0 + rr / p.g) * p.H_q + (int64_t)kvh * p.g + rr % p.g) * DH + e % DH] = 0.f;
+            }
+        } else if (!split_mode) {
             for (int e = threadIdx.x; e < p.g * DH; e += blockDim.x)
                 p.out[((int64_t)b * p.H_q + (int64_t)kvh * p.g) * DH + e] = 0.f;
         }
@@ -161,7 +183,7 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if constexpr (!kFP8) {
+        if constexpr (!kFP8 && !QM) {
             if (p.k_new != nullptr && first + n_local == n_pages) append_new_token(p, b, kvh, len, P, DH * 2, lane);
         }
         const int32_t* row = p.block_tables + (int64_t)b * p.max_blocks + first;
@@ -241,15 +263,28 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
     const bool active = wp < p.WP;
     const int quad = lane & 3;   // column pair within a fragment
     const int r0 = lane >> 2;    // fragment rows r0 and r0 + 8
-    const int rows = min(16, p.g - hs * 16);  // real heads in this slice
-    constexpr bool lo_rows = LO;               // padding rows 8..15 carry the P residual
-    const int hbase = kvh * p.g + hs * 16;    // query head of row 0
+    const int rows = min(16, nt * p.g - hs * 16);  // real rows (heads, or token-head pairs) in this slice
+    constexpr bool lo_rows = LO;                    // padding rows 8..15 carry the P residual
+    const int hbase = kvh * p.g + hs * 16;         // query head of row 0 (single-token query)
+    // Global q row of slice row r, and (multi-token) the first key position row r may not see.
+    auto q_row = [&](int r) -> int64_t {
+        if constexpr (QM) {
+            const int rr = hs * 16 + r;
+            return (int64_t)(qs0 + t0 + rr / p.g) * p.H_q + (int64_t)kvh * p.g + rr % p.g;
+        } else {
+            return (int64_t)b * p.H_q + hbase + r;
+        }
+    };
+    int key_lim[2] = {0x7fffffff, 0x7fffffff};
+    if constexpr (QM) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) key_lim[h] = len - n_q + t0 + (hs * 16 + r0 + 8 * h) / p.g + 1;
+    }
 
     // Q as the A operand of S = Q K^T: rows = heads, k = dims (pairs of elements per register).
     uint32_t qa[C::kKSteps][4];
     {
         const uint32_t* q32 = static_cast<const uint32_t*>(p.q);
-        const int64_t row0 = (int64_t)b * p.H_q + hbase;
 #pragma unroll
         for (int kk = 0; kk < C::kKSteps; ++kk) {
 #pragma unroll
@@ -260,7 +295,7 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
                     // 16-bit K/V: k-step kk covers dims kk*16 .. +15 in ldmatrix order. E4M3: the
                     // thread's K words hold dims quad*Dh/4 + 4*kk .. +3, so its q pairs follow them.
                     const int d = kFP8 ? quad * (DH / 4) + 4 * kk + 2 * ch : kk * 16 + ch * 8 + 2 * quad;
-                    uint32_t v = (r < rows) ? q32[((row0 + r) * DH + d) >> 1] : 0u;
+                    uint32_t v = (r < rows) ? q32[(q_row(r) * DH + d) >> 1] : 0u;
                     if constexpr (kFP8 && QT == KV_DTYPE_BF16)  // bf16 q -> f16 operands (exact in f16's range)
                         v = pack2_satfinite_f16(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
                     qa[kk][rr + 2 * ch] = v;
@@ -338,12 +373,18 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
 
                 // ---- scale, mask, row max (4 lanes of a quad share a row)
                 float mx[2] = {-INFINITY, -INFINITY};
+                int tlim[2] = {nvalid, nvalid};  // first masked token of the stage per row
+                if constexpr (QM) {
+                    const int kbase = (first + i * PPS) * P;
+                    tlim[0] = min(nvalid, key_lim[0] - kbase);
+                    tlim[1] = min(nvalid, key_lim[1] - kbase);
+                }
 #pragma unroll
                 for (int n = 0; n < C::kNT; ++n)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int t = n * 8 + 2 * quad + (e & 1);
-                        const float v = (t < nvalid) ? sc[n][e] * sl2 : -INFINITY;
+                        const float v = (t < tlim[e >> 1]) ? sc[n][e] * sl2 : -INFINITY;
                         sc[n][e] = v;
                         mx[e >> 1] = fmaxf(mx[e >> 1], v);
                     }
@@ -500,7 +541,7 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
     named_bar_sync(1, 32 * NW);
 
     const int tid = threadIdx.x - 32;
-    for (int e = tid; e < p.g * DH; e += 32 * NW) {
+    for (int e = tid; e < nt * p.g * DH; e += 32 * NW) {
         const int hh = e / DH;
         const int d = e % DH;
         const int slice = hh >> 4, r = hh & 15;
@@ -517,7 +558,8 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
                 U += sw * src[d];
             }
         }
-        const int64_t hq = (int64_t)b * p.H_q + (int64_t)kvh * p.g + hh;
+        const int64_t hq = QM ? (int64_t)(qs0 + t0 + hh / p.g) * p.H_q + (int64_t)kvh * p.g + hh % p.g
+                              : (int64_t)b * p.H_q + (int64_t)kvh * p.g + hh;
         if (!split_mode) {
             p.out[hq * DH + d] = (L > 0.f) ? U / L : 0.f;
         } else {

@@ -577,6 +577,58 @@ int paged_decode_attention_fp8(float* out, const void* q, int32_t q_dtype, const
                        stream, q_dtype, k_scale, v_scale);
 }
 
+int paged_prefill_attention(float* out, const void* q, const int32_t* q_start, int32_t max_q_len,
+                            const void* k_pages, const void* v_pages, const int32_t* block_tables, int32_t max_blocks,
+                            const int32_t* seq_lens, int32_t B, int32_t H_q, int32_t H_kv, int32_t Dh,
+                            int32_t page_size, int32_t num_pages, float scale, int32_t dtype, int* err_flag,
+                            void* stream) {
+    if (dtype != KV_DTYPE_BF16 && dtype != KV_DTYPE_F16) return dtype == KV_DTYPE_F32 ? KV_ERR_UNSUPPORTED : KV_ERR_ARG;
+    if (H_q <= 0 || H_kv <= 0 || H_q % H_kv != 0) return KV_ERR_ARG;
+    if (Dh != 64 && Dh != 128) return KV_ERR_UNSUPPORTED;
+    if (page_size != 16 && page_size != 32) return KV_ERR_UNSUPPORTED;
+    const int32_t g = H_q / H_kv;
+    if (g > 64) return KV_ERR_UNSUPPORTED;
+    if (B < 0 || max_q_len < 0 || max_blocks <= 0 || num_pages <= 0) return KV_ERR_ARG;
+    if (B == 0 || max_q_len == 0) return KV_OK;
+    if (B > 65535 || H_kv > 65535) return KV_ERR_UNSUPPORTED;
+    if (!out || !q || !q_start || !k_pages || !v_pages || !block_tables || !seq_lens) return KV_ERR_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages)) return KV_ERR_ARG;
+    if (static_cast<int64_t>(num_pages) * H_kv * page_size >= (1LL << 31)) return KV_ERR_UNSUPPORTED;
+    // 64 MMA rows per CTA: q_tile chunk tokens x g heads, four 16-row slices
+    const int32_t q_tile = 64 / g;
+    DecodeParams p{};
+    p.out = out;
+    p.q = q;
+    p.k_pages = k_pages;
+    p.v_pages = v_pages;
+    p.block_tables = block_tables;
+    p.seq_lens = seq_lens;
+    p.err = err_flag;
+    p.max_blocks = max_blocks;
+    p.B = B;
+    p.H_q = H_q;
+    p.H_kv = H_kv;
+    p.num_pages = num_pages;
+    p.g = g;
+    p.HS = (q_tile * g + 15) / 16;
+    p.WP = 4 / p.HS;
+    p.num_splits = 1;
+    p.pages_per_split = max_blocks;
+    p.scale_log2 = scale * kLog2e;
+    p.q_start = q_start;
+    p.q_tile = q_tile;
+    CUtensorMap tk, tv;
+    const int64_t rows = static_cast<int64_t>(num_pages) * H_kv * page_size;
+    if (!make_pool_map(&tk, k_pages, dtype, rows, Dh, page_size) || !make_pool_map(&tv, v_pages, dtype, rows, Dh, page_size))
+        return KV_ERR_CUDA;
+    const dim3 grid(static_cast<unsigned>((max_q_len + q_tile - 1) / q_tile), static_cast<unsigned>(H_kv),
+                    static_cast<unsigned>(B));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const cudaError_t e = dtype == KV_DTYPE_BF16 ? launch_prefill_bf16(p, tk, tv, Dh, page_size, grid, st)
+                                                 : launch_prefill_f16(p, tk, tv, Dh, page_size, grid, st);
+    return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;
+}
+
 int kv_append_fp8(void* k_pages, void* v_pages, const void* k_new, const void* v_new, int32_t src_dtype,
                   const float* k_scale, const float* v_scale, const int64_t* slot_mapping, int32_t B, int32_t H_kv,
                   int32_t Dh, int32_t page_size, int32_t num_pages, int* err_flag, void* stream) {

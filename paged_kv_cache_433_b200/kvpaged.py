@@ -81,6 +81,8 @@ SIGNATURES = [
     ("paged_decode_attention_fp8", ctypes.c_int,
      [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _sz, _vp,
       _vp]),
+    ("paged_prefill_attention", ctypes.c_int,
+     [_vp, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp]),
     ("paged_decode_set_kernel", ctypes.c_int, [_i32]),
     ("paged_decode_num_splits", ctypes.c_int, [_i32, _i32, _i32, _i32, _i32, _pi32]),
     ("paged_decode_workspace_bytes", ctypes.c_int, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, _psz]),
@@ -376,6 +378,26 @@ def paged_decode_attention_fp8(out, q, k_pages, v_pages, k_scale, v_scale, block
         0 if workspace is None else workspace.numel() * workspace.element_size(), _dev(err_flag, "err_flag", torch.int32),
         _stream(stream))
     _check("paged_decode_attention_fp8", rc)
+
+
+def paged_prefill_attention(out, q, q_start, max_q_len: int, k_pages, v_pages, block_tables, seq_lens, scale: float,
+                            err_flag=None, stream=None) -> None:
+    """Causal attention of chunk rows q [N, H_q, Dh] (rows q_start[b] .. q_start[b+1]-1 are the last tokens of
+    sequence b) over the paged cache; out fp32 [N, H_q, Dh]; q_start int32 [B + 1] (device)."""
+    import torch
+
+    num_pages, H_kv, P, Dh = k_pages.shape
+    N, H_q, Dh2 = q.shape
+    B = seq_lens.shape[0]
+    assert Dh2 == Dh and v_pages.shape == k_pages.shape and tuple(out.shape) == (N, H_q, Dh)
+    assert tuple(q_start.shape) == (B + 1,) and block_tables.shape[0] == B
+    rc = lib().paged_prefill_attention(
+        _dev(out, "out", torch.float32), _dev(q, "q", k_pages.dtype), _dev(q_start, "q_start", torch.int32),
+        int(max_q_len), _dev(k_pages, "k_pages"), _dev(v_pages, "v_pages", k_pages.dtype),
+        _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1], _dev(seq_lens, "seq_lens", torch.int32),
+        B, H_q, H_kv, Dh, P, num_pages, float(scale), _torch_dtype_code(k_pages), _dev(err_flag, "err_flag", torch.int32),
+        _stream(stream))
+    _check("paged_prefill_attention", rc)
 
 
 KV_DECODE_KERNEL_AUTO, KV_DECODE_KERNEL_SIMT, KV_DECODE_KERNEL_MMA = 0, 1, 2
