@@ -44,10 +44,12 @@ def parse():
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", type=int, choices=[2, 3, 4, 5, 6, 7], default=2,
+    ap.add_argument("--config", type=int, choices=[2, 3, 4, 5, 6, 7, 8], default=2,
                     help="2: 8B-shaped layer (default); 3: 32K context x 32 layers; 4: shared-prefix batch; "
                          "5: mixed continuous-batching sweep; 6: rotary embedding + append of a prefill chunk; "
-                         "7: the 8B-shaped layer with an E4M3 K/V cache")
+                         "7: the 8B-shaped layer with an E4M3 K/V cache; 8: chunked prefill (8 x 512 new tokens "
+                         "over 4096 cached)")
+    ap.add_argument("--chunk", type=int, default=512, help="config 8: chunk tokens per sequence")
     ap.add_argument("--splits", type=int, default=0, help="num_splits passed to paged_decode_attention (0 = auto)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -485,6 +487,89 @@ def run_fp8_bench(args, world, rank, local):
         "gpu_launches": steps * (1 + (3 if S == 0 else (2 if S > 1 else 1))),
         "e2e": None, "clocks": clocks,
     }
+
+
+def run_prefill_bench(args, world, rank, local):
+    """Chunked prefill on the 8B-shaped layer: 8 sequences each extend a 4096-token cached context by a
+    512-token chunk (its K/V already appended); one step = paged_prefill_attention over the 4096 chunk rows.
+    Tensor-bound: roofline against the measured bf16 dense peak, causal flops only."""
+    import torch
+
+    from paged_kv_cache_433_b200 import kvpaged as K
+    from paged_kv_cache_433_b200 import workloads as W
+
+    cfg = W.LLAMA8B
+    B, ctx, n = 8, 4096, args.chunk
+    steps = args.steps if args.steps is not None else 20
+    warm = args.warmup if args.warmup is not None else 3
+    P = cfg.page_size
+    total = ctx + n
+    lens = np.full(B, total, np.int64)
+    wl = Workload(dataclasses_replace(cfg, B=B), lens, 0, rank, 1)
+    dev = torch.device("cuda")
+    q = torch.randn((B * n, cfg.H_q, cfg.Dh), generator=wl.gen, device=dev).to(wl.dt)
+    out = torch.empty((B * n, cfg.H_q, cfg.Dh), dtype=torch.float32, device=dev)
+    q_start = torch.arange(0, B * n + 1, n, dtype=torch.int32, device=dev)
+    seq = torch.from_numpy(lens.astype(np.int32)).to(dev)
+    tab = torch.from_numpy(wl.tab).to(dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def call():
+        K.paged_prefill_attention(out, q, q_start, n, wl.k_pages[0], wl.v_pages[0], tab, seq, cfg.scale, err_flag=err,
+                                  stream=stream)
+
+    for _ in range(warm):
+        call()
+    torch.cuda.synchronize()
+    clk = ClockSampler(local, enabled=not args.no_clocks)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = clk.stop()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error flag {int(err.item())}")
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    per_s = ms / steps / 1e3
+    keys = B * (n * ctx + n * (n + 1) // 2)                    # sum over chunk rows of the keys each one sees
+    flops = 4.0 * cfg.Dh * cfg.H_q * keys                      # QK^T and PV, 2 flops per multiply-add
+    peak = peaks_tensor()
+    achieved = flops / per_s / 1e12
+    return {
+        "metric": "chunked prefill tokens/s; achieved TFLOP/s", "value": B * n * steps * world / (ms / 1e3),
+        "unit": "tokens/s", "n_gpus": world, "steps": steps, "warmup": warm, "ms_per_step": ms / steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (N(0,1) K/V, q)",
+        "config": {"workload": f"chunked-prefill-{cfg.name}-B{B}-ctx{ctx}-chunk{n}", "B": B, "context": ctx, "chunk": n,
+                   "H_q": cfg.H_q, "H_kv": cfg.H_kv, "Dh": cfg.Dh, "page_size": P,
+                   "l2": "K/V %.0f MB, re-read per 16-token tile mostly from L2; no flush" % (
+                       B * total * cfg.H_kv * cfg.Dh * 4 / 1e6)},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "peak_source": "measured cuBLAS bf16 dense (MEASURED_PEAKS bf16_tflops)",
+                     "traffic": None, "kernel": "paged_decode_mma_kernel (multi-token query)",
+                     "flops_per_launch": flops, "launch_us": per_s * 1e6},
+        "gpu_launches": steps, "e2e": None, "clocks": clocks,
+    }
+
+
+def dataclasses_replace(cfg, **kw):
+    import dataclasses
+
+    return dataclasses.replace(cfg, **kw)
+
+
+def peaks_tensor():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return 1590.0
 
 
 def run_e2e(wl, cfg, warm, steps, args, world):
@@ -1042,7 +1127,7 @@ def main():
     K.paged_decode_set_kernel({"auto": K.KV_DECODE_KERNEL_AUTO, "simt": K.KV_DECODE_KERNEL_SIMT,
                                "mma": K.KV_DECODE_KERNEL_MMA}[args.kernel])
     run = {2: run_layer_bench, 3: run_long_bench, 4: run_prefix_bench, 5: run_mixed_bench, 6: run_rope_bench,
-           7: run_fp8_bench}[args.config]
+           7: run_fp8_bench, 8: run_prefill_bench}[args.config]
     res = run(args, world, rank, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config == 2:
         res["cpu_baseline"] = cpu_baseline()
