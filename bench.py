@@ -478,7 +478,8 @@ def run_fp8_bench(args, world, rank, local):
         "vs_baseline": None, "dtype": "e4m3 K/V, bf16 q, f16 MMA",
         "data": "synthetic (N(0,1) K/V quantised with scale 4.5/448 per head; bf16 q; lengths U[512,4096])",
         "config": {"workload": cfg.name.replace("-bf16-", "-fp8kv-"), "B": B, "H_q": cfg.H_q, "H_kv": cfg.H_kv,
-                   "Dh": cfg.Dh, "page_size": P, "kv_dtype": "e4m3", "num_splits": S,
+                   "Dh": cfg.Dh, "page_size": P, "kv_dtype": "e4m3",
+                   "num_splits": args.splits if args.splits else "auto (E4M3 rule: half the 16-bit CTAs per SM)",
                    "l2": "inputs larger than L2 (K/V working set %.0f MB > 126 MB L2); no flush" % (mean_bytes / 1e6)},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": peak_kind, "traffic": None,
@@ -573,27 +574,39 @@ def peaks_tensor():
 
 
 def run_e2e(wl, cfg, warm, steps, args, world):
-    """Each step: host bookkeeping, H2D of slots/lens/q/k_new/v_new (+ table rows when a page was added),
-    kv_append + paged_decode_attention, D2H of the fp32 output, wait for it."""
+    """Each step: host bookkeeping, one H2D copy of the step's inputs packed in a pinned staging buffer
+    (q, k_new, v_new, slots, lengths, and the block table when a page was added), kv_append +
+    paged_decode_attention (fused by default), D2H of the fp32 output, wait for it. Steps are serial, as in a
+    decode loop whose next input depends on this step's output."""
     import torch
 
     K = wl.K
     B, P = wl.B, cfg.page_size
     dev = torch.device("cuda")
     n = warm + steps
-    host_q = torch.randn((n, B, cfg.H_q, cfg.Dh)).to(wl.dt).pin_memory()
-    host_kn = torch.randn((n, B, cfg.H_kv, cfg.Dh)).to(wl.dt).pin_memory()
-    host_vn = torch.randn((n, B, cfg.H_kv, cfg.Dh)).to(wl.dt).pin_memory()
+    eb = cfg.elem_bytes
+    nq, nkv = B * cfg.H_q * cfg.Dh * eb, B * cfg.H_kv * cfg.Dh * eb
+    off_q, off_kn, off_vn = 0, nq, nq + nkv
+    off_slots = nq + 2 * nkv
+    off_lens = off_slots + 8 * B
+    off_tab = (off_lens + 4 * B + 15) // 16 * 16
+    tab_bytes = wl.tab.nbytes
+    total = off_tab + tab_bytes
+    host_in = [torch.empty(total, dtype=torch.uint8).pin_memory() for _ in range(n)]
+    gen = torch.Generator().manual_seed(cfg.seed + 77)
+    for i in range(n):  # step inputs prepared before timing (q, k_new, v_new as the model would produce them)
+        h = host_in[i]
+        h[off_q:off_q + nq].view(wl.dt).copy_(torch.randn(nq // eb, generator=gen).to(wl.dt))
+        h[off_kn:off_kn + 2 * nkv].view(wl.dt).copy_(torch.randn(2 * nkv // eb, generator=gen).to(wl.dt))
     host_out = torch.empty((B, cfg.H_q, cfg.Dh), dtype=torch.float32).pin_memory()
-    pin_slots = torch.empty(B, dtype=torch.int64).pin_memory()
-    pin_lens = torch.empty(B, dtype=torch.int32).pin_memory()
-    pin_tab = torch.from_numpy(wl.tab).pin_memory()
-    d_slots = torch.empty(B, dtype=torch.int64, device=dev)
-    d_lens = torch.empty(B, dtype=torch.int32, device=dev)
-    d_tab = pin_tab.to(dev)
-    d_q = torch.empty((B, cfg.H_q, cfg.Dh), dtype=wl.dt, device=dev)
-    d_kn = torch.empty((B, cfg.H_kv, cfg.Dh), dtype=wl.dt, device=dev)
-    d_vn = torch.empty_like(d_kn)
+    d_in = torch.empty(total, dtype=torch.uint8, device=dev)
+    d_q = d_in[off_q:off_q + nq].view(wl.dt).view(B, cfg.H_q, cfg.Dh)
+    d_kn = d_in[off_kn:off_kn + nkv].view(wl.dt).view(B, cfg.H_kv, cfg.Dh)
+    d_vn = d_in[off_vn:off_vn + nkv].view(wl.dt).view(B, cfg.H_kv, cfg.Dh)
+    d_slots = d_in[off_slots:off_slots + 8 * B].view(torch.int64)
+    d_lens = d_in[off_lens:off_lens + 4 * B].view(torch.int32)
+    d_tab = d_in[off_tab:off_tab + tab_bytes].view(torch.int32).view(wl.tab.shape)
+    d_tab.copy_(torch.from_numpy(wl.tab))
     d_out = torch.empty((B, cfg.H_q, cfg.Dh), dtype=torch.float32, device=dev)
     ws = wl.workspace()
     err = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -603,19 +616,14 @@ def run_e2e(wl, cfg, warm, steps, args, world):
     def one(i):
         before = wl.lens.copy()
         s, l = wl.bookkeeping()
-        pin_slots.numpy()[:] = s
-        pin_lens.numpy()[:] = l
-        nb = 0
-        if np.any(before % P == 0):  # a page was added: refresh the table
-            pin_tab.numpy()[:] = wl.tab
-            d_tab.copy_(pin_tab, non_blocking=True)
-            nb += wl.tab.nbytes
-        d_slots.copy_(pin_slots, non_blocking=True)
-        d_lens.copy_(pin_lens, non_blocking=True)
-        d_q.copy_(host_q[i], non_blocking=True)
-        d_kn.copy_(host_kn[i], non_blocking=True)
-        d_vn.copy_(host_vn[i], non_blocking=True)
-        nb += s.nbytes + l.nbytes + cfg.elem_bytes * (host_q[i].numel() + 2 * host_kn[i].numel())
+        h = host_in[i].numpy()
+        h[off_slots:off_slots + 8 * B] = s.view(np.uint8)
+        h[off_lens:off_lens + 4 * B] = l.astype(np.int32).view(np.uint8)
+        nb = off_tab
+        if np.any(before % P == 0):  # a page was added: the block table travels too
+            h[off_tab:off_tab + tab_bytes] = wl.tab.view(np.uint8).reshape(-1)
+            nb = total
+        d_in[:nb].copy_(host_in[i][:nb], non_blocking=True)
         hot_path(K, args, cfg, wl.k_pages[0], wl.v_pages[0], d_kn, d_vn, d_slots, d_q, d_tab, d_lens, d_out, ws, err,
                  stream)
         host_out.copy_(d_out, non_blocking=True)
@@ -632,6 +640,8 @@ def run_e2e(wl, cfg, warm, steps, args, world):
         h2d_total[0] += one(i)
     end.record(stream)
     torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error flag {int(err.item())}")
     ms = max_over_ranks(start.elapsed_time(end), world)
     return {"value": replica_value(B, steps, world, ms), "unit": UNIT, "h2d_bytes_per_step": h2d_total[0] / steps,
             "d2h_bytes_per_step": host_out.numel() * 4, "ms_per_step": ms / steps}

@@ -338,7 +338,10 @@ int kv_append_fp8(void* k_pages, void* v_pages, const void* k_new, const void* v
  * E4M3 values are exact in fp16). Tensor-core kernel only (H_q / H_kv <= 64,
  * Dh in {64, 128}, page_size in {16, 32}); num_splits, workspace (same size
  * as paged_decode_workspace_bytes), errors and output as
- * paged_decode_attention. */
+ * paged_decode_attention, except that the automatic split count
+ * (num_splits = 0, B > 1) aims at half as many CTAs per SM, each moving half
+ * the bytes of a 16-bit page: paged_decode_num_splits reports the 16-bit
+ * count, an upper bound. */
 int paged_decode_attention_fp8(float* out, const void* q, int32_t q_dtype, const void* k_pages, const void* v_pages,
                                const float* k_scale, const float* v_scale, const int32_t* block_tables,
                                int32_t max_blocks, const int32_t* seq_lens, int32_t B, int32_t H_q, int32_t H_kv,

@@ -189,7 +189,11 @@ bool plan_group(int32_t g, int* GW, int* HS, int* NW, int* WP) {
 //    CTAs per slot so late short CTAs even out long ones, S = ceil(6 slots /
 //    (B H_kv)), with at least 16 pages per split; S = 1 once rows alone are
 //    that many.
-int resolve_splits(int32_t B, int32_t H_kv, int32_t max_blocks, int32_t num_splits, int32_t* S_out, int32_t* C_out) {
+//  * E4M3 K/V (kv_bytes == 1): a CTA moves half the bytes per page, so half
+//    as many CTAs per slot (8B-shaped layer: S = 2 / 3 / 4 / 6 -> 0.65 /
+//    0.64 / 0.62 / 0.58 of the copy peak).
+int resolve_splits(int32_t B, int32_t H_kv, int32_t max_blocks, int32_t num_splits, int32_t* S_out, int32_t* C_out,
+                   int kv_bytes = 2) {
     int32_t S = num_splits;
     if (S <= 0) {
         int sms = sm_count();
@@ -199,7 +203,8 @@ int resolve_splits(int32_t B, int32_t H_kv, int32_t max_blocks, int32_t num_spli
         if (B == 1) {
             S = static_cast<int32_t>(slots / rows > 1 ? slots / rows : 1);
         } else {
-            S = static_cast<int32_t>((6 * slots + rows - 1) / rows);
+            const int64_t per_slot = kv_bytes == 1 ? 3 : 6;
+            S = static_cast<int32_t>((per_slot * slots + rows - 1) / rows);
             const int32_t cap = max_blocks / 16 > 1 ? max_blocks / 16 : 1;
             if (S > cap) S = cap;
         }
@@ -438,7 +443,7 @@ int decode_impl(float* out, const void* q, const void* k_new, const void* v_new,
         plan_group(g, &GW, &HS, &NW, &WP);
     }
     int32_t S, C;
-    rc = resolve_splits(B, H_kv, max_blocks, num_splits, &S, &C);
+    rc = resolve_splits(B, H_kv, max_blocks, num_splits, &S, &C, elem_bytes(dtype));
     if (rc != KV_OK) return rc;
     const bool planned = planned_ok(mma, B, H_q, H_kv, num_splits);
 
