@@ -237,6 +237,23 @@ int kv_rope_append(void* k_pages, void* v_pages, void* q_out, const void* q, con
                    int32_t rope_style, int32_t B, int32_t H_q, int32_t H_kv, int32_t Dh, int32_t page_size,
                    int32_t num_pages, int32_t dtype, int* err_flag, void* stream);
 
+/* One launch for a layer's whole decode step ([CN-06] 6.1 order: rotate q
+ * and k by the new token's position, append k and v, attend): as
+ * paged_decode_attention_append, with the new token's k row and every query
+ * head rotated at position seq_lens[b] - 1 exactly as kv_rope_append does it
+ * (same cos_sin table, max_pos, rope_style; the stored k bits and the
+ * rotated q bits are the same), and q read unrotated from `q`.
+ * bf16 / fp16 K/V on the tensor-core kernel only (KV_ERR_UNSUPPORTED
+ * otherwise). A position outside [0, max_pos) sets KV_DEV_ERR_POSITION; that
+ * row's output is then undefined. */
+int paged_decode_attention_rope_append(float* out, const void* q, const void* k_new, const void* v_new,
+                                       void* k_pages, void* v_pages, const int32_t* block_tables, int32_t max_blocks,
+                                       const int32_t* seq_lens, const float* cos_sin, int32_t max_pos,
+                                       int32_t rope_style, int32_t B, int32_t H_q, int32_t H_kv, int32_t Dh,
+                                       int32_t page_size, int32_t num_pages, float scale, int32_t dtype,
+                                       int32_t num_splits, void* workspace, size_t ws_bytes, int* err_flag,
+                                       void* stream);
+
 /* Copy whole pages of both pools: for i < n, page src_pages[i] -> page
  * dst_pages[i] (all H_kv heads and page_size slots; src/dst are device int32
  * arrays), e.g. after kv_pool_cow_tails. A page id outside [0, num_pages)

@@ -64,6 +64,8 @@ struct DecodeParams {
     const int4* items;          // planned launch: {b, kvh, chunk, item} per CTA (nullable)
     const float* k_scale;       // E4M3 K/V: per-KV-head scales (read value = code * scale)
     const float* v_scale;
+    const float* cos_sin;       // fused rotary embedding (nullable): fp32 [max_pos][Dh], cos then sin
+    int32_t max_pos, rope_style;
     const int32_t* q_start;     // multi-token query: rows of sequence b are q_start[b] .. q_start[b+1]-1
     int32_t q_tile;             // multi-token query: chunk tokens per CTA
     const int32_t* plan;        // planned launch: [0] pages per chunk, [4 + b] item prefix

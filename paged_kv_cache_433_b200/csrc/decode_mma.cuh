@@ -28,12 +28,65 @@
 
 #include "decode_kernel.cuh"
 #include "fp8.cuh"
+#include "rope.cuh"
 
 #ifndef KVP_MMA_STAGE_BUDGET
 #define KVP_MMA_STAGE_BUDGET (96 * 1024)
 #endif
 
 namespace kvp {
+
+// Fused rotary embedding + append of the new token (position len - 1): the
+// rotated k row and the v row go to their slot exactly as kv_rope_append
+// writes them (same fp32 operations, same rounding). Lane l < Dh/16 rotates
+// the vector pair (l, l + Dh/16) (split halves) or (2l, 2l + 1)
+// (interleaved) of the k row; the next Dh/8 lanes copy the v row. Called by
+// one whole warp before it loads the page.
+template <int DT>
+__device__ __forceinline__ void append_new_token_rope(const DecodeParams& p, int b, int kvh, int len, int P, int DH,
+                                                      int lane) {
+    using V = RopeVec<DT>;
+    constexpr int N = V::kN;
+    const int pos = len - 1;
+    const int32_t page = p.block_tables[(int64_t)b * p.max_blocks + pos / P];
+    if (pos < 0 || pos >= p.max_pos) {
+        if (lane == 0) raise_err(p.err, KV_DEV_ERR_POSITION);
+    } else if (page >= 0 && page < p.num_pages) {
+        const int vpr = DH / N, upr = vpr / 2;
+        const int64_t dst_row = ((int64_t)page * p.H_kv + kvh) * P + pos % P;
+        const int64_t src_row = (int64_t)b * p.H_kv + kvh;
+        if (lane < upr) {
+            const uint4* src = static_cast<const uint4*>(p.k_new) + src_row * vpr;
+            uint4* dst = static_cast<uint4*>(const_cast<void*>(p.k_pages)) + dst_row * vpr;
+            const int va = p.rope_style == KV_ROPE_HALF ? lane : 2 * lane;
+            const int vb = p.rope_style == KV_ROPE_HALF ? lane + upr : 2 * lane + 1;
+            float xa[N], xb[N];
+            V::load(src[va], xa);
+            V::load(src[vb], xb);
+            const float* crow = p.cos_sin + (int64_t)pos * DH;
+            const int k0 = lane * N;
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+                if (p.rope_style == KV_ROPE_HALF) {
+                    rotate_pair(xa[i], xb[i], crow[k0 + i], crow[DH / 2 + k0 + i]);
+                } else if (i < N / 2) {
+                    rotate_pair(xa[2 * i], xa[2 * i + 1], crow[k0 + i], crow[DH / 2 + k0 + i]);
+                    rotate_pair(xb[2 * i], xb[2 * i + 1], crow[k0 + N / 2 + i], crow[DH / 2 + k0 + N / 2 + i]);
+                }
+            }
+            dst[va] = V::store(xa);
+            dst[vb] = V::store(xb);
+        } else if (lane < upr + vpr) {
+            const int c = lane - upr;
+            static_cast<uint4*>(const_cast<void*>(p.v_pages))[dst_row * vpr + c] =
+                static_cast<const uint4*>(p.v_new)[src_row * vpr + c];
+        }
+        fence_proxy_async_global();
+    } else if (lane == 0) {
+        raise_err(p.err, KV_DEV_ERR_PAGE_RANGE);
+    }
+    __syncwarp();
+}
 
 // EB: bytes per K/V element (2: bf16 / fp16; 1: E4M3). A token row of Dh
 // elements is loaded as boxes of at most 128 bytes (rows of 128 bytes use the
@@ -184,7 +237,12 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if constexpr (!kFP8 && !QM) {
-            if (p.k_new != nullptr && first + n_local == n_pages) append_new_token(p, b, kvh, len, P, DH * 2, lane);
+            if (p.k_new != nullptr && first + n_local == n_pages) {
+                if (p.cos_sin != nullptr)
+                    append_new_token_rope<KT>(p, b, kvh, len, P, DH, lane);
+                else
+                    append_new_token(p, b, kvh, len, P, DH * 2, lane);
+            }
         }
         const int32_t* row = p.block_tables + (int64_t)b * p.max_blocks + first;
         const int n_st = (n_local + PPS - 1) / PPS;  // stages of this CTA
@@ -301,6 +359,54 @@ __global__ void __launch_bounds__(32 * (NW + 1), 2)
                     qa[kk][rr + 2 * ch] = v;
                 }
             }
+        }
+    }
+
+    // Fused rotary embedding of q at position len - 1, with the same fp32 operations and rounding as
+    // kv_rope_append. In the fragment a register holds dims (d, d + 1), d = kk*16 + ch*8 + 2*quad; the
+    // split-halves partner d + Dh/2 sits in k-step kk + Dh/32 of the same thread.
+    if constexpr (!kFP8 && !QM) {
+        const int pos = len - 1;
+        if (p.cos_sin != nullptr && pos >= 0 && pos < p.max_pos) {
+            const float* crow = p.cos_sin + (int64_t)pos * DH;
+            auto unpack = [](uint32_t w, float& lo, float& hi) {
+                if constexpr (kBF16) {
+                    lo = __uint_as_float(w << 16);
+                    hi = __uint_as_float(w & 0xffff0000u);
+                } else {
+                    lo = __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xffffu)));
+                    hi = __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16)));
+                }
+            };
+#pragma unroll
+            for (int kk = 0; kk < C::kKSteps; ++kk)
+#pragma unroll
+                for (int ch = 0; ch < 2; ++ch) {
+                    const int d = kk * 16 + ch * 8 + 2 * quad;
+                    if (p.rope_style == KV_ROPE_HALF) {
+                        if (kk >= C::kKSteps / 2) continue;
+                        const float c0 = crow[d], c1 = crow[d + 1], s0 = crow[DH / 2 + d], s1 = crow[DH / 2 + d + 1];
+#pragma unroll
+                        for (int rr = 0; rr < 2; ++rr) {
+                            float x0, x1, y0, y1;
+                            unpack(qa[kk][rr + 2 * ch], x0, x1);
+                            unpack(qa[kk + C::kKSteps / 2][rr + 2 * ch], y0, y1);
+                            rotate_pair(x0, y0, c0, s0);
+                            rotate_pair(x1, y1, c1, s1);
+                            qa[kk][rr + 2 * ch] = pack2<kBF16>(x0, x1);
+                            qa[kk + C::kKSteps / 2][rr + 2 * ch] = pack2<kBF16>(y0, y1);
+                        }
+                    } else {
+                        const float c = crow[d / 2], s = crow[DH / 2 + d / 2];
+#pragma unroll
+                        for (int rr = 0; rr < 2; ++rr) {
+                            float x0, x1;
+                            unpack(qa[kk][rr + 2 * ch], x0, x1);
+                            rotate_pair(x0, x1, c, s);
+                            qa[kk][rr + 2 * ch] = pack2<kBF16>(x0, x1);
+                        }
+                    }
+                }
         }
     }
 

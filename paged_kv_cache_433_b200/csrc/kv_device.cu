@@ -414,7 +414,8 @@ int decode_impl(float* out, const void* q, const void* k_new, const void* v_new,
                 const void* v_pages, const int32_t* block_tables, int32_t max_blocks, const int32_t* seq_lens, int32_t B,
                 int32_t H_q, int32_t H_kv, int32_t Dh, int32_t page_size, int32_t num_pages, float scale, int32_t dtype,
                 int32_t num_splits, void* workspace, size_t ws_bytes, int* err_flag, void* stream,
-                int32_t q_dtype = -1, const float* k_scale = nullptr, const float* v_scale = nullptr) {
+                int32_t q_dtype = -1, const float* k_scale = nullptr, const float* v_scale = nullptr,
+                const float* cos_sin = nullptr, int32_t max_pos = 0, int32_t rope_style = 0) {
     int rc = check_shape(H_q, H_kv, Dh, page_size, dtype);
     if (rc != KV_OK) return rc;
     if (q_dtype < 0) q_dtype = dtype;
@@ -470,6 +471,10 @@ int decode_impl(float* out, const void* q, const void* k_new, const void* v_new,
     p.scale_log2 = scale * kLog2e;
     p.k_scale = k_scale;
     p.v_scale = v_scale;
+    p.cos_sin = cos_sin;
+    p.max_pos = max_pos;
+    p.rope_style = rope_style;
+    if (cos_sin != nullptr && !mma) return KV_ERR_UNSUPPORTED;  // the fused rotation lives in the tensor-core kernel
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     dim3 grid(static_cast<unsigned>(S), static_cast<unsigned>(H_kv), static_cast<unsigned>(B));
     cudaError_t e;
@@ -580,6 +585,22 @@ int paged_decode_attention_fp8(float* out, const void* q, int32_t q_dtype, const
     return decode_impl(out, q, nullptr, nullptr, k_pages, v_pages, block_tables, max_blocks, seq_lens, B, H_q, H_kv, Dh,
                        page_size, num_pages, scale, KV_DTYPE_FP8_E4M3, num_splits, workspace, ws_bytes, err_flag,
                        stream, q_dtype, k_scale, v_scale);
+}
+
+int paged_decode_attention_rope_append(float* out, const void* q, const void* k_new, const void* v_new,
+                                       void* k_pages, void* v_pages, const int32_t* block_tables, int32_t max_blocks,
+                                       const int32_t* seq_lens, const float* cos_sin, int32_t max_pos,
+                                       int32_t rope_style, int32_t B, int32_t H_q, int32_t H_kv, int32_t Dh,
+                                       int32_t page_size, int32_t num_pages, float scale, int32_t dtype,
+                                       int32_t num_splits, void* workspace, size_t ws_bytes, int* err_flag,
+                                       void* stream) {
+    if (dtype != KV_DTYPE_BF16 && dtype != KV_DTYPE_F16) return dtype == KV_DTYPE_F32 ? KV_ERR_UNSUPPORTED : KV_ERR_ARG;
+    if (rope_style != KV_ROPE_HALF && rope_style != KV_ROPE_INTERLEAVED) return KV_ERR_ARG;
+    if (B > 0 && (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new) || !cos_sin || max_pos <= 0))
+        return KV_ERR_ARG;
+    return decode_impl(out, q, k_new, v_new, k_pages, v_pages, block_tables, max_blocks, seq_lens, B, H_q, H_kv, Dh,
+                       page_size, num_pages, scale, dtype, num_splits, workspace, ws_bytes, err_flag, stream, dtype,
+                       nullptr, nullptr, cos_sin, max_pos, rope_style);
 }
 
 int paged_prefill_attention(float* out, const void* q, const int32_t* q_start, int32_t max_q_len,

@@ -81,6 +81,9 @@ SIGNATURES = [
     ("paged_decode_attention_fp8", ctypes.c_int,
      [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _sz, _vp,
       _vp]),
+    ("paged_decode_attention_rope_append", ctypes.c_int,
+     [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32,
+      _i32, _vp, _sz, _vp, _vp]),
     ("paged_prefill_attention", ctypes.c_int,
      [_vp, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp]),
     ("paged_decode_set_kernel", ctypes.c_int, [_i32]),
@@ -378,6 +381,30 @@ def paged_decode_attention_fp8(out, q, k_pages, v_pages, k_scale, v_scale, block
         0 if workspace is None else workspace.numel() * workspace.element_size(), _dev(err_flag, "err_flag", torch.int32),
         _stream(stream))
     _check("paged_decode_attention_fp8", rc)
+
+
+def paged_decode_attention_rope_append(out, q, k_new, v_new, k_pages, v_pages, block_tables, seq_lens, cos_sin,
+                                       scale: float, style: str = "half", num_splits: int = 0, workspace=None,
+                                       err_flag=None, stream=None) -> None:
+    """Rotate (q, the new k) at position seq_lens[b] - 1, append k / v, decode -- one launch (+ combine)."""
+    import torch
+
+    B, H_q, Dh = q.shape
+    num_pages, H_kv, P, Dh2 = k_pages.shape
+    assert Dh2 == Dh and v_pages.shape == k_pages.shape and tuple(out.shape) == (B, H_q, Dh)
+    assert tuple(k_new.shape) == (B, H_kv, Dh) and v_new.shape == k_new.shape and cos_sin.shape[1] == Dh
+    dt = k_pages.dtype
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr = _dev(workspace, "workspace")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib().paged_decode_attention_rope_append(
+        _dev(out, "out", torch.float32), _dev(q, "q", dt), _dev(k_new, "k_new", dt), _dev(v_new, "v_new", dt),
+        _dev(k_pages, "k_pages"), _dev(v_pages, "v_pages", dt), _dev(block_tables, "block_tables", torch.int32),
+        block_tables.shape[1], _dev(seq_lens, "seq_lens", torch.int32), _dev(cos_sin, "cos_sin", torch.float32),
+        cos_sin.shape[0], ROPE_STYLE[style], B, H_q, H_kv, Dh, P, num_pages, float(scale), _torch_dtype_code(k_pages),
+        num_splits, ws_ptr, ws_bytes, _dev(err_flag, "err_flag", torch.int32), _stream(stream))
+    _check("paged_decode_attention_rope_append", rc)
 
 
 def paged_prefill_attention(out, q, q_start, max_q_len: int, k_pages, v_pages, block_tables, seq_lens, scale: float,

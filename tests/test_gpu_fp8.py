@@ -193,3 +193,12 @@ def test_fp8_refusals():
         K.paged_decode_attention(out, q.view(torch.uint8).reshape(2, 8, 256)[..., :128].contiguous(), c.k_pages,
                                  c.v_pages, tab, lens, cfg.scale)
     torch.cuda.synchronize()
+
+
+def test_fp8_llama8b_full_size():
+    """The 8B-shaped layer at full size (B=64, lengths U[512, 4096]) with an E4M3 cache, automatic splits."""
+    cfg = W.LLAMA8B
+    c = Fp8Cache(cfg, W.cached_lengths(cfg))
+    out, ref, err = c.step(0)
+    assert err == 0
+    check_close(out, ref, "bf16", "fp8 8B full")

@@ -101,3 +101,16 @@ def test_prefill_refuses_fp32():
                                   torch.tensor([0, 1], dtype=torch.int32, device="cuda"), 1, k, k,
                                   torch.zeros((1, 2), dtype=torch.int32, device="cuda"),
                                   torch.ones(1, dtype=torch.int32, device="cuda"), 0.1)
+
+
+def test_prefill_bench_shape_sampled():
+    """The chunked-prefill workload the benchmark times (8 sequences x 512-token chunk over 4096 cached
+    tokens); sequences 0 and 7 are checked against the oracle."""
+    cfg = W.DecodeConfig("prefill-bench", "bf16", B=8, H_q=32, H_kv=8, Dh=128, page_size=16, seed=85)
+    totals, chunks = [4096 + 512] * 8, [512] * 8
+    got, q, q_start, st, lens = _run(cfg, totals, chunks)
+    for b in (0, 7):
+        rows = slice(int(q_start[b]), int(q_start[b + 1]))
+        ref = R.paged_prefill(q[rows], np.array([0, 512], np.int32), st.kp, st.vp, st.tab[b:b + 1], lens[b:b + 1],
+                              cfg.scale, "bf16")
+        check_close(got[rows], ref, "bf16", f"prefill bench shape, sequence {b}")

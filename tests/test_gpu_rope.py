@@ -96,3 +96,57 @@ def test_rope_append_error_bits():
     with pytest.raises(K.KvError):  # Dh * 2 bytes not a multiple of 32
         K.kv_rope_append(kp[..., :8].contiguous(), vp[..., :8].contiguous(), kn[..., :8].contiguous(),
                          kn[..., :8].contiguous(), slots, pos, table[:, :8].contiguous(), P)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("style", RP.STYLES)
+@pytest.mark.parametrize("splits", [1, 0])
+def test_fused_rope_append_decode(dtype, style, splits):
+    """paged_decode_attention_rope_append: pools bit-exact vs the oracle's rotate-then-append, output within the
+    attention tolerance of the oracle, and bit-identical to kv_rope_append followed by paged_decode_attention."""
+    from gpu_cases import build_cache, check_close
+    from oracle import reference as R
+
+    cfg = W.DecodeConfig(f"fused-rope-{dtype}-{style}", dtype, B=12, H_q=32, H_kv=8, Dh=128, page_size=16, seed=44)
+    lens = [15, 16, 1, 300, 47, 1000, 31, 32, 2047, 5, 64, 129]
+    st = build_cache(cfg, lens)
+    P = cfg.page_size
+    lens32 = st.lens.astype(np.int32).copy()
+    mlens = [int(x) for x in st.lens]
+    slots = st.pool.append_slots(st.tab, lens32)
+    mslots = st.mpool.append_slots(st.mtab, st.max_blocks, mlens)
+    assert list(slots) == mslots
+    positions = np.asarray(lens, np.int32)  # the new token's position = its cached length before the append
+    table = RP.rope_table(4096, cfg.Dh, 500000.0)
+    k_new, v_new = W.new_token_kv(cfg, 0, 0)
+    q = W.queries(cfg, 0, 0)
+    # oracle: rotate, append, fp64 decode
+    RP.rope_append(st.kp, st.vp, k_new, v_new, mslots, positions, table, style, dtype)
+    q_rot = RP.apply_rope(q, positions, table, style, dtype)
+    ref = R.paged_decode(q_rot, st.kp, st.vp, np.asarray(st.mtab, np.int32), np.asarray(mlens, np.int32), cfg.scale,
+                         dtype)
+    # product, fused, on a copy of the pools; then the two-step path on the original pools
+    kp2, vp2 = st.k_pages.clone(), st.v_pages.clone()
+    tab = torch.from_numpy(st.tab).cuda()
+    d_lens = torch.from_numpy(lens32).cuda()
+    d_table = torch.from_numpy(table).cuda()
+    nb = K.paged_decode_workspace_bytes(cfg.B, cfg.H_q, cfg.H_kv, cfg.Dh, st.max_blocks, P, splits)
+    ws = torch.zeros(max(nb, 16), dtype=torch.uint8, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.empty((cfg.B, cfg.H_q, cfg.Dh), dtype=torch.float32, device="cuda")
+    K.paged_decode_attention_rope_append(out, to_device(q, dtype), to_device(k_new, dtype), to_device(v_new, dtype), kp2,
+                                         vp2, tab, d_lens, d_table, cfg.scale, style=style, num_splits=splits,
+                                         workspace=ws, err_flag=err)
+    q_out = torch.empty_like(to_device(q, dtype))
+    K.kv_rope_append(st.k_pages, st.v_pages, to_device(k_new, dtype), to_device(v_new, dtype),
+                     torch.from_numpy(slots).cuda(), torch.from_numpy(positions).cuda(), d_table, P, style=style,
+                     q=to_device(q, dtype), q_out=q_out, err_flag=err)
+    out2 = torch.empty_like(out)
+    K.paged_decode_attention(out2, q_out, st.k_pages, st.v_pages, tab, d_lens, cfg.scale, num_splits=splits,
+                             workspace=ws, err_flag=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert np.array_equal(device_bits(kp2), st.kp) and np.array_equal(device_bits(vp2), st.vp), "fused pools"
+    assert np.array_equal(device_bits(q_out), q_rot), "rotated q"
+    check_close(out.cpu().numpy(), ref, dtype, "fused rope + append + decode")
+    assert torch.equal(out, out2), "fused launch differs from rotate-append then decode"
