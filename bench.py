@@ -230,7 +230,7 @@ class Workload:
         """Algorithmic bytes of one decode launch (one layer): K/V rows actually attended,
         q, fp32 out, block-table entries and seq_lens."""
         cfg = self.cfg
-        kv = int(np.sum(lens_after)) * cfg.H_kv * cfg.Dh * 2 * (1 if self.fp8 else cfg.elem_bytes)
+        kv = int(np.sum(lens_after)) * cfg.H_kv * cfg.Dh * 2 * (1 if getattr(self, "fp8", False) else cfg.elem_bytes)
         q = self.B * cfg.H_q * cfg.Dh * cfg.elem_bytes
         out = self.B * cfg.H_q * cfg.Dh * 4
         tables = int(np.sum(-(-lens_after // cfg.page_size))) * 4 + self.B * 4
@@ -802,7 +802,7 @@ class PagedState:
 
     def step_bytes(self, lens_after, fused=True):
         cfg = self.cfg
-        kv = int(np.sum(lens_after)) * cfg.H_kv * cfg.Dh * 2 * (1 if self.fp8 else cfg.elem_bytes)
+        kv = int(np.sum(lens_after)) * cfg.H_kv * cfg.Dh * 2 * (1 if getattr(self, "fp8", False) else cfg.elem_bytes)
         q = self.B * cfg.H_q * cfg.Dh * cfg.elem_bytes
         out = self.B * cfg.H_q * cfg.Dh * 4
         tables = int(np.sum(-(-np.asarray(lens_after) // self.P))) * 4 + self.B * 4
