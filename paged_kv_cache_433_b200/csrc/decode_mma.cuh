@@ -1,4 +1,8 @@
-// Paged decode attention on the tensor cores (bf16 / fp16 K/V), sm_100a.
+// Paged decode attention on the tensor cores (bf16 / fp16 / E4M3 K/V), sm_100a.
+// One kernel template serves four uses: single-token decode (the default),
+// E4M3 K/V (codes converted to f16 pairs in registers, two pages per stage),
+// multi-token query (chunked prefill: MMA rows are (token, head) pairs with a
+// per-row causal limit), and the fused rotate + append + decode step.
 //
 // Same contract and the same online (m, l, u) merge as decode_kernel.cuh
 // ("07｜KV Cache、FlashAttention与PagedAttention的内部过程", Q027; attention
