@@ -372,6 +372,52 @@ def test_device_entry_argument_checks_without_gpu():
     assert L.kv_append(None, None, None, None, None, 3, 8, 128, 16, 10, 9, None, None) == K.KV_ERR_ARG
 
 
+def test_extension_entry_argument_checks_without_gpu():
+    """E4M3, RoPE, fused and multi-token entry points refuse bad arguments before any CUDA call."""
+    L = K.lib()
+    # kv_append_fp8: source must be a 16/32-bit type, Dh a multiple of 16, scales and pointers present
+    assert L.kv_append_fp8(None, None, None, None, 3, None, None, None, 2, 8, 128, 16, 10, None, None) == K.KV_ERR_ARG
+    assert L.kv_append_fp8(None, None, None, None, 1, None, None, None, 2, 8, 120, 16, 10, None, None) == \
+        K.KV_ERR_UNSUPPORTED
+    assert L.kv_append_fp8(None, None, None, None, 1, None, None, None, 0, 8, 128, 16, 10, None, None) == K.KV_OK
+    assert L.kv_append_fp8(None, None, None, None, 1, None, None, None, 2, 8, 128, 16, 10, None, None) == K.KV_ERR_ARG
+    # paged_decode_attention_fp8: q must be bf16 / fp16, scales present
+    fp8 = [None, None, 0, None, None, None, None, None, 16, None, 2, 32, 8, 128, 16, 64, 0.1, 0, None, 0, None, None]
+    assert L.paged_decode_attention_fp8(*fp8) == K.KV_ERR_ARG  # q of fp32
+    fp8[2] = 1
+    assert L.paged_decode_attention_fp8(*fp8) == K.KV_ERR_ARG  # no scales
+    # kv_rope_append: style, q / q_out pairing, row size
+    rope = [None] * 9 + [64, 0, 2, 32, 8, 128, 16, 10, 1, None, None]
+    rope[9] = 64
+    assert L.kv_rope_append(*rope) == K.KV_ERR_ARG  # null pointers
+    rope[10] = 5
+    assert L.kv_rope_append(*rope) == K.KV_ERR_ARG  # unknown pairing
+    rope[10] = 0
+    rope[14] = 8
+    assert L.kv_rope_append(*rope) == K.KV_ERR_UNSUPPORTED  # 16-byte rows cannot hold vector pairs
+    rope[14], rope[11] = 128, 0
+    assert L.kv_rope_append(*rope) == K.KV_OK  # no tokens
+    # fused rotate + append + decode: 16-bit K/V only, table required
+    fused = [None] * 7 + [16, None, None, 64, 0, 2, 32, 8, 128, 16, 64, 0.1, 0, 0, None, 0, None, None]
+    assert L.paged_decode_attention_rope_append(*fused) == K.KV_ERR_UNSUPPORTED  # fp32 K/V
+    fused[19] = 1
+    assert L.paged_decode_attention_rope_append(*fused) == K.KV_ERR_ARG  # no k_new / table
+    # multi-token query: fp32 unsupported, shapes checked, nothing to do for empty batches
+    pre = [None, None, None, 16, None, None, None, 8, None, 2, 32, 8, 128, 16, 64, 0.1, 0, None, None]
+    assert L.paged_prefill_attention(*pre) == K.KV_ERR_UNSUPPORTED  # fp32
+    pre[16] = 1
+    pre[12] = 96
+    assert L.paged_prefill_attention(*pre) == K.KV_ERR_UNSUPPORTED  # Dh = 96
+    pre[12] = 128
+    pre[10] = 130
+    assert L.paged_prefill_attention(*pre) == K.KV_ERR_ARG  # H_q % H_kv != 0
+    pre[10] = 32
+    pre[3] = 0
+    assert L.paged_prefill_attention(*pre) == K.KV_OK  # no chunk rows
+    pre[3] = 16
+    assert L.paged_prefill_attention(*pre) == K.KV_ERR_ARG  # null pointers
+
+
 # ------------------------------------------------------------------ copy-on-write vs model
 @pytest.mark.parametrize("seed", range(4))
 def test_cow_tails_matches_model(seed):
