@@ -7,6 +7,8 @@ import socket
 
 import pytest
 
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
 
 def _free_port():
     with socket.socket() as s:
@@ -52,3 +54,21 @@ def test_two_gloo_ranks_take_the_slowest_rank():
     assert m0 == m1 == 15.0
     assert v0 == v1 == pytest.approx(64 * 100 * 2 / 0.015)
     assert o0 != o1
+
+
+def test_reference_arm_prints_one_contract_line():
+    """bench.py --impl reference (the fp64 oracle on the host cores) runs without a GPU and prints the
+    JSON line the driver compares against."""
+    import json
+    import subprocess
+    import sys
+
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "1"], capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "seq-steps/s" and d["value"] > 0 and d["higher_is_better"]
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
