@@ -272,7 +272,9 @@ int kv_copy_pages(void* k_pages, void* v_pages, const int32_t* src_pages, const 
  *   out: fp32 [B][H_q][Dh].   q: [B][H_q][Dh] of `dtype` (same as K/V).
  *   block_tables: int32 [B][max_blocks]; seq_lens: int32 [B] (0 -> zeros).
  *   Supported: Dh in {64, 128}; page_size in {16, 32}; H_q % H_kv == 0 with
- *   H_q / H_kv <= 32; dtype F32/BF16/F16. Else KV_ERR_UNSUPPORTED/KV_ERR_ARG.
+ *   H_q / H_kv <= 64 for bf16/fp16 on the tensor-core kernel, <= 32 for fp32
+ *   or the CUDA-core kernel; dtype F32/BF16/F16 (E4M3 pools go through
+ *   paged_decode_attention_fp8). Else KV_ERR_UNSUPPORTED/KV_ERR_ARG.
  *   num_splits: 1 = single pass; >1 = split each sequence's pages into that
  *   many contiguous ranges (split-KV) merged by a second combine kernel;
  *   0 = choose automatically from B, H_kv, max_blocks and the SM count;
