@@ -1,20 +1,25 @@
 #!/usr/bin/env python
 """Paged decode attention benchmark (one JSON line on rank 0).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2|3] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2..8] [--impl ours|reference]
 
 A step is one pass of the hot path over one batch: the host slot bookkeeping
 (page allocation at block boundaries), kv_append of the new token's K/V and
 paged_decode_attention (split-KV + combine where chosen).
 Workloads (synthetic, seeded; no dataset is involved):
   --config 2  Llama-3.1-8B-shaped decode layer, bf16 K/V: B=64, H_q=32, H_kv=8,
-              Dh=128, page 16, cached lengths U[512, 4096] (the default).
+              Dh=128, page 16, cached lengths U[512, 4096] (the default). On
+              one GPU the line also carries, under "configs", the 32K-context
+              and mixed-sweep records measured in the same process.
   --config 3  one 32K-token sequence, 32 layers, fp16 K/V (4 GiB cache); the
               32 per-layer calls of a step are replayed as one CUDA graph.
-`value` is device-timed with all step inputs resident in HBM; `e2e` repeats
-the loop through the same calls with the step's inputs copied from pinned
-host memory and the output read back every step. Multi-GPU runs are
-replicas (each rank its own batch, no data-path collective): weak scaling.
+  --config 4..8  shared prefix, mixed sweep, RoPE append, E4M3 cache, prefill.
+`value` is device-timed over exactly K steps with all step inputs resident in
+HBM; `sustained` replays the timed window for >= 1 s, five times, and gives
+the median; `e2e` repeats the loop through the same calls with the step's
+inputs copied from pinned host memory and the output read back every step.
+Multi-GPU runs are replicas (each rank its own batch, no data-path
+collective): weak scaling.
 """
 from __future__ import annotations
 
@@ -52,6 +57,10 @@ def parse():
     ap.add_argument("--chunk", type=int, default=512, help="config 8: chunk tokens per sequence")
     ap.add_argument("--splits", type=int, default=0, help="num_splits passed to paged_decode_attention (0 = auto)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-sustained", action="store_true",
+                    help="skip the >= 1 s repeats (median of 5) that follow the timed steps")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="default run: do not add the 32K-context and mixed-sweep records to the config-2 line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="config 3: launch the 32 layers without a CUDA graph")
@@ -306,6 +315,60 @@ def replica_value(seqs_per_rank, steps, world, elapsed_ms_max):
     return seqs_per_rank * steps * world / (elapsed_ms_max / 1e3)
 
 
+KERNEL_NAMES = {1: "cuda cores", 2: "warp mma (mma.sync)", 3: "tcgen05 (tensor memory)"}
+DATASHEET_HBM_GBS = 8000.0  # B200 HBM3e datasheet figure (~8 TB/s), shown beside the measured-copy fraction
+
+
+def kv_byte_variants(cfg, lens_after, B, kv_elem_bytes, S, C, plan_C=None, layers=1):
+    """Per-launch byte figures beside the algorithmic bytes (one layer unless `layers`):
+    K/V bytes when whole pages are read (page-rounded), and the split partials' fp32 (m, l, u) bytes written by
+    the decode kernel and read back by the combine (grid split: every non-empty split of a row; planned launch:
+    every chunk of a row that has more than one, with the device's chunk size plan_C)."""
+    P = cfg.page_size
+    lens_after = np.asarray(lens_after, np.int64)
+    pages = -(-lens_after // P)
+    rounded = int(pages.sum()) * P * cfg.H_kv * cfg.Dh * 2 * kv_elem_bytes
+    row_partial = cfg.g * (cfg.Dh + 2) * 4  # one (m, l, u) per query head of a (row, chunk)
+    if plan_C:
+        n_chunks = -(-pages // plan_C)
+        parts = int(np.sum(np.where(n_chunks > 1, n_chunks, 0))) * cfg.H_kv
+    elif S > 1:
+        parts = int(np.sum(-(-pages // C))) * cfg.H_kv  # splits that hold pages of the row
+    else:
+        parts = 0
+    return {"kv_bytes_page_rounded": layers * rounded, "partials_bytes_write_read": layers * 2 * parts * row_partial}
+
+
+def roofline_fracs(achieved_gbs, peak):
+    return {"frac": achieved_gbs / peak, "frac_datasheet": achieved_gbs / DATASHEET_HBM_GBS,
+            "datasheet_gbs": DATASHEET_HBM_GBS}
+
+
+def sustained_repeats(launch, n_window, stream, est_ms_per_call, local, args, repeats=5, min_s=1.0):
+    """Median of `repeats` device-timed runs, each at least `min_s` long: the recorded window of n_window
+    calls is replayed in order (launch(i), i cycling over the window), CUDA events on the launching stream;
+    nvidia-smi clocks sampled over all repeats."""
+    import torch
+
+    iters = max(n_window, int(math.ceil(min_s * 1e3 / max(est_ms_per_call, 1e-3))))
+    iters = -(-iters // n_window) * n_window
+    clk = ClockSampler(local, enabled=not args.no_clocks)
+    per_call = []
+    for _ in range(repeats):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for i in range(iters):
+            launch(i % n_window)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        per_call.append(e0.elapsed_time(e1) / iters)
+    clocks = clk.stop()
+    return {"ms_per_step_median": float(np.median(per_call)), "ms_per_step_repeats": per_call, "repeats": repeats,
+            "steps_per_repeat": iters, "repeat_s_median": float(np.median(per_call)) * iters / 1e3,
+            "clocks": clocks}
+
+
 # ---------------------------------------------------------------------------- our arm: config 2
 def run_layer_bench(args, world, rank, local):
     import torch
@@ -322,7 +385,8 @@ def run_layer_bench(args, world, rank, local):
     warm = args.warmup if args.warmup is not None else cfg.warmup_steps
     lens = W.cached_lengths(cfg)
     e2e_steps = 0 if args.no_e2e else steps
-    n_steps = warm + steps + (warm + e2e_steps if e2e_steps else 0)
+    # room for the timed pass and the e2e pass (which books one step ahead)
+    n_steps = warm + steps + (warm + e2e_steps + 1 if e2e_steps else 0)
     wl = Workload(cfg, lens, n_steps, rank, args.splits, sequential=args.page_order == "sequential")
     B, P = wl.B, cfg.page_size
     dev = torch.device("cuda")
@@ -343,7 +407,7 @@ def run_layer_bench(args, world, rank, local):
     out = torch.empty((B, cfg.H_q, cfg.Dh), dtype=torch.float32, device=dev)
     ws = wl.workspace()
     err = torch.zeros(1, dtype=torch.int32, device=dev)
-    S = K.paged_decode_num_splits(B, cfg.H_kv, wl.max_blocks, P, args.splits)
+    S, kernel_kind = K.paged_decode_launch_info(B, cfg.H_q, cfg.H_kv, cfg.Dh, wl.max_blocks, P, cfg.dtype, args.splits)
     stream = torch.cuda.current_stream()
     kp, vp = wl.k_pages[0], wl.v_pages[0]
 
@@ -372,6 +436,14 @@ def run_layer_bench(args, world, rank, local):
     bytes_per_launch = [wl.step_bytes(lens_list[i]) + append_bytes for i in range(warm, T1)]
     if int(err.item()) != 0:
         raise RuntimeError(f"device error flag {int(err.item())}")
+    plan_C = int(ws[:4].view(torch.int32).item()) if S == 0 else None
+    C = -(-wl.max_blocks // S) if S > 0 else 0
+
+    # ---- sustained: the timed window replayed for >= 1 s, median of 5 repeats (replaying step i rewrites
+    # step i's token at its own slot, so the cache stays that of the window)
+    sus = None
+    if not args.no_sustained:
+        sus = sustained_repeats(lambda i: step(warm + i), steps, stream, elapsed_ms / steps, local, args)
 
     # ---- end-to-end: same calls, inputs from pinned host memory, output read back each step
     e2e = None
@@ -385,6 +457,17 @@ def run_layer_bench(args, world, rank, local):
     achieved = mean_bytes / mean_dec_s / 1e9
     ratio = measured_traffic_ratio() if args.kernel != "simt" and P == 16 else None
     traffic = ratio * mean_bytes if ratio is not None else None
+    variants = kv_byte_variants(cfg, np.mean(np.stack(lens_list[warm:T1]), axis=0), B, cfg.elem_bytes, S, C, plan_C)
+    roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", **roofline_fracs(achieved, peak),
+            "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS hbm_gbs)" if peak_kind == "measured" else "fallback",
+            "traffic": traffic,
+            "traffic_source": ("ncu dram bytes of the decode kernel (profiles/" + os.path.basename(PROFILE_DECODE)
+                               + "), scaled to this run's algorithmic bytes") if traffic else None,
+            "kernel": "paged_decode_attention" + (" (split + combine)" if S != 1 else " (single pass)"),
+            "bytes_per_launch": mean_bytes, "launch_us": mean_dec_s * 1e6, **variants}
+    if sus is not None:
+        sus["frac_median"] = mean_bytes / (sus["ms_per_step_median"] / 1e3) / 1e9 / peak
+        sus["value_median"] = replica_value(B, 1, world, sus["ms_per_step_median"])
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps, "warmup": warm,
         "ms_per_step": elapsed_ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -392,15 +475,11 @@ def run_layer_bench(args, world, rank, local):
         "config": {"workload": cfg.name, "B": B, "H_q": cfg.H_q, "H_kv": cfg.H_kv, "Dh": cfg.Dh, "page_size": P,
                    "layers": 1, "num_splits": S, "page_order": args.page_order, "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
                    "l2": "inputs larger than L2 (K/V working set %.0f MB > 126 MB L2); no flush" % (mean_bytes / 1e6)},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS hbm_gbs)" if peak_kind == "measured" else "fallback",
-                     "traffic": traffic,
-                     "traffic_source": ("ncu dram bytes of the decode kernel (profiles/" + os.path.basename(PROFILE_DECODE)
-                                        + "), scaled to this run's algorithmic bytes") if traffic else None, "kernel": "paged_decode_attention" + (" (split + combine)" if S > 1 else " (single pass)"),
-                     "bytes_per_launch": mean_bytes, "launch_us": mean_dec_s * 1e6},
+        "roofline": roof,
         "gpu_launches": steps * launches_per_call(S, args),
         "e2e": e2e,
         "clocks": clocks,
+        "sustained": sus,
     }
     return res
 
@@ -435,7 +514,7 @@ def run_fp8_bench(args, world, rank, local):
     out = torch.empty((B, cfg.H_q, cfg.Dh), dtype=torch.float32, device=dev)
     ws = wl.workspace()
     err = torch.zeros(1, dtype=torch.int32, device=dev)
-    S = K.paged_decode_num_splits(B, cfg.H_kv, wl.max_blocks, P, args.splits)
+    S, kernel_kind = K.paged_decode_launch_info(B, cfg.H_q, cfg.H_kv, cfg.Dh, wl.max_blocks, P, cfg.dtype, args.splits)
     stream = torch.cuda.current_stream()
     kp, vp = wl.k_pages[0], wl.v_pages[0]
 
@@ -574,10 +653,11 @@ def peaks_tensor():
 
 
 def run_e2e(wl, cfg, warm, steps, args, world):
-    """Each step: host bookkeeping, one H2D copy of the step's inputs packed in a pinned staging buffer
-    (q, k_new, v_new, slots, lengths, and the block table when a page was added), kv_append +
-    paged_decode_attention (fused by default), D2H of the fp32 output, wait for it. Steps are serial, as in a
-    decode loop whose next input depends on this step's output."""
+    """Each step: one H2D copy of the step's inputs packed in a pinned staging buffer (q, k_new, v_new, slots,
+    lengths, and the block table when a page was added), kv_append + paged_decode_attention (fused by default),
+    D2H of the fp32 output, wait for it. Steps are serial, as in a decode loop whose next input depends on this
+    step's output; only the host slot bookkeeping of the next step (which does not depend on the output) is done
+    while the device runs this one."""
     import torch
 
     K = wl.K
@@ -592,7 +672,7 @@ def run_e2e(wl, cfg, warm, steps, args, world):
     off_tab = (off_lens + 4 * B + 15) // 16 * 16
     tab_bytes = wl.tab.nbytes
     total = off_tab + tab_bytes
-    host_in = [torch.empty(total, dtype=torch.uint8).pin_memory() for _ in range(n)]
+    host_in = [torch.empty(total, dtype=torch.uint8).pin_memory() for _ in range(n + 1)]
     gen = torch.Generator().manual_seed(cfg.seed + 77)
     for i in range(n):  # step inputs prepared before timing (q, k_new, v_new as the model would produce them)
         h = host_in[i]
@@ -611,44 +691,53 @@ def run_e2e(wl, cfg, warm, steps, args, world):
     ws = wl.workspace()
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
-    h2d_total = [0]
 
-    def one(i):
+    def prep(i):
+        """Host step a1 for step i, packed into its staging buffer; returns the bytes to copy."""
         before = wl.lens.copy()
         s, l = wl.bookkeeping()
         h = host_in[i].numpy()
         h[off_slots:off_slots + 8 * B] = s.view(np.uint8)
         h[off_lens:off_lens + 4 * B] = l.astype(np.int32).view(np.uint8)
-        nb = off_tab
         if np.any(before % P == 0):  # a page was added: the block table travels too
             h[off_tab:off_tab + tab_bytes] = wl.tab.view(np.uint8).reshape(-1)
-            nb = total
+            return total
+        return off_tab
+
+    def one(i, nb):
         d_in[:nb].copy_(host_in[i][:nb], non_blocking=True)
         hot_path(K, args, cfg, wl.k_pages[0], wl.v_pages[0], d_kn, d_vn, d_slots, d_q, d_tab, d_lens, d_out, ws, err,
                  stream)
         host_out.copy_(d_out, non_blocking=True)
+        nxt = prep(i + 1)  # overlaps the device work of step i
         stream.synchronize()
-        return nb
+        return nxt
 
+    nb = prep(0)
     for i in range(warm):
-        one(i)
+        nb = one(i, nb)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
+    h2d = 0
     start.record(stream)
     for i in range(warm, n):
-        h2d_total[0] += one(i)
+        h2d += nb
+        nb = one(i, nb)
     end.record(stream)
     torch.cuda.synchronize()
     if int(err.item()) != 0:
         raise RuntimeError(f"device error flag {int(err.item())}")
     ms = max_over_ranks(start.elapsed_time(end), world)
-    return {"value": replica_value(B, steps, world, ms), "unit": UNIT, "h2d_bytes_per_step": h2d_total[0] / steps,
-            "d2h_bytes_per_step": host_out.numel() * 4, "ms_per_step": ms / steps}
+    return {"value": replica_value(B, steps, world, ms), "unit": UNIT, "h2d_bytes_per_step": h2d / steps,
+            "d2h_bytes_per_step": host_out.numel() * 4, "ms_per_step": ms / steps,
+            "copies_declared": True}
 
 
 # ---------------------------------------------------------------------------- our arm: config 3
 def run_long_bench(args, world, rank, local):
+    """One 32K-token sequence, 32 layers (fp16, 4 GiB cache): a step is 32 x (append + decode + combine),
+    captured once as a CUDA graph that reads its inputs from one staging buffer and replayed every step."""
     import torch
 
     from paged_kv_cache_433_b200 import kvpaged as K
@@ -660,7 +749,9 @@ def run_long_bench(args, world, rank, local):
     L = cfg.layers
     lens = W.cached_lengths(cfg)
     T1 = warm + steps
-    wl = Workload(cfg, lens, T1 + 1, rank, args.splits, layers=L, sequential=args.page_order == "sequential")
+    e2e_steps = 0 if args.no_e2e else steps
+    wl = Workload(cfg, lens, T1 + 1 + (warm + e2e_steps + 1 if e2e_steps else 0), rank, args.splits, layers=L,
+                  sequential=args.page_order == "sequential")
     B, P = wl.B, cfg.page_size
     dev = torch.device("cuda")
     slot_list, lens_list = [], []
@@ -668,20 +759,32 @@ def run_long_bench(args, world, rank, local):
         s, l = wl.bookkeeping()
         slot_list.append(s)
         lens_list.append(l)
+    eb = cfg.elem_bytes
+    # staging layout of one step's inputs: q, k_new, v_new of every layer, slots, lengths, block table
+    nq, nkv = L * B * cfg.H_q * cfg.Dh * eb, L * B * cfg.H_kv * cfg.Dh * eb
+    off_kn, off_vn, off_slots = nq, nq + nkv, nq + 2 * nkv
+    off_lens = off_slots + 8 * B
+    off_tab = (off_lens + 4 * B + 15) // 16 * 16
+    tab_bytes = wl.tab.nbytes
+    total = off_tab + tab_bytes
+    d_stage = torch.empty(total, dtype=torch.uint8, device=dev)
+    cur = {"q": d_stage[:nq].view(wl.dt).view(L, B, cfg.H_q, cfg.Dh),
+           "kn": d_stage[off_kn:off_kn + nkv].view(wl.dt).view(L, B, cfg.H_kv, cfg.Dh),
+           "vn": d_stage[off_vn:off_vn + nkv].view(wl.dt).view(L, B, cfg.H_kv, cfg.Dh),
+           "slots": d_stage[off_slots:off_slots + 8 * B].view(torch.int64),
+           "lens": d_stage[off_lens:off_lens + 4 * B].view(torch.int32)}
+    tab_dev = d_stage[off_tab:].view(torch.int32).view(wl.tab.shape)
+    tab_dev.copy_(torch.from_numpy(wl.tab))
     slots_dev = torch.from_numpy(np.stack(slot_list)).to(dev)
     lens_dev = torch.from_numpy(np.stack(lens_list)).to(dev)
-    tab_dev = torch.from_numpy(wl.tab).to(dev)
     q_dev = torch.randn((T1, L, B, cfg.H_q, cfg.Dh), generator=wl.gen, device=dev).to(wl.dt)
     kn_dev = torch.randn((T1, L, B, cfg.H_kv, cfg.Dh), generator=wl.gen, device=dev).to(wl.dt)
     vn_dev = torch.randn((T1, L, B, cfg.H_kv, cfg.Dh), generator=wl.gen, device=dev).to(wl.dt)
     out = torch.empty((L, B, cfg.H_q, cfg.Dh), dtype=torch.float32, device=dev)
     ws = wl.workspace()
     err = torch.zeros(1, dtype=torch.int32, device=dev)
-    S = K.paged_decode_num_splits(B, cfg.H_kv, wl.max_blocks, P, args.splits)
+    S, kernel_kind = K.paged_decode_launch_info(B, cfg.H_q, cfg.H_kv, cfg.Dh, wl.max_blocks, P, cfg.dtype, args.splits)
     side = torch.cuda.Stream()
-    # Step inputs are addressed through one staging slot so the captured graph replays any step.
-    cur = {"slots": torch.empty_like(slots_dev[0]), "lens": torch.empty_like(lens_dev[0]),
-           "q": torch.empty_like(q_dev[0]), "kn": torch.empty_like(kn_dev[0]), "vn": torch.empty_like(vn_dev[0])}
 
     def layers_pass(stream):
         for layer in range(L):
@@ -706,10 +809,14 @@ def run_long_bench(args, world, rank, local):
         with torch.cuda.graph(graph, stream=side):
             layers_pass(side)
         torch.cuda.synchronize()
-    # the warm-up pass above consumed step 0's slots: rebuild state by replaying from step 0
-    for i in range(warm):
+
+    def run_step(i):
         stage(i, stream)
         graph.replay() if graph is not None else layers_pass(stream)
+
+    # the warm-up pass above consumed step 0's slots: rebuild state by replaying from step 0
+    for i in range(warm):
+        run_step(i)
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     stage_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
@@ -730,10 +837,70 @@ def run_long_bench(args, world, rank, local):
     pass_ms = [a.elapsed_time(b) for a, b in stage_ev]
     if int(err.item()) != 0:
         raise RuntimeError(f"device error flag {int(err.item())}")
+    sus = None
+    if not args.no_sustained:
+        sus = sustained_repeats(lambda i: run_step(warm + i), steps, stream, elapsed_ms / steps, local, args)
+    C = -(-wl.max_blocks // S) if S > 0 else 0
+
+    # ---- end-to-end: each step's inputs (all 32 layers) from one pinned buffer, outputs read back
+    e2e = None
+    if e2e_steps and graph is not None:
+        n = warm + e2e_steps
+        host_in = [torch.empty(total, dtype=torch.uint8).pin_memory() for _ in range(n + 1)]
+        gen = torch.Generator().manual_seed(cfg.seed + 77)
+        for i in range(n):
+            host_in[i][:off_slots].view(wl.dt).copy_(torch.randn(off_slots // eb, generator=gen).to(wl.dt))
+        host_out = torch.empty(tuple(out.shape), dtype=torch.float32).pin_memory()
+
+        def prep(i):
+            before = wl.lens.copy()
+            s_, l_ = wl.bookkeeping()
+            h = host_in[i].numpy()
+            h[off_slots:off_slots + 8 * B] = s_.view(np.uint8)
+            h[off_lens:off_lens + 4 * B] = l_.astype(np.int32).view(np.uint8)
+            if np.any(before % P == 0):
+                h[off_tab:off_tab + tab_bytes] = wl.tab.view(np.uint8).reshape(-1)
+                return total
+            return off_tab
+
+        def one(i, nb):
+            d_stage[:nb].copy_(host_in[i][:nb], non_blocking=True)
+            graph.replay()
+            host_out.copy_(out, non_blocking=True)
+            nxt = prep(i + 1)
+            stream.synchronize()
+            return nxt
+
+        nb = prep(0)
+        for i in range(warm):
+            nb = one(i, nb)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        h2d = 0
+        e0.record(stream)
+        for i in range(warm, n):
+            h2d += nb
+            nb = one(i, nb)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if int(err.item()) != 0:
+            raise RuntimeError(f"device error flag {int(err.item())}")
+        ms = max_over_ranks(e0.elapsed_time(e1), world)
+        e2e = {"value": replica_value(B, e2e_steps, world, ms), "unit": UNIT, "h2d_bytes_per_step": h2d / e2e_steps,
+               "d2h_bytes_per_step": host_out.numel() * 4, "ms_per_step": ms / e2e_steps, "copies_declared": True,
+               "path": "one H2D of the step's packed inputs, the captured 32-layer graph, D2H of all outputs"}
     bytes_step = [L * wl.step_bytes(lens_list[i]) for i in range(warm, T1)]
     value = replica_value(B, steps, world, elapsed_ms)
     peak, peak_kind = peaks()
-    achieved = float(np.mean(bytes_step)) / (float(np.mean(pass_ms)) / 1e3) / 1e9
+    mean_bytes = float(np.mean(bytes_step))
+    achieved = mean_bytes / (float(np.mean(pass_ms)) / 1e3) / 1e9
+    variants = kv_byte_variants(cfg, np.mean(np.stack(lens_list[warm:T1]), axis=0), B, cfg.elem_bytes, S, C,
+                                layers=L)
+    if sus is not None:
+        sus["frac_median"] = mean_bytes / (sus["ms_per_step_median"] / 1e3) / 1e9 / peak
+        sus["value_median"] = replica_value(B, 1, world, sus["ms_per_step_median"])
+        sus["note"] = "each repeat: staging copies + graph replay per step, back to back"
     return {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps, "warmup": warm,
         "ms_per_step": elapsed_ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -741,14 +908,16 @@ def run_long_bench(args, world, rank, local):
         "config": {"workload": cfg.name, "B": B, "T": int(lens[0]), "layers": L, "H_q": cfg.H_q, "H_kv": cfg.H_kv,
                    "Dh": cfg.Dh, "page_size": P, "num_splits": S, "cuda_graph": graph is not None,
                    "l2": "inputs larger than L2 (4 GiB cache); no flush"},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     **roofline_fracs(achieved, peak),
                      "peak_source": f"{peak_kind} copy bandwidth", "traffic": None,
                      "kernel": ("32 x (paged_decode_attention_append + combine) per step" if args.append == "fused"
                                 else "32 x (kv_append + paged_decode_attention + combine) per step"),
-                     "bytes_per_step": float(np.mean(bytes_step)), "pass_us": float(np.mean(pass_ms)) * 1e3},
+                     "bytes_per_step": mean_bytes, "pass_us": float(np.mean(pass_ms)) * 1e3, **variants},
         "gpu_launches": steps * L * launches_per_call(S, args),
-        "e2e": None,
+        "e2e": e2e,
         "clocks": clocks,
+        "sustained": sus,
     }
 
 
@@ -812,7 +981,8 @@ class PagedState:
 
 def time_steps(args, st, steps, warm, before_step=None):
     """Run warm + steps decode steps on `st`; each step: optional untimed host work (before_step),
-    bookkeeping + uploads (untimed), then the timed append + decode call. Returns per-step (ms, bytes)."""
+    bookkeeping + uploads (untimed), then the timed append + decode call. Returns per-step (ms, bytes) and a
+    closure that re-issues the last step's call (same inputs), for the sustained repeats."""
     import torch
 
     K, cfg = st.K, st.cfg
@@ -823,8 +993,11 @@ def time_steps(args, st, steps, warm, before_step=None):
     nb = K.paged_decode_workspace_bytes(st.B, cfg.H_q, cfg.H_kv, cfg.Dh, st.max_blocks, st.P, args.splits)
     ws = torch.zeros(max(nb, 16), dtype=torch.uint8, device=dev)
     res = []
-    S = K.paged_decode_num_splits(st.B, cfg.H_kv, st.max_blocks, st.P, args.splits)
+    S, st.kernel_kind = K.paged_decode_launch_info(st.B, cfg.H_q, cfg.H_kv, cfg.Dh, st.max_blocks, st.P, cfg.dtype,
+                                                    args.splits)
     st.launches_per_step = launches_per_call(S, args)
+    st.splits_used = S
+    last = None
     for i in range(warm + steps):
         if before_step is not None:
             before_step(i)
@@ -841,9 +1014,16 @@ def time_steps(args, st, steps, warm, before_step=None):
         torch.cuda.synchronize()
         if i >= warm:
             res.append((ev[0].elapsed_time(ev[1]), st.step_bytes(st.lens, args.append == "fused")))
+        last = (kn, vn, d_slots, q, d_tab, d_lens)
     if int(err.item()) != 0:
         raise RuntimeError(f"device error flag {int(err.item())}")
-    return res
+    st.plan_C = int(ws[:4].view(torch.int32).item()) if S == 0 else None
+
+    def again(_i, last=last):
+        kn, vn, d_slots, q, d_tab, d_lens = last
+        hot_path(K, args, cfg, st.k_pages, st.v_pages, kn, vn, d_slots, q, d_tab, d_lens, out, ws, err, stream)
+
+    return res, again
 
 
 def run_prefix_bench(args, world, rank, local):
@@ -875,7 +1055,7 @@ def run_prefix_bench(args, world, rank, local):
         ix.register(st.pool, toks, row)
         st.fill(b, len(hit) * P, len(toks) - len(hit) * P)
         hits += len(hit)
-    res = time_steps(args, st, steps, warm)
+    res, _ = time_steps(args, st, steps, warm)
     ms = float(np.sum([r[0] for r in res]))
     logical = float(np.mean([r[1] for r in res]))
     unique = (W.PREFIX_LEN + float(np.sum(st.lens - W.PREFIX_LEN))) * cfg.H_kv * cfg.Dh * 2 * cfg.elem_bytes
@@ -899,7 +1079,11 @@ def run_prefix_bench(args, world, rank, local):
 def run_mixed_bench(args, world, rank, local):
     """Mixed continuous-batching sweep: B=256, log-normal lengths, H_kv in {1, 8, 32}, P in {16, 32}; before
     every step each sequence exits with probability 1/32 and a new one is admitted in its row (pages freed /
-    allocated on the host, its K/V written outside the timed region); the timed part is append + decode."""
+    allocated on the host, its K/V written outside the timed region); the timed part is append + decode.
+    Per point: the device-timed steps with their clocks, and (sustained) the last step's call repeated
+    back to back for >= 1 s, median of 5 repeats."""
+    import torch
+
     from paged_kv_cache_433_b200 import workloads as W
 
     steps = args.steps if args.steps is not None else 20
@@ -911,6 +1095,8 @@ def run_mixed_bench(args, world, rank, local):
     if args.mixed_point:
         h, p = (int(x) for x in args.mixed_point.split(","))
         pts = [(h, p)]
+    peak, _ = peaks()
+    stream = torch.cuda.current_stream()
     for H_kv, P in pts:
         cfg = W.mixed_config(H_kv, P)
         lens = W.cached_lengths(cfg)
@@ -927,22 +1113,33 @@ def run_mixed_bench(args, world, rank, local):
                 st.release(int(b))
                 st.admit(int(b), int(L))
 
-        res = time_steps(args, st, steps, warm, before_step=churn)
+        clk = ClockSampler(local, enabled=not args.no_clocks)
+        res, again = time_steps(args, st, steps, warm, before_step=churn)
+        clocks = clk.stop()
         ms = float(np.sum([r[0] for r in res]))
         byts = float(np.sum([r[1] for r in res]))
-        peak, _ = peaks()
-        points.append({"H_kv": H_kv, "page_size": P, "seq_steps_per_s": cfg.B * steps / (ms / 1e3),
-                       "GBps": byts / (ms / 1e3) / 1e9, "frac": byts / (ms / 1e3) / 1e9 / peak,
-                       "us_per_step": ms / steps * 1e3, "mean_len": float(np.mean(st.lens))})
+        S = st.splits_used
+        C = -(-max_blocks // S) if S > 0 else 0
+        variants = kv_byte_variants(cfg, st.lens, cfg.B, cfg.elem_bytes, S, C, st.plan_C)
+        pt = {"H_kv": H_kv, "page_size": P, "seq_steps_per_s": cfg.B * steps / (ms / 1e3),
+              "GBps": byts / (ms / 1e3) / 1e9, "frac": byts / (ms / 1e3) / 1e9 / peak,
+              "us_per_step": ms / steps * 1e3, "mean_len": float(np.mean(st.lens)),
+              "launch": "planned" if S == 0 else f"grid split S={S}", "plan_chunk_pages": st.plan_C,
+              "kernel": KERNEL_NAMES.get(st.kernel_kind, str(st.kernel_kind)),
+              "bytes_per_step": byts / steps, **variants, "clocks": clocks}
+        if not args.no_sustained:
+            sus = sustained_repeats(again, 1, stream, ms / steps, local, args)
+            last_bytes = res[-1][1]
+            sus["frac_median"] = last_bytes / (sus["ms_per_step_median"] / 1e3) / 1e9 / peak
+            sus["note"] = "the last step's append + decode call repeated back to back"
+            pt["sustained"] = sus
+        points.append(pt)
         tot_ms += ms
         tot_seq += cfg.B * steps
         launches += steps * st.launches_per_step
         tot_bytes += byts
         del st
-        import torch
-
         torch.cuda.empty_cache()
-    peak, _ = peaks()
     achieved = tot_bytes / (tot_ms / 1e3) / 1e9
     return {
         "metric": METRIC, "value": tot_seq * world / (max_over_ranks(tot_ms, world) / 1e3), "unit": UNIT,
@@ -951,9 +1148,10 @@ def run_mixed_bench(args, world, rank, local):
         "data": "synthetic (seeded log-normal lengths, churn 1/32 per step; N(0,1) K/V, q)",
         "config": {"workload": "mixed-bf16-B256-lognormal1024-sweep", "B": 256, "H_q": 32, "Dh": 128,
                    "points": "H_kv x page_size = {1,8,32} x {16,32}", "l2": "inputs larger than L2; no flush"},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": None},
-        "sweep": points, "gpu_launches": launches, "e2e": None, "clocks": None,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     **roofline_fracs(achieved, peak), "traffic": None},
+        "sweep": points, "gpu_launches": launches, "e2e": None,
+        "clocks": {"per_point": "see sweep[i].clocks"},
     }
 
 
@@ -1012,6 +1210,42 @@ def cpu_baseline(budget_s=10.0):
     return {"value": B * runs / dt, "unit": UNIT, "cores": o.cores(), "kind": "oracle",
             "sample": f"{runs} full decode steps of the 64-sequence Llama-3.1-8B-shaped layer (bf16 K/V, fp64 math), "
                       f"{dt:.1f} s"}
+
+
+def oracle_rows_baseline(cfg, rows, row_lens, budget_s=10.0, layers_per_step=1, what=""):
+    """The fp64 oracle as it stands, timed on the host cores over a bounded sample: the K/V of the given rows
+    (one layer) drawn from the seeded host generators into a compact pool, one decode of those rows repeated
+    for ~budget_s. value = sequences decoded per second / layers_per_step (a step covers every layer)."""
+    from oracle import reference as R
+    from paged_kv_cache_433_b200 import workloads as W
+
+    P = cfg.page_size
+    npg = [-(-int(n) // P) for n in row_lens]
+    kp = np.zeros((sum(npg), cfg.H_kv, P, cfg.Dh), np.uint16 if cfg.dtype != "fp32" else np.float32)
+    vp = np.zeros_like(kp)
+    tab = np.full((len(rows), max(npg)), -1, np.int32)
+    first = 0
+    for i, (b, n) in enumerate(zip(rows, row_lens)):
+        tab[i, :npg[i]] = np.arange(first, first + npg[i], dtype=np.int32)
+        first += npg[i]
+        kr, vr = W.kv_rows(cfg, 0, int(b), int(n))
+        R.scatter_to_pages(kp, tab[i], kr)
+        R.scatter_to_pages(vp, tab[i], vr)
+    q = W.queries(cfg, 0, 0)[np.asarray(rows)]
+    lens = np.asarray(row_lens, np.int32)
+    t0 = time.perf_counter()
+    runs = 0
+    while True:
+        R.paged_decode(q, kp, vp, tab, lens, cfg.scale, cfg.dtype)
+        runs += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": len(rows) * runs / dt / layers_per_step, "unit": UNIT, "cores": R.max_threads(),
+            "kind": "oracle",
+            "sample": f"{runs} decodes of {len(rows)} row(s) of {what or cfg.name} (one layer"
+                      f"{f' of {layers_per_step}, scaled by 1/{layers_per_step}' if layers_per_step > 1 else ''}; "
+                      f"fp64 over {cfg.dtype} K/V), {dt:.1f} s"}
 
 
 def run_reference(args):
@@ -1124,6 +1358,36 @@ def run_rope_bench(args, world, rank, local):
     }
 
 
+def W_mod():
+    from paged_kv_cache_433_b200 import workloads as W
+
+    return W
+
+
+def args_for(args, **kw):
+    """A copy of the parsed arguments with some fields replaced (the sub-records use their own step counts)."""
+    import copy
+
+    a = copy.copy(args)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def long_context_baseline(W):
+    """Oracle baseline of the 32K-context step: one layer (of 32) of one step, scaled by 1/32."""
+    cfg = W.LONG32K
+    return oracle_rows_baseline(cfg, [0], [W.LONG_T + 1], budget_s=10.0, layers_per_step=cfg.layers)
+
+
+def mixed_baseline(W):
+    """Oracle baseline of the mixed sweep: 16 rows of the GQA point (H_kv = 8, P = 16) at their log-normal lengths."""
+    cfg = W.mixed_config(8, 16)
+    lens = W.cached_lengths(cfg) + 1
+    rows = list(range(16))
+    return oracle_rows_baseline(cfg, rows, lens[rows], budget_s=10.0, what=cfg.name + " (16 rows)")
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -1139,8 +1403,32 @@ def main():
     run = {2: run_layer_bench, 3: run_long_bench, 4: run_prefix_bench, 5: run_mixed_bench, 6: run_rope_bench,
            7: run_fp8_bench, 8: run_prefill_bench}[args.config]
     res = run(args, world, rank, local)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config == 2:
+    base = rank == 0 and world == 1 and not args.no_cpu_baseline
+    if base and args.config == 2:
         res["cpu_baseline"] = cpu_baseline()
+    if base:
+        from paged_kv_cache_433_b200 import workloads as W
+
+        if args.config == 3:
+            res["cpu_baseline"] = long_context_baseline(W)
+        elif args.config == 4:
+            lens = W.cached_lengths(W.SHARED_PREFIX) + 1
+            res["cpu_baseline"] = oracle_rows_baseline(W.SHARED_PREFIX, [0, 1, 2, 3], lens[:4], budget_s=10.0)
+        elif args.config == 5:
+            res["cpu_baseline"] = mixed_baseline(W)
+    if args.config == 2 and world == 1 and not args.no_extra:
+        # the other gated workload and the sweep, measured in the same process (sub-records)
+        import torch
+
+        torch.cuda.empty_cache()
+        long = run_long_bench(args_for(args, steps=None, warmup=None), world, rank, local)
+        if base:
+            long["cpu_baseline"] = long_context_baseline(W_mod())
+        torch.cuda.empty_cache()
+        mixed = run_mixed_bench(args_for(args, steps=20, warmup=3), world, rank, local)
+        if base:
+            mixed["cpu_baseline"] = mixed_baseline(W_mod())
+        res["configs"] = {long["config"]["workload"]: long, mixed["config"]["workload"]: mixed}
     if world > 1:
         import torch.distributed as dist
 

@@ -13,8 +13,11 @@
  *     exception crosses the ABI. On error nothing is launched and host state
  *     is unchanged unless stated otherwise.
  *   - Device pointers are owned by the caller (e.g. PyTorch tensors) and must
- *     be 16-byte aligned. The library never allocates device memory; kernels
- *     needing scratch take a caller-provided workspace.
+ *     be 16-byte aligned. No entry point allocates device memory when it is
+ *     called; kernels needing scratch take a caller-provided workspace. The
+ *     one piece of device memory the library holds is a fixed module array of
+ *     KV_NOALLOC_SCRATCH_BYTES per GPU (the scratch of
+ *     paged_decode_attention_noalloc), present from module load until exit.
  *   - Host handles (kv_pool_t, kv_prefix_t) are owned by the library and
  *     released with their _destroy call. They are not thread-safe.
  *   - Launches are asynchronous on `stream` (a cudaStream_t; NULL = legacy
@@ -197,7 +200,7 @@ int kv_prefix_num_entries(const kv_prefix_t* index, int32_t* out);
  * ======================================================================= */
 
 /* KV append -- [HB-07] Q025 (each layer appends the new token's K/V to its
- * own cache before attending); [CN-06] 6.1-6.2; [KV-03] lifecycle "填充".
+ * own cache before attending); [CN-06] 6.1-6.2; [KV-03] lifecycle section, fill step.
  * For every b in [0, B) with slot_mapping[b] >= 0 and every head h:
  *   k_pages[slot / P][h][slot % P][:] = k_new[b][h][:], same for V.
  * k_new, v_new: [B][H_kv][Dh] contiguous, same dtype as the pools.
@@ -368,28 +371,45 @@ int paged_decode_attention_fp8(float* out, const void* q, int32_t q_dtype, const
                                void* workspace, size_t ws_bytes, int* err_flag, void* stream);
 
 /* Which decode kernel paged_decode_attention uses (process-wide; default AUTO):
- *   KV_DECODE_KERNEL_AUTO  tensor cores (warp MMA on TMA-staged swizzled tiles)
- *                          for bf16/fp16 K/V with H_q / H_kv <= 64, CUDA cores
- *                          (packed f32x2 FMA) for fp32 K/V;
+ *   KV_DECODE_KERNEL_AUTO  bf16/fp16 K/V with H_q / H_kv = 32 and Dh = 128
+ *                          (MQA-shaped groups), no fused rotation: the
+ *                          fifth-generation tensor-core kernel (tcgen05; the
+ *                          128 tokens of a stage are the MMA rows, scores and
+ *                          output accumulate in tensor memory; persistent, one
+ *                          CTA per SM; with num_splits = 0 and B > 1 always
+ *                          device-planned). Other bf16/fp16 shapes with
+ *                          H_q / H_kv <= 64: warp MMA on TMA-staged swizzled
+ *                          tiles. fp32 K/V: CUDA cores (packed f32x2 FMA);
  *   KV_DECODE_KERNEL_SIMT  CUDA cores for every dtype (H_q / H_kv <= 32);
- *   KV_DECODE_KERNEL_MMA   same as AUTO (fp32 K/V still use CUDA cores).
- * Both kernels compute the same function; this exists to compare them.
- * KV_ERR_ARG for an unknown kind. */
+ *   KV_DECODE_KERNEL_MMA   warp MMA for every bf16/fp16 shape (never the
+ *                          tcgen05 kernel; fp32 K/V still use CUDA cores).
+ * All kernels compute the same function; this exists to compare them.
+ * KV_ERR_ARG for an unknown kind (KV_DECODE_KERNEL_TCGEN05 is only reported
+ * by paged_decode_launch_info, not selectable on its own). */
 #define KV_DECODE_KERNEL_AUTO 0
 #define KV_DECODE_KERNEL_SIMT 1
 #define KV_DECODE_KERNEL_MMA 2
+#define KV_DECODE_KERNEL_TCGEN05 3
 int paged_decode_set_kernel(int32_t kind);
 
-/* The split count paged_decode_attention will use for these arguments
- * (resolves num_splits = 0 on the current device). 0 means the launch is
- * planned on the device (see paged_decode_attention) -- which holds for
- * bf16/fp16 K/V on the tensor-core kernel; fp32 K/V and the CUDA-core kernel
- * use the grid rule's split count even then. */
+/* How paged_decode_attention (dtype = the K/V type) would launch for these
+ * arguments under the current kernel selection: *splits = the split count
+ * (0 = planned on the device), *kernel = KV_DECODE_KERNEL_SIMT, _MMA or
+ * _TCGEN05. KV_ERR_ARG for bad shapes. */
+int paged_decode_launch_info(int32_t B, int32_t H_q, int32_t H_kv, int32_t Dh, int32_t max_blocks, int32_t page_size,
+                             int32_t dtype, int32_t num_splits, int32_t* splits, int32_t* kernel);
+
+/* The split count the warp-MMA kernel uses for these arguments (resolves
+ * num_splits = 0 on the current device). 0 means the launch is planned on
+ * the device (see paged_decode_attention); fp32 K/V and the CUDA-core kernel
+ * use the grid rule's split count even then. paged_decode_launch_info also
+ * covers the tcgen05 kernel. */
 int paged_decode_num_splits(int32_t B, int32_t H_kv, int32_t max_blocks, int32_t page_size, int32_t num_splits,
                             int32_t* out);
 
 /* Workspace bytes needed by paged_decode_attention for the same arguments
- * (0 when no split is used). */
+ * (0 when no split is used), for 16-bit K/V under the current kernel
+ * selection (an upper bound for the other types). */
 int paged_decode_workspace_bytes(int32_t B, int32_t H_q, int32_t H_kv, int32_t Dh, int32_t max_blocks,
                                  int32_t page_size, int32_t num_splits, size_t* out);
 
@@ -406,9 +426,14 @@ int paged_decode_workspace_bytes(int32_t B, int32_t H_q, int32_t H_kv, int32_t D
  *     stream capture on that device.
  *   - All calls share the array and it keeps the last call's contents; calls
  *     whose kernels may overlap on the GPU (unordered streams) race on it.
- *   - KV_ERR_WORKSPACE when the partials for these arguments
- *     (paged_decode_workspace_bytes) exceed KV_NOALLOC_SCRATCH_BYTES; use
- *     fewer splits or the workspace entry point then.
+ *   - The address is kept for the life of the process: it does not survive
+ *     cudaDeviceReset of that device, after which this entry point must not
+ *     be called on it.
+ *   - num_splits = 0: the automatic choice, or, when its partials would not
+ *     fit the array, the largest explicit split count whose partials do
+ *     (down to 1, which needs none). An explicit num_splits whose partials
+ *     (paged_decode_workspace_bytes) exceed KV_NOALLOC_SCRATCH_BYTES returns
+ *     KV_ERR_WORKSPACE; use fewer splits or the workspace entry point then.
  * Other arguments, errors and results: as paged_decode_attention. */
 #define KV_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
 int paged_decode_attention_noalloc(float* out, const void* q, const void* k_pages, const void* v_pages,

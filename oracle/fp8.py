@@ -1,7 +1,7 @@
 """FP8 (E4M3) K/V cache: quantising append and decode -- TEST INFRASTRUCTURE ONLY.
 
 "03. KV Cache：用显存换计算" (the follow-up on KV quantisation) and the course
-notes' table of KV-size levers ("每个数存得更小": from 16 bits down to 8)
+notes' table of KV-size levers (the row on storing each number in fewer bits: from 16 down to 8)
 name storing K / V in 8 bits, with the warning that the error must be checked,
 but fix no format. The plainest reading, taken here:
 

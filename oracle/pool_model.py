@@ -3,7 +3,7 @@
 The rules restated here (page titles behind the tags: see the package docstring):
 
 * Physical blocks form a pool; a sequence gets blocks on demand and returns
-  them when it finishes ([HB-07] Q028; [CN-06] 6.5 "流程"; [KV-03]
+  them when it finishes ([HB-07] Q028; [CN-06] 6.5 allocation flow; [KV-03]
   "一个请求的 KV Cache 怎样产生和消失").
 * A block shared by several sequences carries a reference count and is not
   reclaimed while any user remains ([KV-04] "深入：引擎怎样找状态"; [HB-07]

@@ -199,14 +199,6 @@ def scatter_to_pages(pool: np.ndarray, table_row: Sequence[int], rows: np.ndarra
     pool[pages, :, t % P, :] = rows
 
 
-def gather_from_pages(pool: np.ndarray, table_row: Sequence[int], n: int) -> np.ndarray:
-    """Logical rows [n, H_kv, Dh] of one sequence read back through its block-table row."""
-    P = pool.shape[2]
-    t = np.arange(n)
-    pages = np.asarray(table_row, dtype=np.int64)[t // P]
-    return pool[pages, :, t % P, :]
-
-
 # --------------------------------------------------------------------------
 # fp64 paged decode in C (OpenMP over (sequence, query head))
 # --------------------------------------------------------------------------

@@ -143,6 +143,12 @@ cudaError_t launch_mma_bf16(const DecodeParams& p, const CUtensorMap& tk, const 
                             cudaStream_t st);
 cudaError_t launch_mma_f16(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int DH, int P, dim3 grid,
                            cudaStream_t st);
+// tcgen05 kernel (decode_tc.cu): g = 32, Dh = 128, bf16 / fp16 K/V; n_work items over `grid` persistent CTAs.
+cudaError_t launch_tc(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
+                      int dtype, int P, int n_work, int grid, cudaStream_t st);
+// tcgen05 multi-token query kernel (prefill_tc.cu): Dh = 128, 128 % g == 0, bf16 / fp16 K/V.
+cudaError_t launch_prefill_tc(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int dtype, int P,
+                              dim3 grid, cudaStream_t st);
 // E4M3 K/V with q of type q_dtype (bf16 or fp16).
 cudaError_t launch_mma_fp8(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int q_dtype, int DH,
                            int P, dim3 grid, cudaStream_t st);

@@ -1,0 +1,37 @@
+// Compiled instances of the tcgen05 decode kernel (g = 32, Dh = 128; bf16 and
+// fp16 K/V; page size 16 and 32) and their launch.
+#include <atomic>
+
+#include "decode_launch.cuh"
+#include "decode_tc.cuh"
+
+namespace kvp {
+
+template <int KT, int P>
+cudaError_t launch_tc_inst(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
+                           int n_work, int grid, cudaStream_t st) {
+    using C = TcCfg<128, P, 32>;
+    auto* kern = paged_decode_tc_kernel<KT, 128, P, 32>;
+    static std::atomic<uint64_t> configured{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(configured.load(std::memory_order_acquire) & bit)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        if (e != cudaSuccess) return e;
+        configured.fetch_or(bit, std::memory_order_acq_rel);
+    }
+    return launch_pdl(kern, dim3(grid), dim3(C::kThreads), C::kSmem, st, p, tk, tv, tq, n_work);
+}
+
+cudaError_t launch_tc(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
+                      int dtype, int P, int n_work, int grid, cudaStream_t st) {
+    if (dtype == KV_DTYPE_BF16)
+        return P == 16 ? launch_tc_inst<KV_DTYPE_BF16, 16>(p, tk, tv, tq, n_work, grid, st)
+                       : launch_tc_inst<KV_DTYPE_BF16, 32>(p, tk, tv, tq, n_work, grid, st);
+    return P == 16 ? launch_tc_inst<KV_DTYPE_F16, 16>(p, tk, tv, tq, n_work, grid, st)
+                   : launch_tc_inst<KV_DTYPE_F16, 32>(p, tk, tv, tq, n_work, grid, st);
+}
+
+}  // namespace kvp

@@ -221,17 +221,17 @@ int resolve_splits(int32_t B, int32_t H_kv, int32_t max_blocks, int32_t num_spli
 std::atomic<int> g_kernel_kind{KV_DECODE_KERNEL_AUTO};
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+// Looked up once; the function-local static makes concurrent first calls from
+// several host threads safe.
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::atomic<bool> tried{false};
-    if (!tried.load(std::memory_order_acquire)) {
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
         void* f = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-        tried.store(true, std::memory_order_release);
-    }
+            return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+        return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+    }();
     return fn;
 }
 
@@ -265,6 +265,13 @@ bool use_mma(int32_t dtype, int32_t g) {
     if (dtype == KV_DTYPE_F32) return false;
     if (kind == KV_DECODE_KERNEL_SIMT && dtype != KV_DTYPE_FP8_E4M3) return false;
     return g <= 64;
+}
+
+// The tcgen05 kernel (decode_tc.cuh): 16-bit K/V, GQA group of 32 heads,
+// Dh = 128, no fused rotation; chosen by the automatic kernel selection.
+bool tc_ok(int32_t dtype, int32_t g, int32_t Dh, bool rope) {
+    return g_kernel_kind.load(std::memory_order_relaxed) == KV_DECODE_KERNEL_AUTO &&
+           (dtype == KV_DTYPE_BF16 || dtype == KV_DTYPE_F16) && g == 32 && Dh == 128 && !rope;
 }
 
 size_t workspace_for(int32_t B, int32_t H_q, int32_t Dh, int32_t S) {
@@ -309,6 +316,28 @@ bool planned_ok(bool mma, int32_t B, int32_t H_q, int32_t H_kv, int32_t num_spli
     const int sms = sm_count();
     return mma && num_splits == 0 && B > 1 && B <= kPlanThreads * kPlanRowsPerThread && (H_q / H_kv) <= 64 &&
            sms > 0 && static_cast<int64_t>(B) * H_kv > 4LL * sms;
+}
+
+// The tcgen05 kernel is persistent (one CTA per SM walking work items), so it
+// takes the device plan for every multi-row batch with the automatic split:
+// chunks follow the actual lengths instead of the table width.
+bool planned_tc(int32_t B, int32_t num_splits) {
+    return num_splits == 0 && B > 1 && B <= kPlanThreads * kPlanRowsPerThread;
+}
+
+// A q tensor [rows][Dh] (16-bit) seen as boxes of `box_rows` rows x 128 bytes, 128-byte swizzle.
+bool make_q_map(CUtensorMap* m, const void* q, int32_t dtype, int64_t rows, int32_t Dh, int32_t box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc || rows >= (1LL << 32)) return false;
+    cuuint64_t gdim[2] = {static_cast<cuuint64_t>(Dh), static_cast<cuuint64_t>(rows)};
+    cuuint64_t gstride[1] = {static_cast<cuuint64_t>(Dh) * 2};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estride[2] = {1, 1};
+    const CUtensorMapDataType t =
+        dtype == KV_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    CUresult r = enc(m, t, 2, const_cast<void*>(q), gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
 }
 
 int check_shape(int32_t H_q, int32_t H_kv, int32_t Dh, int32_t page_size, int32_t dtype) {
@@ -371,7 +400,8 @@ int kv_copy_pages(void* k_pages, void* v_pages, const int32_t* src_pages, const 
 }
 
 int paged_decode_set_kernel(int32_t kind) {
-    if (kind != KV_DECODE_KERNEL_AUTO && kind != KV_DECODE_KERNEL_SIMT && kind != KV_DECODE_KERNEL_MMA) return KV_ERR_ARG;
+    if (kind != KV_DECODE_KERNEL_AUTO && kind != KV_DECODE_KERNEL_SIMT && kind != KV_DECODE_KERNEL_MMA)
+        return KV_ERR_ARG;
     g_kernel_kind.store(kind, std::memory_order_relaxed);
     return KV_OK;
 }
@@ -393,13 +423,30 @@ int paged_decode_workspace_bytes(int32_t B, int32_t H_q, int32_t H_kv, int32_t D
     int rc = resolve_splits(B, H_kv, max_blocks, num_splits, &S, &C);
     if (rc != KV_OK) return rc;
     size_t need = workspace_for(B, H_q, Dh, S);
-    if (planned_ok(true, B, H_q, H_kv, num_splits)) {
+    const bool tc = tc_ok(KV_DTYPE_BF16, H_q / H_kv, Dh, false) && H_q % H_kv == 0;
+    if (tc ? planned_tc(B, num_splits) : planned_ok(true, B, H_q, H_kv, num_splits)) {
         const int64_t grid = planned_grid(B, H_kv);
         if (grid < 0) return KV_ERR_CUDA;
         const size_t pl = planned_layout(B, H_q, H_kv, Dh, grid).total;
         if (pl > need) need = pl;
     }
     *out = need;
+    return KV_OK;
+}
+
+int paged_decode_launch_info(int32_t B, int32_t H_q, int32_t H_kv, int32_t Dh, int32_t max_blocks, int32_t page_size,
+                             int32_t dtype, int32_t num_splits, int32_t* splits, int32_t* kernel) {
+    if (!splits || !kernel || B < 0 || H_q <= 0 || H_kv <= 0 || H_q % H_kv != 0 || Dh <= 0 || max_blocks <= 0 ||
+        page_size <= 0 || num_splits < 0 || elem_bytes(dtype) == 0)
+        return KV_ERR_ARG;
+    const int32_t g = H_q / H_kv;
+    int32_t S, C;
+    int rc = resolve_splits(B, H_kv, max_blocks, num_splits, &S, &C, elem_bytes(dtype));
+    if (rc != KV_OK) return rc;
+    const bool mma = use_mma(dtype, g);
+    const bool tc = mma && tc_ok(dtype, g, Dh, false);
+    *kernel = tc ? KV_DECODE_KERNEL_TCGEN05 : (mma ? KV_DECODE_KERNEL_MMA : KV_DECODE_KERNEL_SIMT);
+    *splits = (tc ? planned_tc(B, num_splits) : planned_ok(mma, B, H_q, H_kv, num_splits)) ? 0 : S;
     return KV_OK;
 }
 
@@ -446,7 +493,8 @@ int decode_impl(float* out, const void* q, const void* k_new, const void* v_new,
     int32_t S, C;
     rc = resolve_splits(B, H_kv, max_blocks, num_splits, &S, &C, elem_bytes(dtype));
     if (rc != KV_OK) return rc;
-    const bool planned = planned_ok(mma, B, H_q, H_kv, num_splits);
+    const bool tc = mma && tc_ok(dtype, g, Dh, cos_sin != nullptr);
+    const bool planned = tc ? planned_tc(B, num_splits) : planned_ok(mma, B, H_q, H_kv, num_splits);
 
     DecodeParams p{};
     p.out = out;
@@ -498,9 +546,10 @@ int decode_impl(float* out, const void* q, const void* k_new, const void* v_new,
         const int64_t partial_bytes = static_cast<int64_t>(H_q / H_kv) * (Dh + 2) * 4;
         const int32_t c_floor = static_cast<int32_t>(std::max<int64_t>(8, (16 * partial_bytes + chunk_bytes_per_page - 1) /
                                                                                 chunk_bytes_per_page));
+        // resident CTAs: two per SM for the warp-MMA kernel, one (persistent) for the tcgen05 kernel
+        const int32_t slots = static_cast<int32_t>((tc ? 1 : 2) * sm_count());
         e = launch_pdl(paged_plan_kernel, dim3(1), dim3(kPlanThreads), 0, st, seq_lens, B, H_kv, page_size, max_blocks,
-                       static_cast<int32_t>(2 * sm_count()), static_cast<int32_t>(pgrid), c_floor, plan, items,
-                       err_flag);
+                       slots, static_cast<int32_t>(pgrid), c_floor, plan, items, err_flag);
         if (e != cudaSuccess) return KV_ERR_CUDA;
         grid = dim3(static_cast<unsigned>(pgrid), 1, 1);
     } else if (S > 1) {
@@ -510,7 +559,20 @@ int decode_impl(float* out, const void* q, const void* k_new, const void* v_new,
         p.part_u = static_cast<float*>(workspace);
         p.part_ml = reinterpret_cast<float2*>(static_cast<char*>(workspace) + rows * Dh * sizeof(float));
     }
-    if (mma) {
+    if (tc) {
+        CUtensorMap tk, tv, tq;
+        const int64_t rows = static_cast<int64_t>(num_pages) * H_kv * page_size;
+        if (!make_pool_map(&tk, k_pages, dtype, rows, Dh, page_size) ||
+            !make_pool_map(&tv, v_pages, dtype, rows, Dh, page_size) ||
+            !make_q_map(&tq, q, dtype, static_cast<int64_t>(B) * H_q, Dh, g))
+            return KV_ERR_CUDA;
+        const int64_t n_work = planned ? pgrid : static_cast<int64_t>(S) * H_kv * B;
+        if (n_work > 0x7fffffffLL) return KV_ERR_UNSUPPORTED;
+        const int sms = sm_count();
+        if (sms <= 0) return KV_ERR_CUDA;
+        const int tc_grid = static_cast<int>(std::min<int64_t>(n_work, sms));
+        e = launch_tc(p, tk, tv, tq, dtype, page_size, static_cast<int>(n_work), tc_grid, st);
+    } else if (mma) {
         CUtensorMap tk, tv;
         const int64_t rows = static_cast<int64_t>(num_pages) * H_kv * page_size;
         if (!make_pool_map(&tk, k_pages, dtype, rows, Dh, page_size) ||
@@ -620,8 +682,10 @@ int paged_prefill_attention(float* out, const void* q, const int32_t* q_start, i
     if (!out || !q || !q_start || !k_pages || !v_pages || !block_tables || !seq_lens) return KV_ERR_ARG;
     if (!aligned16(out) || !aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages)) return KV_ERR_ARG;
     if (static_cast<int64_t>(num_pages) * H_kv * page_size >= (1LL << 31)) return KV_ERR_UNSUPPORTED;
-    // 64 MMA rows per CTA: q_tile chunk tokens x g heads, four 16-row slices
-    const int32_t q_tile = 64 / g;
+    // tcgen05 kernel: 128 MMA rows per CTA (128 / g chunk tokens x g heads); warp-MMA kernel: 64 rows
+    // (64 / g tokens, four 16-row slices)
+    const bool tc = g_kernel_kind.load(std::memory_order_relaxed) == KV_DECODE_KERNEL_AUTO && Dh == 128 && 128 % g == 0;
+    const int32_t q_tile = tc ? 128 / g : 64 / g;
     DecodeParams p{};
     p.out = out;
     p.q = q;
@@ -650,8 +714,9 @@ int paged_prefill_attention(float* out, const void* q, const int32_t* q_start, i
     const dim3 grid(static_cast<unsigned>((max_q_len + q_tile - 1) / q_tile), static_cast<unsigned>(H_kv),
                     static_cast<unsigned>(B));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const cudaError_t e = dtype == KV_DTYPE_BF16 ? launch_prefill_bf16(p, tk, tv, Dh, page_size, grid, st)
-                                                 : launch_prefill_f16(p, tk, tv, Dh, page_size, grid, st);
+    const cudaError_t e = tc                       ? launch_prefill_tc(p, tk, tv, dtype, page_size, grid, st)
+                          : dtype == KV_DTYPE_BF16 ? launch_prefill_bf16(p, tk, tv, Dh, page_size, grid, st)
+                                                   : launch_prefill_f16(p, tk, tv, Dh, page_size, grid, st);
     return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;
 }
 

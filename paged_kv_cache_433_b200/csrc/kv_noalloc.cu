@@ -20,7 +20,14 @@
 //     GPU (different streams without ordering) race on it. Calls on one
 //     stream are ordered and safe. Nothing in it needs to start at zero (each
 //     split writes its partial before the combine kernel reads it);
-//   * a launch whose partials would not fit returns KV_ERR_WORKSPACE.
+//   * the array's device address is looked up once per device and kept for
+//     the life of the process; it does not survive cudaDeviceReset of that
+//     device (a process that resets a device must not call this entry point
+//     on it afterwards);
+//   * with num_splits == 0, when the automatic choice's partials would not
+//     fit, the largest explicit split count whose partials fit is used
+//     instead (down to 1, which needs no scratch); an explicit num_splits
+//     whose partials would not fit returns KV_ERR_WORKSPACE.
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -69,6 +76,20 @@ extern "C" int paged_decode_attention_noalloc(float* out, const void* q, const v
     size_t need = 0;
     int rc = paged_decode_workspace_bytes(B, H_q, H_kv, Dh, max_blocks, page_size, num_splits, &need);
     if (rc != KV_OK) return rc;
+    if (need > kScratchBytes && num_splits == 0) {
+        // automatic choice too large for the array: the largest explicit split count that fits
+        int32_t s0 = 0;
+        rc = paged_decode_num_splits(B, H_kv, max_blocks, page_size, 0, &s0);
+        if (rc != KV_OK) return rc;
+        for (int32_t s = s0 > 1 ? s0 - 1 : 8; s >= 1; --s) {
+            rc = paged_decode_workspace_bytes(B, H_q, H_kv, Dh, max_blocks, page_size, s, &need);
+            if (rc != KV_OK) return rc;
+            if (need <= kScratchBytes) {
+                num_splits = s;
+                break;
+            }
+        }
+    }
     if (need > kScratchBytes) return KV_ERR_WORKSPACE;  // partials exceed the fixed scratch
     void* scratch = nullptr;
     if (need > 0) {

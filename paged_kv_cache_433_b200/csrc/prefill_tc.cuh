@@ -1,0 +1,412 @@
+// Multi-token query (chunked prefill) over the paged cache on the
+// fifth-generation tensor cores (tcgen05), sm_100a.
+//
+// What is computed: row i of sequence b's chunk sits at position
+// p_i = seq_lens[b] - n_b + i and attends to the keys at positions 0 .. p_i
+// (causal within the chunk, "04. 注意力与 KV 缓存" and
+// "07｜KV Cache、FlashAttention与PagedAttention的内部过程" Q025), read through
+// the block table (Q028) and folded in with the online (m, l, u) merge of Q027.
+// Chunked prefill itself is the workload of "06 KV Cache、Prefix Cache、
+// PagedAttention 与 vLLM", 6.2 / 6.6.
+//
+// Tile: 128 MMA rows = 128 / g chunk tokens x the g query heads of one KV
+// head, so every K/V byte staged in shared memory serves the whole GQA group
+// of 128 / g tokens. Per stage of 128 keys:
+//   S[128 x 128]  = Q[128 x Dh] . K_stage^T             (SS: both K-major)
+//   O[128 x Dh]  += P[128 x 128] . V_stage               (TS: P in tensor memory,
+//                                                          V MN-major)
+// S is triple-buffered in tensor memory (3 x 128 columns) and O takes the
+// last 128 columns. Thread r of the four softmax warps owns row r: the whole
+// row max, exponentials and sum stay in its registers (no shuffles). P is
+// written back over its own S columns as a bf16 (fp16) pair: hi = RN(p) in
+// columns 0..63, lo = RN(p - hi) in 64..127; the P.V MMA runs on both, so the
+// probabilities carry ~2^-16 relative precision into the product.
+// The reference maximum of a row moves only when a score exceeds it by more
+// than 2^8; the row's O and l are then rescaled (o = u / l for any common
+// reference).
+//
+// Warps (192 threads, one CTA per SM by tensor memory and shared memory):
+//   warp 0     producer: per stage the K then V boxes of its pages (P rows x
+//              128 bytes, 128-byte swizzle) into a ring of six 32 KB entries;
+//   warp 1     tensor memory allocation; lane 0 issues QK(0), QK(1), then per
+//              stage PV(j) and QK(j + 2);
+//   warps 2-5  load the Q tile (swizzled stores), softmax, epilogue.
+// Every wait is bounded (KV_DEV_ERR_TIMEOUT); block-table entries outside
+// [0, num_pages) are never loaded (their keys are masked,
+// KV_DEV_ERR_PAGE_RANGE).
+#pragma once
+
+#include <cuda.h>
+
+#include "decode_kernel.cuh"
+#include "tc05.cuh"
+
+namespace kvp {
+
+template <int DH, int P>
+struct PfCfg {
+    static constexpr int kTP = 128;              // keys per stage
+    static constexpr int kPPS = kTP / P;         // pages per stage
+    static constexpr int kBoxCols = DH / 64;
+    static constexpr int kBoxB = kTP * 128;      // one 128-byte box column of an entry
+    static constexpr int kEntry = kBoxCols * kBoxB;
+    static constexpr int kRing = 6;              // K, V of three stages
+    static constexpr int kQB = 128 * DH * 2;     // Q tile: 128 rows
+    static constexpr int kOffQ = kRing * kEntry;
+    static constexpr int kOffBad = kOffQ + kQB;
+    static constexpr int kOffBar = (kOffBad + 4 * kRing + 7) / 8 * 8;
+    // full[6], empty[6], q_full, s_full[3], p_full[2], p_empty, o_full, done
+    static constexpr int kNumBars = 2 * kRing + 1 + 3 + 5;
+    static constexpr int kOffTmem = kOffBar + 8 * kNumBars;
+    static constexpr int kSmem = 1024 + kOffTmem + 16;
+    static constexpr int kThreads = 192;
+    static constexpr uint32_t kTmemCols = 512;   // S x 3 (384) + O (128)
+    static_assert(DH == 128, "instance: Dh = 128");
+    static_assert(kPPS * kBoxCols <= 32, "one TMA box per lane");
+    static_assert(kSmem <= 227 * 1024, "shared memory");
+};
+
+template <int KT, int DH, int P>
+__global__ void __launch_bounds__(192, 1)
+    paged_prefill_tc_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
+                            const __grid_constant__ CUtensorMap tmap_v) {
+    using C = PfCfg<DH, P>;
+    constexpr bool kBF16 = KT == KV_DTYPE_BF16;
+    constexpr uint32_t kIdescQK = idesc_f16(kBF16, 128, C::kTP, false, false);
+    constexpr uint32_t kIdescPV = idesc_f16(kBF16, 128, DH, false, true);
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        prefetch_tmap(&tmap_k);
+        prefetch_tmap(&tmap_v);
+    }
+    grid_dependency_wait();
+    if (threadIdx.x == 0) grid_launch_dependents();
+
+    // ---- this CTA's tile: chunk tokens t0 .. t0 + nt - 1 of sequence b, KV head kvh
+    const int kvh = blockIdx.y, b = blockIdx.z;
+    const int g = p.g;
+    const int qs0 = p.q_start[b];
+    const int n_q = p.q_start[b + 1] - qs0;
+    const int t0 = blockIdx.x * p.q_tile;
+    if (t0 >= n_q) return;
+    const int nt = min(p.q_tile, n_q - t0);
+    int len = p.seq_lens[b];
+    if (len < 0 || len > p.max_blocks * P || n_q > len) {
+        if (threadIdx.x == 0 && t0 == 0 && kvh == 0) raise_err(p.err, KV_DEV_ERR_SEQ_LEN);
+        // rows of this tile are zero
+        for (int e = threadIdx.x; e < nt * g * DH; e += blockDim.x) {
+            const int rr = e / DH;
+            p.out[((int64_t)(qs0 + t0 + rr / g) * p.H_q + (int64_t)kvh * g + rr % g) * DH + e % DH] = 0.f;
+        }
+        return;
+    }
+    const int pos0 = len - n_q + t0;          // position of the tile's first token
+    const int key_end = pos0 + nt;            // keys 0 .. key_end - 1 are seen by some row
+    const int n_pages = (key_end + P - 1) / P;
+    const int n_st = (key_end + C::kTP - 1) / C::kTP;
+
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;
+    unsigned char* smem = smem_raw + (sbase - raw);
+    const uint32_t bar0 = sbase + C::kOffBar;
+    auto full = [&](int e) { return bar0 + 8u * e; };
+    auto empty = [&](int e) { return bar0 + 8u * (C::kRing + e); };
+    const uint32_t q_full = bar0 + 8u * (2 * C::kRing);
+    auto s_full = [&](int i) { return q_full + 8u + 8u * i; };
+    // P of stage j is announced on p_full(j & 1): the softmax of stage j + 1 may finish before the MMA
+    // thread has waited for stage j, so one barrier would run a whole phase ahead of its waiter
+    auto p_full = [&](int i) { return q_full + 32u + 8u * i; };
+    const uint32_t p_empty = q_full + 48;
+    const uint32_t o_full = q_full + 56;
+    const uint32_t done_bar = q_full + 64;
+    volatile int* stage_bad = reinterpret_cast<volatile int*>(smem + C::kOffBad);
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::kOffTmem);
+
+    if (threadIdx.x == 0) {
+        for (int e = 0; e < C::kRing; ++e) {
+            mbar_init(full(e), 1);
+            mbar_init(empty(e), 1);
+        }
+        mbar_init(q_full, 4);
+        for (int i = 0; i < 3; ++i) mbar_init(s_full(i), 1);
+        mbar_init(p_full(0), 4);
+        mbar_init(p_full(1), 4);
+        mbar_init(p_empty, 1);
+        mbar_init(o_full, 1);
+        mbar_init(done_bar, 1);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tO = tmem + 3 * C::kTP;
+    const uint32_t ring = sbase;
+    const uint32_t sQ = sbase + C::kOffQ;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        bool ok = true;
+        uint32_t fill = 0;
+        const int32_t* row = p.block_tables + (int64_t)b * p.max_blocks;
+        for (int j = 0; j < n_st && ok; ++j) {
+            const int np = min(C::kPPS, n_pages - j * C::kPPS);
+            const int pg = lane < np ? row[j * C::kPPS + lane] : -1;
+            const bool good = lane < np && pg >= 0 && pg < p.num_pages;
+            if (lane < np && !good) raise_err(p.err, KV_DEV_ERR_PAGE_RANGE);
+            const unsigned gmask = __ballot_sync(0xffffffffu, good);
+            const int box_page = lane / C::kBoxCols, bb = lane % C::kBoxCols;
+            const int pgl = __shfl_sync(0xffffffffu, pg, box_page & 31);
+#pragma unroll 1
+            for (int half = 0; half < 2 && ok; ++half) {
+                const int e = fill % C::kRing;
+                if (lane == 0) {
+                    if (fill >= (uint32_t)C::kRing &&
+                        !mbar_wait_bounded(empty(e), ((fill / C::kRing) - 1) & 1, kWaitLimitNs)) {
+                        raise_err(p.err, KV_DEV_ERR_TIMEOUT);
+                        ok = false;
+                    } else {
+                        stage_bad[e] = (int)(~gmask & ((1u << np) - 1u));
+                        mbar_arrive_expect_tx(full(e), __popc(gmask) * C::kBoxCols * P * 128);
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                if (box_page < np && ((gmask >> box_page) & 1u)) {
+                    const uint32_t dst = ring + e * C::kEntry + bb * C::kBoxB + box_page * P * 128;
+                    tma_load_2d(dst, half ? static_cast<const void*>(&tmap_v) : static_cast<const void*>(&tmap_k),
+                                bb * 64, (pgl * p.H_kv + kvh) * P, full(e));
+                }
+                ++fill;
+            }
+        }
+        if (lane == 0) {
+            for (uint32_t i = fill > (uint32_t)C::kRing ? fill - C::kRing : 0; i < fill; ++i)
+                if (!mbar_wait_bounded(full(i % C::kRing), (i / C::kRing) & 1, kWaitLimitNs))
+                    raise_err(p.err, KV_DEV_ERR_TIMEOUT);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issue
+        if (lane == 0) {
+            bool ok = true;
+            auto wait = [&](uint32_t bar, uint32_t parity) {
+                if (ok && !mbar_wait_bounded(bar, parity, kWaitLimitNs)) {
+                    raise_err(p.err, KV_DEV_ERR_TIMEOUT);
+                    ok = false;
+                }
+                return ok;
+            };
+            auto qk = [&](int j) {
+                const uint32_t f = 2 * j;
+                const int e = f % C::kRing;
+                if (!wait(full(e), (f / C::kRing) & 1)) return;
+                tc_fence_after();
+                const uint32_t sK = ring + e * C::kEntry;
+                const uint32_t tS = tmem + (j % 3) * C::kTP;
+#pragma unroll
+                for (int kk = 0; kk < DH / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::kBoxB + (kk & 3) * 32;
+                    umma_ss(tS, smem_desc(sQ + off, 16, 1024, kSwz128), smem_desc(sK + off, 16, 1024, kSwz128),
+                            kIdescQK, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(s_full(j % 3));
+                umma_commit(empty(e));
+            };
+            if (wait(q_full, 0)) {
+                qk(0);
+                if (n_st > 1) qk(1);
+                for (int j = 0; j < n_st && ok; ++j) {
+                    const uint32_t f = 2 * j + 1;
+                    const int e = f % C::kRing;
+                    if (!wait(full(e), (f / C::kRing) & 1)) break;
+                    if (!wait(p_full(j & 1), (j >> 1) & 1)) break;
+                    // P.V(j - 1) has finished before P.V(j) is committed (so p_empty never runs two phases
+                    // ahead of this wait) and before QK(j + 2) reuses its S columns
+                    if (j >= 1 && !wait(p_empty, (j - 1) & 1)) break;
+                    tc_fence_after();
+                    const uint32_t sV = ring + e * C::kEntry;
+                    const uint32_t tP = tmem + (j % 3) * C::kTP;
+#pragma unroll
+                    for (int kk = 0; kk < C::kTP / 16; ++kk)
+                        umma_ts(tO, tP + kk * 8, smem_desc(sV + kk * 16 * 128, C::kBoxB, 1024, kSwz128), kIdescPV,
+                                (j > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                    for (int kk = 0; kk < C::kTP / 16; ++kk)
+                        umma_ts(tO, tP + C::kTP / 2 + kk * 8, smem_desc(sV + kk * 16 * 128, C::kBoxB, 1024, kSwz128),
+                                kIdescPV, 1u);
+                    umma_commit(empty(e));
+                    umma_commit(p_empty);
+                    if (j + 2 < n_st) qk(j + 2);  // S columns (j + 2) % 3 last held P(j - 1), now consumed
+                }
+                if (ok) umma_commit(o_full);
+            }
+            umma_commit(done_bar);
+            if (!mbar_wait_bounded(done_bar, 0, kWaitLimitNs)) raise_err(p.err, KV_DEV_ERR_TIMEOUT);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ Q tile, softmax, epilogue
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;   // MMA row: chunk token t0 + r / g, head kvh * g + r % g
+        const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+        const int tr = r / g;
+        const bool row_valid = tr < nt;
+        const int pos = pos0 + tr;           // this row sees keys 0 .. pos
+        const int64_t qrow = ((int64_t)(qs0 + t0 + tr) * p.H_q + (int64_t)kvh * g + r % g);
+        // Q row r -> swizzled K-major tile (two 128-byte box columns of 128 rows)
+        {
+            const uint4* src = static_cast<const uint4*>(p.q) + qrow * (DH / 8);
+#pragma unroll
+            for (int c = 0; c < DH / 8; ++c) {
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (row_valid) v = src[c];
+                const uint32_t dst = sQ + (c >> 3) * (128 * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x), "r"(v.y), "r"(v.z),
+                             "r"(v.w)
+                             : "memory");
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(q_full);
+        }
+        bool ok = true;
+        // warp-uniform outcome: the tensor-memory loads and stores after a wait are warp-collective
+        auto wait = [&](uint32_t bar, uint32_t parity) {
+            if (ok && !mbar_wait_bounded(bar, parity, kWaitLimitNs)) {
+                raise_err(p.err, KV_DEV_ERR_TIMEOUT);
+                ok = false;
+            }
+            ok = __all_sync(0xffffffffu, ok);
+            return ok;
+        };
+        const float sl2 = p.scale_log2;
+        float m_ref = -INFINITY, l = 0.f;
+        for (int j = 0; j < n_st; ++j) {
+            if (!wait(s_full(j % 3), (j / 3) & 1)) break;
+            tc_fence_after();
+            const uint32_t tS = tmem + (j % 3) * C::kTP + lane_addr;
+            float s[C::kTP];
+            {
+                uint32_t a[32];
+#pragma unroll
+                for (int q4 = 0; q4 < C::kTP / 32; ++q4) {
+                    tmem_ld32(tS + q4 * 32, a);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) s[q4 * 32 + i] = __uint_as_float(a[i]);
+                }
+            }
+            // keys of this stage: kbase .. kbase + 127; the V entry carries the skipped-page mask
+            const uint32_t fv = 2 * j + 1;
+            const int ev = fv % C::kRing;
+            if (!wait(full(ev), (fv / C::kRing) & 1)) break;
+            const int kbase = j * C::kTP;
+            const int np = min(C::kPPS, n_pages - j * C::kPPS);
+            const int bad = stage_bad[ev];
+            // keys this row may see in the stage: [0, lim); pages skipped or not loaded are masked
+            const int lim = row_valid ? min(C::kTP, pos + 1 - kbase) : 0;
+            const bool full_stage = lim == C::kTP && np == C::kPPS && bad == 0;
+            if (!full_stage) {
+#pragma unroll
+                for (int c = 0; c < C::kTP; ++c) {
+                    const int pgi = c / P;
+                    if (c >= lim || pgi >= np || ((bad >> pgi) & 1)) s[c] = -INFINITY;
+                }
+            }
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < C::kTP; ++c) mx = fmaxf(mx, s[c]);
+            const float mx2 = mx * sl2;  // sl2 > 0: the scaled maximum
+            // reference maximum: moves only when the row's max exceeds it by more than 2^8
+            const bool need = mx2 > m_ref + 8.f;
+            float alpha = 1.f;
+            if (need) {
+                alpha = exp2f(m_ref - mx2);  // 0 while m_ref is -inf
+                m_ref = mx2;
+                l *= alpha;
+            }
+            if (j > 0 && __any_sync(0xffffffffu, need)) {
+                // O holds P.V of the earlier stages: wait for the last one, then rescale the rows that moved
+                if (!wait(p_empty, (j - 1) & 1)) break;
+                tc_fence_after();
+                uint32_t a[32];
+#pragma unroll
+                for (int q4 = 0; q4 < DH / 32; ++q4) {
+                    tmem_ld32(tO + lane_addr + q4 * 32, a);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) a[i] = __float_as_uint(__uint_as_float(a[i]) * alpha);
+                    tmem_st32(tO + lane_addr + q4 * 32, a);
+                }
+                tmem_wait_st();
+            }
+            // probabilities -> P over this S buffer: hi pairs in columns 0..63, residual pairs in 64..127
+            const float neg = (m_ref == -INFINITY) ? 0.f : -m_ref;
+#pragma unroll
+            for (int q4 = 0; q4 < C::kTP / 32; ++q4) {
+                uint32_t hi[16], lo[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float x0 = s[q4 * 32 + 2 * i], x1 = s[q4 * 32 + 2 * i + 1];
+                    const float p0 = x0 == -INFINITY ? 0.f : exp2f(fmaf(x0, sl2, neg));
+                    const float p1 = x1 == -INFINITY ? 0.f : exp2f(fmaf(x1, sl2, neg));
+                    l += p0 + p1;
+                    pack2_split<kBF16>(p0, p1, hi[i], lo[i]);
+                }
+                tmem_st16(tmem + (j % 3) * C::kTP + lane_addr + q4 * 16, hi);
+                tmem_st16(tmem + (j % 3) * C::kTP + lane_addr + C::kTP / 2 + q4 * 16, lo);
+            }
+            tmem_wait_st();
+            // a key no row may see (past the tile, or on a page not loaded) may hold stale bytes: zero its V row
+            {
+                const int pgi = r / P;
+                if (kbase + r >= key_end || pgi >= np || ((bad >> pgi) & 1)) {
+                    const uint32_t vrow = ring + ev * C::kEntry + r * 128;
+#pragma unroll
+                    for (int bb = 0; bb < C::kBoxCols; ++bb)
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) sts128_zero(vrow + bb * C::kBoxB + c * 16);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full(j & 1));
+        }
+        // ---- epilogue: O row / l
+        if (wait(o_full, 0)) {
+            tc_fence_after();
+            float* dst = p.out + qrow * DH;
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            uint32_t a[32];
+#pragma unroll
+            for (int q4 = 0; q4 < DH / 32; ++q4) {
+                tmem_ld32(tO + lane_addr + q4 * 32, a);
+                tmem_wait_ld();
+                if (row_valid) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4)
+                        *reinterpret_cast<float4*>(dst + q4 * 32 + i) =
+                            make_float4(__uint_as_float(a[i]) * inv, __uint_as_float(a[i + 1]) * inv,
+                                        __uint_as_float(a[i + 2]) * inv, __uint_as_float(a[i + 3]) * inv);
+                }
+            }
+        } else if (row_valid) {
+            for (int d = 0; d < DH; ++d) p.out[qrow * DH + d] = 0.f;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
+}
+
+}  // namespace kvp

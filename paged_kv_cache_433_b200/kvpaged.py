@@ -88,6 +88,7 @@ SIGNATURES = [
      [_vp, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp]),
     ("paged_decode_set_kernel", ctypes.c_int, [_i32]),
     ("paged_decode_num_splits", ctypes.c_int, [_i32, _i32, _i32, _i32, _i32, _pi32]),
+    ("paged_decode_launch_info", ctypes.c_int, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _pi32, _pi32]),
     ("paged_decode_workspace_bytes", ctypes.c_int, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, _psz]),
 ]
 
@@ -427,7 +428,7 @@ def paged_prefill_attention(out, q, q_start, max_q_len: int, k_pages, v_pages, b
     _check("paged_prefill_attention", rc)
 
 
-KV_DECODE_KERNEL_AUTO, KV_DECODE_KERNEL_SIMT, KV_DECODE_KERNEL_MMA = 0, 1, 2
+KV_DECODE_KERNEL_AUTO, KV_DECODE_KERNEL_SIMT, KV_DECODE_KERNEL_MMA, KV_DECODE_KERNEL_TCGEN05 = 0, 1, 2, 3
 
 
 def paged_decode_set_kernel(kind: int) -> None:
@@ -452,6 +453,15 @@ def paged_decode_num_splits(B: int, H_kv: int, max_blocks: int, page_size: int, 
     out = ctypes.c_int32()
     _check("paged_decode_num_splits", lib().paged_decode_num_splits(B, H_kv, max_blocks, page_size, num_splits, out))
     return out.value
+
+
+def paged_decode_launch_info(B: int, H_q: int, H_kv: int, Dh: int, max_blocks: int, page_size: int,
+                             dtype: str = "bf16", num_splits: int = 0):
+    """(split count, 0 = device-planned; kernel kind KV_DECODE_KERNEL_SIMT / _MMA / _TCGEN05)."""
+    S, kind = ctypes.c_int32(), ctypes.c_int32()
+    _check("paged_decode_launch_info", lib().paged_decode_launch_info(B, H_q, H_kv, Dh, max_blocks, page_size,
+                                                                      DTYPE_CODE[dtype], num_splits, S, kind))
+    return S.value, kind.value
 
 
 def paged_decode_workspace_bytes(B: int, H_q: int, H_kv: int, Dh: int, max_blocks: int, page_size: int,

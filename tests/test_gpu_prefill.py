@@ -114,3 +114,17 @@ def test_prefill_bench_shape_sampled():
         ref = R.paged_prefill(q[rows], np.array([0, 512], np.int32), st.kp, st.vp, st.tab[b:b + 1], lens[b:b + 1],
                               cfg.scale, "bf16")
         check_close(got[rows], ref, "bf16", f"prefill bench shape, sequence {b}")
+
+
+@pytest.mark.parametrize("dtype,P,H_q,H_kv", [("bf16", 16, 32, 8), ("fp16", 32, 32, 1)])
+def test_prefill_warp_mma_kernel(dtype, P, H_q, H_kv):
+    """Dh = 128 chunks through the warp-MMA kernel (the automatic choice there is the tcgen05 kernel)."""
+    cfg = W.DecodeConfig(f"prefill-mma-{dtype}-{P}-{H_q}-{H_kv}", dtype, B=3, H_q=H_q, H_kv=H_kv, Dh=128,
+                         page_size=P, seed=86)
+    K.paged_decode_set_kernel(K.KV_DECODE_KERNEL_MMA)
+    try:
+        got, q, q_start, st, lens = _run(cfg, [300, 95, 40], [100, 95, 17])
+    finally:
+        K.paged_decode_set_kernel(K.KV_DECODE_KERNEL_AUTO)
+    ref = R.paged_prefill(q, q_start, st.kp, st.vp, st.tab, lens, cfg.scale, dtype)
+    check_close(got, ref, dtype, cfg.name)
