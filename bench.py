@@ -74,8 +74,9 @@ def parse():
                     help="append the new token inside the decode launch (paged_decode_attention_append) "
                          "or with kv_append before paged_decode_attention")
     ap.add_argument("--tokens", type=int, default=8192, help="config 6: tokens in the prefill chunk")
-    ap.add_argument("--kernel", choices=["auto", "simt", "mma"], default="auto",
-                    help="decode kernel: tensor cores (auto/mma, 16-bit K/V) or CUDA cores (simt)")
+    ap.add_argument("--kernel", choices=["auto", "simt", "mma", "tc"], default="auto",
+                    help="decode kernel: automatic choice, CUDA cores (simt), warp MMA (mma) or the tcgen05 kernel "
+                         "wherever it applies (tc)")
     return ap.parse_args()
 
 
@@ -1399,7 +1400,7 @@ def main():
     from paged_kv_cache_433_b200 import kvpaged as K
 
     K.paged_decode_set_kernel({"auto": K.KV_DECODE_KERNEL_AUTO, "simt": K.KV_DECODE_KERNEL_SIMT,
-                               "mma": K.KV_DECODE_KERNEL_MMA}[args.kernel])
+                               "mma": K.KV_DECODE_KERNEL_MMA, "tc": K.KV_DECODE_KERNEL_TCGEN05}[args.kernel])
     run = {2: run_layer_bench, 3: run_long_bench, 4: run_prefix_bench, 5: run_mixed_bench, 6: run_rope_bench,
            7: run_fp8_bench, 8: run_prefill_bench}[args.config]
     res = run(args, world, rank, local)

@@ -382,10 +382,14 @@ int paged_decode_attention_fp8(float* out, const void* q, int32_t q_dtype, const
  *                          tiles. fp32 K/V: CUDA cores (packed f32x2 FMA);
  *   KV_DECODE_KERNEL_SIMT  CUDA cores for every dtype (H_q / H_kv <= 32);
  *   KV_DECODE_KERNEL_MMA   warp MMA for every bf16/fp16 shape (never the
- *                          tcgen05 kernel; fp32 K/V still use CUDA cores).
+ *                          tcgen05 kernel; fp32 K/V still use CUDA cores);
+ *   KV_DECODE_KERNEL_TCGEN05  the tcgen05 kernel wherever it applies: bf16/fp16
+ *                          K/V, Dh = 128, H_q / H_kv in {4, 8, 16, 32}, no
+ *                          fused rotation (else as AUTO).
  * All kernels compute the same function; this exists to compare them.
- * KV_ERR_ARG for an unknown kind (KV_DECODE_KERNEL_TCGEN05 is only reported
- * by paged_decode_launch_info, not selectable on its own). */
+ * KV_ERR_ARG for an unknown kind. The multi-token query
+ * (paged_prefill_attention) takes its tcgen05 kernel under AUTO and TCGEN05
+ * for Dh = 128 and groups that divide 128, its warp-MMA kernel otherwise. */
 #define KV_DECODE_KERNEL_AUTO 0
 #define KV_DECODE_KERNEL_SIMT 1
 #define KV_DECODE_KERNEL_MMA 2

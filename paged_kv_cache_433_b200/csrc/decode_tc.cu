@@ -1,5 +1,5 @@
-// Compiled instances of the tcgen05 decode kernel (g = 32, Dh = 128; bf16 and
-// fp16 K/V; page size 16 and 32) and their launch.
+// Compiled instances of the tcgen05 decode kernel (GQA groups of 4, 8, 16 and
+// 32 heads, Dh = 128; bf16 and fp16 K/V; page size 16 and 32) and their launch.
 #include <atomic>
 
 #include "decode_launch.cuh"
@@ -7,11 +7,11 @@
 
 namespace kvp {
 
-template <int KT, int P>
+template <int KT, int P, int G>
 cudaError_t launch_tc_inst(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
                            int n_work, int grid, cudaStream_t st) {
-    using C = TcCfg<128, P, 32>;
-    auto* kern = paged_decode_tc_kernel<KT, 128, P, 32>;
+    using C = TcCfg<128, P, G>;
+    auto* kern = paged_decode_tc_kernel<KT, 128, P, G>;
     static std::atomic<uint64_t> configured{0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -25,13 +25,28 @@ cudaError_t launch_tc_inst(const DecodeParams& p, const CUtensorMap& tk, const C
     return launch_pdl(kern, dim3(grid), dim3(C::kThreads), C::kSmem, st, p, tk, tv, tq, n_work);
 }
 
+template <int KT, int G>
+cudaError_t launch_tc_page(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
+                           int P, int n_work, int grid, cudaStream_t st) {
+    return P == 16 ? launch_tc_inst<KT, 16, G>(p, tk, tv, tq, n_work, grid, st)
+                   : launch_tc_inst<KT, 32, G>(p, tk, tv, tq, n_work, grid, st);
+}
+
+template <int KT>
+cudaError_t launch_tc_dt(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
+                         int P, int n_work, int grid, cudaStream_t st) {
+    switch (p.g) {
+        case 4: return launch_tc_page<KT, 4>(p, tk, tv, tq, P, n_work, grid, st);
+        case 8: return launch_tc_page<KT, 8>(p, tk, tv, tq, P, n_work, grid, st);
+        case 16: return launch_tc_page<KT, 16>(p, tk, tv, tq, P, n_work, grid, st);
+        default: return launch_tc_page<KT, 32>(p, tk, tv, tq, P, n_work, grid, st);
+    }
+}
+
 cudaError_t launch_tc(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
                       int dtype, int P, int n_work, int grid, cudaStream_t st) {
-    if (dtype == KV_DTYPE_BF16)
-        return P == 16 ? launch_tc_inst<KV_DTYPE_BF16, 16>(p, tk, tv, tq, n_work, grid, st)
-                       : launch_tc_inst<KV_DTYPE_BF16, 32>(p, tk, tv, tq, n_work, grid, st);
-    return P == 16 ? launch_tc_inst<KV_DTYPE_F16, 16>(p, tk, tv, tq, n_work, grid, st)
-                   : launch_tc_inst<KV_DTYPE_F16, 32>(p, tk, tv, tq, n_work, grid, st);
+    return dtype == KV_DTYPE_BF16 ? launch_tc_dt<KV_DTYPE_BF16>(p, tk, tv, tq, P, n_work, grid, st)
+                                  : launch_tc_dt<KV_DTYPE_F16>(p, tk, tv, tq, P, n_work, grid, st);
 }
 
 }  // namespace kvp

@@ -14,9 +14,10 @@
 //   O^T[Dh x g]        += V_stage^T[Dh x 128] . P^T[128 x g]  (MN-major A and B)
 // S^T and O^T live in tensor memory (fp32); thread t of the four softmax
 // warps owns token row t of S^T (all g scores of one token) and dimension
-// row t of O^T. P^T goes to shared memory as a bf16 (fp16) pair hi + lo:
-// hi = RN(p), lo = RN(p - hi); the second P.V MMA on lo carries p to ~2^-16
-// relative, so short rows keep the accuracy of the fp32 softmax.
+// row t of O^T. P^T goes to shared memory as a 16-bit pair hi + lo (bf16:
+// hi = p truncated, lo = p - hi truncated, integer operations only; fp16: both
+// rounded to nearest); the second P.V MMA on lo carries p to ~2^-14 relative,
+// so short rows keep the accuracy of the fp32 softmax.
 //
 // Reference maximum (log2 units, per head, shared by the whole CTA): it moves
 // only when some score of a stage exceeds it by more than 2^8; then the stage
@@ -28,8 +29,9 @@
 //              the K then the V boxes of its pages (P rows x 128 bytes each)
 //              into a ring of six 32 KB entries (K and V of three stages);
 //              fused append of the new token when the item owns the last page.
-//   warp 1     allocates tensor memory; lane 0 issues QK(j) then PV(j - 1),
-//              committing each onto the mbarriers the other roles wait on.
+//   warp 1     allocates tensor memory and resolves the CTA's work items
+//              into shared memory; lane 0 issues the QK(j), lane 1 the
+//              P.V(j), each committing onto the mbarriers the others wait on.
 //   warps 2-5  softmax and epilogue (tensor-memory lane quarter = warp % 4).
 // A work item is (sequence, KV head, chunk of pages): from the device plan
 // (planned launch) or from the grid rule (split); partials use the layout of
@@ -49,27 +51,39 @@ namespace kvp {
 
 template <int DH, int P, int G>
 struct TcCfg {
+    static constexpr int kN = G < 16 ? 16 : G;   // MMA N (head columns; heads >= G are zero padding)
     static constexpr int kTP = 128;              // tokens per stage = MMA rows
     static constexpr int kPPS = kTP / P;         // pages per stage
     static constexpr int kBoxCols = DH / 64;     // 128-byte box columns per token row
     static constexpr int kBoxB = kTP * 128;      // one box column of an entry
     static constexpr int kEntry = kBoxCols * kBoxB;  // K (or V) of one stage
-    static constexpr int kRing = 6;              // entries: K, V of three stages
-    static constexpr int kQB = kBoxCols * G * 128;
-    static constexpr int kPB = kTP * G * 2;      // one P^T tile (hi or lo)
+    static constexpr int kPB0 = kTP * kN * 2;    // one P^T tile (hi or lo)
+    // ring entries (K or V of a stage) that fit beside Q, two P^T buffers (hi + lo each) and the small arrays
+    static constexpr int kRing0 = (227 * 1024 - 1024 - 2048 - kBoxCols * kN * 128 - 4 * kPB0) / kEntry;
+    static constexpr int kRing = kRing0 > 6 ? 6 : kRing0;
+    static constexpr int kQRowsB = kN * 128;     // one box column of the Q tile
+    static constexpr int kQB = kBoxCols * kQRowsB;
+    static constexpr int kPRow = kN * 2;         // bytes of one P^T row (token)
+    static constexpr int kPB = kTP * kPRow;      // one P^T tile (hi or lo); equals kPB0
+    // P^T rows of 32 / 64 bytes: MN-major with the 32- / 64-byte swizzle; 8-row atoms
+    static constexpr uint32_t kPSwz = kPRow == 32 ? kSwz32 : kSwz64;
+    static constexpr int kPAtom = 8 * kPRow;
     static constexpr int kOffQ = kRing * kEntry;
     static constexpr int kOffP = kOffQ + kQB;
-    static constexpr int kOffRed = kOffP + 2 * kPB;          // 2 x [G][4] floats
+    static constexpr int kOffRed = kOffP + 4 * kPB;          // 2 x [G][4] floats (after 2 x (hi, lo) P^T)
     static constexpr int kOffFlag = kOffRed + 2 * G * 4 * 4;  // 2 x 4 ints
     static constexpr int kOffBad = kOffFlag + 32;             // int per ring entry
-    static constexpr int kOffBar = (kOffBad + 4 * kRing + 7) / 8 * 8;
-    // full[6], empty[6], q_full, q_empty, s_full[2], s_empty[2], p_full, p_empty, o_full, o_empty, done
-    static constexpr int kNumBars = 2 * kRing + 2 + 4 + 4 + 1;
+    static constexpr int kMaxList = 96;          // work items of a CTA resolved once into shared memory
+    static constexpr int kOffList = (kOffBad + 4 * kRing + 15) / 16 * 16;  // int4 x 2 per item
+    static constexpr int kOffBar = kOffList + kMaxList * 32;
+    // full[R], empty[R], q_full, q_empty, s_full[2], s_empty[2], p_full[2], p_empty[2], o_full, o_empty,
+    // done (QK issuer), done (PV issuer)
+    static constexpr int kNumBars = 2 * kRing + 2 + 4 + 4 + 2 + 2;
     static constexpr int kOffTmem = kOffBar + 8 * kNumBars;
     static constexpr int kSmem = 1024 + kOffTmem + 16;
     static constexpr int kThreads = 192;
-    static constexpr uint32_t kTmemCols = 128;   // S^T x 2 (2g) + O^T (g)
-    static_assert(G == 32 && DH == 128, "instance: g = 32, Dh = 128");
+    static constexpr uint32_t kTmemCols = 3 * kN <= 64 ? 64 : 128;  // S^T x 2 + O^T, N columns each
+    static_assert((G == 4 || G == 8 || G == 16 || G == 32) && DH == 128, "instances: g in {4, 8, 16, 32}, Dh = 128");
     static_assert(kPPS * kBoxCols <= 32, "one TMA box per lane");
     static_assert(kSmem <= 227 * 1024, "shared memory");
 };
@@ -110,14 +124,54 @@ __device__ __forceinline__ bool tc_work(const DecodeParams& p, int w, int P, TcW
     return true;
 }
 
-// Per-head reduction over the 32 lanes of a warp: afterwards lane l holds the
-// reduction of x[l] (halving exchange: each step ships half of the values).
-template <bool MAX>
-__device__ __forceinline__ float warp_heads_reduce(float (&x)[32], int lane) {
+__host__ __device__ constexpr int ilog2(int n) { return n <= 1 ? 0 : 1 + ilog2(n / 2); }
+
+// A CTA's candidate work items (w = blockIdx.x + k gridDim.x) resolved once by
+// one warp into shared memory, so the roles walk them without the dependent
+// global loads of tc_work; candidates past the list are resolved on the fly.
+struct TcList {
+    int4* e;        // [kMaxList][2]: {b, kvh, split, item}, {first, n_local, len, flags}
+    int n_list;     // candidates held
+};
+
+__device__ __forceinline__ void tc_list_build(const DecodeParams& p, int n_work, int P, int4* e, int max_list,
+                                              int lane) {
+    for (int k = lane; k < max_list; k += 32) {
+        const int w = blockIdx.x + k * gridDim.x;
+        TcWork wk;
+        int flags = 0;
+        if (w < n_work && tc_work(p, w, P, wk)) flags = 4 | (wk.split_mode ? 1 : 0) | (wk.bad_len ? 2 : 0);
+        else wk = TcWork{0, 0, 0, 0, 0, 0, 0, 0, false, false};
+        e[2 * k] = make_int4(wk.b, wk.kvh, wk.split, wk.item);
+        e[2 * k + 1] = make_int4(wk.first, wk.n_local, wk.len, flags);
+    }
+}
+
+// Candidate k of this CTA: false when it carries no work item.
+__device__ __forceinline__ bool tc_get(const DecodeParams& p, const TcList& L, int k, int P, TcWork& wk) {
+    if (k < L.n_list) {
+        const int4 a = L.e[2 * k], c = L.e[2 * k + 1];
+        if (!(c.w & 4)) return false;
+        wk.b = a.x, wk.kvh = a.y, wk.split = a.z, wk.item = a.w;
+        wk.first = c.x, wk.n_local = c.y, wk.len = c.z;
+        wk.split_mode = (c.w & 1) != 0, wk.bad_len = (c.w & 2) != 0;
+        wk.n_pages = (wk.len + P - 1) / P;
+        return true;
+    }
+    return tc_work(p, blockIdx.x + k * gridDim.x, P, wk);
+}
+
+// Per-head reduction over the 32 lanes of a warp of NV values per lane (NV a
+// power of two <= 32): halving exchanges (each step ships half of the values)
+// until one value is left, then a butterfly. Afterwards the lanes of group
+// lane >> (5 - log2 NV) hold the reduction of that head.
+template <int NV, bool MAX>
+__device__ __forceinline__ float warp_heads_reduce(float (&x)[NV], int lane) {
+    constexpr int kL = ilog2(NV);
 #pragma unroll
-    for (int k = 0; k < 5; ++k) {
+    for (int k = 0; k < kL; ++k) {
         const int off = 16 >> k;
-        const int half = 16 >> k;
+        const int half = NV >> (k + 1);
         const bool up = (lane & off) != 0;
 #pragma unroll
         for (int i = 0; i < half; ++i) {
@@ -127,24 +181,58 @@ __device__ __forceinline__ float warp_heads_reduce(float (&x)[32], int lane) {
             x[i] = MAX ? fmaxf(keep, got) : keep + got;
         }
     }
-    return x[0];
+    float v = x[0];
+#pragma unroll
+    for (int off = 16 >> kL; off >= 1; off >>= 1) {
+        const float got = __shfl_xor_sync(0xffffffffu, v, off);
+        v = MAX ? fmaxf(v, got) : v + got;
+    }
+    return v;
 }
 
 // The same reduction over the four softmax warps (128 threads, named barrier
-// 1); every thread receives all 32 results. `buf` alternates between calls.
-template <bool MAX>
-__device__ __forceinline__ void cta_heads_reduce(float (&x)[32], float* red, int sw, int lane, int& buf) {
-    const float v = warp_heads_reduce<MAX>(x, lane);
-    float* r = red + buf * 32 * 4;
-    r[lane * 4 + sw] = v;
+// 1); every thread receives all NV results. `buf` alternates between calls.
+template <int NV, bool MAX>
+__device__ __forceinline__ void cta_heads_reduce(float (&x)[NV], float* red, int sw, int lane, int& buf) {
+    constexpr int kShift = 5 - ilog2(NV);
+    const float v = warp_heads_reduce<NV, MAX>(x, lane);
+    float* r = red + buf * NV * 4;
+    if ((lane & ((1 << kShift) - 1)) == 0) r[(lane >> kShift) * 4 + sw] = v;
     named_bar_sync(1, 128);
     const float4* r4 = reinterpret_cast<const float4*>(r);
 #pragma unroll
-    for (int h = 0; h < 32; ++h) {
+    for (int h = 0; h < NV; ++h) {
         const float4 a = r4[h];
         x[h] = MAX ? fmaxf(fmaxf(a.x, a.y), fmaxf(a.z, a.w)) : (a.x + a.y) + (a.z + a.w);
     }
     buf ^= 1;
+}
+
+// kN consecutive fp32 columns of this thread's lane (16 or 32).
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&a)[N]) {
+    if constexpr (N == 16) {
+        tmem_ld16(taddr, a);
+    } else {
+        uint32_t lo[16], hi[16];
+        tmem_ld16(taddr, lo);
+        tmem_ld16(taddr + 16, hi);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) a[i] = lo[i], a[16 + i] = hi[i];
+    }
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&a)[N]) {
+    if constexpr (N == 16) {
+        tmem_st16(taddr, a);
+    } else {
+        uint32_t lo[16], hi[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) lo[i] = a[i], hi[i] = a[16 + i];
+        tmem_st16(taddr, lo);
+        tmem_st16(taddr + 16, hi);
+    }
 }
 
 __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
@@ -158,8 +246,9 @@ __global__ void __launch_bounds__(192, 1)
                            int n_work) {
     using C = TcCfg<DH, P, G>;
     constexpr bool kBF16 = KT == KV_DTYPE_BF16;
-    constexpr uint32_t kIdescQK = idesc_f16(kBF16, 128, G, false, false);
-    constexpr uint32_t kIdescPV = idesc_f16(kBF16, 128, G, true, true);
+    constexpr int N = C::kN;
+    constexpr uint32_t kIdescQK = idesc_f16(kBF16, 128, N, false, false);
+    constexpr uint32_t kIdescPV = idesc_f16(kBF16, 128, N, true, true);
     extern __shared__ __align__(1024) unsigned char smem_raw[];
 
     const int warp = threadIdx.x >> 5;
@@ -182,11 +271,13 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t q_empty = q_full + 8;
     auto s_full = [&](int i) { return q_full + 16u + 8u * i; };
     auto s_empty = [&](int i) { return q_full + 32u + 8u * i; };
-    const uint32_t p_full = q_full + 48;
-    const uint32_t p_empty = q_full + 56;
-    const uint32_t o_full = q_full + 64;
-    const uint32_t o_empty = q_full + 72;
-    const uint32_t done_bar = q_full + 80;
+    // P^T is double-buffered (stage J in buffer J & 1): the softmax of stage J writes while P.V(J - 1) runs
+    auto p_full = [&](int i) { return q_full + 48u + 8u * i; };
+    auto p_empty = [&](int i) { return q_full + 64u + 8u * i; };
+    const uint32_t o_full = q_full + 80;
+    const uint32_t o_empty = q_full + 88;
+    const uint32_t done_qk = q_full + 96;
+    const uint32_t done_pv = q_full + 104;
     volatile int* stage_bad = reinterpret_cast<volatile int*>(smem + C::kOffBad);
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::kOffTmem);
 
@@ -201,36 +292,52 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(s_full(i), 1);
             mbar_init(s_empty(i), 4);
         }
-        mbar_init(p_full, 4);
-        mbar_init(p_empty, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(p_full(i), 4);
+            mbar_init(p_empty(i), 1);
+        }
         mbar_init(o_full, 1);
         mbar_init(o_empty, 4);
-        mbar_init(done_bar, 1);
+        mbar_init(done_qk, 1);
+        mbar_init(done_pv, 1);
         fence_barrier_init();
     }
+    int4* list_e = reinterpret_cast<int4*>(smem + C::kOffList);
+    const int n_cand = n_work > (int)blockIdx.x ? (n_work - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+    const TcList L{list_e, min(n_cand, C::kMaxList)};
     if (warp == 1) {
         tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), C::kTmemCols);
         tmem_relinquish();
+        tc_list_build(p, n_work, P, list_e, L.n_list, lane);
+    }
+    if constexpr (G < N) {
+        // Q rows G .. N-1 are MMA padding: zero once (the TMA box writes rows 0 .. G-1 only)
+        for (int i = threadIdx.x; i < C::kBoxCols * (N - G) * 8; i += blockDim.x) {
+            const int bb = i / ((N - G) * 8), rest = i % ((N - G) * 8);
+            sts128_zero(sbase + C::kOffQ + bb * C::kQRowsB + (G + rest / 8) * 128 + (rest % 8) * 16);
+        }
+        fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem;           // S^T buffers: columns [0, 2g)
-    const uint32_t tO = tmem + 2 * G;   // O^T: columns [2g, 3g)
+    const uint32_t tS = tmem;           // S^T buffers: columns [0, 2N)
+    const uint32_t tO = tmem + 2 * N;   // O^T: columns [2N, 3N)
     const uint32_t ring = sbase;
     const uint32_t sQ = sbase + C::kOffQ;
-    const uint32_t sPhi = sbase + C::kOffP;
-    const uint32_t sPlo = sPhi + C::kPB;
+    // P^T buffer b: hi tile at sP + 2b kPB, residual lo tile right after it
+    const uint32_t sP = sbase + C::kOffP;
+    auto sPhi = [&](uint32_t j) { return sP + (j & 1) * 2 * C::kPB; };
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         bool ok = true;
         uint32_t fill = 0;
         int item_i = 0;
-        for (int w = blockIdx.x; w < n_work && ok; w += gridDim.x) {
+        for (int k = 0; k < n_cand && ok; ++k) {
             TcWork wk;
-            if (!tc_work(p, w, P, wk) || wk.n_local <= 0) continue;
+            if (!tc_get(p, L, k, P, wk) || wk.n_local <= 0) continue;
             if (p.k_new != nullptr && wk.first + wk.n_local == wk.n_pages)
                 append_new_token(p, wk.b, wk.kvh, wk.len, P, DH * 2, lane);
             if (lane == 0) {
@@ -238,10 +345,10 @@ __global__ void __launch_bounds__(192, 1)
                     raise_err(p.err, KV_DEV_ERR_TIMEOUT);
                     ok = false;
                 } else {
-                    mbar_arrive_expect_tx(q_full, C::kQB);
+                    mbar_arrive_expect_tx(q_full, C::kBoxCols * G * 128);
 #pragma unroll
                     for (int bb = 0; bb < C::kBoxCols; ++bb)
-                        tma_load_2d(sQ + bb * G * 128, &tmap_q, bb * 64, wk.b * p.H_q + wk.kvh * G, q_full);
+                        tma_load_2d(sQ + bb * C::kQRowsB, &tmap_q, bb * 64, wk.b * p.H_q + wk.kvh * G, q_full);
                 }
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -289,10 +396,13 @@ __global__ void __launch_bounds__(192, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issue
-        if (lane == 0) {
+        // Lane 0 issues the score products QK(j) as soon as K(j) has landed and an S^T buffer is free;
+        // lane 1 issues P.V(j) once the softmax has written P^T(j). Neither waits on the other's
+        // barriers, so QK runs up to two stages ahead of the softmax.
+        if (lane < 2) {
             bool ok = true;
             uint32_t fbase = 0;  // ring fills of the earlier items
-            uint32_t J = 0;      // stages issued so far (all items)
+            uint32_t J = 0;      // stages of the earlier items and this one
             int item_i = 0;
             auto wait = [&](uint32_t bar, uint32_t parity) {
                 if (ok && !mbar_wait_bounded(bar, parity, kWaitLimitNs)) {
@@ -301,64 +411,65 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 return ok;
             };
-            // P.V of stage jj (global stage JJ) of the current item
-            auto pv = [&](int jj, uint32_t JJ) {
-                const uint32_t f = fbase + 2 * jj + 1;
-                const int e = f % C::kRing;
-                if (!wait(full(e), (f / C::kRing) & 1)) return;
-                if (!wait(p_full, JJ & 1)) return;
-                if (jj == 0 && item_i > 0 && !wait(o_empty, (item_i - 1) & 1)) return;
-                tc_fence_after();
-                const uint32_t sV = ring + e * C::kEntry;
-#pragma unroll
-                for (int kk = 0; kk < C::kTP / 16; ++kk) {
-                    const uint64_t a = smem_desc(sV + kk * 16 * 128, C::kBoxB, 1024, kSwz128);
-                    umma_ss(tO, a, smem_desc(sPhi + kk * 16 * 64, C::kTP * 64, 512, kSwz64), kIdescPV,
-                            (jj > 0 || kk > 0) ? 1u : 0u);
-                }
-#pragma unroll
-                for (int kk = 0; kk < C::kTP / 16; ++kk) {
-                    const uint64_t a = smem_desc(sV + kk * 16 * 128, C::kBoxB, 1024, kSwz128);
-                    umma_ss(tO, a, smem_desc(sPlo + kk * 16 * 64, C::kTP * 64, 512, kSwz64), kIdescPV, 1u);
-                }
-                umma_commit(empty(e));
-                umma_commit(p_empty);
-            };
-            for (int w = blockIdx.x; w < n_work && ok; w += gridDim.x) {
+            for (int k = 0; k < n_cand && ok; ++k) {
                 TcWork wk;
-                if (!tc_work(p, w, P, wk) || wk.n_local <= 0) continue;
+                if (!tc_get(p, L, k, P, wk) || wk.n_local <= 0) continue;
                 const int n_st = (wk.n_local + C::kPPS - 1) / C::kPPS;
-                if (!wait(q_full, item_i & 1)) break;
-                for (int j = 0; j < n_st && ok; ++j) {
-                    const uint32_t f = fbase + 2 * j;
-                    const int e = f % C::kRing;
-                    const int sb = J & 1;
-                    if (!wait(full(e), (f / C::kRing) & 1)) break;
-                    if (J >= 2 && !wait(s_empty(sb), ((J >> 1) - 1) & 1)) break;
-                    tc_fence_after();
-                    const uint32_t sK = ring + e * C::kEntry;
+                if (lane == 0) {
+                    if (!wait(q_full, item_i & 1)) break;
+                    for (int j = 0; j < n_st; ++j, ++J) {
+                        const uint32_t f = fbase + 2 * j;
+                        const int e = f % C::kRing;
+                        const int sb = J & 1;
+                        if (!wait(full(e), (f / C::kRing) & 1)) break;
+                        if (J >= 2 && !wait(s_empty(sb), ((J >> 1) - 1) & 1)) break;
+                        tc_fence_after();
+                        const uint32_t sK = ring + e * C::kEntry;
 #pragma unroll
-                    for (int kk = 0; kk < DH / 16; ++kk) {
-                        const uint32_t koff = (kk >> 2) * C::kBoxB + (kk & 3) * 32;
-                        const uint32_t qoff = (kk >> 2) * G * 128 + (kk & 3) * 32;
-                        umma_ss(tS + sb * G, smem_desc(sK + koff, 16, 1024, kSwz128),
-                                smem_desc(sQ + qoff, 16, 1024, kSwz128), kIdescQK, kk > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < DH / 16; ++kk) {
+                            const uint32_t koff = (kk >> 2) * C::kBoxB + (kk & 3) * 32;
+                            const uint32_t qoff = (kk >> 2) * C::kQRowsB + (kk & 3) * 32;
+                            umma_ss(tS + sb * N, smem_desc(sK + koff, 16, 1024, kSwz128),
+                                    smem_desc(sQ + qoff, 16, 1024, kSwz128), kIdescQK, kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit(s_full(sb));
+                        umma_commit(empty(e));
+                        if (j == n_st - 1) umma_commit(q_empty);
                     }
-                    umma_commit(s_full(sb));
-                    umma_commit(empty(e));
-                    if (j == n_st - 1) umma_commit(q_empty);
-                    if (j > 0) pv(j - 1, J - 1);
-                    ++J;
+                } else {
+                    for (int j = 0; j < n_st; ++j, ++J) {
+                        const uint32_t f = fbase + 2 * j + 1;
+                        const int e = f % C::kRing;
+                        if (!wait(full(e), (f / C::kRing) & 1)) break;
+                        if (!wait(p_full(J & 1), (J >> 1) & 1)) break;
+                        if (j == 0 && item_i > 0 && !wait(o_empty, (item_i - 1) & 1)) break;
+                        tc_fence_after();
+                        const uint32_t sV = ring + e * C::kEntry;
+#pragma unroll
+                        for (int kk = 0; kk < C::kTP / 16; ++kk) {
+                            const uint64_t a = smem_desc(sV + kk * 16 * 128, C::kBoxB, 1024, kSwz128);
+                            umma_ss(tO, a, smem_desc(sPhi(J) + kk * 16 * C::kPRow, C::kPB, C::kPAtom, C::kPSwz),
+                                    kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+                        }
+#pragma unroll
+                        for (int kk = 0; kk < C::kTP / 16; ++kk) {
+                            const uint64_t a = smem_desc(sV + kk * 16 * 128, C::kBoxB, 1024, kSwz128);
+                            umma_ss(tO, a,
+                                    smem_desc(sPhi(J) + C::kPB + kk * 16 * C::kPRow, C::kPB, C::kPAtom, C::kPSwz),
+                                    kIdescPV, 1u);
+                        }
+                        umma_commit(empty(e));
+                        umma_commit(p_empty(J & 1));
+                    }
+                    if (ok) umma_commit(o_full);
                 }
-                if (!ok) break;
-                pv(n_st - 1, J - 1);
-                umma_commit(o_full);
                 fbase += 2 * n_st;
                 ++item_i;
             }
-            // every MMA issued has completed before tensor memory is released
-            umma_commit(done_bar);
-            if (!mbar_wait_bounded(done_bar, 0, kWaitLimitNs)) raise_err(p.err, KV_DEV_ERR_TIMEOUT);
+            // every MMA this thread issued has completed before tensor memory is released
+            const uint32_t done = lane == 0 ? done_qk : done_pv;
+            umma_commit(done);
+            if (!mbar_wait_bounded(done, 0, kWaitLimitNs)) raise_err(p.err, KV_DEV_ERR_TIMEOUT);
         }
         __syncwarp();
     } else {
@@ -397,9 +508,9 @@ __global__ void __launch_bounds__(192, 1)
             if (!wk.split_mode)
                 for (int h = 0; h < G; ++h) p.out[((int64_t)wk.b * p.H_q + wk.kvh * G + h) * DH + r] = 0.f;
         };
-        for (int w = blockIdx.x; w < n_work; w += gridDim.x) {
+        for (int k = 0; k < n_cand; ++k) {
             TcWork wk;
-            if (!tc_work(p, w, P, wk)) continue;
+            if (!tc_get(p, L, k, P, wk)) continue;
             if (wk.bad_len && r == 0 && wk.split == 0 && p.items == nullptr) raise_err(p.err, KV_DEV_ERR_SEQ_LEN);
             if (wk.n_local <= 0 || !ok) {
                 zero_rows(wk);
@@ -417,12 +528,11 @@ __global__ void __launch_bounds__(192, 1)
                 for (int h = 0; h < G; ++h) s[h] = -INFINITY;
                 if (wait(okl, s_full(sb), (J >> 1) & 1)) {
                     tc_fence_after();
-                    uint32_t a[16], b2[16];
-                    tmem_ld16(tS + sb * G + lane_addr, a);
-                    tmem_ld16(tS + sb * G + 16 + lane_addr, b2);
+                    uint32_t a[N];
+                    tmem_ld_cols<N>(tS + sb * N + lane_addr, a);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int h = 0; h < 16; ++h) s[h] = __uint_as_float(a[h]), s[16 + h] = __uint_as_float(b2[h]);
+                    for (int h = 0; h < G; ++h) s[h] = __uint_as_float(a[h]);
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(s_empty(sb));
@@ -454,7 +564,7 @@ __global__ void __launch_bounds__(192, 1)
                     float mx[G];
 #pragma unroll
                     for (int h = 0; h < G; ++h) mx[h] = s[h];
-                    cta_heads_reduce<true>(mx, red, sw, lane, rbuf);
+                    cta_heads_reduce<G, true>(mx, red, sw, lane, rbuf);
 #pragma unroll
                     for (int h = 0; h < G; ++h) {
                         const float mn = fmaxf(m_ref[h], mx[h]);
@@ -464,42 +574,46 @@ __global__ void __launch_bounds__(192, 1)
                     }
                     rescale_o = j > 0;
                 }
-                // P.V of the previous stage has finished: the P^T tiles are free and O^T is settled
-                if (J > 0 && !wait(okl, p_empty, (J - 1) & 1)) {
+                // P^T buffer J & 1 is free once P.V(J - 2) has finished; a rescale of O^T also needs P.V(J - 1)
+                bool okw = true;
+                if (J >= 2) okw = wait(okl, p_empty(J & 1), ((J >> 1) - 1) & 1);
+                if (okw && rescale_o) okw = wait(okl, p_empty((J - 1) & 1), ((J - 1) >> 1) & 1);
+                if (!okw) {
                     ok = false;  // the next flag exchange stops every warp
                     ++J;
                     continue;
                 }
                 if (rescale_o) {
                     tc_fence_after();
-                    uint32_t a[16], b2[16];
-                    tmem_ld16(tO + lane_addr, a);
-                    tmem_ld16(tO + 16 + lane_addr, b2);
+                    uint32_t a[N];
+                    tmem_ld_cols<N>(tO + lane_addr, a);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int h = 0; h < 16; ++h) {
-                        a[h] = __float_as_uint(__uint_as_float(a[h]) * alpha[h]);
-                        b2[h] = __float_as_uint(__uint_as_float(b2[h]) * alpha[16 + h]);
-                    }
-                    tmem_st16(tO + lane_addr, a);
-                    tmem_st16(tO + 16 + lane_addr, b2);
+                    for (int h = 0; h < G; ++h) a[h] = __float_as_uint(__uint_as_float(a[h]) * alpha[h]);
+                    tmem_st_cols<N>(tO + lane_addr, a);
                     tmem_wait_st();
                 }
-                // probabilities -> P^T row r (hi and residual lo), 64-byte swizzle
-                uint32_t hi[G / 2], lo[G / 2];
+                // probabilities -> P^T row r (hi and residual lo; padding heads are zero), swizzled rows
+                uint32_t hi[N / 2], lo[N / 2];
 #pragma unroll
-                for (int i = 0; i < G / 2; ++i) {
-                    const float p0 = s[2 * i] == -INFINITY ? 0.f : exp2f(s[2 * i] - m_ref[2 * i]);
-                    const float p1 = s[2 * i + 1] == -INFINITY ? 0.f : exp2f(s[2 * i + 1] - m_ref[2 * i + 1]);
-                    lp[2 * i] += p0;
-                    lp[2 * i + 1] += p1;
-                    pack2_split<kBF16>(p0, p1, hi[i], lo[i]);
+                for (int i = 0; i < N / 2; ++i) {
+                    if (2 * i < G) {
+                        const float p0 = s[2 * i] == -INFINITY ? 0.f : exp2f(s[2 * i] - m_ref[2 * i]);
+                        const float p1 = s[2 * i + 1] == -INFINITY ? 0.f : exp2f(s[2 * i + 1] - m_ref[2 * i + 1]);
+                        lp[2 * i] += p0;
+                        lp[2 * i + 1] += p1;
+                        pack2_split_fast<kBF16>(p0, p1, hi[i], lo[i]);
+                    } else {
+                        hi[i] = lo[i] = 0u;
+                    }
                 }
 #pragma unroll
-                for (int c = 0; c < G / 8; ++c) {
-                    const uint32_t off = r * 64 + ((c ^ ((r >> 1) & 3)) << 4);
-                    sts128(sPhi + off, hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
-                    sts128(sPlo + off, lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
+                for (int c = 0; c < N / 8; ++c) {
+                    // 16-byte chunk c of the row, placed as the MN-major swizzle of rows of kPRow bytes expects
+                    const uint32_t phys = C::kPRow == 32 ? (c ^ ((r >> 2) & 1)) : (c ^ ((r >> 1) & 3));
+                    const uint32_t off = r * C::kPRow + (phys << 4);
+                    sts128(sPhi(J) + off, hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
+                    sts128(sPhi(J) + C::kPB + off, lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
                 }
                 // a masked token's V row may hold stale bytes (even NaN): zero it before P.V
                 if (!valid) {
@@ -512,7 +626,7 @@ __global__ void __launch_bounds__(192, 1)
                 fence_proxy_async_smem();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(p_full);
+                if (lane == 0) mbar_arrive(p_full(J & 1));
                 ++J;
             }
             // ---- epilogue: O^T row r, row sums over the CTA, output or partials
@@ -528,18 +642,17 @@ __global__ void __launch_bounds__(192, 1)
             fbase += 2 * n_st;
             float o[G];
             {
-                uint32_t a[16], b2[16];
-                tmem_ld16(tO + lane_addr, a);
-                tmem_ld16(tO + 16 + lane_addr, b2);
+                uint32_t a[N];
+                tmem_ld_cols<N>(tO + lane_addr, a);
                 tmem_wait_ld();
 #pragma unroll
-                for (int h = 0; h < 16; ++h) o[h] = __uint_as_float(a[h]), o[16 + h] = __uint_as_float(b2[h]);
+                for (int h = 0; h < G; ++h) o[h] = __uint_as_float(a[h]);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(o_empty);
             ++item_i;
-            cta_heads_reduce<false>(lp, red, sw, lane, rbuf);
+            cta_heads_reduce<G, false>(lp, red, sw, lane, rbuf);
             const int64_t hq0 = (int64_t)wk.b * p.H_q + (int64_t)wk.kvh * G;
             if (!wk.split_mode) {
 #pragma unroll

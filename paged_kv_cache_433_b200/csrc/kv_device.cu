@@ -267,11 +267,15 @@ bool use_mma(int32_t dtype, int32_t g) {
     return g <= 64;
 }
 
-// The tcgen05 kernel (decode_tc.cuh): 16-bit K/V, GQA group of 32 heads,
-// Dh = 128, no fused rotation; chosen by the automatic kernel selection.
+// The tcgen05 kernel (decode_tc.cuh): 16-bit K/V, Dh = 128, no fused rotation,
+// GQA groups of 4, 8, 16 or 32 heads when selected explicitly; the automatic
+// selection takes it for groups of 32 (MQA-shaped), where the warp-MMA
+// kernel is bound by its per-page MMA work.
 bool tc_ok(int32_t dtype, int32_t g, int32_t Dh, bool rope) {
-    return g_kernel_kind.load(std::memory_order_relaxed) == KV_DECODE_KERNEL_AUTO &&
-           (dtype == KV_DTYPE_BF16 || dtype == KV_DTYPE_F16) && g == 32 && Dh == 128 && !rope;
+    const int kind = g_kernel_kind.load(std::memory_order_relaxed);
+    if ((dtype != KV_DTYPE_BF16 && dtype != KV_DTYPE_F16) || Dh != 128 || rope) return false;
+    if (kind == KV_DECODE_KERNEL_TCGEN05) return g == 4 || g == 8 || g == 16 || g == 32;
+    return kind == KV_DECODE_KERNEL_AUTO && g == 32;
 }
 
 size_t workspace_for(int32_t B, int32_t H_q, int32_t Dh, int32_t S) {
@@ -400,7 +404,8 @@ int kv_copy_pages(void* k_pages, void* v_pages, const int32_t* src_pages, const 
 }
 
 int paged_decode_set_kernel(int32_t kind) {
-    if (kind != KV_DECODE_KERNEL_AUTO && kind != KV_DECODE_KERNEL_SIMT && kind != KV_DECODE_KERNEL_MMA)
+    if (kind != KV_DECODE_KERNEL_AUTO && kind != KV_DECODE_KERNEL_SIMT && kind != KV_DECODE_KERNEL_MMA &&
+        kind != KV_DECODE_KERNEL_TCGEN05)
         return KV_ERR_ARG;
     g_kernel_kind.store(kind, std::memory_order_relaxed);
     return KV_OK;
@@ -684,7 +689,8 @@ int paged_prefill_attention(float* out, const void* q, const int32_t* q_start, i
     if (static_cast<int64_t>(num_pages) * H_kv * page_size >= (1LL << 31)) return KV_ERR_UNSUPPORTED;
     // tcgen05 kernel: 128 MMA rows per CTA (128 / g chunk tokens x g heads); warp-MMA kernel: 64 rows
     // (64 / g tokens, four 16-row slices)
-    const bool tc = g_kernel_kind.load(std::memory_order_relaxed) == KV_DECODE_KERNEL_AUTO && Dh == 128 && 128 % g == 0;
+    const int kind = g_kernel_kind.load(std::memory_order_relaxed);
+    const bool tc = (kind == KV_DECODE_KERNEL_AUTO || kind == KV_DECODE_KERNEL_TCGEN05) && Dh == 128 && 128 % g == 0;
     const int32_t q_tile = tc ? 128 / g : 64 / g;
     DecodeParams p{};
     p.out = out;

@@ -16,21 +16,26 @@
 //   O[128 x Dh]  += P[128 x 128] . V_stage               (TS: P in tensor memory,
 //                                                          V MN-major)
 // S is triple-buffered in tensor memory (3 x 128 columns) and O takes the
-// last 128 columns. Thread r of the four softmax warps owns row r: the whole
-// row max, exponentials and sum stay in its registers (no shuffles). P is
-// written back over its own S columns as a bf16 (fp16) pair: hi = RN(p) in
-// columns 0..63, lo = RN(p - hi) in 64..127; the P.V MMA runs on both, so the
-// probabilities carry ~2^-16 relative precision into the product.
+// last 128 columns. Each row is owned by two threads of the eight softmax
+// warps (warps w and w + 4 share a tensor-memory lane quarter; one takes
+// columns 0..63, the other 64..127): exponentials and partial sums stay in
+// registers, the two halves of a row meet once per stage in shared memory to
+// agree on the row maximum. P is
+// written back over its own S columns as a 16-bit pair: hi in columns 0..63,
+// the residual lo = p - hi in 64..127 (bf16: both truncated with integer
+// operations; fp16: rounded); the P.V MMA runs on both, so the probabilities
+// carry ~2^-14 relative precision into the product.
 // The reference maximum of a row moves only when a score exceeds it by more
 // than 2^8; the row's O and l are then rescaled (o = u / l for any common
 // reference).
 //
-// Warps (192 threads, one CTA per SM by tensor memory and shared memory):
+// Warps (320 threads, one CTA per SM by tensor memory and shared memory):
 //   warp 0     producer: per stage the K then V boxes of its pages (P rows x
-//              128 bytes, 128-byte swizzle) into a ring of six 32 KB entries;
-//   warp 1     tensor memory allocation; lane 0 issues QK(0), QK(1), then per
-//              stage PV(j) and QK(j + 2);
-//   warps 2-5  load the Q tile (swizzled stores), softmax, epilogue.
+//              128 bytes, 128-byte swizzle) into a ring of five 32 KB entries;
+//   warp 1     tensor memory allocation; lane 0 issues the QK(j), lane 1 the
+//              P.V(j), each paced only by its own barriers;
+//   warps 2-9  load the Q tile (swizzled stores), softmax, epilogue; each pair
+//              of warps of one lane quarter syncs on its own named barrier.
 // Every wait is bounded (KV_DEV_ERR_TIMEOUT); block-table entries outside
 // [0, num_pages) are never loaded (their keys are masked,
 // KV_DEV_ERR_PAGE_RANGE).
@@ -50,16 +55,18 @@ struct PfCfg {
     static constexpr int kBoxCols = DH / 64;
     static constexpr int kBoxB = kTP * 128;      // one 128-byte box column of an entry
     static constexpr int kEntry = kBoxCols * kBoxB;
-    static constexpr int kRing = 6;              // K, V of three stages
+    static constexpr int kRing = 5;              // K / V entries (two and a half stages)
     static constexpr int kQB = 128 * DH * 2;     // Q tile: 128 rows
     static constexpr int kOffQ = kRing * kEntry;
     static constexpr int kOffBad = kOffQ + kQB;
-    static constexpr int kOffBar = (kOffBad + 4 * kRing + 7) / 8 * 8;
-    // full[6], empty[6], q_full, s_full[3], p_full[2], p_empty, o_full, done
-    static constexpr int kNumBars = 2 * kRing + 1 + 3 + 5;
+    static constexpr int kOffX = (kOffBad + 4 * kRing + 15) / 16 * 16;  // row exchange: [2][2][128] floats + ints
+    static constexpr int kOffBar = kOffX + 2 * 2 * 128 * 4 * 2;
+    // full[R], empty[R], q_full, s_full[3], p_full[2], p_empty[3], o_full, done (QK), done (PV)
+    static constexpr int kNumBars = 2 * kRing + 1 + 3 + 2 + 3 + 3;
     static constexpr int kOffTmem = kOffBar + 8 * kNumBars;
     static constexpr int kSmem = 1024 + kOffTmem + 16;
-    static constexpr int kThreads = 192;
+    static constexpr int kThreads = 320;
+    static constexpr int kSoftmaxWarps = 8;
     static constexpr uint32_t kTmemCols = 512;   // S x 3 (384) + O (128)
     static_assert(DH == 128, "instance: Dh = 128");
     static_assert(kPPS * kBoxCols <= 32, "one TMA box per lane");
@@ -67,7 +74,7 @@ struct PfCfg {
 };
 
 template <int KT, int DH, int P>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     paged_prefill_tc_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                             const __grid_constant__ CUtensorMap tmap_v) {
     using C = PfCfg<DH, P>;
@@ -119,9 +126,11 @@ __global__ void __launch_bounds__(192, 1)
     // P of stage j is announced on p_full(j & 1): the softmax of stage j + 1 may finish before the MMA
     // thread has waited for stage j, so one barrier would run a whole phase ahead of its waiter
     auto p_full = [&](int i) { return q_full + 32u + 8u * i; };
-    const uint32_t p_empty = q_full + 48;
-    const uint32_t o_full = q_full + 56;
-    const uint32_t done_bar = q_full + 64;
+    // P.V(j) completion is announced on p_empty(j % 3), the barrier of the S columns it read
+    auto p_empty = [&](int i) { return q_full + 48u + 8u * i; };
+    const uint32_t o_full = q_full + 72;
+    const uint32_t done_qk = q_full + 80;
+    const uint32_t done_pv = q_full + 88;
     volatile int* stage_bad = reinterpret_cast<volatile int*>(smem + C::kOffBad);
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::kOffTmem);
 
@@ -130,13 +139,14 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(full(e), 1);
             mbar_init(empty(e), 1);
         }
-        mbar_init(q_full, 4);
+        mbar_init(q_full, C::kSoftmaxWarps);
         for (int i = 0; i < 3; ++i) mbar_init(s_full(i), 1);
-        mbar_init(p_full(0), 4);
-        mbar_init(p_full(1), 4);
-        mbar_init(p_empty, 1);
+        mbar_init(p_full(0), C::kSoftmaxWarps);
+        mbar_init(p_full(1), C::kSoftmaxWarps);
+        for (int i = 0; i < 3; ++i) mbar_init(p_empty(i), 1);
         mbar_init(o_full, 1);
-        mbar_init(done_bar, 1);
+        mbar_init(done_qk, 1);
+        mbar_init(done_pv, 1);
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -194,7 +204,9 @@ __global__ void __launch_bounds__(192, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issue
-        if (lane == 0) {
+        // Lane 0 issues QK(j) once K(j) has landed and P.V(j - 3) has released S columns j % 3; lane 1
+        // issues P.V(j) once the softmax has written P(j). Neither waits on the other's barriers.
+        if (lane < 2) {
             bool ok = true;
             auto wait = [&](uint32_t bar, uint32_t parity) {
                 if (ok && !mbar_wait_bounded(bar, parity, kWaitLimitNs)) {
@@ -203,33 +215,32 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 return ok;
             };
-            auto qk = [&](int j) {
-                const uint32_t f = 2 * j;
-                const int e = f % C::kRing;
-                if (!wait(full(e), (f / C::kRing) & 1)) return;
-                tc_fence_after();
-                const uint32_t sK = ring + e * C::kEntry;
-                const uint32_t tS = tmem + (j % 3) * C::kTP;
+            if (lane == 0) {
+                if (wait(q_full, 0)) {
+                    for (int j = 0; j < n_st; ++j) {
+                        const uint32_t f = 2 * j;
+                        const int e = f % C::kRing;
+                        if (!wait(full(e), (f / C::kRing) & 1)) break;
+                        if (j >= 3 && !wait(p_empty(j % 3), ((j - 3) / 3) & 1)) break;
+                        tc_fence_after();
+                        const uint32_t sK = ring + e * C::kEntry;
+                        const uint32_t tS = tmem + (j % 3) * C::kTP;
 #pragma unroll
-                for (int kk = 0; kk < DH / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * C::kBoxB + (kk & 3) * 32;
-                    umma_ss(tS, smem_desc(sQ + off, 16, 1024, kSwz128), smem_desc(sK + off, 16, 1024, kSwz128),
-                            kIdescQK, kk > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < DH / 16; ++kk) {
+                            const uint32_t off = (kk >> 2) * C::kBoxB + (kk & 3) * 32;
+                            umma_ss(tS, smem_desc(sQ + off, 16, 1024, kSwz128), smem_desc(sK + off, 16, 1024, kSwz128),
+                                    kIdescQK, kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit(s_full(j % 3));
+                        umma_commit(empty(e));
+                    }
                 }
-                umma_commit(s_full(j % 3));
-                umma_commit(empty(e));
-            };
-            if (wait(q_full, 0)) {
-                qk(0);
-                if (n_st > 1) qk(1);
-                for (int j = 0; j < n_st && ok; ++j) {
+            } else {
+                for (int j = 0; j < n_st; ++j) {
                     const uint32_t f = 2 * j + 1;
                     const int e = f % C::kRing;
                     if (!wait(full(e), (f / C::kRing) & 1)) break;
                     if (!wait(p_full(j & 1), (j >> 1) & 1)) break;
-                    // P.V(j - 1) has finished before P.V(j) is committed (so p_empty never runs two phases
-                    // ahead of this wait) and before QK(j + 2) reuses its S columns
-                    if (j >= 1 && !wait(p_empty, (j - 1) & 1)) break;
                     tc_fence_after();
                     const uint32_t sV = ring + e * C::kEntry;
                     const uint32_t tP = tmem + (j % 3) * C::kTP;
@@ -242,32 +253,37 @@ __global__ void __launch_bounds__(192, 1)
                         umma_ts(tO, tP + C::kTP / 2 + kk * 8, smem_desc(sV + kk * 16 * 128, C::kBoxB, 1024, kSwz128),
                                 kIdescPV, 1u);
                     umma_commit(empty(e));
-                    umma_commit(p_empty);
-                    if (j + 2 < n_st) qk(j + 2);  // S columns (j + 2) % 3 last held P(j - 1), now consumed
+                    umma_commit(p_empty(j % 3));
                 }
                 if (ok) umma_commit(o_full);
             }
-            umma_commit(done_bar);
-            if (!mbar_wait_bounded(done_bar, 0, kWaitLimitNs)) raise_err(p.err, KV_DEV_ERR_TIMEOUT);
+            const uint32_t done = lane == 0 ? done_qk : done_pv;
+            umma_commit(done);
+            if (!mbar_wait_bounded(done, 0, kWaitLimitNs)) raise_err(p.err, KV_DEV_ERR_TIMEOUT);
         }
         __syncwarp();
     } else {
         // ------------------------------------------------------------ Q tile, softmax, epilogue
         const int quarter = warp & 3;
+        const int half = (warp - 2) >> 2;    // key columns [64 half, 64 half + 64) of S, dims of O likewise
         const int r = quarter * 32 + lane;   // MMA row: chunk token t0 + r / g, head kvh * g + r % g
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+        const uint32_t pair_bar = 1 + quarter;  // named barrier of the two warps that share row r
         const int tr = r / g;
         const bool row_valid = tr < nt;
         const int pos = pos0 + tr;           // this row sees keys 0 .. pos
         const int64_t qrow = ((int64_t)(qs0 + t0 + tr) * p.H_q + (int64_t)kvh * g + r % g);
-        // Q row r -> swizzled K-major tile (two 128-byte box columns of 128 rows)
+        float* xm = reinterpret_cast<float*>(smem + C::kOffX);        // [buf][half][row] partial maxima / sums
+        int* xok = reinterpret_cast<int*>(smem + C::kOffX) + 2 * 2 * 128;
+        int xbuf = 0;
+        // this thread's half of Q row r -> box column `half` of the swizzled K-major tile
         {
-            const uint4* src = static_cast<const uint4*>(p.q) + qrow * (DH / 8);
+            const uint4* src = static_cast<const uint4*>(p.q) + qrow * (DH / 8) + half * 8;
 #pragma unroll
-            for (int c = 0; c < DH / 8; ++c) {
+            for (int c = 0; c < 8; ++c) {
                 uint4 v = make_uint4(0u, 0u, 0u, 0u);
                 if (row_valid) v = src[c];
-                const uint32_t dst = sQ + (c >> 3) * (128 * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+                const uint32_t dst = sQ + half * (128 * 128) + r * 128 + ((c ^ (r & 7)) << 4);
                 asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x), "r"(v.y), "r"(v.z),
                              "r"(v.w)
                              : "memory");
@@ -278,52 +294,66 @@ __global__ void __launch_bounds__(192, 1)
         }
         bool ok = true;
         // warp-uniform outcome: the tensor-memory loads and stores after a wait are warp-collective
-        auto wait = [&](uint32_t bar, uint32_t parity) {
-            if (ok && !mbar_wait_bounded(bar, parity, kWaitLimitNs)) {
+        auto wait = [&](bool& okl, uint32_t bar, uint32_t parity) {
+            if (okl && !mbar_wait_bounded(bar, parity, kWaitLimitNs)) {
                 raise_err(p.err, KV_DEV_ERR_TIMEOUT);
-                ok = false;
+                okl = false;
             }
-            ok = __all_sync(0xffffffffu, ok);
-            return ok;
+            okl = __all_sync(0xffffffffu, okl);
+            return okl;
+        };
+        // the two halves of row r meet: returns the partner's value; `okl` becomes the AND of both
+        auto meet = [&](float v, bool& okl) {
+            xm[(xbuf * 2 + half) * 128 + r] = v;
+            xok[(xbuf * 2 + half) * 128 + r] = okl ? 1 : 0;
+            named_bar_sync(pair_bar, 64);
+            const float other = xm[(xbuf * 2 + (half ^ 1)) * 128 + r];
+            okl = __all_sync(0xffffffffu, okl && xok[(xbuf * 2 + (half ^ 1)) * 128 + r] != 0);
+            xbuf ^= 1;
+            return other;
         };
         const float sl2 = p.scale_log2;
         float m_ref = -INFINITY, l = 0.f;
+        constexpr int kH = C::kTP / 2;       // key columns per thread
         for (int j = 0; j < n_st; ++j) {
-            if (!wait(s_full(j % 3), (j / 3) & 1)) break;
-            tc_fence_after();
+            bool okl = ok;
             const uint32_t tS = tmem + (j % 3) * C::kTP + lane_addr;
-            float s[C::kTP];
-            {
-                uint32_t a[32];
+            float s[kH];
+            if (wait(okl, s_full(j % 3), (j / 3) & 1)) {
+                tc_fence_after();
+                uint32_t a[32], b2[32];
+                tmem_ld32(tS + half * kH, a);
+                tmem_ld32(tS + half * kH + 32, b2);
+                tmem_wait_ld();
 #pragma unroll
-                for (int q4 = 0; q4 < C::kTP / 32; ++q4) {
-                    tmem_ld32(tS + q4 * 32, a);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) s[q4 * 32 + i] = __uint_as_float(a[i]);
-                }
+                for (int i = 0; i < 32; ++i) s[i] = __uint_as_float(a[i]), s[32 + i] = __uint_as_float(b2[i]);
             }
             // keys of this stage: kbase .. kbase + 127; the V entry carries the skipped-page mask
             const uint32_t fv = 2 * j + 1;
             const int ev = fv % C::kRing;
-            if (!wait(full(ev), (fv / C::kRing) & 1)) break;
             const int kbase = j * C::kTP;
             const int np = min(C::kPPS, n_pages - j * C::kPPS);
-            const int bad = stage_bad[ev];
+            int bad = 0;
+            if (wait(okl, full(ev), (fv / C::kRing) & 1)) bad = stage_bad[ev];
             // keys this row may see in the stage: [0, lim); pages skipped or not loaded are masked
             const int lim = row_valid ? min(C::kTP, pos + 1 - kbase) : 0;
             const bool full_stage = lim == C::kTP && np == C::kPPS && bad == 0;
-            if (!full_stage) {
+            if (!full_stage || !okl) {
 #pragma unroll
-                for (int c = 0; c < C::kTP; ++c) {
-                    const int pgi = c / P;
-                    if (c >= lim || pgi >= np || ((bad >> pgi) & 1)) s[c] = -INFINITY;
+                for (int c = 0; c < kH; ++c) {
+                    const int cc = half * kH + c, pgi = cc / P;
+                    if (!okl || cc >= lim || pgi >= np || ((bad >> pgi) & 1)) s[c] = -INFINITY;
                 }
             }
             float mx = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < C::kTP; ++c) mx = fmaxf(mx, s[c]);
-            const float mx2 = mx * sl2;  // sl2 > 0: the scaled maximum
+            for (int c = 0; c < kH; ++c) mx = fmaxf(mx, s[c]);
+            mx = fmaxf(mx, meet(mx, okl));
+            if (!okl) {
+                ok = false;  // both halves of every row of this pair stop here
+                break;
+            }
+            const float mx2 = mx * sl2;  // sl2 > 0: the scaled maximum of the whole row
             // reference maximum: moves only when the row's max exceeds it by more than 2^8
             const bool need = mx2 > m_ref + 8.f;
             float alpha = 1.f;
@@ -333,46 +363,50 @@ __global__ void __launch_bounds__(192, 1)
                 l *= alpha;
             }
             if (j > 0 && __any_sync(0xffffffffu, need)) {
-                // O holds P.V of the earlier stages: wait for the last one, then rescale the rows that moved
-                if (!wait(p_empty, (j - 1) & 1)) break;
-                tc_fence_after();
-                uint32_t a[32];
-#pragma unroll
-                for (int q4 = 0; q4 < DH / 32; ++q4) {
-                    tmem_ld32(tO + lane_addr + q4 * 32, a);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) a[i] = __float_as_uint(__uint_as_float(a[i]) * alpha);
-                    tmem_st32(tO + lane_addr + q4 * 32, a);
+                // O holds P.V of the earlier stages: wait for the last one, then rescale this half of the rows
+                if (!wait(okl, p_empty((j - 1) % 3), ((j - 1) / 3) & 1)) {
+                    ok = false;  // the next meeting stops the pair
+                    continue;
                 }
+                tc_fence_after();
+                uint32_t a[32], b2[32];
+                tmem_ld32(tO + lane_addr + half * kH, a);
+                tmem_ld32(tO + lane_addr + half * kH + 32, b2);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    a[i] = __float_as_uint(__uint_as_float(a[i]) * alpha);
+                    b2[i] = __float_as_uint(__uint_as_float(b2[i]) * alpha);
+                }
+                tmem_st32(tO + lane_addr + half * kH, a);
+                tmem_st32(tO + lane_addr + half * kH + 32, b2);
                 tmem_wait_st();
             }
             // probabilities -> P over this S buffer: hi pairs in columns 0..63, residual pairs in 64..127
+            // (this thread's keys: hi columns 32 half .., lo columns 64 + 32 half ..)
             const float neg = (m_ref == -INFINITY) ? 0.f : -m_ref;
 #pragma unroll
-            for (int q4 = 0; q4 < C::kTP / 32; ++q4) {
+            for (int q2 = 0; q2 < 2; ++q2) {
                 uint32_t hi[16], lo[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const float x0 = s[q4 * 32 + 2 * i], x1 = s[q4 * 32 + 2 * i + 1];
-                    const float p0 = x0 == -INFINITY ? 0.f : exp2f(fmaf(x0, sl2, neg));
-                    const float p1 = x1 == -INFINITY ? 0.f : exp2f(fmaf(x1, sl2, neg));
+                    const float p0 = exp2f(fmaf(s[q2 * 32 + 2 * i], sl2, neg));  // exp2(-inf) = 0 for masked keys
+                    const float p1 = exp2f(fmaf(s[q2 * 32 + 2 * i + 1], sl2, neg));
                     l += p0 + p1;
-                    pack2_split<kBF16>(p0, p1, hi[i], lo[i]);
+                    pack2_split_fast<kBF16>(p0, p1, hi[i], lo[i]);
                 }
-                tmem_st16(tmem + (j % 3) * C::kTP + lane_addr + q4 * 16, hi);
-                tmem_st16(tmem + (j % 3) * C::kTP + lane_addr + C::kTP / 2 + q4 * 16, lo);
+                tmem_st16(tmem + (j % 3) * C::kTP + lane_addr + half * 32 + q2 * 16, hi);
+                tmem_st16(tmem + (j % 3) * C::kTP + lane_addr + C::kTP / 2 + half * 32 + q2 * 16, lo);
             }
             tmem_wait_st();
             // a key no row may see (past the tile, or on a page not loaded) may hold stale bytes: zero its V row
+            // (this thread: box column `half` of V row r)
             {
                 const int pgi = r / P;
                 if (kbase + r >= key_end || pgi >= np || ((bad >> pgi) & 1)) {
-                    const uint32_t vrow = ring + ev * C::kEntry + r * 128;
+                    const uint32_t vrow = ring + ev * C::kEntry + half * C::kBoxB + r * 128;
 #pragma unroll
-                    for (int bb = 0; bb < C::kBoxCols; ++bb)
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) sts128_zero(vrow + bb * C::kBoxB + c * 16);
+                    for (int c = 0; c < 8; ++c) sts128_zero(vrow + c * 16);
                 }
             }
             fence_proxy_async_smem();
@@ -380,26 +414,30 @@ __global__ void __launch_bounds__(192, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(p_full(j & 1));
         }
-        // ---- epilogue: O row / l
-        if (wait(o_full, 0)) {
-            tc_fence_after();
-            float* dst = p.out + qrow * DH;
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            uint32_t a[32];
+        // ---- epilogue: O row / l (this thread: dims 64 half .. 64 half + 63)
+        bool okl = ok;
+        if (wait(okl, o_full, 0)) tc_fence_after();
+        const float l_all = l + meet(l, okl);
+        if (okl) {
+            float* dst = p.out + qrow * DH + half * kH;
+            const float inv = l_all > 0.f ? 1.f / l_all : 0.f;
+            uint32_t a[32], b2[32];
+            tmem_ld32(tO + lane_addr + half * kH, a);
+            tmem_ld32(tO + lane_addr + half * kH + 32, b2);
+            tmem_wait_ld();
+            if (row_valid) {
 #pragma unroll
-            for (int q4 = 0; q4 < DH / 32; ++q4) {
-                tmem_ld32(tO + lane_addr + q4 * 32, a);
-                tmem_wait_ld();
-                if (row_valid) {
-#pragma unroll
-                    for (int i = 0; i < 32; i += 4)
-                        *reinterpret_cast<float4*>(dst + q4 * 32 + i) =
-                            make_float4(__uint_as_float(a[i]) * inv, __uint_as_float(a[i + 1]) * inv,
-                                        __uint_as_float(a[i + 2]) * inv, __uint_as_float(a[i + 3]) * inv);
+                for (int i = 0; i < 32; i += 4) {
+                    *reinterpret_cast<float4*>(dst + i) =
+                        make_float4(__uint_as_float(a[i]) * inv, __uint_as_float(a[i + 1]) * inv,
+                                    __uint_as_float(a[i + 2]) * inv, __uint_as_float(a[i + 3]) * inv);
+                    *reinterpret_cast<float4*>(dst + 32 + i) =
+                        make_float4(__uint_as_float(b2[i]) * inv, __uint_as_float(b2[i + 1]) * inv,
+                                    __uint_as_float(b2[i + 2]) * inv, __uint_as_float(b2[i + 3]) * inv);
                 }
             }
         } else if (row_valid) {
-            for (int d = 0; d < DH; ++d) p.out[qrow * DH + d] = 0.f;
+            for (int d = 0; d < kH; ++d) p.out[qrow * DH + half * kH + d] = 0.f;
         }
     }
 

@@ -20,7 +20,24 @@
 
 #include <cstdint>
 
+#include "ptx.cuh"
+
 namespace kvp {
+
+// The same split with integer arithmetic for bf16 (no conversion instruction):
+// hi = x truncated to bf16 (x - hi is then exact in fp32), lo = that residual
+// truncated to bf16. hi + lo carries x to ~2^-14 relative. fp16 pairs use the
+// rounding conversions above.
+template <bool IS_BF16>
+__device__ __forceinline__ void pack2_split_fast(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+    if constexpr (IS_BF16) {
+        const uint32_t h0 = __float_as_uint(x0) & 0xffff0000u, h1 = __float_as_uint(x1) & 0xffff0000u;
+        hi = __byte_perm(h0, h1, 0x7632);
+        lo = __byte_perm(__float_as_uint(x0 - __uint_as_float(h0)), __float_as_uint(x1 - __uint_as_float(h1)), 0x7632);
+    } else {
+        pack2_split<false>(x0, x1, hi, lo);
+    }
+}
 
 // ---- tensor memory allocation (one whole warp executes these) -------------
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {

@@ -1,6 +1,7 @@
-"""GPU parity of the fifth-generation tensor-core (tcgen05) decode kernel, the
-automatic choice for bf16/fp16 K/V with 32 query heads per KV head and
-Dh = 128 (MQA-shaped groups), against the fp64 oracle.
+"""GPU parity of the fifth-generation tensor-core (tcgen05) decode kernel
+against the fp64 oracle: selected explicitly (KV_DECODE_KERNEL_TCGEN05) for
+GQA groups of 4, 8, 16 and 32 heads, the automatic choice for groups of 32
+(MQA-shaped), bf16/fp16 K/V, Dh = 128.
 
 Covers: ragged and edge lengths (1, P-1, P, P+1, a full table, a row longer
 than one 128-token stage), grid splits and device-planned launches, the fused
@@ -26,6 +27,8 @@ def _built():
 
     build.build()
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    K.paged_decode_set_kernel(K.KV_DECODE_KERNEL_TCGEN05)
+    yield
     K.paged_decode_set_kernel(K.KV_DECODE_KERNEL_AUTO)
 
 
@@ -35,7 +38,8 @@ def _assert_tc(cfg, max_blocks, splits):
     return S
 
 
-TC_SHAPES = [("bf16", 16, 32, 1), ("fp16", 32, 32, 1), ("bf16", 32, 64, 2), ("fp16", 16, 96, 3)]
+TC_SHAPES = [("bf16", 16, 32, 1), ("fp16", 32, 32, 1), ("bf16", 32, 64, 2), ("fp16", 16, 96, 3),
+             ("bf16", 16, 32, 8), ("fp16", 32, 16, 2), ("bf16", 16, 32, 2), ("fp16", 16, 8, 1)]
 
 
 @pytest.mark.parametrize("dtype,P,H_q,H_kv", TC_SHAPES)
@@ -44,10 +48,11 @@ TC_SHAPES = [("bf16", 16, 32, 1), ("fp16", 32, 32, 1), ("bf16", 32, 64, 2), ("fp
 def test_tc_edge_lengths(dtype, P, H_q, H_kv, splits, fused):
     cfg = W.DecodeConfig(f"tc-edge-{dtype}-{P}-{H_q}-{H_kv}", dtype, B=7, H_q=H_q, H_kv=H_kv, Dh=128, page_size=P,
                          seed=41)
-    # after the append: 1, P-1, P, P+1, one 128-token stage + 5, three stages + 1, and a full table
-    lens = [0, P - 2, P - 1, P, 133 - 1, 3 * 128, 20 * P - 1]
-    st = build_cache(cfg, lens, extra_blocks=0)
-    assert st.max_blocks * P == lens[-1] + 1
+    # after the append: 1, P-1, P, P+1, one 128-token stage + 5, three stages + 1, and (one step) a full table
+    lens = [0, P - 2, P - 1, P, 133 - 1, 3 * 128, 30 * P - 1]
+    st = build_cache(cfg, lens, extra_blocks=1 if fused else 0, slack_pages=8)
+    if not fused:
+        assert st.max_blocks * P == lens[-1] + 1
     S = _assert_tc(cfg, st.max_blocks, splits)
     assert (S == 0) == (splits == 0)
     for step in range(2 if fused else 1):
@@ -149,6 +154,17 @@ def test_tc_empty_rows_and_error_bits():
     assert int(err.item()) & K.KV_DEV_ERR_SEQ_LEN and torch.count_nonzero(out).item() == 0
 
 
+def test_auto_selection_takes_tc_for_32_head_groups():
+    K.paged_decode_set_kernel(K.KV_DECODE_KERNEL_AUTO)
+    try:
+        assert K.paged_decode_launch_info(256, 32, 1, 128, 1030, 16, "bf16", 0) == (0, K.KV_DECODE_KERNEL_TCGEN05)
+        assert K.paged_decode_launch_info(64, 32, 8, 128, 270, 16, "bf16", 0)[1] == K.KV_DECODE_KERNEL_MMA
+        assert K.paged_decode_launch_info(4, 32, 1, 64, 100, 16, "bf16", 0)[1] == K.KV_DECODE_KERNEL_MMA
+        assert K.paged_decode_launch_info(4, 32, 1, 128, 100, 16, "fp32", 0)[1] == K.KV_DECODE_KERNEL_SIMT
+    finally:
+        K.paged_decode_set_kernel(K.KV_DECODE_KERNEL_TCGEN05)
+
+
 def test_tc_matches_warp_mma_kernel():
     """Same inputs through the tcgen05 kernel and the warp-MMA kernel: both within the oracle's tolerance."""
     cfg = W.DecodeConfig("tc-vs-mma", "bf16", B=9, H_q=32, H_kv=1, Dh=128, page_size=16, seed=45)
@@ -168,5 +184,5 @@ def test_tc_matches_warp_mma_kernel():
                                  torch.from_numpy(lens32).cuda(), cfg.scale, num_splits=0, workspace=ws)
         torch.cuda.synchronize()
     finally:
-        K.paged_decode_set_kernel(K.KV_DECODE_KERNEL_AUTO)
+        K.paged_decode_set_kernel(K.KV_DECODE_KERNEL_TCGEN05)
     check_close(out.cpu().numpy(), ref, "bf16", "warp mma")

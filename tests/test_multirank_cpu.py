@@ -72,3 +72,25 @@ def test_reference_arm_prints_one_contract_line():
     assert d["impl"] == "reference" and d["unit"] == "seq-steps/s" and d["value"] > 0 and d["higher_is_better"]
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_bench_byte_variants():
+    """Page-rounded K/V bytes and the split partials' bytes that the bench line reports beside the
+    algorithmic bytes (bench-side arithmetic, no GPU)."""
+    import sys
+
+    sys.path.insert(0, ROOT)
+    import bench
+    from paged_kv_cache_433_b200 import workloads as W
+
+    cfg = W.DecodeConfig("t", "bf16", B=2, H_q=8, H_kv=2, Dh=128, page_size=16)
+    lens = [17, 32]  # 2 and 2 pages
+    v = bench.kv_byte_variants(cfg, lens, 2, 2, S=1, C=0)
+    assert v["kv_bytes_page_rounded"] == 4 * 16 * 2 * 128 * 2 * 2 and v["partials_bytes_write_read"] == 0
+    # grid split of 2 splits, 1 page each: every row fills both splits -> 2 partials per (row, KV head)
+    v = bench.kv_byte_variants(cfg, lens, 2, 2, S=2, C=1)
+    assert v["partials_bytes_write_read"] == 2 * (2 * 2 * 2) * 4 * (128 + 2) * 4
+    # planned chunks of 2 pages: each row has one chunk -> no partials
+    assert bench.kv_byte_variants(cfg, lens, 2, 2, S=0, C=0, plan_C=2)["partials_bytes_write_read"] == 0
+    f = bench.roofline_fracs(4000.0, 8000.0)
+    assert f["frac"] == 0.5 and f["frac_datasheet"] == 0.5
