@@ -620,8 +620,12 @@ def run_prefill_bench(args, world, rank, local):
     per_s = ms / steps / 1e3
     keys = B * (n * ctx + n * (n + 1) // 2)                    # sum over chunk rows of the keys each one sees
     flops = 4.0 * cfg.Dh * cfg.H_q * keys                      # QK^T and PV, 2 flops per multiply-add
-    peak = peaks_tensor()
+    peak, peak_src = peaks_tensor()
     achieved = flops / per_s / 1e12
+    g = cfg.H_q // cfg.H_kv
+    # the library's choice for a chunk (automatic kernel kind): tcgen05 for Dh 128 when the group divides 128
+    prefill_kernel = ("paged_prefill_tc_kernel (tcgen05, 128-row tiles)" if cfg.Dh == 128 and 128 % g == 0
+                      else "paged_decode_mma_kernel (multi-token query)")
     return {
         "metric": "chunked prefill tokens/s; achieved TFLOP/s", "value": B * n * steps * world / (ms / 1e3),
         "unit": "tokens/s", "n_gpus": world, "steps": steps, "warmup": warm, "ms_per_step": ms / steps,
@@ -629,11 +633,11 @@ def run_prefill_bench(args, world, rank, local):
         "data": "synthetic (N(0,1) K/V, q)",
         "config": {"workload": f"chunked-prefill-{cfg.name}-B{B}-ctx{ctx}-chunk{n}", "B": B, "context": ctx, "chunk": n,
                    "H_q": cfg.H_q, "H_kv": cfg.H_kv, "Dh": cfg.Dh, "page_size": P,
-                   "l2": "K/V %.0f MB, re-read per 16-token tile mostly from L2; no flush" % (
+                   "l2": "K/V %.0f MB, re-read per query tile mostly from L2; no flush" % (
                        B * total * cfg.H_kv * cfg.Dh * 4 / 1e6)},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "peak_source": "measured cuBLAS bf16 dense (MEASURED_PEAKS bf16_tflops)",
-                     "traffic": None, "kernel": "paged_decode_mma_kernel (multi-token query)",
+                     "frac": achieved / peak, "peak_source": peak_src,
+                     "traffic": None, "kernel": prefill_kernel,
                      "flops_per_launch": flops, "launch_us": per_s * 1e6},
         "gpu_launches": steps, "e2e": None, "clocks": clocks,
     }
@@ -646,11 +650,13 @@ def dataclasses_replace(cfg, **kw):
 
 
 def peaks_tensor():
+    """(dense bf16 TFLOP/s, source): the measured cuBLAS burst figure when the peaks file is present, else the
+    earlier B200 measurement (1590 TFLOP/s burst)."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            return float(json.load(f)["bf16_tflops"])
+            return float(json.load(f)["bf16_tflops"]), "measured cuBLAS bf16 dense (burst)"
     except Exception:
-        return 1590.0
+        return 1590.0, "fallback (1590 TFLOP/s cuBLAS bf16 burst)"
 
 
 def run_e2e(wl, cfg, warm, steps, args, world):

@@ -24,11 +24,11 @@
 // maximum is reduced over the CTA, and O^T and the partial row sums are
 // rescaled (o = u / l holds for any common reference).
 //
-// Warp roles (192 threads, one CTA per SM, persistent over work items):
-//   warp 0     producer: Q tile (2-D TMA, 128-byte swizzle) and, per stage,
-//              the K then the V boxes of its pages (P rows x 128 bytes each)
-//              into a ring of six 32 KB entries (K and V of three stages);
-//              fused append of the new token when the item owns the last page.
+// Warp roles (224 threads, one CTA per SM, persistent over work items):
+//   warps 0, 6 producers: warp 0 the Q tile (2-D TMA, 128-byte swizzle) and
+//              the K boxes of each stage, warp 6 the V boxes (P rows x 128
+//              bytes each), into K and V entries of 32 KB; each writes its
+//              half of the fused append when the item owns the last page.
 //   warp 1     allocates tensor memory and resolves the CTA's work items
 //              into shared memory; lane 0 issues the QK(j), lane 1 the
 //              P.V(j), each committing onto the mbarriers the others wait on.
@@ -58,9 +58,13 @@ struct TcCfg {
     static constexpr int kBoxB = kTP * 128;      // one box column of an entry
     static constexpr int kEntry = kBoxCols * kBoxB;  // K (or V) of one stage
     static constexpr int kPB0 = kTP * kN * 2;    // one P^T tile (hi or lo)
-    // ring entries (K or V of a stage) that fit beside Q, two P^T buffers (hi + lo each) and the small arrays
-    static constexpr int kRing0 = (227 * 1024 - 1024 - 2048 - kBoxCols * kN * 128 - 4 * kPB0) / kEntry;
+    // ring entries (K or V of a stage) that fit beside two Q tiles, two P^T buffers (hi + lo each), the
+    // work list (3 KB) and the small arrays
+    static constexpr int kRing0 = (227 * 1024 - 1024 - 2048 - 3072 - 2 * kBoxCols * kN * 128 - 4 * kPB0) / kEntry;
     static constexpr int kRing = kRing0 > 6 ? 6 : kRing0;
+    // K of global stage J in entry J % kKSlots, V in kKSlots + J % kVSlots: a K entry is refilled as soon as
+    // its QK has run, whatever the P.V of older stages
+    static constexpr int kKSlots = (kRing + 1) / 2, kVSlots = kRing / 2;
     static constexpr int kQRowsB = kN * 128;     // one box column of the Q tile
     static constexpr int kQB = kBoxCols * kQRowsB;
     static constexpr int kPRow = kN * 2;         // bytes of one P^T row (token)
@@ -69,20 +73,21 @@ struct TcCfg {
     static constexpr uint32_t kPSwz = kPRow == 32 ? kSwz32 : kSwz64;
     static constexpr int kPAtom = 8 * kPRow;
     static constexpr int kOffQ = kRing * kEntry;
-    static constexpr int kOffP = kOffQ + kQB;
+    static constexpr int kOffP = kOffQ + 2 * kQB;  // two Q tiles (item parity)
     static constexpr int kOffRed = kOffP + 4 * kPB;          // 2 x [G][4] floats (after 2 x (hi, lo) P^T)
     static constexpr int kOffFlag = kOffRed + 2 * G * 4 * 4;  // 2 x 4 ints
     static constexpr int kOffBad = kOffFlag + 32;             // int per ring entry
     static constexpr int kMaxList = 96;          // work items of a CTA resolved once into shared memory
     static constexpr int kOffList = (kOffBad + 4 * kRing + 15) / 16 * 16;  // int4 x 2 per item
     static constexpr int kOffBar = kOffList + kMaxList * 32;
-    // full[R], empty[R], q_full, q_empty, s_full[2], s_empty[2], p_full[2], p_empty[2], o_full, o_empty,
-    // done (QK issuer), done (PV issuer)
-    static constexpr int kNumBars = 2 * kRing + 2 + 4 + 4 + 2 + 2;
+    // full[R], empty[R], q_full[2], q_empty[2], s_full[2], s_empty[2], p_full[2], p_empty[2], o_full[2],
+    // o_empty[2], done (QK issuer), done (PV issuer)
+    static constexpr int kNumBars = 2 * kRing + 4 + 4 + 4 + 4 + 2;
     static constexpr int kOffTmem = kOffBar + 8 * kNumBars;
     static constexpr int kSmem = 1024 + kOffTmem + 16;
-    static constexpr int kThreads = 192;
-    static constexpr uint32_t kTmemCols = 3 * kN <= 64 ? 64 : 128;  // S^T x 2 + O^T, N columns each
+    static constexpr int kThreads = 224;
+    static constexpr int kVWarp = 6;             // the V producer (warp 0 produces Q and K)
+    static constexpr uint32_t kTmemCols = 4 * kN <= 64 ? 64 : 128;  // S^T x 2 + O^T x 2, N columns each
     static_assert((G == 4 || G == 8 || G == 16 || G == 32) && DH == 128, "instances: g in {4, 8, 16, 32}, Dh = 128");
     static_assert(kPPS * kBoxCols <= 32, "one TMA box per lane");
     static_assert(kSmem <= 227 * 1024, "shared memory");
@@ -159,6 +164,27 @@ __device__ __forceinline__ bool tc_get(const DecodeParams& p, const TcList& L, i
         return true;
     }
     return tc_work(p, blockIdx.x + k * gridDim.x, P, wk);
+}
+
+// Fused append of the new token (position len - 1) for one of the pools: part 0
+// writes the K row, part 1 the V row (each producer warp writes the rows its own
+// TMA boxes will read, then fences them against the async proxy).
+__device__ __forceinline__ void append_new_token_part(const DecodeParams& p, int b, int kvh, int len, int P,
+                                                      int row_bytes, int lane, int part) {
+    const int pos = len - 1;
+    const int32_t page = p.block_tables[(int64_t)b * p.max_blocks + pos / P];
+    if (page >= 0 && page < p.num_pages) {
+        const int nch = row_bytes / 16;
+        const int64_t dst_row = ((int64_t)page * p.H_kv + kvh) * P + pos % P;
+        const int64_t src_row = (int64_t)b * p.H_kv + kvh;
+        const uint4* src = static_cast<const uint4*>(part ? p.v_new : p.k_new) + src_row * nch;
+        uint4* dst = static_cast<uint4*>(const_cast<void*>(part ? p.v_pages : p.k_pages)) + dst_row * nch;
+        for (int c = lane; c < nch; c += 32) dst[c] = src[c];
+        fence_proxy_async_global();
+    } else if (lane == 0 && part == 0) {
+        raise_err(p.err, KV_DEV_ERR_PAGE_RANGE);
+    }
+    __syncwarp();
 }
 
 // Per-head reduction over the 32 lanes of a warp of NV values per lane (NV a
@@ -240,7 +266,7 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, ui
 }
 
 template <int KT, int DH, int P, int G>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(224, 1)
     paged_decode_tc_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                            const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_q,
                            int n_work) {
@@ -267,17 +293,25 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t bar0 = sbase + C::kOffBar;
     auto full = [&](int e) { return bar0 + 8u * e; };
     auto empty = [&](int e) { return bar0 + 8u * (C::kRing + e); };
-    const uint32_t q_full = bar0 + 8u * (2 * C::kRing);
-    const uint32_t q_empty = q_full + 8;
-    auto s_full = [&](int i) { return q_full + 16u + 8u * i; };
-    auto s_empty = [&](int i) { return q_full + 32u + 8u * i; };
+    auto kslot = [](uint32_t j) { return static_cast<int>(j % C::kKSlots); };
+    auto vslot = [](uint32_t j) { return static_cast<int>(C::kKSlots + j % C::kVSlots); };
+    auto kphase = [](uint32_t j) { return (j / C::kKSlots) & 1u; };
+    auto vphase = [](uint32_t j) { return (j / C::kVSlots) & 1u; };
+    // Q tile, its barriers and the O^T accumulator are double-buffered by item parity, so the producer
+    // loads the next item's Q and pages, and its first P.V starts, while this item finishes
+    const uint32_t bq0 = bar0 + 8u * (2 * C::kRing);
+    auto q_full = [&](int i) { return bq0 + 8u * i; };
+    auto q_empty = [&](int i) { return bq0 + 16u + 8u * i; };
+    const uint32_t bs0 = bq0 + 32u;
+    auto s_full = [&](int i) { return bs0 + 8u * i; };
+    auto s_empty = [&](int i) { return bs0 + 16u + 8u * i; };
     // P^T is double-buffered (stage J in buffer J & 1): the softmax of stage J writes while P.V(J - 1) runs
-    auto p_full = [&](int i) { return q_full + 48u + 8u * i; };
-    auto p_empty = [&](int i) { return q_full + 64u + 8u * i; };
-    const uint32_t o_full = q_full + 80;
-    const uint32_t o_empty = q_full + 88;
-    const uint32_t done_qk = q_full + 96;
-    const uint32_t done_pv = q_full + 104;
+    auto p_full = [&](int i) { return bs0 + 32u + 8u * i; };
+    auto p_empty = [&](int i) { return bs0 + 48u + 8u * i; };
+    auto o_full = [&](int i) { return bs0 + 64u + 8u * i; };
+    auto o_empty = [&](int i) { return bs0 + 80u + 8u * i; };
+    const uint32_t done_qk = bs0 + 96u;
+    const uint32_t done_pv = bs0 + 104u;
     volatile int* stage_bad = reinterpret_cast<volatile int*>(smem + C::kOffBad);
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::kOffTmem);
 
@@ -286,8 +320,12 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(full(e), 1);
             mbar_init(empty(e), 1);
         }
-        mbar_init(q_full, 1);
-        mbar_init(q_empty, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(q_full(i), 1);
+            mbar_init(q_empty(i), 1);
+            mbar_init(o_full(i), 1);
+            mbar_init(o_empty(i), 4);
+        }
         for (int i = 0; i < 2; ++i) {
             mbar_init(s_full(i), 1);
             mbar_init(s_empty(i), 4);
@@ -296,8 +334,6 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(p_full(i), 4);
             mbar_init(p_empty(i), 1);
         }
-        mbar_init(o_full, 1);
-        mbar_init(o_empty, 4);
         mbar_init(done_qk, 1);
         mbar_init(done_pv, 1);
         fence_barrier_init();
@@ -323,52 +359,65 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t tS = tmem;           // S^T buffers: columns [0, 2N)
-    const uint32_t tO = tmem + 2 * N;   // O^T: columns [2N, 3N)
+    auto tO = [&](int i) { return tmem + 2 * N + i * N; };  // O^T of item parity i: columns [2N + iN, 3N + iN)
     const uint32_t ring = sbase;
-    const uint32_t sQ = sbase + C::kOffQ;
+    auto sQ = [&](int i) { return sbase + C::kOffQ + i * C::kQB; };
     // P^T buffer b: hi tile at sP + 2b kPB, residual lo tile right after it
     const uint32_t sP = sbase + C::kOffP;
     auto sPhi = [&](uint32_t j) { return sP + (j & 1) * 2 * C::kPB; };
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
+    if (warp == 0 || warp == C::kVWarp) {
+        // ------------------------------------------------------------ producers
+        // Two warps issue the TMA boxes, one the K entries (and Q), the other the V entries: each
+        // producer's boxes are handled in order, so two streams keep more of them moving.
+        const int half = warp == 0 ? 0 : 1;
         bool ok = true;
-        uint32_t fill = 0;
+        uint32_t Jp = 0;  // stages issued (all items)
+        int fills = 0;
         int item_i = 0;
         for (int k = 0; k < n_cand && ok; ++k) {
             TcWork wk;
             if (!tc_get(p, L, k, P, wk) || wk.n_local <= 0) continue;
             if (p.k_new != nullptr && wk.first + wk.n_local == wk.n_pages)
-                append_new_token(p, wk.b, wk.kvh, wk.len, P, DH * 2, lane);
-            if (lane == 0) {
-                if (item_i > 0 && !mbar_wait_bounded(q_empty, (item_i - 1) & 1, kWaitLimitNs)) {
+                append_new_token_part(p, wk.b, wk.kvh, wk.len, P, DH * 2, lane, half);
+            if (half == 0 && lane == 0) {
+                if (item_i > 1 && !mbar_wait_bounded(q_empty(item_i & 1), ((item_i >> 1) - 1) & 1, kWaitLimitNs)) {
                     raise_err(p.err, KV_DEV_ERR_TIMEOUT);
                     ok = false;
                 } else {
-                    mbar_arrive_expect_tx(q_full, C::kBoxCols * G * 128);
+                    mbar_arrive_expect_tx(q_full(item_i & 1), C::kBoxCols * G * 128);
 #pragma unroll
                     for (int bb = 0; bb < C::kBoxCols; ++bb)
-                        tma_load_2d(sQ + bb * C::kQRowsB, &tmap_q, bb * 64, wk.b * p.H_q + wk.kvh * G, q_full);
+                        tma_load_2d(sQ(item_i & 1) + bb * C::kQRowsB, &tmap_q, bb * 64, wk.b * p.H_q + wk.kvh * G,
+                                    q_full(item_i & 1));
                 }
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
             ++item_i;
             const int32_t* row = p.block_tables + (int64_t)wk.b * p.max_blocks + wk.first;
+            int tab_cur = lane < wk.n_local ? row[lane] : -1, tab_nxt = -1;
             const int n_st = (wk.n_local + C::kPPS - 1) / C::kPPS;
-            for (int j = 0; j < n_st && ok; ++j) {
+            for (int j = 0; j < n_st && ok; ++j, ++Jp) {
                 const int np = min(C::kPPS, wk.n_local - j * C::kPPS);
-                const int pg = lane < np ? row[j * C::kPPS + lane] : -1;
+                // block-table entries come 32 at a time, one per lane, the next 32 fetched while these are used
+                // (stages never straddle a group: 32 is a multiple of the pages per stage)
+                if (((j * C::kPPS) & 31) == 0) {
+                    const int base = j * C::kPPS;
+                    tab_cur = base == 0 ? tab_cur : tab_nxt;
+                    tab_nxt = (base + 32 + lane < wk.n_local) ? row[base + 32 + lane] : -1;
+                }
+                const int pg_all = __shfl_sync(0xffffffffu, tab_cur, (j * C::kPPS + lane) & 31);
+                const int pg = lane < np ? pg_all : -1;
                 const bool good = lane < np && pg >= 0 && pg < p.num_pages;
                 if (lane < np && !good) raise_err(p.err, KV_DEV_ERR_PAGE_RANGE);
                 const unsigned gmask = __ballot_sync(0xffffffffu, good);
                 const int box_page = lane / C::kBoxCols, bb = lane % C::kBoxCols;
                 const int pgl = __shfl_sync(0xffffffffu, pg, box_page & 31);
-#pragma unroll 1
-                for (int half = 0; half < 2 && ok; ++half) {
-                    const int e = fill % C::kRing;
+                {
+                    const int e = half ? vslot(Jp) : kslot(Jp);
+                    const uint32_t use = half ? Jp / C::kVSlots : Jp / C::kKSlots;  // earlier fills of the entry
                     if (lane == 0) {
-                        if (fill >= (uint32_t)C::kRing &&
-                            !mbar_wait_bounded(empty(e), ((fill / C::kRing) - 1) & 1, kWaitLimitNs)) {
+                        if (use > 0 && !mbar_wait_bounded(empty(e), (use - 1) & 1, kWaitLimitNs)) {
                             raise_err(p.err, KV_DEV_ERR_TIMEOUT);
                             ok = false;
                         } else {
@@ -383,16 +432,19 @@ __global__ void __launch_bounds__(192, 1)
                         tma_load_2d(dst, half ? static_cast<const void*>(&tmap_v) : static_cast<const void*>(&tmap_k),
                                     bb * 64, (pgl * p.H_kv + wk.kvh) * P, full(e));
                     }
-                    ++fill;
+                    fills = Jp + 1;
                 }
             }
         }
         if (lane == 0) {  // let every copy in flight land before the CTA exits
-            for (uint32_t i = fill > (uint32_t)C::kRing ? fill - C::kRing : 0; i < fill; ++i)
-                if (!mbar_wait_bounded(full(i % C::kRing), (i / C::kRing) & 1, kWaitLimitNs))
+            const int slots = half ? C::kVSlots : C::kKSlots;
+            for (int j = max(0, fills - slots); j < fills; ++j)
+                if (!mbar_wait_bounded(full(half ? vslot(j) : kslot(j)), half ? vphase(j) : kphase(j), kWaitLimitNs))
                     raise_err(p.err, KV_DEV_ERR_TIMEOUT);
-            if (item_i > 0 && !mbar_wait_bounded(q_full, (item_i - 1) & 1, kWaitLimitNs))
-                raise_err(p.err, KV_DEV_ERR_TIMEOUT);
+            if (half == 0)
+                for (int i = item_i > 2 ? item_i - 2 : 0; i < item_i; ++i)
+                    if (!mbar_wait_bounded(q_full(i & 1), (i >> 1) & 1, kWaitLimitNs))
+                        raise_err(p.err, KV_DEV_ERR_TIMEOUT);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issue
@@ -401,7 +453,6 @@ __global__ void __launch_bounds__(192, 1)
         // barriers, so QK runs up to two stages ahead of the softmax.
         if (lane < 2) {
             bool ok = true;
-            uint32_t fbase = 0;  // ring fills of the earlier items
             uint32_t J = 0;      // stages of the earlier items and this one
             int item_i = 0;
             auto wait = [&](uint32_t bar, uint32_t parity) {
@@ -416,12 +467,11 @@ __global__ void __launch_bounds__(192, 1)
                 if (!tc_get(p, L, k, P, wk) || wk.n_local <= 0) continue;
                 const int n_st = (wk.n_local + C::kPPS - 1) / C::kPPS;
                 if (lane == 0) {
-                    if (!wait(q_full, item_i & 1)) break;
+                    if (!wait(q_full(item_i & 1), (item_i >> 1) & 1)) break;
                     for (int j = 0; j < n_st; ++j, ++J) {
-                        const uint32_t f = fbase + 2 * j;
-                        const int e = f % C::kRing;
+                        const int e = kslot(J);
                         const int sb = J & 1;
-                        if (!wait(full(e), (f / C::kRing) & 1)) break;
+                        if (!wait(full(e), kphase(J))) break;
                         if (J >= 2 && !wait(s_empty(sb), ((J >> 1) - 1) & 1)) break;
                         tc_fence_after();
                         const uint32_t sK = ring + e * C::kEntry;
@@ -430,40 +480,38 @@ __global__ void __launch_bounds__(192, 1)
                             const uint32_t koff = (kk >> 2) * C::kBoxB + (kk & 3) * 32;
                             const uint32_t qoff = (kk >> 2) * C::kQRowsB + (kk & 3) * 32;
                             umma_ss(tS + sb * N, smem_desc(sK + koff, 16, 1024, kSwz128),
-                                    smem_desc(sQ + qoff, 16, 1024, kSwz128), kIdescQK, kk > 0 ? 1u : 0u);
+                                    smem_desc(sQ(item_i & 1) + qoff, 16, 1024, kSwz128), kIdescQK, kk > 0 ? 1u : 0u);
                         }
                         umma_commit(s_full(sb));
                         umma_commit(empty(e));
-                        if (j == n_st - 1) umma_commit(q_empty);
+                        if (j == n_st - 1) umma_commit(q_empty(item_i & 1));
                     }
                 } else {
                     for (int j = 0; j < n_st; ++j, ++J) {
-                        const uint32_t f = fbase + 2 * j + 1;
-                        const int e = f % C::kRing;
-                        if (!wait(full(e), (f / C::kRing) & 1)) break;
+                        const int e = vslot(J);
+                        if (!wait(full(e), vphase(J))) break;
                         if (!wait(p_full(J & 1), (J >> 1) & 1)) break;
-                        if (j == 0 && item_i > 0 && !wait(o_empty, (item_i - 1) & 1)) break;
+                        if (j == 0 && item_i > 1 && !wait(o_empty(item_i & 1), ((item_i >> 1) - 1) & 1)) break;
                         tc_fence_after();
                         const uint32_t sV = ring + e * C::kEntry;
 #pragma unroll
                         for (int kk = 0; kk < C::kTP / 16; ++kk) {
                             const uint64_t a = smem_desc(sV + kk * 16 * 128, C::kBoxB, 1024, kSwz128);
-                            umma_ss(tO, a, smem_desc(sPhi(J) + kk * 16 * C::kPRow, C::kPB, C::kPAtom, C::kPSwz),
+                            umma_ss(tO(item_i & 1), a, smem_desc(sPhi(J) + kk * 16 * C::kPRow, C::kPB, C::kPAtom, C::kPSwz),
                                     kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
                         }
 #pragma unroll
                         for (int kk = 0; kk < C::kTP / 16; ++kk) {
                             const uint64_t a = smem_desc(sV + kk * 16 * 128, C::kBoxB, 1024, kSwz128);
-                            umma_ss(tO, a,
+                            umma_ss(tO(item_i & 1), a,
                                     smem_desc(sPhi(J) + C::kPB + kk * 16 * C::kPRow, C::kPB, C::kPAtom, C::kPSwz),
                                     kIdescPV, 1u);
                         }
                         umma_commit(empty(e));
                         umma_commit(p_empty(J & 1));
                     }
-                    if (ok) umma_commit(o_full);
+                    if (ok) umma_commit(o_full(item_i & 1));
                 }
-                fbase += 2 * n_st;
                 ++item_i;
             }
             // every MMA this thread issued has completed before tensor memory is released
@@ -484,7 +532,7 @@ __global__ void __launch_bounds__(192, 1)
         volatile int* flags = reinterpret_cast<volatile int*>(smem + C::kOffFlag);
         int rbuf = 0, fbuf = 0;
         bool ok = true;  // equal in the four warps at every flag exchange
-        uint32_t fbase = 0, J = 0;
+        uint32_t J = 0;
         int item_i = 0;
         // warp-uniform outcome: the tensor-memory loads and stores after a wait are warp-collective
         auto wait = [&](bool& okl, uint32_t bar, uint32_t parity) {
@@ -538,10 +586,9 @@ __global__ void __launch_bounds__(192, 1)
                     if (lane == 0) mbar_arrive(s_empty(sb));
                 }
                 // the stage's V entry (and its skipped-page mask) must have landed
-                const uint32_t fv = fbase + 2 * j + 1;
-                const int ev = fv % C::kRing;
+                const int ev = vslot(J);
                 bool valid = false;
-                if (wait(okl, full(ev), (fv / C::kRing) & 1)) {
+                if (wait(okl, full(ev), vphase(J))) {
                     const int np = min(C::kPPS, wk.n_local - j * C::kPPS);
                     const int bad = stage_bad[ev];
                     const int pg_in = r / P;
@@ -586,11 +633,11 @@ __global__ void __launch_bounds__(192, 1)
                 if (rescale_o) {
                     tc_fence_after();
                     uint32_t a[N];
-                    tmem_ld_cols<N>(tO + lane_addr, a);
+                    tmem_ld_cols<N>(tO(item_i & 1) + lane_addr, a);
                     tmem_wait_ld();
 #pragma unroll
                     for (int h = 0; h < G; ++h) a[h] = __float_as_uint(__uint_as_float(a[h]) * alpha[h]);
-                    tmem_st_cols<N>(tO + lane_addr, a);
+                    tmem_st_cols<N>(tO(item_i & 1) + lane_addr, a);
                     tmem_wait_st();
                 }
                 // probabilities -> P^T row r (hi and residual lo; padding heads are zero), swizzled rows
@@ -631,7 +678,7 @@ __global__ void __launch_bounds__(192, 1)
             }
             // ---- epilogue: O^T row r, row sums over the CTA, output or partials
             bool okl = ok;
-            if (wait(okl, o_full, item_i & 1)) {
+            if (wait(okl, o_full(item_i & 1), (item_i >> 1) & 1)) {
                 tc_fence_after();
             }
             if (exchange(okl ? 0 : 2) & 2) ok = false;
@@ -639,18 +686,17 @@ __global__ void __launch_bounds__(192, 1)
                 zero_rows(wk);
                 continue;
             }
-            fbase += 2 * n_st;
             float o[G];
             {
                 uint32_t a[N];
-                tmem_ld_cols<N>(tO + lane_addr, a);
+                tmem_ld_cols<N>(tO(item_i & 1) + lane_addr, a);
                 tmem_wait_ld();
 #pragma unroll
                 for (int h = 0; h < G; ++h) o[h] = __uint_as_float(a[h]);
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(o_empty);
+            if (lane == 0) mbar_arrive(o_empty(item_i & 1));
             ++item_i;
             cta_heads_reduce<G, false>(lp, red, sw, lane, rbuf);
             const int64_t hq0 = (int64_t)wk.b * p.H_q + (int64_t)wk.kvh * G;

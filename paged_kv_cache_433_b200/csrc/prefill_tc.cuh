@@ -29,9 +29,11 @@
 // than 2^8; the row's O and l are then rescaled (o = u / l for any common
 // reference).
 //
-// Warps (320 threads, one CTA per SM by tensor memory and shared memory):
-//   warp 0     producer: per stage the K then V boxes of its pages (P rows x
-//              128 bytes, 128-byte swizzle) into a ring of five 32 KB entries;
+// Warps (352 threads, one CTA per SM by tensor memory and shared memory):
+//   warps 0, 10 producers: per stage warp 0 the K boxes, warp 10 the V boxes
+//              of its pages (P rows x 128 bytes, 128-byte swizzle) into three
+//              K and two V entries of 32 KB (a K entry is refilled once its
+//              QK has run);
 //   warp 1     tensor memory allocation; lane 0 issues the QK(j), lane 1 the
 //              P.V(j), each paced only by its own barriers;
 //   warps 2-9  load the Q tile (swizzled stores), softmax, epilogue; each pair
@@ -55,7 +57,10 @@ struct PfCfg {
     static constexpr int kBoxCols = DH / 64;
     static constexpr int kBoxB = kTP * 128;      // one 128-byte box column of an entry
     static constexpr int kEntry = kBoxCols * kBoxB;
-    static constexpr int kRing = 5;              // K / V entries (two and a half stages)
+    // entries 0..2 hold K of stages j % 3, entries 3..4 V of stages j % 2: a K entry is refilled as soon
+    // as its QK has run, independently of the P.V of older stages
+    static constexpr int kKSlots = 3, kVSlots = 2;
+    static constexpr int kRing = kKSlots + kVSlots;
     static constexpr int kQB = 128 * DH * 2;     // Q tile: 128 rows
     static constexpr int kOffQ = kRing * kEntry;
     static constexpr int kOffBad = kOffQ + kQB;
@@ -65,7 +70,8 @@ struct PfCfg {
     static constexpr int kNumBars = 2 * kRing + 1 + 3 + 2 + 3 + 3;
     static constexpr int kOffTmem = kOffBar + 8 * kNumBars;
     static constexpr int kSmem = 1024 + kOffTmem + 16;
-    static constexpr int kThreads = 320;
+    static constexpr int kThreads = 352;
+    static constexpr int kVWarp = 10;            // the V producer (warp 0 produces K)
     static constexpr int kSoftmaxWarps = 8;
     static constexpr uint32_t kTmemCols = 512;   // S x 3 (384) + O (128)
     static_assert(DH == 128, "instance: Dh = 128");
@@ -74,7 +80,7 @@ struct PfCfg {
 };
 
 template <int KT, int DH, int P>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     paged_prefill_tc_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                             const __grid_constant__ CUtensorMap tmap_v) {
     using C = PfCfg<DH, P>;
@@ -121,6 +127,10 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t bar0 = sbase + C::kOffBar;
     auto full = [&](int e) { return bar0 + 8u * e; };
     auto empty = [&](int e) { return bar0 + 8u * (C::kRing + e); };
+    auto kslot = [](int j) { return j % C::kKSlots; };
+    auto vslot = [](int j) { return C::kKSlots + j % C::kVSlots; };
+    auto kphase = [](int j) { return static_cast<uint32_t>((j / C::kKSlots) & 1); };
+    auto vphase = [](int j) { return static_cast<uint32_t>((j / C::kVSlots) & 1); };
     const uint32_t q_full = bar0 + 8u * (2 * C::kRing);
     auto s_full = [&](int i) { return q_full + 8u + 8u * i; };
     // P of stage j is announced on p_full(j & 1): the softmax of stage j + 1 may finish before the MMA
@@ -161,25 +171,35 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t ring = sbase;
     const uint32_t sQ = sbase + C::kOffQ;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
+    if (warp == 0 || warp == C::kVWarp) {
+        // ------------------------------------------------------------ producers
+        // warp 0 issues the K boxes of every stage, warp kVWarp the V boxes: two streams of TMA requests
+        const int half = warp == 0 ? 0 : 1;
         bool ok = true;
-        uint32_t fill = 0;
+        int kfills = 0, vfills = 0;  // stages whose K / V boxes were issued
         const int32_t* row = p.block_tables + (int64_t)b * p.max_blocks;
+        int tab_cur = lane < n_pages ? row[lane] : -1, tab_nxt = -1;
         for (int j = 0; j < n_st && ok; ++j) {
             const int np = min(C::kPPS, n_pages - j * C::kPPS);
-            const int pg = lane < np ? row[j * C::kPPS + lane] : -1;
+            // block-table entries come 32 at a time, one per lane, the next 32 fetched while these are used
+            // (stages never straddle a group: 32 is a multiple of the pages per stage)
+            if (((j * C::kPPS) & 31) == 0) {
+                const int base = j * C::kPPS;
+                tab_cur = base == 0 ? tab_cur : tab_nxt;
+                tab_nxt = (base + 32 + lane < n_pages) ? row[base + 32 + lane] : -1;
+            }
+            const int pg_all = __shfl_sync(0xffffffffu, tab_cur, (j * C::kPPS + lane) & 31);
+            const int pg = lane < np ? pg_all : -1;
             const bool good = lane < np && pg >= 0 && pg < p.num_pages;
             if (lane < np && !good) raise_err(p.err, KV_DEV_ERR_PAGE_RANGE);
             const unsigned gmask = __ballot_sync(0xffffffffu, good);
             const int box_page = lane / C::kBoxCols, bb = lane % C::kBoxCols;
             const int pgl = __shfl_sync(0xffffffffu, pg, box_page & 31);
-#pragma unroll 1
-            for (int half = 0; half < 2 && ok; ++half) {
-                const int e = fill % C::kRing;
+            {
+                const int e = half ? vslot(j) : kslot(j);
+                const int use = half ? j / C::kVSlots : j / C::kKSlots;  // earlier fills of this entry
                 if (lane == 0) {
-                    if (fill >= (uint32_t)C::kRing &&
-                        !mbar_wait_bounded(empty(e), ((fill / C::kRing) - 1) & 1, kWaitLimitNs)) {
+                    if (use > 0 && !mbar_wait_bounded(empty(e), (use - 1) & 1, kWaitLimitNs)) {
                         raise_err(p.err, KV_DEV_ERR_TIMEOUT);
                         ok = false;
                     } else {
@@ -194,13 +214,20 @@ __global__ void __launch_bounds__(320, 1)
                     tma_load_2d(dst, half ? static_cast<const void*>(&tmap_v) : static_cast<const void*>(&tmap_k),
                                 bb * 64, (pgl * p.H_kv + kvh) * P, full(e));
                 }
-                ++fill;
+                if (half) vfills = j + 1;
+                else kfills = j + 1;
             }
         }
-        if (lane == 0) {
-            for (uint32_t i = fill > (uint32_t)C::kRing ? fill - C::kRing : 0; i < fill; ++i)
-                if (!mbar_wait_bounded(full(i % C::kRing), (i / C::kRing) & 1, kWaitLimitNs))
-                    raise_err(p.err, KV_DEV_ERR_TIMEOUT);
+        if (lane == 0) {  // the last fill of every entry has landed before the CTA exits
+            if (half == 0) {
+                for (int j = max(0, kfills - C::kKSlots); j < kfills; ++j)
+                    if (!mbar_wait_bounded(full(kslot(j)), kphase(j), kWaitLimitNs))
+                        raise_err(p.err, KV_DEV_ERR_TIMEOUT);
+            } else {
+                for (int j = max(0, vfills - C::kVSlots); j < vfills; ++j)
+                    if (!mbar_wait_bounded(full(vslot(j)), vphase(j), kWaitLimitNs))
+                        raise_err(p.err, KV_DEV_ERR_TIMEOUT);
+            }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issue
@@ -218,9 +245,8 @@ __global__ void __launch_bounds__(320, 1)
             if (lane == 0) {
                 if (wait(q_full, 0)) {
                     for (int j = 0; j < n_st; ++j) {
-                        const uint32_t f = 2 * j;
-                        const int e = f % C::kRing;
-                        if (!wait(full(e), (f / C::kRing) & 1)) break;
+                        const int e = kslot(j);
+                        if (!wait(full(e), kphase(j))) break;
                         if (j >= 3 && !wait(p_empty(j % 3), ((j - 3) / 3) & 1)) break;
                         tc_fence_after();
                         const uint32_t sK = ring + e * C::kEntry;
@@ -237,9 +263,8 @@ __global__ void __launch_bounds__(320, 1)
                 }
             } else {
                 for (int j = 0; j < n_st; ++j) {
-                    const uint32_t f = 2 * j + 1;
-                    const int e = f % C::kRing;
-                    if (!wait(full(e), (f / C::kRing) & 1)) break;
+                    const int e = vslot(j);
+                    if (!wait(full(e), vphase(j))) break;
                     if (!wait(p_full(j & 1), (j >> 1) & 1)) break;
                     tc_fence_after();
                     const uint32_t sV = ring + e * C::kEntry;
@@ -329,12 +354,11 @@ __global__ void __launch_bounds__(320, 1)
                 for (int i = 0; i < 32; ++i) s[i] = __uint_as_float(a[i]), s[32 + i] = __uint_as_float(b2[i]);
             }
             // keys of this stage: kbase .. kbase + 127; the V entry carries the skipped-page mask
-            const uint32_t fv = 2 * j + 1;
-            const int ev = fv % C::kRing;
+            const int ev = vslot(j);
             const int kbase = j * C::kTP;
             const int np = min(C::kPPS, n_pages - j * C::kPPS);
             int bad = 0;
-            if (wait(okl, full(ev), (fv / C::kRing) & 1)) bad = stage_bad[ev];
+            if (wait(okl, full(ev), vphase(j))) bad = stage_bad[ev];
             // keys this row may see in the stage: [0, lim); pages skipped or not loaded are masked
             const int lim = row_valid ? min(C::kTP, pos + 1 - kbase) : 0;
             const bool full_stage = lim == C::kTP && np == C::kPPS && bad == 0;
