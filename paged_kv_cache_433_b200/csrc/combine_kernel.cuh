@@ -6,6 +6,7 @@
 
 #include <cstdint>
 
+#include "plan_layout.cuh"
 #include "ptx.cuh"
 
 namespace kvp {
@@ -20,12 +21,14 @@ namespace kvp {
 // and (WPR > 1) a shared-memory sum over the row's warps, all relative to the
 // same m*.
 constexpr int kCombineWarps = 8;
-constexpr int kPlanHdrCombine = 4;  // first S_b entry of a plan
 
 // Planned launches (plan != nullptr, WPR == 1 only): the row's chunk size and
 // first item come from the plan; rows with one chunk were written by the
 // decode kernel and are skipped, empty rows are zeroed here; partial s of
 // (b, query head h) sits at item t0 + s, row h of that item's [g][Dh] block.
+// Balanced plans (plan[0] == kPlanStream): the row's pages lie in the ranges
+// of CTAs c0 .. c1; its first piece left its partial in slot 2 c0 + 1, piece
+// s >= 1 in slot 2 (c0 + s).
 template <int DH, int WPR>
 __global__ void __launch_bounds__(32 * kCombineWarps) paged_combine_kernel(
     float* __restrict__ out, const float* __restrict__ part_u, const float2* __restrict__ part_ml,
@@ -45,20 +48,40 @@ __global__ void __launch_bounds__(32 * kCombineWarps) paged_combine_kernel(
     if (threadIdx.x == 0) grid_launch_dependents();
     bool live = item < (int64_t)B * H_q;
     int ns = 0;
-    int64_t base = item * S, stride = 1;
+    int64_t base = item * S, stride = 1, first = 0;  // partial s at base + (s == 0 ? first : s * stride)
     if (live) {
         const int b = static_cast<int>(item / H_q);
         int len = seq_lens[b];
         if (len < 0 || len > max_blocks * P) len = 0;
         const int n_pages = (len + P - 1) / P;
-        if (plan != nullptr) {
+        if (plan != nullptr && plan[0] == kPlanStream) {
+            const int G = plan[1];
+            const long long T = static_cast<long long>(static_cast<uint32_t>(plan[2])) |
+                                (static_cast<long long>(plan[3]) << 32);
+            const int64_t* pre = plan_stream_prefix(plan);
+            const int g = H_q / H_kv;
+            const int hq = static_cast<int>(item % H_q);
+            const long long s0 = pre[b], n = pre[b + 1] - s0;
+            if (n > 0 && G > 0) {
+                const long long r0 = (long long)H_kv * s0 + (long long)(hq / g) * n;
+                const int c0 = plan_stream_cta(r0, T, G), c1 = plan_stream_cta(r0 + n - 1, T, G);
+                if (c0 == c1) {
+                    live = false;  // the decode kernel wrote this row
+                } else {
+                    ns = c1 - c0 + 1;
+                    base = 2LL * g * c0 + hq % g;
+                    stride = 2LL * g;
+                    first = g;
+                }
+            }
+        } else if (plan != nullptr) {
             const int C = plan[0];
             const int items_b = (n_pages + C - 1) / C;
             const int g = H_q / H_kv;
             const int hq = static_cast<int>(item % H_q);
             if (items_b == 1) live = false;  // the decode kernel wrote this row
             ns = items_b > 1 ? items_b : 0;
-            const int64_t t0 = (int64_t)H_kv * plan[kPlanHdrCombine + b] + (int64_t)(hq / g) * items_b;
+            const int64_t t0 = (int64_t)H_kv * plan[kPlanHdr + b] + (int64_t)(hq / g) * items_b;
             base = t0 * g + hq % g;
             stride = g;
         } else {
@@ -80,8 +103,9 @@ __global__ void __launch_bounds__(32 * kCombineWarps) paged_combine_kernel(
         for (int j = 0; j < kPer; ++j) {
             const int s = r0 + rw + j * WPR;
             if (s < ns) {
-                st[j] = ml[s * stride];
-                const float* src = pu + (int64_t)s * stride * DH;
+                const int64_t off = s == 0 ? first : (int64_t)s * stride;
+                st[j] = ml[off];
+                const float* src = pu + off * DH;
                 if constexpr (kD == 4) {
                     const float4 x = *reinterpret_cast<const float4*>(src);
                     v[j][0] = x.x; v[j][1] = x.y; v[j][2] = x.z; v[j][3] = x.w;
@@ -96,7 +120,7 @@ __global__ void __launch_bounds__(32 * kCombineWarps) paged_combine_kernel(
             }
         }
         if (r0 == 0) {
-            for (int s = lane; s < ns; s += 32) mstar = fmaxf(mstar, ml[s * stride].x);
+            for (int s = lane; s < ns; s += 32) mstar = fmaxf(mstar, ml[s == 0 ? first : (int64_t)s * stride].x);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) mstar = fmaxf(mstar, __shfl_xor_sync(0xffffffffu, mstar, o));
         }

@@ -24,14 +24,16 @@
 // maximum is reduced over the CTA, and O^T and the partial row sums are
 // rescaled (o = u / l holds for any common reference).
 //
-// Warp roles (224 threads, one CTA per SM, persistent over work items):
+// Warp roles (256 threads, one CTA per SM, persistent over work items):
 //   warps 0, 6 producers: warp 0 the Q tile (2-D TMA, 128-byte swizzle) and
 //              the K boxes of each stage, warp 6 the V boxes (P rows x 128
 //              bytes each), into K and V entries of 32 KB; each writes its
 //              half of the fused append when the item owns the last page.
 //   warp 1     allocates tensor memory and resolves the CTA's work items
-//              into shared memory; lane 0 issues the QK(j), lane 1 the
-//              P.V(j), each committing onto the mbarriers the others wait on.
+//              into shared memory; its lane 0 issues the QK(j).
+//   warp 7     lane 0 issues the P.V(j). The two issuers sit in different
+//              warps so that neither one's wait holds up the other (two
+//              lanes of one warp would take turns).
 //   warps 2-5  softmax and epilogue (tensor-memory lane quarter = warp % 4).
 // A work item is (sequence, KV head, chunk of pages): from the device plan
 // (planned launch) or from the grid rule (split); partials use the layout of
@@ -45,6 +47,7 @@
 #include <cuda.h>
 
 #include "decode_kernel.cuh"
+#include "plan_layout.cuh"
 #include "tc05.cuh"
 
 namespace kvp {
@@ -60,7 +63,7 @@ struct TcCfg {
     static constexpr int kPB0 = kTP * kN * 2;    // one P^T tile (hi or lo)
     // ring entries (K or V of a stage) that fit beside two Q tiles, two P^T buffers (hi + lo each), the
     // work list (3 KB) and the small arrays
-    static constexpr int kRing0 = (227 * 1024 - 1024 - 2048 - 3072 - 2 * kBoxCols * kN * 128 - 4 * kPB0) / kEntry;
+    static constexpr int kRing0 = (227 * 1024 - 1024 - 2048 - 3104 - 2 * kBoxCols * kN * 128 - 4 * kPB0) / kEntry;
     static constexpr int kRing = kRing0 > 6 ? 6 : kRing0;
     // K of global stage J in entry J % kKSlots, V in kKSlots + J % kVSlots: a K entry is refilled as soon as
     // its QK has run, whatever the P.V of older stages
@@ -79,14 +82,16 @@ struct TcCfg {
     static constexpr int kOffBad = kOffFlag + 32;             // int per ring entry
     static constexpr int kMaxList = 96;          // work items of a CTA resolved once into shared memory
     static constexpr int kOffList = (kOffBad + 4 * kRing + 15) / 16 * 16;  // int4 x 2 per item
-    static constexpr int kOffBar = kOffList + kMaxList * 32;
+    static constexpr int kOffStream = kOffList + kMaxList * 32;   // TcStream of a balanced plan (32 bytes)
+    static constexpr int kOffBar = kOffStream + 32;
     // full[R], empty[R], q_full[2], q_empty[2], s_full[2], s_empty[2], p_full[2], p_empty[2], o_full[2],
     // o_empty[2], done (QK issuer), done (PV issuer)
     static constexpr int kNumBars = 2 * kRing + 4 + 4 + 4 + 4 + 2;
     static constexpr int kOffTmem = kOffBar + 8 * kNumBars;
     static constexpr int kSmem = 1024 + kOffTmem + 16;
-    static constexpr int kThreads = 224;
+    static constexpr int kThreads = 256;
     static constexpr int kVWarp = 6;             // the V producer (warp 0 produces Q and K)
+    static constexpr int kPVWarp = 7;            // issues P.V (warp 1 issues QK)
     static constexpr uint32_t kTmemCols = 4 * kN <= 64 ? 64 : 128;  // S^T x 2 + O^T x 2, N columns each
     static_assert((G == 4 || G == 8 || G == 16 || G == 32) && DH == 128, "instances: g in {4, 8, 16, 32}, Dh = 128");
     static_assert(kPPS * kBoxCols <= 32, "one TMA box per lane");
@@ -96,7 +101,63 @@ struct TcCfg {
 struct TcWork {
     int b, kvh, split, item, first, n_local, len, n_pages;
     bool split_mode, bad_len;
+    bool planned;  // partial at slot `item` ([item][g][Dh]); else at (row, split) of the grid layout
 };
+
+// This CTA's share of a balanced plan (paged_plan_stream_kernel): pages [lo, hi) of the line of
+// (sequence, KV head) rows, the first of which, row0 = b * H_kv + kvh, holds page lo.
+struct TcStream {
+    long long lo, hi, row0;
+    int active;  // a balanced plan with pages for this CTA
+    int pad;
+};
+
+__device__ __forceinline__ bool tc_is_stream(const DecodeParams& p) {
+    return p.items == nullptr && p.plan != nullptr && p.plan[0] == kPlanStream;
+}
+
+__device__ __forceinline__ TcStream tc_stream_range(const DecodeParams& p) {
+    TcStream r{0, 0, 0, 0, 0};
+    const int G = p.plan[1];
+    const int c = blockIdx.x;
+    if (c >= G) return r;
+    const long long T = static_cast<long long>(static_cast<uint32_t>(p.plan[2])) | (static_cast<long long>(p.plan[3]) << 32);
+    const int64_t* pre = plan_stream_prefix(p.plan);
+    const int b0 = p.plan[kPlanHdr + 2 * (p.B + 1) + c];
+    r.lo = T * c / G;
+    r.hi = T * (c + 1) / G;
+    const long long s0 = pre[b0], n0 = pre[b0 + 1] - s0;
+    if (r.hi <= r.lo || n0 <= 0) return r;
+    r.row0 = static_cast<long long>(b0) * p.H_kv + (r.lo - p.H_kv * s0) / n0;
+    r.active = 1;
+    return r;
+}
+
+// Piece k of the CTA's range: row row0 + k cut to [lo, hi). 1: work, 0: an empty row, -1: past the range.
+__device__ __forceinline__ int tc_stream_piece(const DecodeParams& p, const TcStream& st, int k, int P, TcWork& wk) {
+    if (!st.active) return -1;
+    const long long row = st.row0 + k;
+    const int b = static_cast<int>(row / p.H_kv), kvh = static_cast<int>(row % p.H_kv);
+    if (b >= p.B) return -1;
+    const int64_t* pre = plan_stream_prefix(p.plan);
+    const long long s0 = pre[b], n = pre[b + 1] - s0;
+    const long long r0 = p.H_kv * s0 + kvh * n;
+    if (r0 >= st.hi) return -1;
+    const long long x0 = r0 > st.lo ? r0 : st.lo, x1 = r0 + n < st.hi ? r0 + n : st.hi;
+    if (x1 <= x0) return 0;
+    wk.b = b;
+    wk.kvh = kvh;
+    wk.split = 0;
+    wk.item = 2 * static_cast<int>(blockIdx.x) + (r0 >= st.lo ? 1 : 0);
+    wk.first = static_cast<int>(x0 - r0);
+    wk.n_local = static_cast<int>(x1 - x0);
+    wk.len = p.seq_lens[b];
+    wk.n_pages = static_cast<int>(n);
+    wk.split_mode = !(x0 == r0 && x1 == r0 + n);
+    wk.bad_len = false;  // the plan raised it and gave the row no pages
+    wk.planned = true;
+    return 1;
+}
 
 // Work item w: planned (items list) or grid (split, KV head, sequence).
 __device__ __forceinline__ bool tc_work(const DecodeParams& p, int w, int P, TcWork& k) {
@@ -126,6 +187,7 @@ __device__ __forceinline__ bool tc_work(const DecodeParams& p, int w, int P, TcW
     k.n_pages = (len + P - 1) / P;
     k.n_local = chunked ? min(chunk_pages, k.n_pages - k.first) : k.n_pages;
     k.split_mode = p.items != nullptr ? k.n_pages > chunk_pages : p.num_splits > 1;
+    k.planned = p.items != nullptr;
     return true;
 }
 
@@ -135,35 +197,60 @@ __host__ __device__ constexpr int ilog2(int n) { return n <= 1 ? 0 : 1 + ilog2(n
 // one warp into shared memory, so the roles walk them without the dependent
 // global loads of tc_work; candidates past the list are resolved on the fly.
 struct TcList {
-    int4* e;        // [kMaxList][2]: {b, kvh, split, item}, {first, n_local, len, flags}
-    int n_list;     // candidates held
+    int4* e;            // [kMaxList][2]: {b, kvh, split, item}, {first, n_local, len, flags}
+    int n_list;         // entries held
+    int n_cand;         // candidates of a grid or chunked launch (a balanced plan ends at its range)
+    const TcStream* st;  // balanced plan: this CTA's range (shared memory), else nullptr
 };
 
+// list entry flags
+constexpr int kTcSplit = 1, kTcBad = 2, kTcWork = 4, kTcPlanned = 8, kTcEnd = 16;
+
+__device__ __forceinline__ void tc_list_put(int4* e, int k, const TcWork& wk, int flags) {
+    e[2 * k] = make_int4(wk.b, wk.kvh, wk.split, wk.item);
+    e[2 * k + 1] = make_int4(wk.first, wk.n_local, wk.len,
+                             flags | (wk.split_mode ? kTcSplit : 0) | (wk.bad_len ? kTcBad : 0) |
+                                 (wk.planned ? kTcPlanned : 0));
+}
+
+// One warp: the stream range (balanced plan) and the first candidates, into shared memory.
 __device__ __forceinline__ void tc_list_build(const DecodeParams& p, int n_work, int P, int4* e, int max_list,
-                                              int lane) {
+                                              TcStream* st_out, int lane) {
+    const bool stream = tc_is_stream(p);
+    TcStream st{0, 0, 0, 0, 0};
+    if (stream) st = tc_stream_range(p);  // the same loads in every lane
+    if (lane == 0) *st_out = st;
     for (int k = lane; k < max_list; k += 32) {
-        const int w = blockIdx.x + k * gridDim.x;
-        TcWork wk;
+        TcWork wk{0, 0, 0, 0, 0, 0, 0, 0, false, false, false};
         int flags = 0;
-        if (w < n_work && tc_work(p, w, P, wk)) flags = 4 | (wk.split_mode ? 1 : 0) | (wk.bad_len ? 2 : 0);
-        else wk = TcWork{0, 0, 0, 0, 0, 0, 0, 0, false, false};
-        e[2 * k] = make_int4(wk.b, wk.kvh, wk.split, wk.item);
-        e[2 * k + 1] = make_int4(wk.first, wk.n_local, wk.len, flags);
+        if (stream) {
+            const int got = tc_stream_piece(p, st, k, P, wk);
+            flags = got > 0 ? kTcWork : (got < 0 ? kTcEnd : 0);
+        } else {
+            const int w = blockIdx.x + k * gridDim.x;
+            if (w >= n_work) flags = kTcEnd;
+            else if (tc_work(p, w, P, wk)) flags = kTcWork;
+        }
+        tc_list_put(e, k, wk, flags);
     }
 }
 
-// Candidate k of this CTA: false when it carries no work item.
-__device__ __forceinline__ bool tc_get(const DecodeParams& p, const TcList& L, int k, int P, TcWork& wk) {
+// Candidate k of this CTA: 1 a work item, 0 none (skip it), -1 past the CTA's last candidate.
+__device__ __forceinline__ int tc_get(const DecodeParams& p, const TcList& L, int k, int P, TcWork& wk) {
     if (k < L.n_list) {
         const int4 a = L.e[2 * k], c = L.e[2 * k + 1];
-        if (!(c.w & 4)) return false;
+        if (c.w & kTcEnd) return -1;
+        if (!(c.w & kTcWork)) return 0;
         wk.b = a.x, wk.kvh = a.y, wk.split = a.z, wk.item = a.w;
         wk.first = c.x, wk.n_local = c.y, wk.len = c.z;
-        wk.split_mode = (c.w & 1) != 0, wk.bad_len = (c.w & 2) != 0;
+        wk.split_mode = (c.w & kTcSplit) != 0, wk.bad_len = (c.w & kTcBad) != 0, wk.planned = (c.w & kTcPlanned) != 0;
         wk.n_pages = (wk.len + P - 1) / P;
-        return true;
+        return 1;
     }
-    return tc_work(p, blockIdx.x + k * gridDim.x, P, wk);
+    if (L.n_list > 0 && (L.e[2 * (L.n_list - 1) + 1].w & kTcEnd)) return -1;
+    if (L.st != nullptr) return tc_stream_piece(p, *L.st, k, P, wk);
+    if (k >= L.n_cand) return -1;
+    return tc_work(p, blockIdx.x + k * gridDim.x, P, wk) ? 1 : 0;
 }
 
 // Fused append of the new token (position len - 1) for one of the pools: part 0
@@ -266,7 +353,7 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, ui
 }
 
 template <int KT, int DH, int P, int G>
-__global__ void __launch_bounds__(224, 1)
+__global__ void __launch_bounds__(256, 1)
     paged_decode_tc_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                            const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_q,
                            int n_work) {
@@ -340,11 +427,13 @@ __global__ void __launch_bounds__(224, 1)
     }
     int4* list_e = reinterpret_cast<int4*>(smem + C::kOffList);
     const int n_cand = n_work > (int)blockIdx.x ? (n_work - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
-    const TcList L{list_e, min(n_cand, C::kMaxList)};
+    const bool stream = tc_is_stream(p);
+    TcStream* st_smem = reinterpret_cast<TcStream*>(smem + C::kOffStream);
+    const TcList L{list_e, stream ? C::kMaxList : min(n_cand, C::kMaxList), n_cand, stream ? st_smem : nullptr};
     if (warp == 1) {
         tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), C::kTmemCols);
         tmem_relinquish();
-        tc_list_build(p, n_work, P, list_e, L.n_list, lane);
+        tc_list_build(p, n_work, P, list_e, L.n_list, st_smem, lane);
     }
     if constexpr (G < N) {
         // Q rows G .. N-1 are MMA padding: zero once (the TMA box writes rows 0 .. G-1 only)
@@ -375,9 +464,11 @@ __global__ void __launch_bounds__(224, 1)
         uint32_t Jp = 0;  // stages issued (all items)
         int fills = 0;
         int item_i = 0;
-        for (int k = 0; k < n_cand && ok; ++k) {
+        for (int k = 0; ok; ++k) {
             TcWork wk;
-            if (!tc_get(p, L, k, P, wk) || wk.n_local <= 0) continue;
+            const int got = tc_get(p, L, k, P, wk);
+            if (got < 0) break;
+            if (got == 0 || wk.n_local <= 0) continue;
             if (p.k_new != nullptr && wk.first + wk.n_local == wk.n_pages)
                 append_new_token_part(p, wk.b, wk.kvh, wk.len, P, DH * 2, lane, half);
             if (half == 0 && lane == 0) {
@@ -446,12 +537,13 @@ __global__ void __launch_bounds__(224, 1)
                     if (!mbar_wait_bounded(q_full(i & 1), (i >> 1) & 1, kWaitLimitNs))
                         raise_err(p.err, KV_DEV_ERR_TIMEOUT);
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 || warp == C::kPVWarp) {
         // ------------------------------------------------------------ MMA issue
-        // Lane 0 issues the score products QK(j) as soon as K(j) has landed and an S^T buffer is free;
-        // lane 1 issues P.V(j) once the softmax has written P^T(j). Neither waits on the other's
+        // Warp 1 issues the score products QK(j) as soon as K(j) has landed and an S^T buffer is free;
+        // the P.V warp issues P.V(j) once the softmax has written P^T(j). Neither waits on the other's
         // barriers, so QK runs up to two stages ahead of the softmax.
-        if (lane < 2) {
+        const bool qk = warp == 1;
+        if (lane == 0) {
             bool ok = true;
             uint32_t J = 0;      // stages of the earlier items and this one
             int item_i = 0;
@@ -462,11 +554,13 @@ __global__ void __launch_bounds__(224, 1)
                 }
                 return ok;
             };
-            for (int k = 0; k < n_cand && ok; ++k) {
+            for (int k = 0; ok; ++k) {
                 TcWork wk;
-                if (!tc_get(p, L, k, P, wk) || wk.n_local <= 0) continue;
+                const int got = tc_get(p, L, k, P, wk);
+                if (got < 0) break;
+                if (got == 0 || wk.n_local <= 0) continue;
                 const int n_st = (wk.n_local + C::kPPS - 1) / C::kPPS;
-                if (lane == 0) {
+                if (qk) {
                     if (!wait(q_full(item_i & 1), (item_i >> 1) & 1)) break;
                     for (int j = 0; j < n_st; ++j, ++J) {
                         const int e = kslot(J);
@@ -515,7 +609,7 @@ __global__ void __launch_bounds__(224, 1)
                 ++item_i;
             }
             // every MMA this thread issued has completed before tensor memory is released
-            const uint32_t done = lane == 0 ? done_qk : done_pv;
+            const uint32_t done = qk ? done_qk : done_pv;
             umma_commit(done);
             if (!mbar_wait_bounded(done, 0, kWaitLimitNs)) raise_err(p.err, KV_DEV_ERR_TIMEOUT);
         }
@@ -556,9 +650,11 @@ __global__ void __launch_bounds__(224, 1)
             if (!wk.split_mode)
                 for (int h = 0; h < G; ++h) p.out[((int64_t)wk.b * p.H_q + wk.kvh * G + h) * DH + r] = 0.f;
         };
-        for (int k = 0; k < n_cand; ++k) {
+        for (int k = 0;; ++k) {
             TcWork wk;
-            if (!tc_get(p, L, k, P, wk)) continue;
+            const int got = tc_get(p, L, k, P, wk);
+            if (got < 0) break;
+            if (got == 0) continue;
             if (wk.bad_len && r == 0 && wk.split == 0 && p.items == nullptr) raise_err(p.err, KV_DEV_ERR_SEQ_LEN);
             if (wk.n_local <= 0 || !ok) {
                 zero_rows(wk);
@@ -706,7 +802,7 @@ __global__ void __launch_bounds__(224, 1)
             } else {
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
-                    const int64_t ps = p.items != nullptr ? (int64_t)wk.item * G + h : (hq0 + h) * p.num_splits + wk.split;
+                    const int64_t ps = wk.planned ? (int64_t)wk.item * G + h : (hq0 + h) * p.num_splits + wk.split;
                     p.part_u[ps * DH + r] = o[h];
                     if (r == 0) p.part_ml[ps] = make_float2(m_ref[h], lp[h]);
                 }

@@ -309,6 +309,20 @@ PlannedLayout planned_layout(int32_t B, int32_t H_q, int32_t H_kv, int32_t Dh, i
     return L;
 }
 
+// Balanced plan of the persistent tcgen05 kernel (paged_plan_stream_kernel):
+// the plan words, then two partial slots per CTA.
+PlannedLayout stream_layout(int32_t B, int32_t H_q, int32_t H_kv, int32_t Dh, int64_t grid) {
+    auto r16 = [](size_t x) { return (x + 15) / 16 * 16; };
+    const size_t g = static_cast<size_t>(H_q / H_kv);
+    PlannedLayout L{};
+    L.plan_off = 0;
+    L.items_off = r16(sizeof(int32_t) * static_cast<size_t>(plan_stream_words(B, grid)));
+    L.u_off = L.items_off;  // no item list
+    L.ml_off = L.u_off + r16(sizeof(float) * 2 * static_cast<size_t>(grid) * g * Dh);
+    L.total = L.ml_off + r16(sizeof(float2) * 2 * static_cast<size_t>(grid) * g);
+    return L;
+}
+
 // Automatic split choice between the two launch forms. With no more
 // (sequence, KV head) rows than two waves of resident CTAs, the grid rule
 // splits every row into equal ranges of the longest possible row and keeps
@@ -428,8 +442,16 @@ int paged_decode_workspace_bytes(int32_t B, int32_t H_q, int32_t H_kv, int32_t D
     int rc = resolve_splits(B, H_kv, max_blocks, num_splits, &S, &C);
     if (rc != KV_OK) return rc;
     size_t need = workspace_for(B, H_q, Dh, S);
+    // the pool dtype is not known here: cover the tcgen05 kernel's balanced plan (16-bit pools) and the
+    // chunked plan of the warp-MMA kernel (the other dtypes) wherever either may be chosen
     const bool tc = tc_ok(KV_DTYPE_BF16, H_q / H_kv, Dh, false) && H_q % H_kv == 0;
-    if (tc ? planned_tc(B, num_splits) : planned_ok(true, B, H_q, H_kv, num_splits)) {
+    if (tc && planned_tc(B, num_splits)) {
+        const int sms = sm_count();
+        if (sms <= 0) return KV_ERR_CUDA;
+        const size_t pl = stream_layout(B, H_q, H_kv, Dh, sms).total;
+        if (pl > need) need = pl;
+    }
+    if (planned_ok(true, B, H_q, H_kv, num_splits)) {
         const int64_t grid = planned_grid(B, H_kv);
         if (grid < 0) return KV_ERR_CUDA;
         const size_t pl = planned_layout(B, H_q, H_kv, Dh, grid).total;
@@ -532,7 +554,25 @@ int decode_impl(float* out, const void* q, const void* k_new, const void* v_new,
     dim3 grid(static_cast<unsigned>(S), static_cast<unsigned>(H_kv), static_cast<unsigned>(B));
     cudaError_t e;
     int64_t pgrid = 0;
-    if (planned) {
+    const int sms_all = sm_count();
+    if (sms_all <= 0) return KV_ERR_CUDA;
+    if (planned && tc) {
+        // balanced plan: one persistent CTA per SM, each streaming the same number of pages
+        pgrid = sms_all;
+        const PlannedLayout L = stream_layout(B, H_q, H_kv, Dh, pgrid);
+        if (!workspace || ws_bytes < L.total || !aligned16(workspace)) return KV_ERR_WORKSPACE;
+        char* w = static_cast<char*>(workspace);
+        int32_t* plan = reinterpret_cast<int32_t*>(w + L.plan_off);
+        p.plan = plan;
+        p.items = nullptr;
+        p.part_u = reinterpret_cast<float*>(w + L.u_off);
+        p.part_ml = reinterpret_cast<float2*>(w + L.ml_off);
+        p.num_splits = 0;
+        const int32_t min_pages = 2 * std::max<int32_t>(1, 128 / page_size);  // two stages of 128 keys
+        e = launch_pdl(paged_plan_stream_kernel, dim3(1), dim3(kPlanThreads), 0, st, seq_lens, B, H_kv, page_size,
+                       max_blocks, static_cast<int32_t>(pgrid), min_pages, plan, err_flag);
+        if (e != cudaSuccess) return KV_ERR_CUDA;
+    } else if (planned) {
         pgrid = planned_grid(B, H_kv);
         if (pgrid < 0) return KV_ERR_CUDA;
         if (pgrid > 0x7fffffffLL) return KV_ERR_UNSUPPORTED;
@@ -551,8 +591,8 @@ int decode_impl(float* out, const void* q, const void* k_new, const void* v_new,
         const int64_t partial_bytes = static_cast<int64_t>(H_q / H_kv) * (Dh + 2) * 4;
         const int32_t c_floor = static_cast<int32_t>(std::max<int64_t>(8, (16 * partial_bytes + chunk_bytes_per_page - 1) /
                                                                                 chunk_bytes_per_page));
-        // resident CTAs: two per SM for the warp-MMA kernel, one (persistent) for the tcgen05 kernel
-        const int32_t slots = static_cast<int32_t>((tc ? 1 : 2) * sm_count());
+        // resident CTAs of the warp-MMA kernel: two per SM
+        const int32_t slots = static_cast<int32_t>(2 * sms_all);
         e = launch_pdl(paged_plan_kernel, dim3(1), dim3(kPlanThreads), 0, st, seq_lens, B, H_kv, page_size, max_blocks,
                        slots, static_cast<int32_t>(pgrid), c_floor, plan, items, err_flag);
         if (e != cudaSuccess) return KV_ERR_CUDA;
@@ -573,9 +613,7 @@ int decode_impl(float* out, const void* q, const void* k_new, const void* v_new,
             return KV_ERR_CUDA;
         const int64_t n_work = planned ? pgrid : static_cast<int64_t>(S) * H_kv * B;
         if (n_work > 0x7fffffffLL) return KV_ERR_UNSUPPORTED;
-        const int sms = sm_count();
-        if (sms <= 0) return KV_ERR_CUDA;
-        const int tc_grid = static_cast<int>(std::min<int64_t>(n_work, sms));
+        const int tc_grid = static_cast<int>(std::min<int64_t>(n_work, sms_all));
         e = launch_tc(p, tk, tv, tq, dtype, page_size, static_cast<int>(n_work), tc_grid, st);
     } else if (mma) {
         CUtensorMap tk, tv;

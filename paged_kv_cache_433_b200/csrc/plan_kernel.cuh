@@ -22,12 +22,12 @@
 #include <cstdint>
 
 #include "kvpaged.h"
+#include "plan_layout.cuh"
 #include "ptx.cuh"
 
 namespace kvp {
 
 constexpr int kPlanThreads = 1024;
-constexpr int kPlanHdr = 4;
 constexpr int kPlanRowsPerThread = 8;  // rows held in registers per thread (B <= 8192)
 
 // Block-wide exclusive scan of one 64-bit value per thread; returns the block total.
@@ -156,6 +156,81 @@ __global__ void __launch_bounds__(kPlanThreads) paged_plan_kernel(const int32_t*
         if (total > grid && err) atomicOr(err, KV_DEV_ERR_PIPELINE);  // the host sizes the grid so this cannot happen
     }
     for (long long pos = n_full + tid; pos < grid - n_tail; pos += kPlanThreads) items[pos] = make_int4(-1, 0, 0, 0);
+}
+
+// Balanced ("stream") plan for the persistent tcgen05 decode kernel. The
+// (sequence, KV head) rows are laid end to end in (b, kvh) order -- row
+// (b, kvh) holds pages [H_kv S_b + kvh n_b, + n_b) of a line of
+// T = H_kv sum_b n_b pages -- and CTA c of G takes the pages
+// [floor(c T / G), floor((c + 1) T / G)): every CTA streams the same number
+// of pages (+-1), whatever the length mix. A row cut by a CTA boundary is
+// processed in pieces by consecutive CTAs; a piece leaves its (m, l, u)
+// partial in one of two slots of its CTA -- slot 2c + 1 when the row starts
+// inside the CTA's range (the CTA's last piece), slot 2c when it started
+// before (the CTA's first piece) -- and the combine kernel merges them. Rows
+// inside one CTA's range are written to the output directly.
+// G = min(grid, ceil(T / min_pages)) keeps at least `min_pages` per CTA.
+//
+// Plan layout (int32 words): [0] kPlanStream, [1] G, [2], [3] T (int64),
+// [4 ..] S_b (int64, B + 1 entries: exclusive prefix of n_b), then cta_row[G]:
+// the sequence whose rows hold page floor(c T / G).
+
+__global__ void __launch_bounds__(kPlanThreads) paged_plan_stream_kernel(const int32_t* __restrict__ seq_lens,
+                                                                         int32_t B, int32_t H_kv, int32_t P,
+                                                                         int32_t max_blocks, int32_t grid,
+                                                                         int32_t min_pages, int32_t* __restrict__ plan,
+                                                                         int* err) {
+    __shared__ unsigned long long warp_sums[32];
+    grid_dependency_wait();
+    if (threadIdx.x == 0) grid_launch_dependents();
+    const int tid = threadIdx.x;
+    int64_t* pre = plan_stream_prefix(plan);
+    int32_t* cta_row = plan + kPlanHdr + 2 * (B + 1);
+    // rows tid, tid + 1024, ...: page counts and their exclusive prefix in registers
+    int n[kPlanRowsPerThread];
+    long long s[kPlanRowsPerThread];
+    long long carry = 0;
+#pragma unroll
+    for (int r = 0; r < kPlanRowsPerThread; ++r) {
+        const int b = tid + r * kPlanThreads;
+        n[r] = 0;
+        s[r] = 0;
+        if (r * kPlanThreads >= B) continue;  // uniform over the block
+        if (b < B) {
+            int len = seq_lens[b];
+            if (len < 0 || len > max_blocks * P) {
+                if (err) atomicOr(err, KV_DEV_ERR_SEQ_LEN);
+                len = 0;
+            }
+            n[r] = (len + P - 1) / P;
+        }
+        unsigned long long tot;
+        const unsigned long long ex = block_exclusive_scan(static_cast<unsigned long long>(n[r]), warp_sums, tot);
+        s[r] = carry + static_cast<long long>(ex);
+        if (b < B) pre[b] = s[r];
+        carry += static_cast<long long>(tot);
+    }
+    const long long T = carry * H_kv;
+    long long G = min_pages > 0 ? (T + min_pages - 1) / min_pages : T;
+    if (G > grid) G = grid;
+    if (tid == 0) {
+        plan[0] = kPlanStream;
+        plan[1] = static_cast<int32_t>(G);
+        plan[2] = static_cast<int32_t>(T & 0xffffffffLL);
+        plan[3] = static_cast<int32_t>(T >> 32);
+        pre[B] = carry;
+    }
+    if (G <= 0) return;
+    // CTA c starts in the rows of sequence b when floor(c T / G) lies in [H_kv S_b, H_kv S_{b+1}), i.e.
+    // c in [ceil(H_kv S_b G / T), ceil(H_kv S_{b+1} G / T)); empty sequences own no CTA
+#pragma unroll
+    for (int r = 0; r < kPlanRowsPerThread; ++r) {
+        const int b = tid + r * kPlanThreads;
+        if (b >= B || n[r] == 0) continue;
+        const long long a0 = s[r] * H_kv, a1 = (s[r] + n[r]) * H_kv;
+        const long long c0 = (a0 * G + T - 1) / T, c1 = (a1 * G + T - 1) / T;
+        for (long long c = c0; c < c1; ++c) cta_row[c] = b;
+    }
 }
 
 }  // namespace kvp

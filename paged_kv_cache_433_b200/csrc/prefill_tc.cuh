@@ -29,15 +29,20 @@
 // than 2^8; the row's O and l are then rescaled (o = u / l for any common
 // reference).
 //
-// Warps (352 threads, one CTA per SM by tensor memory and shared memory):
-//   warps 0, 10 producers: per stage warp 0 the K boxes, warp 10 the V boxes
+// Warps (384 threads = three warpgroups, one CTA per SM by tensor memory and
+// shared memory):
+//   warps 0, 2 producers: per stage warp 0 the K boxes, warp 2 the V boxes
 //              of its pages (P rows x 128 bytes, 128-byte swizzle) into three
 //              K and two V entries of 32 KB (a K entry is refilled once its
 //              QK has run);
-//   warp 1     tensor memory allocation; lane 0 issues the QK(j), lane 1 the
-//              P.V(j), each paced only by its own barriers;
-//   warps 2-9  load the Q tile (swizzled stores), softmax, epilogue; each pair
+//   warp 1     tensor memory allocation; lane 0 issues the QK(j);
+//   warp 3     lane 0 issues the P.V(j); each issuer is paced only by its own
+//              barriers (in different warps, so one's wait never holds up
+//              the other);
+//   warps 4-11 load the Q tile (swizzled stores), softmax, epilogue; each pair
 //              of warps of one lane quarter syncs on its own named barrier.
+// The first warpgroup gives registers back (setmaxnreg) to the two softmax
+// warpgroups, which hold a 64-score half row each.
 // Every wait is bounded (KV_DEV_ERR_TIMEOUT); block-table entries outside
 // [0, num_pages) are never loaded (their keys are masked,
 // KV_DEV_ERR_PAGE_RANGE).
@@ -70,8 +75,14 @@ struct PfCfg {
     static constexpr int kNumBars = 2 * kRing + 1 + 3 + 2 + 3 + 3;
     static constexpr int kOffTmem = kOffBar + 8 * kNumBars;
     static constexpr int kSmem = 1024 + kOffTmem + 16;
-    static constexpr int kThreads = 352;
-    static constexpr int kVWarp = 10;            // the V producer (warp 0 produces K)
+    static constexpr int kThreads = 384;
+    static constexpr int kVWarp = 2;             // the V producer (warp 0 produces K)
+    static constexpr int kPVWarp = 3;            // issues P.V (warp 1 issues QK)
+    static constexpr int kFirstSoftmaxWarp = 4;
+    // registers per thread after the split: warpgroup 0 (producers, issuers) and warpgroups 1-2 (softmax);
+    // 128 x kRegsLow + 256 x kRegsHigh must not exceed the launch's 384 x (registers per thread), which the
+    // host checks before the first launch
+    static constexpr uint32_t kRegsLow = 56, kRegsHigh = 216;
     static constexpr int kSoftmaxWarps = 8;
     static constexpr uint32_t kTmemCols = 512;   // S x 3 (384) + O (128)
     static_assert(DH == 128, "instance: Dh = 128");
@@ -80,7 +91,7 @@ struct PfCfg {
 };
 
 template <int KT, int DH, int P>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(384, 1)
     paged_prefill_tc_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                             const __grid_constant__ CUtensorMap tmap_v) {
     using C = PfCfg<DH, P>;
@@ -171,6 +182,10 @@ __global__ void __launch_bounds__(352, 1)
     const uint32_t ring = sbase;
     const uint32_t sQ = sbase + C::kOffQ;
 
+    // the register split sits at the top of each warpgroup's branch, so every code path after it is
+    // compiled for its own budget
+    if (warp < C::kFirstSoftmaxWarp) {
+    regs_dec<C::kRegsLow>();
     if (warp == 0 || warp == C::kVWarp) {
         // ------------------------------------------------------------ producers
         // warp 0 issues the K boxes of every stage, warp kVWarp the V boxes: two streams of TMA requests
@@ -229,11 +244,12 @@ __global__ void __launch_bounds__(352, 1)
                         raise_err(p.err, KV_DEV_ERR_TIMEOUT);
             }
         }
-    } else if (warp == 1) {
+    } else {
         // ------------------------------------------------------------ MMA issue
-        // Lane 0 issues QK(j) once K(j) has landed and P.V(j - 3) has released S columns j % 3; lane 1
-        // issues P.V(j) once the softmax has written P(j). Neither waits on the other's barriers.
-        if (lane < 2) {
+        // Warp 1 issues QK(j) once K(j) has landed and P.V(j - 3) has released S columns j % 3; the P.V
+        // warp issues P.V(j) once the softmax has written P(j). Neither waits on the other's barriers.
+        const bool qk = warp == 1;
+        if (lane == 0) {
             bool ok = true;
             auto wait = [&](uint32_t bar, uint32_t parity) {
                 if (ok && !mbar_wait_bounded(bar, parity, kWaitLimitNs)) {
@@ -242,7 +258,7 @@ __global__ void __launch_bounds__(352, 1)
                 }
                 return ok;
             };
-            if (lane == 0) {
+            if (qk) {
                 if (wait(q_full, 0)) {
                     for (int j = 0; j < n_st; ++j) {
                         const int e = kslot(j);
@@ -282,15 +298,17 @@ __global__ void __launch_bounds__(352, 1)
                 }
                 if (ok) umma_commit(o_full);
             }
-            const uint32_t done = lane == 0 ? done_qk : done_pv;
+            const uint32_t done = qk ? done_qk : done_pv;
             umma_commit(done);
             if (!mbar_wait_bounded(done, 0, kWaitLimitNs)) raise_err(p.err, KV_DEV_ERR_TIMEOUT);
         }
         __syncwarp();
+    }
     } else {
+        regs_inc<C::kRegsHigh>();
         // ------------------------------------------------------------ Q tile, softmax, epilogue
         const int quarter = warp & 3;
-        const int half = (warp - 2) >> 2;    // key columns [64 half, 64 half + 64) of S, dims of O likewise
+        const int half = (warp - C::kFirstSoftmaxWarp) >> 2;  // key columns [64 half, 64 half + 64) of S, dims of O likewise
         const int r = quarter * 32 + lane;   // MMA row: chunk token t0 + r / g, head kvh * g + r % g
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
         const uint32_t pair_bar = 1 + quarter;  // named barrier of the two warps that share row r
@@ -393,17 +411,16 @@ __global__ void __launch_bounds__(352, 1)
                     continue;
                 }
                 tc_fence_after();
-                uint32_t a[32], b2[32];
-                tmem_ld32(tO + lane_addr + half * kH, a);
-                tmem_ld32(tO + lane_addr + half * kH + 32, b2);
-                tmem_wait_ld();
+                // 32 columns at a time: the 64 scores stay live across this block
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    a[i] = __float_as_uint(__uint_as_float(a[i]) * alpha);
-                    b2[i] = __float_as_uint(__uint_as_float(b2[i]) * alpha);
+                for (int q2 = 0; q2 < 2; ++q2) {
+                    uint32_t a[32];
+                    tmem_ld32(tO + lane_addr + half * kH + q2 * 32, a);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) a[i] = __float_as_uint(__uint_as_float(a[i]) * alpha);
+                    tmem_st32(tO + lane_addr + half * kH + q2 * 32, a);
                 }
-                tmem_st32(tO + lane_addr + half * kH, a);
-                tmem_st32(tO + lane_addr + half * kH + 32, b2);
                 tmem_wait_st();
             }
             // probabilities -> P over this S buffer: hi pairs in columns 0..63, residual pairs in 64..127

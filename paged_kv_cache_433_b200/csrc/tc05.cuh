@@ -51,6 +51,20 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 
+// Per-warpgroup register budget (the four warps of a warpgroup execute the same one): `dec` returns
+// registers to the CTA's pool, `inc` waits until the pool holds enough. The pool is what the CTA was
+// launched with (threads x registers per thread), so the shares of all warpgroups must fit in it.
+template <uint32_t R>
+__device__ __forceinline__ void regs_dec() {
+    static_assert(R % 8 == 0 && R >= 24 && R <= 256, "setmaxnreg range");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <uint32_t R>
+__device__ __forceinline__ void regs_inc() {
+    static_assert(R % 8 == 0 && R >= 24 && R <= 256, "setmaxnreg range");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+}
+
 // ---- ordering of tcgen05 operations around thread synchronisation ---------
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }

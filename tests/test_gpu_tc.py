@@ -88,6 +88,32 @@ def test_tc_mixed_batch_with_churn(P):
         check_close(out, ref, "bf16", f"tc mixed P={P} step {step}")
 
 
+# Balanced plan (num_splits = 0): CTA c streams pages [c T / G, (c + 1) T / G) of the rows laid end to end;
+# rows cut by a boundary are merged by the combine kernel from two partial slots per CTA.
+BALANCED_CASES = [
+    # one row spanning every CTA's range (many pieces of one row), beside a one-token row
+    ("span", "bf16", 16, 32, 1, [0, 148 * 3 * 128 + 37]),
+    # 16384 one-page rows: about 110 pieces per CTA, past the shared-memory work list
+    ("many", "bf16", 16, 32, 8, [0] * 2048),
+    # 296 rows of 16 pages: every CTA takes exactly two whole rows (boundaries coincide, no partials)
+    ("aligned", "fp16", 16, 32, 1, [16 * 16 - 1] * 296),
+    # fewer pages than two stages per CTA: a handful of CTAs carry the work
+    ("small", "bf16", 32, 32, 2, [3, 40, 0, 17, 100]),
+]
+
+
+@pytest.mark.parametrize("name,dtype,P,H_q,H_kv,lens", BALANCED_CASES, ids=[c[0] for c in BALANCED_CASES])
+def test_tc_balanced_plan(name, dtype, P, H_q, H_kv, lens):
+    cfg = W.DecodeConfig(f"tc-balanced-{name}", dtype, B=len(lens), H_q=H_q, H_kv=H_kv, Dh=128, page_size=P,
+                         seed=46)
+    st = build_cache(cfg, lens, extra_blocks=1, slack_pages=len(lens) + 8)  # a page per row for the second step
+    assert _assert_tc(cfg, st.max_blocks, 0) == 0
+    for step in range(2):
+        out, ref, err = append_and_decode(st, step=step, num_splits=0, fused=True, check_pools=(step == 1))
+        assert err == 0
+        check_close(out, ref, dtype, f"{cfg.name} step {step}")
+
+
 @pytest.mark.parametrize("splits", [0, 3])
 def test_tc_growing_scores_rescale(splits):
     """Keys whose scores rise far above the first stage's maximum: the reference maximum moves
