@@ -79,9 +79,8 @@ struct TcCfg {
     static constexpr int kOffP = kOffQ + 2 * kQB;  // two Q tiles (item parity)
     static constexpr int kOffRed = kOffP + 4 * kPB;          // 2 x [G][4] floats (after 2 x (hi, lo) P^T)
     static constexpr int kOffFlag = kOffRed + 2 * G * 4 * 4;  // 2 x 4 ints
-    static constexpr int kOffBad = kOffFlag + 32;             // int per ring entry
     static constexpr int kMaxList = 96;          // work items of a CTA resolved once into shared memory
-    static constexpr int kOffList = (kOffBad + 4 * kRing + 15) / 16 * 16;  // int4 x 2 per item
+    static constexpr int kOffList = kOffFlag + 32;            // int4 x 2 per item
     static constexpr int kOffStream = kOffList + kMaxList * 32;   // TcStream of a balanced plan (32 bytes)
     static constexpr int kOffBar = kOffStream + 32;
     // full[R], empty[R], q_full[2], q_empty[2], s_full[2], s_empty[2], p_full[2], p_empty[2], o_full[2],
@@ -399,7 +398,6 @@ __global__ void __launch_bounds__(256, 1)
     auto o_empty = [&](int i) { return bs0 + 80u + 8u * i; };
     const uint32_t done_qk = bs0 + 96u;
     const uint32_t done_pv = bs0 + 104u;
-    volatile int* stage_bad = reinterpret_cast<volatile int*>(smem + C::kOffBad);
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::kOffTmem);
 
     if (threadIdx.x == 0) {
@@ -512,7 +510,6 @@ __global__ void __launch_bounds__(256, 1)
                             raise_err(p.err, KV_DEV_ERR_TIMEOUT);
                             ok = false;
                         } else {
-                            stage_bad[e] = (int)(~gmask & ((1u << np) - 1u));
                             mbar_arrive_expect_tx(full(e), __popc(gmask) * C::kBoxCols * P * 128);
                         }
                     }
@@ -664,9 +661,16 @@ __global__ void __launch_bounds__(256, 1)
             float m_ref[G], lp[G];
 #pragma unroll
             for (int h = 0; h < G; ++h) m_ref[h] = -INFINITY, lp[h] = 0.f;
+            // the page of row r in each stage, read one stage ahead: the mask of pages the producers skip
+            // (entries outside the pool) is known without waiting for the V entry
+            const int32_t* trow = p.block_tables + (int64_t)wk.b * p.max_blocks + wk.first;
+            const int pr = r / P;
+            int pg_cur = pr < wk.n_local ? __ldg(trow + pr) : -1;
             for (int j = 0; j < n_st; ++j) {
                 bool okl = ok;
                 const int sb = J & 1;
+                const int nxt = (j + 1) * C::kPPS + pr;
+                const int pg_nxt = nxt < wk.n_local ? __ldg(trow + nxt) : -1;
                 float s[G];
 #pragma unroll
                 for (int h = 0; h < G; ++h) s[h] = -INFINITY;
@@ -681,15 +685,12 @@ __global__ void __launch_bounds__(256, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(s_empty(sb));
                 }
-                // the stage's V entry (and its skipped-page mask) must have landed
+                // token row r of the stage: inside the sequence, on a page of this stage that was loaded
                 const int ev = vslot(J);
-                bool valid = false;
-                if (wait(okl, full(ev), vphase(J))) {
-                    const int np = min(C::kPPS, wk.n_local - j * C::kPPS);
-                    const int bad = stage_bad[ev];
-                    const int pg_in = r / P;
-                    valid = (wk.first + j * C::kPPS) * P + r < wk.len && pg_in < np && !((bad >> pg_in) & 1);
-                }
+                const int np = min(C::kPPS, wk.n_local - j * C::kPPS);
+                const bool valid = okl && (wk.first + j * C::kPPS) * P + r < wk.len && pr < np && pg_cur >= 0 &&
+                                   pg_cur < p.num_pages;
+                pg_cur = pg_nxt;
 #pragma unroll
                 for (int h = 0; h < G; ++h) s[h] = valid ? s[h] * p.scale_log2 : -INFINITY;
                 // reference maximum: moves only when a score exceeds it by more than 2^8
@@ -758,13 +759,21 @@ __global__ void __launch_bounds__(256, 1)
                     sts128(sPhi(J) + off, hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
                     sts128(sPhi(J) + C::kPB + off, lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
                 }
-                // a masked token's V row may hold stale bytes (even NaN): zero it before P.V
-                if (!valid) {
-                    const uint32_t vrow = ring + ev * C::kEntry + r * 128;
+                // a masked token's V row may hold stale bytes (even NaN): zero it before P.V, once the V entry
+                // has landed (only warps with such a row wait for it; the P.V issuer waits for every entry)
+                if (__any_sync(0xffffffffu, !valid)) {
+                    if (!wait(okl, full(ev), vphase(J))) {
+                        ok = false;  // the next flag exchange stops every warp
+                        ++J;
+                        continue;
+                    }
+                    if (!valid) {
+                        const uint32_t vrow = ring + ev * C::kEntry + r * 128;
 #pragma unroll
-                    for (int bb = 0; bb < C::kBoxCols; ++bb)
+                        for (int bb = 0; bb < C::kBoxCols; ++bb)
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) sts128_zero(vrow + bb * C::kBoxB + c * 16);
+                            for (int c = 0; c < 8; ++c) sts128_zero(vrow + bb * C::kBoxB + c * 16);
+                    }
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();

@@ -68,8 +68,7 @@ struct PfCfg {
     static constexpr int kRing = kKSlots + kVSlots;
     static constexpr int kQB = 128 * DH * 2;     // Q tile: 128 rows
     static constexpr int kOffQ = kRing * kEntry;
-    static constexpr int kOffBad = kOffQ + kQB;
-    static constexpr int kOffX = (kOffBad + 4 * kRing + 15) / 16 * 16;  // row exchange: [2][2][128] floats + ints
+    static constexpr int kOffX = kOffQ + kQB;   // row exchange: [2][2][128] floats + ints
     static constexpr int kOffBar = kOffX + 2 * 2 * 128 * 4 * 2;
     // full[R], empty[R], q_full, s_full[3], p_full[2], p_empty[3], o_full, done (QK), done (PV)
     static constexpr int kNumBars = 2 * kRing + 1 + 3 + 2 + 3 + 3;
@@ -82,7 +81,7 @@ struct PfCfg {
     // registers per thread after the split: warpgroup 0 (producers, issuers) and warpgroups 1-2 (softmax);
     // 128 x kRegsLow + 256 x kRegsHigh must not exceed the launch's 384 x (registers per thread), which the
     // host checks before the first launch
-    static constexpr uint32_t kRegsLow = 56, kRegsHigh = 216;
+    static constexpr uint32_t kRegsLow = 64, kRegsHigh = 216;
     static constexpr int kSoftmaxWarps = 8;
     static constexpr uint32_t kTmemCols = 512;   // S x 3 (384) + O (128)
     static_assert(DH == 128, "instance: Dh = 128");
@@ -152,7 +151,6 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t o_full = q_full + 72;
     const uint32_t done_qk = q_full + 80;
     const uint32_t done_pv = q_full + 88;
-    volatile int* stage_bad = reinterpret_cast<volatile int*>(smem + C::kOffBad);
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::kOffTmem);
 
     if (threadIdx.x == 0) {
@@ -218,7 +216,6 @@ __global__ void __launch_bounds__(384, 1)
                         raise_err(p.err, KV_DEV_ERR_TIMEOUT);
                         ok = false;
                     } else {
-                        stage_bad[e] = (int)(~gmask & ((1u << np) - 1u));
                         mbar_arrive_expect_tx(full(e), __popc(gmask) * C::kBoxCols * P * 128);
                     }
                 }
@@ -358,9 +355,15 @@ __global__ void __launch_bounds__(384, 1)
         const float sl2 = p.scale_log2;
         float m_ref = -INFINITY, l = 0.f;
         constexpr int kH = C::kTP / 2;       // key columns per thread
+        // lanes 0 .. kPPS-1: the page ids of stage j, read one stage ahead; the mask of pages the producers
+        // skip (entries outside the pool) is then known without waiting for the V entry
+        const int32_t* trow = p.block_tables + (int64_t)b * p.max_blocks;
+        int pg_cur = lane < C::kPPS && lane < n_pages ? __ldg(trow + lane) : -1;
         for (int j = 0; j < n_st; ++j) {
             bool okl = ok;
             const uint32_t tS = tmem + (j % 3) * C::kTP + lane_addr;
+            const int nxt = (j + 1) * C::kPPS + lane;
+            const int pg_nxt = lane < C::kPPS && nxt < n_pages ? __ldg(trow + nxt) : -1;
             float s[kH];
             if (wait(okl, s_full(j % 3), (j / 3) & 1)) {
                 tc_fence_after();
@@ -375,8 +378,9 @@ __global__ void __launch_bounds__(384, 1)
             const int ev = vslot(j);
             const int kbase = j * C::kTP;
             const int np = min(C::kPPS, n_pages - j * C::kPPS);
-            int bad = 0;
-            if (wait(okl, full(ev), vphase(j))) bad = stage_bad[ev];
+            const unsigned loaded = __ballot_sync(0xffffffffu, lane < np && pg_cur >= 0 && pg_cur < p.num_pages);
+            const int bad = static_cast<int>(~loaded & ((1u << np) - 1u));
+            pg_cur = pg_nxt;
             // keys this row may see in the stage: [0, lim); pages skipped or not loaded are masked
             const int lim = row_valid ? min(C::kTP, pos + 1 - kbase) : 0;
             const bool full_stage = lim == C::kTP && np == C::kPPS && bad == 0;
@@ -441,13 +445,21 @@ __global__ void __launch_bounds__(384, 1)
             }
             tmem_wait_st();
             // a key no row may see (past the tile, or on a page not loaded) may hold stale bytes: zero its V row
-            // (this thread: box column `half` of V row r)
+            // (this thread: box column `half` of V row r) once the V entry has landed; only warps with such a
+            // row wait for it (the P.V issuer waits for every entry)
             {
                 const int pgi = r / P;
-                if (kbase + r >= key_end || pgi >= np || ((bad >> pgi) & 1)) {
-                    const uint32_t vrow = ring + ev * C::kEntry + half * C::kBoxB + r * 128;
+                const bool stale = kbase + r >= key_end || pgi >= np || ((bad >> pgi) & 1);
+                if (__any_sync(0xffffffffu, stale)) {
+                    if (!wait(okl, full(ev), vphase(j))) {
+                        ok = false;  // the next meeting stops the pair
+                        continue;
+                    }
+                    if (stale) {
+                        const uint32_t vrow = ring + ev * C::kEntry + half * C::kBoxB + r * 128;
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) sts128_zero(vrow + c * 16);
+                        for (int c = 0; c < 8; ++c) sts128_zero(vrow + c * 16);
+                    }
                 }
             }
             fence_proxy_async_smem();
