@@ -26,9 +26,6 @@ constexpr int kCombineWarps = 8;
 // first item come from the plan; rows with one chunk were written by the
 // decode kernel and are skipped, empty rows are zeroed here; partial s of
 // (b, query head h) sits at item t0 + s, row h of that item's [g][Dh] block.
-// Balanced plans (plan[0] == kPlanStream): the row's pages lie in the ranges
-// of CTAs c0 .. c1; its first piece left its partial in slot 2 c0 + 1, piece
-// s >= 1 in slot 2 (c0 + s).
 template <int DH, int WPR>
 __global__ void __launch_bounds__(32 * kCombineWarps) paged_combine_kernel(
     float* __restrict__ out, const float* __restrict__ part_u, const float2* __restrict__ part_ml,
@@ -48,33 +45,13 @@ __global__ void __launch_bounds__(32 * kCombineWarps) paged_combine_kernel(
     if (threadIdx.x == 0) grid_launch_dependents();
     bool live = item < (int64_t)B * H_q;
     int ns = 0;
-    int64_t base = item * S, stride = 1, first = 0;  // partial s at base + (s == 0 ? first : s * stride)
+    int64_t base = item * S, stride = 1;
     if (live) {
         const int b = static_cast<int>(item / H_q);
         int len = seq_lens[b];
         if (len < 0 || len > max_blocks * P) len = 0;
         const int n_pages = (len + P - 1) / P;
-        if (plan != nullptr && plan[0] == kPlanStream) {
-            const int G = plan[1];
-            const long long T = static_cast<long long>(static_cast<uint32_t>(plan[2])) |
-                                (static_cast<long long>(plan[3]) << 32);
-            const int64_t* pre = plan_stream_prefix(plan);
-            const int g = H_q / H_kv;
-            const int hq = static_cast<int>(item % H_q);
-            const long long s0 = pre[b], n = pre[b + 1] - s0;
-            if (n > 0 && G > 0) {
-                const long long r0 = (long long)H_kv * s0 + (long long)(hq / g) * n;
-                const int c0 = plan_stream_cta(r0, T, G), c1 = plan_stream_cta(r0 + n - 1, T, G);
-                if (c0 == c1) {
-                    live = false;  // the decode kernel wrote this row
-                } else {
-                    ns = c1 - c0 + 1;
-                    base = 2LL * g * c0 + hq % g;
-                    stride = 2LL * g;
-                    first = g;
-                }
-            }
-        } else if (plan != nullptr) {
+        if (plan != nullptr) {
             const int C = plan[0];
             const int items_b = (n_pages + C - 1) / C;
             const int g = H_q / H_kv;
@@ -103,9 +80,8 @@ __global__ void __launch_bounds__(32 * kCombineWarps) paged_combine_kernel(
         for (int j = 0; j < kPer; ++j) {
             const int s = r0 + rw + j * WPR;
             if (s < ns) {
-                const int64_t off = s == 0 ? first : (int64_t)s * stride;
-                st[j] = ml[off];
-                const float* src = pu + off * DH;
+                st[j] = ml[s * stride];
+                const float* src = pu + (int64_t)s * stride * DH;
                 if constexpr (kD == 4) {
                     const float4 x = *reinterpret_cast<const float4*>(src);
                     v[j][0] = x.x; v[j][1] = x.y; v[j][2] = x.z; v[j][3] = x.w;
@@ -120,7 +96,7 @@ __global__ void __launch_bounds__(32 * kCombineWarps) paged_combine_kernel(
             }
         }
         if (r0 == 0) {
-            for (int s = lane; s < ns; s += 32) mstar = fmaxf(mstar, ml[s == 0 ? first : (int64_t)s * stride].x);
+            for (int s = lane; s < ns; s += 32) mstar = fmaxf(mstar, ml[s * stride].x);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) mstar = fmaxf(mstar, __shfl_xor_sync(0xffffffffu, mstar, o));
         }
@@ -164,6 +140,90 @@ __global__ void __launch_bounds__(32 * kCombineWarps) paged_combine_kernel(
             }
         }
     }
+}
+
+// Combine of a balanced plan (paged_plan_stream_kernel): only rows cut by a
+// CTA boundary have partials, at most one per boundary, so CTA c of the grid
+// merges the row that starts in CTA c's page range and runs past its end (if
+// any): its first piece is in slot 2c + 1, piece s >= 1 in slot 2 (c + s).
+// One warp per head of the row's GQA group (g <= 32); lane s holds piece s's
+// (m, l) and weight, then every lane sums DH / 32 dims over the pieces with
+// all loads of a round issued before any is used. Rows inside one range were
+// written by the decode kernel, rows without pages by the plan kernel.
+constexpr int kCombineStreamWarps = 32;
+
+template <int DH>
+__global__ void __launch_bounds__(32 * kCombineStreamWarps) paged_combine_stream_kernel(
+    float* __restrict__ out, const float* __restrict__ part_u, const float2* __restrict__ part_ml,
+    const int32_t* __restrict__ plan, int32_t B, int32_t H_q, int32_t H_kv) {
+    constexpr int kD = DH / 32;
+    constexpr int kRound = 4;  // pieces whose dims are loaded together
+    const int h = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    grid_dependency_wait();  // the decode kernel's partials
+    if (threadIdx.x == 0) grid_launch_dependents();
+    const int g = H_q / H_kv;
+    if (h >= g) return;
+    const int G = plan[1];
+    const int c = blockIdx.x;
+    if (c + 1 >= G) return;  // the last range ends the line
+    const long long T = static_cast<long long>(static_cast<uint32_t>(plan[2])) | (static_cast<long long>(plan[3]) << 32);
+    const int64_t* pre = plan_stream_prefix(plan);
+    const long long lo = T * c / G, hi = T * (c + 1) / G;
+    // the row holding page hi: its sequence starts CTA c + 1's range
+    const int b = plan[kPlanHdr + 2 * (B + 1) + c + 1];
+    const long long s0 = pre[b], n = pre[b + 1] - s0;
+    if (n <= 0) return;
+    const int kvh = static_cast<int>((hi - (long long)H_kv * s0) / n);
+    const long long r0 = (long long)H_kv * s0 + (long long)kvh * n;
+    if (r0 >= hi || r0 < lo) return;  // starts at the boundary (not cut) or in an earlier range
+    const int ns = plan_stream_cta(r0 + n - 1, T, G) - c + 1;
+    auto slot = [&](int s) { return (s == 0 ? 2LL * c + 1 : 2LL * (c + s)) * g + h; };
+    float acc[kD];
+#pragma unroll
+    for (int i = 0; i < kD; ++i) acc[i] = 0.f;
+    float L = 0.f;
+    // the maximum over all pieces, then passes of 32 pieces (lane s: piece base + s's weight)
+    float mstar = -INFINITY;
+    for (int s = lane; s < ns; s += 32) mstar = fmaxf(mstar, part_ml[slot(s)].x);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mstar = fmaxf(mstar, __shfl_xor_sync(0xffffffffu, mstar, o));
+    for (int base = 0; base < ns && mstar != -INFINITY; base += 32) {
+        const int s_l = base + lane;
+        float w = 0.f;
+        if (s_l < ns) {
+            const float2 st = part_ml[slot(s_l)];
+            if (st.x != -INFINITY) w = exp2f(st.x - mstar);
+            L += w * st.y;
+        }
+        const int cnt = min(32, ns - base);
+        for (int s = 0; s < cnt; s += kRound) {
+            float v[kRound][kD];
+            float ws[kRound];
+#pragma unroll
+            for (int q = 0; q < kRound; ++q) {
+                ws[q] = __shfl_sync(0xffffffffu, w, (s + q) & 31);
+                if (s + q < cnt && ws[q] != 0.f) {
+                    const float* src = part_u + slot(base + s + q) * DH + lane * kD;
+#pragma unroll
+                    for (int i = 0; i < kD; ++i) v[q][i] = src[i];
+                } else {
+#pragma unroll
+                    for (int i = 0; i < kD; ++i) v[q][i] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < kRound; ++q)
+#pragma unroll
+                for (int i = 0; i < kD; ++i) acc[i] += ws[q] * v[q][i];
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    float* dst = out + ((int64_t)b * H_q + (int64_t)kvh * g + h) * DH + lane * kD;
+#pragma unroll
+    for (int i = 0; i < kD; ++i) dst[i] = acc[i] * inv;
 }
 
 }  // namespace kvp

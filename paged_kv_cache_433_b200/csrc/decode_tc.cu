@@ -18,6 +18,14 @@ cudaError_t launch_tc_inst(const DecodeParams& p, const CUtensorMap& tk, const C
     if (e != cudaSuccess) return e;
     const uint64_t bit = 1ull << (dev & 63);
     if (!(configured.load(std::memory_order_acquire) & bit)) {
+        // the kernel moves registers between its warpgroups (setmaxnreg): the shares must fit in what a CTA
+        // is launched with, or a warpgroup asking for more would wait for ever
+        cudaFuncAttributes fa{};
+        e = cudaFuncGetAttributes(&fa, kern);
+        if (e != cudaSuccess) return e;
+        const long long pool = static_cast<long long>(fa.numRegs) * C::kThreads;
+        const long long need = 128LL * (C::kRegsLow + C::kRegsSoftmax + C::kRegsEpi);
+        if (need > pool) return cudaErrorInvalidConfiguration;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         if (e != cudaSuccess) return e;
         configured.fetch_or(bit, std::memory_order_acq_rel);

@@ -24,17 +24,23 @@
 // maximum is reduced over the CTA, and O^T and the partial row sums are
 // rescaled (o = u / l holds for any common reference).
 //
-// Warp roles (256 threads, one CTA per SM, persistent over work items):
-//   warps 0, 6 producers: warp 0 the Q tile (2-D TMA, 128-byte swizzle) and
-//              the K boxes of each stage, warp 6 the V boxes (P rows x 128
+// Warp roles (384 threads = three warpgroups, one CTA per SM, persistent over
+// work items):
+//   warps 0, 2 producers: warp 0 the Q tile (2-D TMA, 128-byte swizzle) and
+//              the K boxes of each stage, warp 2 the V boxes (P rows x 128
 //              bytes each), into K and V entries of 32 KB; each writes its
 //              half of the fused append when the item owns the last page.
 //   warp 1     allocates tensor memory and resolves the CTA's work items
 //              into shared memory; its lane 0 issues the QK(j).
-//   warp 7     lane 0 issues the P.V(j). The two issuers sit in different
+//   warp 3     lane 0 issues the P.V(j). The two issuers sit in different
 //              warps so that neither one's wait holds up the other (two
 //              lanes of one warp would take turns).
-//   warps 2-5  softmax and epilogue (tensor-memory lane quarter = warp % 4).
+//   warps 4-7  softmax (tensor-memory lane quarter = warp % 4); at the end of
+//              an item they hand its row sums and maxima to
+//   warps 8-11 the epilogue: O^T of the item over the sums, or its partial,
+//              while the softmax warps already work on the next item.
+// The first and last warpgroups give registers (setmaxnreg) to the softmax
+// warpgroup, whose threads hold G scores, maxima and sums each.
 // A work item is (sequence, KV head, chunk of pages): from the device plan
 // (planned launch) or from the grid rule (split); partials use the layout of
 // decode_mma.cuh, so paged_combine_kernel merges them.
@@ -80,17 +86,25 @@ struct TcCfg {
     static constexpr int kOffRed = kOffP + 4 * kPB;          // 2 x [G][4] floats (after 2 x (hi, lo) P^T)
     static constexpr int kOffFlag = kOffRed + 2 * G * 4 * 4;  // 2 x 4 ints
     static constexpr int kMaxList = 96;          // work items of a CTA resolved once into shared memory
-    static constexpr int kOffList = kOffFlag + 32;            // int4 x 2 per item
+    static constexpr int kOffMask = kOffFlag + 32;            // ints: skipped-page mask per K entry, per S^T buffer
+    static constexpr int kOffStats = kOffMask + 32;           // 2 x [l, m][G] floats: an item's sums and maxima
+    static constexpr int kOffList = kOffStats + 2 * 2 * G * 4;  // int4 x 2 per item
     static constexpr int kOffStream = kOffList + kMaxList * 32;   // TcStream of a balanced plan (32 bytes)
     static constexpr int kOffBar = kOffStream + 32;
     // full[R], empty[R], q_full[2], q_empty[2], s_full[2], s_empty[2], p_full[2], p_empty[2], o_full[2],
-    // o_empty[2], done (QK issuer), done (PV issuer)
-    static constexpr int kNumBars = 2 * kRing + 4 + 4 + 4 + 4 + 2;
+    // o_empty[2], done (QK issuer), done (PV issuer), stats_full[2], stats_empty[2]
+    static constexpr int kNumBars = 2 * kRing + 4 + 4 + 4 + 4 + 2 + 4 + 2;  // + mask_full[2]
     static constexpr int kOffTmem = kOffBar + 8 * kNumBars;
     static constexpr int kSmem = 1024 + kOffTmem + 16;
-    static constexpr int kThreads = 256;
-    static constexpr int kVWarp = 6;             // the V producer (warp 0 produces Q and K)
-    static constexpr int kPVWarp = 7;            // issues P.V (warp 1 issues QK)
+    static constexpr int kThreads = 384;         // three warpgroups
+    static constexpr int kVWarp = 2;             // the V producer (warp 0 produces Q and K)
+    static constexpr int kPVWarp = 3;            // issues P.V (warp 1 issues QK)
+    static constexpr int kFirstSoftmaxWarp = 4;  // warps 4-7: softmax
+    static constexpr int kFirstEpiWarp = 8;      // warps 8-11: epilogue
+    // registers per thread after the split (setmaxnreg) of warpgroup 0 (producers, issuers), 1 (softmax,
+    // G scores per thread) and 2 (epilogue): 128 x their sum must fit in the launch's 384 x (registers per
+    // thread), which the host checks before the first launch
+    static constexpr uint32_t kRegsLow = 64, kRegsSoftmax = 248, kRegsEpi = 136;
     static constexpr uint32_t kTmemCols = 4 * kN <= 64 ? 64 : 128;  // S^T x 2 + O^T x 2, N columns each
     static_assert((G == 4 || G == 8 || G == 16 || G == 32) && DH == 128, "instances: g in {4, 8, 16, 32}, Dh = 128");
     static_assert(kPPS * kBoxCols <= 32, "one TMA box per lane");
@@ -352,7 +366,7 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, ui
 }
 
 template <int KT, int DH, int P, int G>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     paged_decode_tc_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                            const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_q,
                            int n_work) {
@@ -398,6 +412,15 @@ __global__ void __launch_bounds__(256, 1)
     auto o_empty = [&](int i) { return bs0 + 80u + 8u * i; };
     const uint32_t done_qk = bs0 + 96u;
     const uint32_t done_pv = bs0 + 104u;
+    // an item's row sums and reference maxima, softmax -> epilogue warps (double-buffered by item parity)
+    auto stats_full = [&](int i) { return bs0 + 112u + 8u * i; };
+    auto stats_empty = [&](int i) { return bs0 + 128u + 8u * i; };
+    // the skipped-page mask of a stage travels producer -> K entry word -> QK issuer -> S^T buffer word, the
+    // last hop announced on mask_full (the softmax needs it before the V entry lands)
+    auto mask_full = [&](int i) { return bs0 + 144u + 8u * i; };
+    volatile int* kmask = reinterpret_cast<volatile int*>(smem + C::kOffMask);      // [kKSlots]
+    volatile int* smask = reinterpret_cast<volatile int*>(smem + C::kOffMask + 16);  // [2]
+    float* stats = reinterpret_cast<float*>(smem + C::kOffStats);
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::kOffTmem);
 
     if (threadIdx.x == 0) {
@@ -421,6 +444,11 @@ __global__ void __launch_bounds__(256, 1)
         }
         mbar_init(done_qk, 1);
         mbar_init(done_pv, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(stats_full(i), 4);
+            mbar_init(stats_empty(i), 4);
+            mbar_init(mask_full(i), 1);
+        }
         fence_barrier_init();
     }
     int4* list_e = reinterpret_cast<int4*>(smem + C::kOffList);
@@ -453,6 +481,10 @@ __global__ void __launch_bounds__(256, 1)
     const uint32_t sP = sbase + C::kOffP;
     auto sPhi = [&](uint32_t j) { return sP + (j & 1) * 2 * C::kPB; };
 
+    // the register split sits at the top of each warpgroup's branch, so every code path after it is
+    // compiled for its own budget
+    if (warp < C::kFirstSoftmaxWarp) {
+    regs_dec<C::kRegsLow>();
     if (warp == 0 || warp == C::kVWarp) {
         // ------------------------------------------------------------ producers
         // Two warps issue the TMA boxes, one the K entries (and Q), the other the V entries: each
@@ -510,6 +542,7 @@ __global__ void __launch_bounds__(256, 1)
                             raise_err(p.err, KV_DEV_ERR_TIMEOUT);
                             ok = false;
                         } else {
+                            if (half == 0) kmask[e] = static_cast<int>(~gmask & ((1u << np) - 1u));
                             mbar_arrive_expect_tx(full(e), __popc(gmask) * C::kBoxCols * P * 128);
                         }
                     }
@@ -534,7 +567,7 @@ __global__ void __launch_bounds__(256, 1)
                     if (!mbar_wait_bounded(q_full(i & 1), (i >> 1) & 1, kWaitLimitNs))
                         raise_err(p.err, KV_DEV_ERR_TIMEOUT);
         }
-    } else if (warp == 1 || warp == C::kPVWarp) {
+    } else {
         // ------------------------------------------------------------ MMA issue
         // Warp 1 issues the score products QK(j) as soon as K(j) has landed and an S^T buffer is free;
         // the P.V warp issues P.V(j) once the softmax has written P^T(j). Neither waits on the other's
@@ -563,6 +596,7 @@ __global__ void __launch_bounds__(256, 1)
                         const int e = kslot(J);
                         const int sb = J & 1;
                         if (!wait(full(e), kphase(J))) break;
+                        const int bad = kmask[e];
                         if (J >= 2 && !wait(s_empty(sb), ((J >> 1) - 1) & 1)) break;
                         tc_fence_after();
                         const uint32_t sK = ring + e * C::kEntry;
@@ -574,6 +608,8 @@ __global__ void __launch_bounds__(256, 1)
                                     smem_desc(sQ(item_i & 1) + qoff, 16, 1024, kSwz128), kIdescQK, kk > 0 ? 1u : 0u);
                         }
                         umma_commit(s_full(sb));
+                        smask[sb] = bad;  // S^T buffer sb is free (s_empty above), so is its mask word
+                        mbar_arrive(mask_full(sb));
                         umma_commit(empty(e));
                         if (j == n_st - 1) umma_commit(q_empty(item_i & 1));
                     }
@@ -611,11 +647,13 @@ __global__ void __launch_bounds__(256, 1)
             if (!mbar_wait_bounded(done, 0, kWaitLimitNs)) raise_err(p.err, KV_DEV_ERR_TIMEOUT);
         }
         __syncwarp();
-    } else {
-        // ------------------------------------------------------------ softmax + epilogue
+    }
+    } else if (warp < C::kFirstEpiWarp) {
+        regs_inc<C::kRegsSoftmax>();
+        // ------------------------------------------------------------ softmax
         // Named barrier 1 (these 128 threads) is only ever reached by all four warps together: a
         // failed wait is shared at the next flag exchange and every warp then stops at once.
-        const int sw = warp - 2;           // softmax warp 0..3
+        const int sw = warp - C::kFirstSoftmaxWarp;  // softmax warp 0..3
         const int quarter = warp & 3;      // tensor-memory lane quarter of this warp
         const int r = quarter * 32 + lane;  // token row of S^T, dimension row of O^T
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
@@ -643,34 +681,20 @@ __global__ void __launch_bounds__(256, 1)
             fbuf ^= 1;
             return all;
         };
-        auto zero_rows = [&](const TcWork& wk) {
-            if (!wk.split_mode)
-                for (int h = 0; h < G; ++h) p.out[((int64_t)wk.b * p.H_q + wk.kvh * G + h) * DH + r] = 0.f;
-        };
         for (int k = 0;; ++k) {
             TcWork wk;
             const int got = tc_get(p, L, k, P, wk);
             if (got < 0) break;
-            if (got == 0) continue;
-            if (wk.bad_len && r == 0 && wk.split == 0 && p.items == nullptr) raise_err(p.err, KV_DEV_ERR_SEQ_LEN);
-            if (wk.n_local <= 0 || !ok) {
-                zero_rows(wk);
-                continue;
-            }
+            if (got == 0 || wk.n_local <= 0 || !ok) continue;  // the epilogue warps zero such rows
             const int n_st = (wk.n_local + C::kPPS - 1) / C::kPPS;
             float m_ref[G], lp[G];
 #pragma unroll
             for (int h = 0; h < G; ++h) m_ref[h] = -INFINITY, lp[h] = 0.f;
-            // the page of row r in each stage, read one stage ahead: the mask of pages the producers skip
-            // (entries outside the pool) is known without waiting for the V entry
-            const int32_t* trow = p.block_tables + (int64_t)wk.b * p.max_blocks + wk.first;
-            const int pr = r / P;
-            int pg_cur = pr < wk.n_local ? __ldg(trow + pr) : -1;
+            const int pr = r / P;  // page of row r within a stage
             for (int j = 0; j < n_st; ++j) {
                 bool okl = ok;
                 const int sb = J & 1;
-                const int nxt = (j + 1) * C::kPPS + pr;
-                const int pg_nxt = nxt < wk.n_local ? __ldg(trow + nxt) : -1;
+                int bad = -1;
                 float s[G];
 #pragma unroll
                 for (int h = 0; h < G; ++h) s[h] = -INFINITY;
@@ -682,15 +706,15 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
                     for (int h = 0; h < G; ++h) s[h] = __uint_as_float(a[h]);
                     tc_fence_before();
+                    // the stage's skipped-page mask, read before S^T buffer sb (and its mask word) is released
+                    if (wait(okl, mask_full(sb), (J >> 1) & 1)) bad = smask[sb];
                     __syncwarp();
                     if (lane == 0) mbar_arrive(s_empty(sb));
                 }
                 // token row r of the stage: inside the sequence, on a page of this stage that was loaded
                 const int ev = vslot(J);
                 const int np = min(C::kPPS, wk.n_local - j * C::kPPS);
-                const bool valid = okl && (wk.first + j * C::kPPS) * P + r < wk.len && pr < np && pg_cur >= 0 &&
-                                   pg_cur < p.num_pages;
-                pg_cur = pg_nxt;
+                const bool valid = okl && (wk.first + j * C::kPPS) * P + r < wk.len && pr < np && !((bad >> pr) & 1);
 #pragma unroll
                 for (int h = 0; h < G; ++h) s[h] = valid ? s[h] * p.scale_log2 : -INFINITY;
                 // reference maximum: moves only when a score exceeds it by more than 2^8
@@ -781,16 +805,65 @@ __global__ void __launch_bounds__(256, 1)
                 if (lane == 0) mbar_arrive(p_full(J & 1));
                 ++J;
             }
-            // ---- epilogue: O^T row r, row sums over the CTA, output or partials
-            bool okl = ok;
-            if (wait(okl, o_full(item_i & 1), (item_i >> 1) & 1)) {
-                tc_fence_after();
+            // ---- hand the item to the epilogue warps: row sums over the CTA and the reference maxima
+            cta_heads_reduce<G, false>(lp, red, sw, lane, rbuf);
+            bool oks = ok;
+            if (item_i >= 2) wait(oks, stats_empty(item_i & 1), ((item_i >> 1) - 1) & 1);
+            if (exchange(oks ? 0 : 2) & 2) {
+                ok = false;
+                continue;
             }
-            if (exchange(okl ? 0 : 2) & 2) ok = false;
-            if (!ok) {
+            if (r == 0) {
+                float* stl = stats + (item_i & 1) * 2 * G;
+#pragma unroll
+                for (int h = 0; h < G; ++h) stl[h] = lp[h], stl[G + h] = m_ref[h];
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(stats_full(item_i & 1));
+            ++item_i;
+        }
+    } else {
+        regs_dec<C::kRegsEpi>();
+        // ------------------------------------------------------------ epilogue
+        // Row r of O^T of each item (once its last P.V has completed) over the CTA's row sums, or kept
+        // as a partial (u, m, l) for the combine kernel; the softmax warps meanwhile go on with the next
+        // item. Frees O^T and the statistics slot for item i + 2.
+        const int quarter = warp & 3;       // tensor-memory lane quarter of this warp
+        const int r = quarter * 32 + lane;  // dimension row of O^T
+        const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+        bool ok = true;
+        int item_i = 0;
+        auto wait = [&](bool& okl, uint32_t bar, uint32_t parity) {
+            if (okl && !mbar_wait_bounded(bar, parity, kWaitLimitNs)) {
+                raise_err(p.err, KV_DEV_ERR_TIMEOUT);
+                okl = false;
+            }
+            okl = __all_sync(0xffffffffu, okl);
+            return okl;
+        };
+        auto zero_rows = [&](const TcWork& wk) {
+            if (!wk.split_mode)
+                for (int h = 0; h < G; ++h) p.out[((int64_t)wk.b * p.H_q + wk.kvh * G + h) * DH + r] = 0.f;
+        };
+        for (int k = 0;; ++k) {
+            TcWork wk;
+            const int got = tc_get(p, L, k, P, wk);
+            if (got < 0) break;
+            if (got == 0) continue;
+            if (wk.bad_len && r == 0 && wk.split == 0 && p.items == nullptr) raise_err(p.err, KV_DEV_ERR_SEQ_LEN);
+            if (wk.n_local <= 0 || !ok) {
                 zero_rows(wk);
                 continue;
             }
+            bool okl = ok;
+            wait(okl, stats_full(item_i & 1), (item_i >> 1) & 1);
+            wait(okl, o_full(item_i & 1), (item_i >> 1) & 1);
+            if (!okl) {
+                ok = false;  // an earlier stage failed: this and the later rows are zeroed
+                zero_rows(wk);
+                continue;
+            }
+            tc_fence_after();
             float o[G];
             {
                 uint32_t a[N];
@@ -802,18 +875,25 @@ __global__ void __launch_bounds__(256, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(o_empty(item_i & 1));
+            float l[G], m[G];
+            {
+                const float* stl = stats + (item_i & 1) * 2 * G;
+#pragma unroll
+                for (int h = 0; h < G; ++h) l[h] = stl[h], m[h] = stl[G + h];
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(stats_empty(item_i & 1));
             ++item_i;
-            cta_heads_reduce<G, false>(lp, red, sw, lane, rbuf);
             const int64_t hq0 = (int64_t)wk.b * p.H_q + (int64_t)wk.kvh * G;
             if (!wk.split_mode) {
 #pragma unroll
-                for (int h = 0; h < G; ++h) p.out[(hq0 + h) * DH + r] = lp[h] > 0.f ? o[h] / lp[h] : 0.f;
+                for (int h = 0; h < G; ++h) p.out[(hq0 + h) * DH + r] = l[h] > 0.f ? o[h] / l[h] : 0.f;
             } else {
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
                     const int64_t ps = wk.planned ? (int64_t)wk.item * G + h : (hq0 + h) * p.num_splits + wk.split;
                     p.part_u[ps * DH + r] = o[h];
-                    if (r == 0) p.part_ml[ps] = make_float2(m_ref[h], lp[h]);
+                    if (r == 0) p.part_ml[ps] = make_float2(m[h], l[h]);
                 }
             }
         }

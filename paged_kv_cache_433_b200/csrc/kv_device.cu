@@ -570,7 +570,7 @@ int decode_impl(float* out, const void* q, const void* k_new, const void* v_new,
         p.num_splits = 0;
         const int32_t min_pages = 2 * std::max<int32_t>(1, 128 / page_size);  // two stages of 128 keys
         e = launch_pdl(paged_plan_stream_kernel, dim3(1), dim3(kPlanThreads), 0, st, seq_lens, B, H_kv, page_size,
-                       max_blocks, static_cast<int32_t>(pgrid), min_pages, plan, err_flag);
+                       max_blocks, static_cast<int32_t>(pgrid), min_pages, plan, out, H_q, Dh, err_flag);
         if (e != cudaSuccess) return KV_ERR_CUDA;
     } else if (planned) {
         pgrid = planned_grid(B, H_kv);
@@ -632,7 +632,15 @@ int decode_impl(float* out, const void* q, const void* k_new, const void* v_new,
         }
     }
     if (e != cudaSuccess) return KV_ERR_CUDA;
-    if (planned || S > 1) {
+    if (planned && tc) {
+        // balanced plan: one CTA per range boundary merges the row cut there (if any)
+        const dim3 blocks(static_cast<unsigned>(pgrid)), threads(32 * kCombineStreamWarps);
+        e = Dh == 128 ? launch_pdl(paged_combine_stream_kernel<128>, blocks, threads, 0, st, out, p.part_u, p.part_ml,
+                                   static_cast<const int32_t*>(p.plan), B, H_q, H_kv)
+                      : launch_pdl(paged_combine_stream_kernel<64>, blocks, threads, 0, st, out, p.part_u, p.part_ml,
+                                   static_cast<const int32_t*>(p.plan), B, H_q, H_kv);
+        if (e != cudaSuccess) return KV_ERR_CUDA;
+    } else if (planned || S > 1) {
         // one warp per row when a single round of 8 loads per lane covers the splits (and for
         // planned launches, where rows have different chunk counts), else 8 warps per row
         const int64_t rows = static_cast<int64_t>(B) * H_q;

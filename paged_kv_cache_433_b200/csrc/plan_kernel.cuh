@@ -170,6 +170,7 @@ __global__ void __launch_bounds__(kPlanThreads) paged_plan_kernel(const int32_t*
 // before (the CTA's first piece) -- and the combine kernel merges them. Rows
 // inside one CTA's range are written to the output directly.
 // G = min(grid, ceil(T / min_pages)) keeps at least `min_pages` per CTA.
+// Output rows of sequences without pages are zeroed here (no CTA visits them).
 //
 // Plan layout (int32 words): [0] kPlanStream, [1] G, [2], [3] T (int64),
 // [4 ..] S_b (int64, B + 1 entries: exclusive prefix of n_b), then cta_row[G]:
@@ -179,8 +180,11 @@ __global__ void __launch_bounds__(kPlanThreads) paged_plan_stream_kernel(const i
                                                                          int32_t B, int32_t H_kv, int32_t P,
                                                                          int32_t max_blocks, int32_t grid,
                                                                          int32_t min_pages, int32_t* __restrict__ plan,
-                                                                         int* err) {
+                                                                         float* __restrict__ out, int32_t H_q,
+                                                                         int32_t Dh, int* err) {
     __shared__ unsigned long long warp_sums[32];
+    __shared__ int empties[kPlanThreads];
+    __shared__ int n_empty;
     grid_dependency_wait();
     if (threadIdx.x == 0) grid_launch_dependents();
     const int tid = threadIdx.x;
@@ -209,6 +213,20 @@ __global__ void __launch_bounds__(kPlanThreads) paged_plan_stream_kernel(const i
         s[r] = carry + static_cast<long long>(ex);
         if (b < B) pre[b] = s[r];
         carry += static_cast<long long>(tot);
+    }
+    // sequences without pages (empty, or a length the table cannot hold): the decode kernel never visits
+    // their rows, so their output rows are zeroed here, one round of 1024 sequences at a time
+    const long long row_floats = static_cast<long long>(H_q) * Dh;
+    for (int r = 0; r < kPlanRowsPerThread && r * kPlanThreads < B; ++r) {
+        if (tid == 0) n_empty = 0;
+        __syncthreads();
+        const int b = tid + r * kPlanThreads;
+        if (b < B && n[r] == 0) empties[atomicAdd(&n_empty, 1)] = b;
+        __syncthreads();
+        const long long ne = n_empty;
+        for (long long i = tid; i < ne * row_floats; i += kPlanThreads)
+            out[static_cast<long long>(empties[i / row_floats]) * row_floats + i % row_floats] = 0.f;
+        __syncthreads();
     }
     const long long T = carry * H_kv;
     long long G = min_pages > 0 ? (T + min_pages - 1) / min_pages : T;
