@@ -371,13 +371,16 @@ int paged_decode_attention_fp8(float* out, const void* q, int32_t q_dtype, const
                                void* workspace, size_t ws_bytes, int* err_flag, void* stream);
 
 /* Which decode kernel paged_decode_attention uses (process-wide; default AUTO):
- *   KV_DECODE_KERNEL_AUTO  bf16/fp16 K/V with H_q / H_kv = 32 and Dh = 128
- *                          (MQA-shaped groups), no fused rotation: the
- *                          fifth-generation tensor-core kernel (tcgen05; the
- *                          128 tokens of a stage are the MMA rows, scores and
- *                          output accumulate in tensor memory; persistent, one
- *                          CTA per SM; with num_splits = 0 and B > 1 always
- *                          device-planned). Other bf16/fp16 shapes with
+ *   KV_DECODE_KERNEL_AUTO  bf16/fp16 K/V, Dh = 128, no fused rotation, and
+ *                          either H_q / H_kv = 32 (MQA-shaped groups) or
+ *                          H_q / H_kv in {4, 8, 16} with num_splits = 0 and
+ *                          B * H_kv above four per SM: the fifth-generation
+ *                          tensor-core kernel (tcgen05; the 128 tokens of a
+ *                          stage are the MMA rows, scores and output accumulate
+ *                          in tensor memory; persistent, one CTA per SM; with
+ *                          num_splits = 0 and B > 1 a device plan gives every
+ *                          CTA the same share of the batch's pages, each work
+ *                          item counted one stage extra). Other bf16/fp16 shapes with
  *                          H_q / H_kv <= 64: warp MMA on TMA-staged swizzled
  *                          tiles. fp32 K/V: CUDA cores (packed f32x2 FMA);
  *   KV_DECODE_KERNEL_SIMT  CUDA cores for every dtype (H_q / H_kv <= 32);

@@ -144,8 +144,8 @@ __global__ void __launch_bounds__(32 * kCombineWarps) paged_combine_kernel(
 
 // Combine of a balanced plan (paged_plan_stream_kernel): only rows cut by a
 // CTA boundary have partials, at most one per boundary, so CTA c of the grid
-// merges the row that starts in CTA c's page range and runs past its end (if
-// any): its first piece is in slot 2c + 1, piece s >= 1 in slot 2 (c + s).
+// merges the row whose real pages start in CTA c's range and run past its end
+// (if any): its first piece is in slot 2c + 1, piece s >= 1 in slot 2 (c + s).
 // One warp per head of the row's GQA group (g <= 32); lane s holds piece s's
 // (m, l) and weight, then every lane sums DH / 32 dims over the pieces with
 // all loads of a round issued before any is used. Rows inside one range were
@@ -164,19 +164,20 @@ __global__ void __launch_bounds__(32 * kCombineStreamWarps) paged_combine_stream
     if (threadIdx.x == 0) grid_launch_dependents();
     const int g = H_q / H_kv;
     if (h >= g) return;
-    const int G = plan[1];
+    const int G = plan_stream_G(plan), v = plan_stream_v(plan);
     const int c = blockIdx.x;
     if (c + 1 >= G) return;  // the last range ends the line
-    const long long T = static_cast<long long>(static_cast<uint32_t>(plan[2])) | (static_cast<long long>(plan[3]) << 32);
+    const long long T = plan_stream_T(plan);
     const int64_t* pre = plan_stream_prefix(plan);
     const long long lo = T * c / G, hi = T * (c + 1) / G;
-    // the row holding page hi: its sequence starts CTA c + 1's range
+    // the row whose span holds position hi: its sequence starts CTA c + 1's range
     const int b = plan[kPlanHdr + 2 * (B + 1) + c + 1];
-    const long long s0 = pre[b], n = pre[b + 1] - s0;
-    if (n <= 0) return;
-    const int kvh = static_cast<int>((hi - (long long)H_kv * s0) / n);
-    const long long r0 = (long long)H_kv * s0 + (long long)kvh * n;
-    if (r0 >= hi || r0 < lo) return;  // starts at the boundary (not cut) or in an earlier range
+    const long long s0 = pre[b], d = pre[b + 1] - s0;
+    if (d <= 0) return;
+    const int kvh = static_cast<int>((hi - (long long)H_kv * s0) / d);
+    const long long r0 = (long long)H_kv * s0 + (long long)kvh * d + v, n = d - v;  // the row's real pages
+    // cut at this boundary when its real pages start inside this range (they then run past hi)
+    if (r0 >= hi || r0 < lo) return;
     const int ns = plan_stream_cta(r0 + n - 1, T, G) - c + 1;
     auto slot = [&](int s) { return (s == 0 ? 2LL * c + 1 : 2LL * (c + s)) * g + h; };
     float acc[kD];

@@ -69,6 +69,7 @@ struct DecodeParams {
     const int32_t* q_start;     // multi-token query: rows of sequence b are q_start[b] .. q_start[b+1]-1
     int32_t q_tile;             // multi-token query: chunk tokens per CTA
     const int32_t* plan;        // planned launch: [0] pages per chunk, [4 + b] item prefix
+    int32_t stream_plan;        // 1: `plan` is the balanced plan of the persistent tcgen05 kernel
     int* err;
     int32_t max_blocks, B, H_q, H_kv, num_pages;
     int32_t g, HS, WP;          // GQA group, head slices, page-warps

@@ -69,7 +69,7 @@ struct TcCfg {
     static constexpr int kPB0 = kTP * kN * 2;    // one P^T tile (hi or lo)
     // ring entries (K or V of a stage) that fit beside two Q tiles, two P^T buffers (hi + lo each), the
     // work list (3 KB) and the small arrays
-    static constexpr int kRing0 = (227 * 1024 - 1024 - 2048 - 3104 - 2 * kBoxCols * kN * 128 - 4 * kPB0) / kEntry;
+    static constexpr int kRing0 = (227 * 1024 - 1024 - 2048 - 3120 - 2 * kBoxCols * kN * 128 - 4 * kPB0) / kEntry;
     static constexpr int kRing = kRing0 > 6 ? 6 : kRing0;
     // K of global stage J in entry J % kKSlots, V in kKSlots + J % kVSlots: a K entry is refilled as soon as
     // its QK has run, whatever the P.V of older stages
@@ -89,8 +89,8 @@ struct TcCfg {
     static constexpr int kOffMask = kOffFlag + 32;            // ints: skipped-page mask per K entry, per S^T buffer
     static constexpr int kOffStats = kOffMask + 32;           // 2 x [l, m][G] floats: an item's sums and maxima
     static constexpr int kOffList = kOffStats + 2 * 2 * G * 4;  // int4 x 2 per item
-    static constexpr int kOffStream = kOffList + kMaxList * 32;   // TcStream of a balanced plan (32 bytes)
-    static constexpr int kOffBar = kOffStream + 32;
+    static constexpr int kOffStream = kOffList + kMaxList * 32;   // TcStream of a balanced plan (48 bytes)
+    static constexpr int kOffBar = kOffStream + 48;
     // full[R], empty[R], q_full[2], q_empty[2], s_full[2], s_empty[2], p_full[2], p_empty[2], o_full[2],
     // o_empty[2], done (QK issuer), done (PV issuer), stats_full[2], stats_empty[2]
     static constexpr int kNumBars = 2 * kRing + 4 + 4 + 4 + 4 + 2 + 4 + 2;  // + mask_full[2]
@@ -113,60 +113,73 @@ struct TcCfg {
 
 struct TcWork {
     int b, kvh, split, item, first, n_local, len, n_pages;
+    int n_pieces;  // balanced plan: pieces of the row (CTAs split .. split + n_pieces - 1)
     bool split_mode, bad_len;
     bool planned;  // partial at slot `item` ([item][g][Dh]); else at (row, split) of the grid layout
 };
 
-// This CTA's share of a balanced plan (paged_plan_stream_kernel): pages [lo, hi) of the line of
-// (sequence, KV head) rows, the first of which, row0 = b * H_kv + kvh, holds page lo.
+// This CTA's share of a balanced plan (paged_plan_stream_kernel): positions [lo, hi) of the line of
+// (sequence, KV head) row spans, the first of which, row0 = b * H_kv + kvh, holds position lo; a row's
+// span is its v virtual pages (the fixed cost of a work item), then its real pages.
 struct TcStream {
-    long long lo, hi, row0;
-    int active;  // a balanced plan with pages for this CTA
+    long long lo, hi, row0, T;
+    int G, v;
+    int active;  // a balanced plan with positions for this CTA
     int pad;
 };
 
-__device__ __forceinline__ bool tc_is_stream(const DecodeParams& p) {
-    return p.items == nullptr && p.plan != nullptr && p.plan[0] == kPlanStream;
-}
+static_assert(sizeof(TcStream) == 48, "shared-memory slot of the stream range");
+
+// (a launch parameter: known before the plan kernel this one depends on has finished)
+__device__ __forceinline__ bool tc_is_stream(const DecodeParams& p) { return p.stream_plan != 0; }
 
 __device__ __forceinline__ TcStream tc_stream_range(const DecodeParams& p) {
-    TcStream r{0, 0, 0, 0, 0};
-    const int G = p.plan[1];
+    TcStream r{0, 0, 0, 0, 0, 0, 0, 0};
+    const int G = plan_stream_G(p.plan);
     const int c = blockIdx.x;
     if (c >= G) return r;
-    const long long T = static_cast<long long>(static_cast<uint32_t>(p.plan[2])) | (static_cast<long long>(p.plan[3]) << 32);
+    const long long T = plan_stream_T(p.plan);
     const int64_t* pre = plan_stream_prefix(p.plan);
     const int b0 = p.plan[kPlanHdr + 2 * (p.B + 1) + c];
+    r.T = T;
+    r.G = G;
+    r.v = plan_stream_v(p.plan);
     r.lo = T * c / G;
     r.hi = T * (c + 1) / G;
-    const long long s0 = pre[b0], n0 = pre[b0 + 1] - s0;
-    if (r.hi <= r.lo || n0 <= 0) return r;
-    r.row0 = static_cast<long long>(b0) * p.H_kv + (r.lo - p.H_kv * s0) / n0;
+    const long long s0 = pre[b0], d0 = pre[b0 + 1] - s0;
+    if (r.hi <= r.lo || d0 <= 0) return r;
+    r.row0 = static_cast<long long>(b0) * p.H_kv + (r.lo - p.H_kv * s0) / d0;
     r.active = 1;
     return r;
 }
 
-// Piece k of the CTA's range: row row0 + k cut to [lo, hi). 1: work, 0: an empty row, -1: past the range.
+// Piece k of the CTA's range: the real pages of row row0 + k inside [lo, hi). 1: work, 0: none (an empty
+// row, or only its virtual pages in range), -1: past the range. A row cut by a range boundary records its
+// first CTA (split) and its number of pieces.
 __device__ __forceinline__ int tc_stream_piece(const DecodeParams& p, const TcStream& st, int k, int P, TcWork& wk) {
     if (!st.active) return -1;
     const long long row = st.row0 + k;
     const int b = static_cast<int>(row / p.H_kv), kvh = static_cast<int>(row % p.H_kv);
     if (b >= p.B) return -1;
     const int64_t* pre = plan_stream_prefix(p.plan);
-    const long long s0 = pre[b], n = pre[b + 1] - s0;
-    const long long r0 = p.H_kv * s0 + kvh * n;
-    if (r0 >= st.hi) return -1;
+    const long long s0 = pre[b], d = pre[b + 1] - s0;
+    const long long rs = p.H_kv * s0 + kvh * d;  // the row's span
+    if (rs >= st.hi) return -1;
+    if (d <= 0) return 0;
+    const long long n = d - st.v, r0 = rs + st.v;  // its real pages
     const long long x0 = r0 > st.lo ? r0 : st.lo, x1 = r0 + n < st.hi ? r0 + n : st.hi;
     if (x1 <= x0) return 0;
     wk.b = b;
     wk.kvh = kvh;
-    wk.split = 0;
     wk.item = 2 * static_cast<int>(blockIdx.x) + (r0 >= st.lo ? 1 : 0);
     wk.first = static_cast<int>(x0 - r0);
     wk.n_local = static_cast<int>(x1 - x0);
     wk.len = p.seq_lens[b];
     wk.n_pages = static_cast<int>(n);
     wk.split_mode = !(x0 == r0 && x1 == r0 + n);
+    const int c0 = plan_stream_cta(r0, st.T, st.G);
+    wk.split = c0;
+    wk.n_pieces = plan_stream_cta(r0 + n - 1, st.T, st.G) - c0 + 1;
     wk.bad_len = false;  // the plan raised it and gave the row no pages
     wk.planned = true;
     return 1;
@@ -201,6 +214,7 @@ __device__ __forceinline__ bool tc_work(const DecodeParams& p, int w, int P, TcW
     k.n_local = chunked ? min(chunk_pages, k.n_pages - k.first) : k.n_pages;
     k.split_mode = p.items != nullptr ? k.n_pages > chunk_pages : p.num_splits > 1;
     k.planned = p.items != nullptr;
+    k.n_pieces = 0;
     return true;
 }
 
@@ -216,25 +230,25 @@ struct TcList {
     const TcStream* st;  // balanced plan: this CTA's range (shared memory), else nullptr
 };
 
-// list entry flags
+// list entry flags (bits 0-4; the row's number of pieces from bit 8)
 constexpr int kTcSplit = 1, kTcBad = 2, kTcWork = 4, kTcPlanned = 8, kTcEnd = 16;
 
 __device__ __forceinline__ void tc_list_put(int4* e, int k, const TcWork& wk, int flags) {
     e[2 * k] = make_int4(wk.b, wk.kvh, wk.split, wk.item);
     e[2 * k + 1] = make_int4(wk.first, wk.n_local, wk.len,
                              flags | (wk.split_mode ? kTcSplit : 0) | (wk.bad_len ? kTcBad : 0) |
-                                 (wk.planned ? kTcPlanned : 0));
+                                 (wk.planned ? kTcPlanned : 0) | (wk.n_pieces << 8));
 }
 
 // One warp: the stream range (balanced plan) and the first candidates, into shared memory.
 __device__ __forceinline__ void tc_list_build(const DecodeParams& p, int n_work, int P, int4* e, int max_list,
                                               TcStream* st_out, int lane) {
     const bool stream = tc_is_stream(p);
-    TcStream st{0, 0, 0, 0, 0};
+    TcStream st{0, 0, 0, 0, 0, 0, 0, 0};
     if (stream) st = tc_stream_range(p);  // the same loads in every lane
     if (lane == 0) *st_out = st;
     for (int k = lane; k < max_list; k += 32) {
-        TcWork wk{0, 0, 0, 0, 0, 0, 0, 0, false, false, false};
+        TcWork wk{0, 0, 0, 0, 0, 0, 0, 0, 0, false, false, false};
         int flags = 0;
         if (stream) {
             const int got = tc_stream_piece(p, st, k, P, wk);
@@ -257,6 +271,7 @@ __device__ __forceinline__ int tc_get(const DecodeParams& p, const TcList& L, in
         wk.b = a.x, wk.kvh = a.y, wk.split = a.z, wk.item = a.w;
         wk.first = c.x, wk.n_local = c.y, wk.len = c.z;
         wk.split_mode = (c.w & kTcSplit) != 0, wk.bad_len = (c.w & kTcBad) != 0, wk.planned = (c.w & kTcPlanned) != 0;
+        wk.n_pieces = c.w >> 8;
         wk.n_pages = (wk.len + P - 1) / P;
         return 1;
     }
@@ -384,9 +399,6 @@ __global__ void __launch_bounds__(384, 1)
         prefetch_tmap(&tmap_v);
         prefetch_tmap(&tmap_q);
     }
-    grid_dependency_wait();
-    if (threadIdx.x == 0) grid_launch_dependents();
-
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;
     unsigned char* smem = smem_raw + (sbase - raw);
@@ -459,7 +471,6 @@ __global__ void __launch_bounds__(384, 1)
     if (warp == 1) {
         tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), C::kTmemCols);
         tmem_relinquish();
-        tc_list_build(p, n_work, P, list_e, L.n_list, st_smem, lane);
     }
     if constexpr (G < N) {
         // Q rows G .. N-1 are MMA padding: zero once (the TMA box writes rows 0 .. G-1 only)
@@ -469,6 +480,11 @@ __global__ void __launch_bounds__(384, 1)
         }
         fence_proxy_async_smem();
     }
+    // the setup above touches only this CTA's shared and tensor memory, so it overlaps the kernel this
+    // one depends on (programmatic launch); everything below may read what that kernel wrote
+    grid_dependency_wait();
+    if (threadIdx.x == 0) grid_launch_dependents();
+    if (warp == 1) tc_list_build(p, n_work, P, list_e, L.n_list, st_smem, lane);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();

@@ -271,11 +271,19 @@ bool use_mma(int32_t dtype, int32_t g) {
 // GQA groups of 4, 8, 16 or 32 heads when selected explicitly; the automatic
 // selection takes it for groups of 32 (MQA-shaped), where the warp-MMA
 // kernel is bound by its per-page MMA work.
-bool tc_ok(int32_t dtype, int32_t g, int32_t Dh, bool rope) {
+// The automatic choice takes the tcgen05 kernel for 32-head groups (MQA-shaped), and for groups of 4, 8
+// and 16 when the balanced plan has many rows to even out (B H_kv above four per SM): there it beats the
+// warp-MMA kernel's grid split (8B-shaped GQA, B = 256: 0.98 vs 0.91 of the copy peak); with fewer rows
+// (B = 64) the two are level and the warp-MMA kernel, which needs no plan, is kept.
+bool tc_ok(int32_t dtype, int32_t g, int32_t Dh, bool rope, int32_t B, int32_t H_kv, int32_t num_splits) {
     const int kind = g_kernel_kind.load(std::memory_order_relaxed);
     if ((dtype != KV_DTYPE_BF16 && dtype != KV_DTYPE_F16) || Dh != 128 || rope) return false;
-    if (kind == KV_DECODE_KERNEL_TCGEN05) return g == 4 || g == 8 || g == 16 || g == 32;
-    return kind == KV_DECODE_KERNEL_AUTO && g == 32;
+    const bool shape = g == 4 || g == 8 || g == 16 || g == 32;
+    if (kind == KV_DECODE_KERNEL_TCGEN05) return shape;
+    if (kind != KV_DECODE_KERNEL_AUTO || !shape) return false;
+    if (g == 32) return true;
+    const int sms = sm_count();
+    return num_splits == 0 && B > 1 && sms > 0 && static_cast<int64_t>(B) * H_kv > 4LL * sms;
 }
 
 size_t workspace_for(int32_t B, int32_t H_q, int32_t Dh, int32_t S) {
@@ -444,7 +452,7 @@ int paged_decode_workspace_bytes(int32_t B, int32_t H_q, int32_t H_kv, int32_t D
     size_t need = workspace_for(B, H_q, Dh, S);
     // the pool dtype is not known here: cover the tcgen05 kernel's balanced plan (16-bit pools) and the
     // chunked plan of the warp-MMA kernel (the other dtypes) wherever either may be chosen
-    const bool tc = tc_ok(KV_DTYPE_BF16, H_q / H_kv, Dh, false) && H_q % H_kv == 0;
+    const bool tc = H_q % H_kv == 0 && tc_ok(KV_DTYPE_BF16, H_q / H_kv, Dh, false, B, H_kv, num_splits);
     if (tc && planned_tc(B, num_splits)) {
         const int sms = sm_count();
         if (sms <= 0) return KV_ERR_CUDA;
@@ -471,7 +479,7 @@ int paged_decode_launch_info(int32_t B, int32_t H_q, int32_t H_kv, int32_t Dh, i
     int rc = resolve_splits(B, H_kv, max_blocks, num_splits, &S, &C, elem_bytes(dtype));
     if (rc != KV_OK) return rc;
     const bool mma = use_mma(dtype, g);
-    const bool tc = mma && tc_ok(dtype, g, Dh, false);
+    const bool tc = mma && tc_ok(dtype, g, Dh, false, B, H_kv, num_splits);
     *kernel = tc ? KV_DECODE_KERNEL_TCGEN05 : (mma ? KV_DECODE_KERNEL_MMA : KV_DECODE_KERNEL_SIMT);
     *splits = (tc ? planned_tc(B, num_splits) : planned_ok(mma, B, H_q, H_kv, num_splits)) ? 0 : S;
     return KV_OK;
@@ -520,7 +528,7 @@ int decode_impl(float* out, const void* q, const void* k_new, const void* v_new,
     int32_t S, C;
     rc = resolve_splits(B, H_kv, max_blocks, num_splits, &S, &C, elem_bytes(dtype));
     if (rc != KV_OK) return rc;
-    const bool tc = mma && tc_ok(dtype, g, Dh, cos_sin != nullptr);
+    const bool tc = mma && tc_ok(dtype, g, Dh, cos_sin != nullptr, B, H_kv, num_splits);
     const bool planned = tc ? planned_tc(B, num_splits) : planned_ok(mma, B, H_q, H_kv, num_splits);
 
     DecodeParams p{};
@@ -564,13 +572,16 @@ int decode_impl(float* out, const void* q, const void* k_new, const void* v_new,
         char* w = static_cast<char*>(workspace);
         int32_t* plan = reinterpret_cast<int32_t*>(w + L.plan_off);
         p.plan = plan;
+        p.stream_plan = 1;
         p.items = nullptr;
         p.part_u = reinterpret_cast<float*>(w + L.u_off);
         p.part_ml = reinterpret_cast<float2*>(w + L.ml_off);
         p.num_splits = 0;
-        const int32_t min_pages = 2 * std::max<int32_t>(1, 128 / page_size);  // two stages of 128 keys
+        // at least two stages of 128 keys per CTA; a work item's fixed cost counted as one stage of pages
+        const int32_t stage_pages = std::max<int32_t>(1, 128 / page_size);
         e = launch_pdl(paged_plan_stream_kernel, dim3(1), dim3(kPlanThreads), 0, st, seq_lens, B, H_kv, page_size,
-                       max_blocks, static_cast<int32_t>(pgrid), min_pages, plan, out, H_q, Dh, err_flag);
+                       max_blocks, static_cast<int32_t>(pgrid), 2 * stage_pages, stage_pages, plan, out, H_q, Dh,
+                       err_flag);
         if (e != cudaSuccess) return KV_ERR_CUDA;
     } else if (planned) {
         pgrid = planned_grid(B, H_kv);

@@ -159,11 +159,14 @@ __global__ void __launch_bounds__(kPlanThreads) paged_plan_kernel(const int32_t*
 }
 
 // Balanced ("stream") plan for the persistent tcgen05 decode kernel. The
-// (sequence, KV head) rows are laid end to end in (b, kvh) order -- row
-// (b, kvh) holds pages [H_kv S_b + kvh n_b, + n_b) of a line of
-// T = H_kv sum_b n_b pages -- and CTA c of G takes the pages
-// [floor(c T / G), floor((c + 1) T / G)): every CTA streams the same number
-// of pages (+-1), whatever the length mix. A row cut by a CTA boundary is
+// (sequence, KV head) rows are laid end to end in (b, kvh) order, each
+// preceded by v virtual pages that stand for the fixed cost of a work item
+// (its Q tile, the first stage's maximum, the hand-over to the epilogue):
+// with D_b = n_b + v for a sequence with pages (0 without), row (b, kvh)
+// spans [H_kv S_b + kvh D_b, + D_b) of a line of T = H_kv sum_b D_b, its
+// real pages the last n_b of the span. CTA c of G takes the line positions
+// [floor(c T / G), floor((c + 1) T / G)): every CTA carries the same cost
+// (+-1 page), whatever the length mix. A row cut by a CTA boundary is
 // processed in pieces by consecutive CTAs; a piece leaves its (m, l, u)
 // partial in one of two slots of its CTA -- slot 2c + 1 when the row starts
 // inside the CTA's range (the CTA's last piece), slot 2c when it started
@@ -172,14 +175,15 @@ __global__ void __launch_bounds__(kPlanThreads) paged_plan_kernel(const int32_t*
 // G = min(grid, ceil(T / min_pages)) keeps at least `min_pages` per CTA.
 // Output rows of sequences without pages are zeroed here (no CTA visits them).
 //
-// Plan layout (int32 words): [0] kPlanStream, [1] G, [2], [3] T (int64),
-// [4 ..] S_b (int64, B + 1 entries: exclusive prefix of n_b), then cta_row[G]:
-// the sequence whose rows hold page floor(c T / G).
+// Plan layout (int32 words): [0] kPlanStream, [1] G | v << 16, [2], [3] T
+// (int64), [4 ..] S_b (int64, B + 1 entries: exclusive prefix of D_b), then
+// cta_row[G]: the sequence whose rows' spans hold position floor(c T / G).
 
 __global__ void __launch_bounds__(kPlanThreads) paged_plan_stream_kernel(const int32_t* __restrict__ seq_lens,
                                                                          int32_t B, int32_t H_kv, int32_t P,
                                                                          int32_t max_blocks, int32_t grid,
-                                                                         int32_t min_pages, int32_t* __restrict__ plan,
+                                                                         int32_t min_pages, int32_t v,
+                                                                         int32_t* __restrict__ plan,
                                                                          float* __restrict__ out, int32_t H_q,
                                                                          int32_t Dh, int* err) {
     __shared__ unsigned long long warp_sums[32];
@@ -190,7 +194,8 @@ __global__ void __launch_bounds__(kPlanThreads) paged_plan_stream_kernel(const i
     const int tid = threadIdx.x;
     int64_t* pre = plan_stream_prefix(plan);
     int32_t* cta_row = plan + kPlanHdr + 2 * (B + 1);
-    // rows tid, tid + 1024, ...: page counts and their exclusive prefix in registers
+    // rows tid, tid + 1024, ...: page counts, spans D_b = n_b + v (0 without pages) and their exclusive
+    // prefix in registers
     int n[kPlanRowsPerThread];
     long long s[kPlanRowsPerThread];
     long long carry = 0;
@@ -209,7 +214,8 @@ __global__ void __launch_bounds__(kPlanThreads) paged_plan_stream_kernel(const i
             n[r] = (len + P - 1) / P;
         }
         unsigned long long tot;
-        const unsigned long long ex = block_exclusive_scan(static_cast<unsigned long long>(n[r]), warp_sums, tot);
+        const long long span = n[r] > 0 ? n[r] + v : 0;
+        const unsigned long long ex = block_exclusive_scan(static_cast<unsigned long long>(span), warp_sums, tot);
         s[r] = carry + static_cast<long long>(ex);
         if (b < B) pre[b] = s[r];
         carry += static_cast<long long>(tot);
@@ -233,19 +239,19 @@ __global__ void __launch_bounds__(kPlanThreads) paged_plan_stream_kernel(const i
     if (G > grid) G = grid;
     if (tid == 0) {
         plan[0] = kPlanStream;
-        plan[1] = static_cast<int32_t>(G);
+        plan[1] = static_cast<int32_t>(G | (static_cast<long long>(v) << 16));
         plan[2] = static_cast<int32_t>(T & 0xffffffffLL);
         plan[3] = static_cast<int32_t>(T >> 32);
         pre[B] = carry;
     }
     if (G <= 0) return;
     // CTA c starts in the rows of sequence b when floor(c T / G) lies in [H_kv S_b, H_kv S_{b+1}), i.e.
-    // c in [ceil(H_kv S_b G / T), ceil(H_kv S_{b+1} G / T)); empty sequences own no CTA
+    // c in [ceil(H_kv S_b G / T), ceil(H_kv S_{b+1} G / T)); sequences without pages span nothing
 #pragma unroll
     for (int r = 0; r < kPlanRowsPerThread; ++r) {
         const int b = tid + r * kPlanThreads;
         if (b >= B || n[r] == 0) continue;
-        const long long a0 = s[r] * H_kv, a1 = (s[r] + n[r]) * H_kv;
+        const long long a0 = s[r] * H_kv, a1 = (s[r] + n[r] + v) * H_kv;
         const long long c0 = (a0 * G + T - 1) / T, c1 = (a1 * G + T - 1) / T;
         for (long long c = c0; c < c1; ++c) cta_row[c] = b;
     }

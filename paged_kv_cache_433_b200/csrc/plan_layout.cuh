@@ -8,9 +8,17 @@ namespace kvp {
 
 constexpr int kPlanHdr = 4;  // header words before the per-sequence arrays
 
-// Balanced plan (paged_plan_stream_kernel): [0] kPlanStream, [1] G, [2], [3]
-// T (int64), [4 ..] S_b (int64, B + 1 entries), then cta_row[G].
+// Balanced plan (paged_plan_stream_kernel): [0] kPlanStream, [1] G | v << 16,
+// [2], [3] T (int64), [4 ..] S_b (int64, B + 1 entries), then cta_row[G].
 constexpr int32_t kPlanStream = -2;
+
+__host__ __device__ __forceinline__ int32_t plan_stream_G(const int32_t* plan) { return plan[1] & 0xffff; }
+__host__ __device__ __forceinline__ int32_t plan_stream_v(const int32_t* plan) {
+    return static_cast<int32_t>(static_cast<uint32_t>(plan[1]) >> 16);
+}
+__host__ __device__ __forceinline__ int64_t plan_stream_T(const int32_t* plan) {
+    return static_cast<int64_t>(static_cast<uint32_t>(plan[2])) | (static_cast<int64_t>(plan[3]) << 32);
+}
 
 __host__ __device__ __forceinline__ int64_t* plan_stream_prefix(int32_t* plan) {
     return reinterpret_cast<int64_t*>(plan + kPlanHdr);

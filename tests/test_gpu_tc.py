@@ -180,11 +180,14 @@ def test_tc_empty_rows_and_error_bits():
     assert int(err.item()) & K.KV_DEV_ERR_SEQ_LEN and torch.count_nonzero(out).item() == 0
 
 
-def test_auto_selection_takes_tc_for_32_head_groups():
+def test_auto_selection_takes_tc_for_32_head_groups_and_many_rows():
     K.paged_decode_set_kernel(K.KV_DECODE_KERNEL_AUTO)
     try:
         assert K.paged_decode_launch_info(256, 32, 1, 128, 1030, 16, "bf16", 0) == (0, K.KV_DECODE_KERNEL_TCGEN05)
         assert K.paged_decode_launch_info(64, 32, 8, 128, 270, 16, "bf16", 0)[1] == K.KV_DECODE_KERNEL_MMA
+        # many (sequence, KV head) rows: the balanced plan of the tcgen05 kernel
+        assert K.paged_decode_launch_info(256, 32, 8, 128, 1030, 16, "bf16", 0) == (0, K.KV_DECODE_KERNEL_TCGEN05)
+        assert K.paged_decode_launch_info(256, 32, 8, 128, 1030, 16, "bf16", 2)[1] == K.KV_DECODE_KERNEL_MMA
         assert K.paged_decode_launch_info(4, 32, 1, 64, 100, 16, "bf16", 0)[1] == K.KV_DECODE_KERNEL_MMA
         assert K.paged_decode_launch_info(4, 32, 1, 128, 100, 16, "fp32", 0)[1] == K.KV_DECODE_KERNEL_SIMT
     finally:
