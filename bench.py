@@ -63,7 +63,8 @@ def parse():
                     help="default run: do not add the 32K-context and mixed-sweep records to the config-2 line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
-    ap.add_argument("--no-graph", action="store_true", help="config 3: launch the 32 layers without a CUDA graph")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch without CUDA graphs (config 3's 32 layers; config 2's end-to-end steps)")
     ap.add_argument("--mixed-point", type=str, default=None,
                     help="config 5: run one point only, 'H_kv,page_size' (e.g. 1,16)")
     ap.add_argument("--page-size", type=int, choices=[16, 32], default=None,
@@ -662,10 +663,12 @@ def peaks_tensor():
 
 def run_e2e(wl, cfg, warm, steps, args, world):
     """Each step: one H2D copy of the step's inputs packed in a pinned staging buffer (q, k_new, v_new, slots,
-    lengths, and the block table when a page was added), kv_append + paged_decode_attention (fused by default),
+    lengths; the block table too when a page was added), kv_append + paged_decode_attention (fused by default),
     D2H of the fp32 output, wait for it. Steps are serial, as in a decode loop whose next input depends on this
     step's output; only the host slot bookkeeping of the next step (which does not depend on the output) is done
-    while the device runs this one."""
+    while the device runs this one. Unless --no-graph, each step's copies and launches are captured once as a
+    CUDA graph (as a serving loop captures its decode step) and replayed: the device then runs copy, kernels and
+    copy back to back instead of waiting on the host between them."""
     import torch
 
     K = wl.K
@@ -699,50 +702,76 @@ def run_e2e(wl, cfg, warm, steps, args, world):
     ws = wl.workspace()
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
+    graphs_on = not args.no_graph
 
     def prep(i):
-        """Host step a1 for step i, packed into its staging buffer; returns the bytes to copy."""
+        """Host step a1 for step i, packed into its staging buffer; True when the block table travels too."""
         before = wl.lens.copy()
         s, l = wl.bookkeeping()
         h = host_in[i].numpy()
         h[off_slots:off_slots + 8 * B] = s.view(np.uint8)
         h[off_lens:off_lens + 4 * B] = l.astype(np.int32).view(np.uint8)
-        if np.any(before % P == 0):  # a page was added: the block table travels too
+        if np.any(before % P == 0) or graphs_on:  # a page was added (or the graph copies the table anyway)
             h[off_tab:off_tab + tab_bytes] = wl.tab.view(np.uint8).reshape(-1)
-            return total
-        return off_tab
+            return True
+        return False
 
-    def one(i, nb):
-        d_in[:nb].copy_(host_in[i][:nb], non_blocking=True)
-        hot_path(K, args, cfg, wl.k_pages[0], wl.v_pages[0], d_kn, d_vn, d_slots, d_q, d_tab, d_lens, d_out, ws, err,
-                 stream)
-        host_out.copy_(d_out, non_blocking=True)
+    # the block table travels in the same copy whenever a page was added somewhere in the batch, which at
+    # B = 64 and P = 16 is nearly every step; the graphs copy it every step
+
+    def body(i, st, nb):
+        """Step i's copies (nb bytes of its staging buffer) and launches on stream st."""
+        with torch.cuda.stream(st):
+            d_in[:nb].copy_(host_in[i][:nb], non_blocking=True)
+            hot_path(K, args, cfg, wl.k_pages[0], wl.v_pages[0], d_kn, d_vn, d_slots, d_q, d_tab, d_lens, d_out, ws,
+                     err, st)
+            host_out.copy_(d_out, non_blocking=True)
+
+    graphs = None
+    if graphs_on:
+        # one graph per step (each reads its own staging buffer); the host bookkeeping is not in them
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        graphs = []
+        for i in range(n):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                body(i, torch.cuda.current_stream(), total)
+            graphs.append(g)
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+
+    def one(i, tab_too):
+        if graphs is not None:
+            graphs[i].replay()
+        else:
+            body(i, stream, total if tab_too else off_tab)
         nxt = prep(i + 1)  # overlaps the device work of step i
         stream.synchronize()
         return nxt
 
-    nb = prep(0)
+    tab_too = prep(0)
     for i in range(warm):
-        nb = one(i, nb)
+        tab_too = one(i, tab_too)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
     h2d = 0
     start.record(stream)
     for i in range(warm, n):
-        h2d += nb
-        nb = one(i, nb)
+        h2d += total if (tab_too or graphs is not None) else off_tab
+        tab_too = one(i, tab_too)
     end.record(stream)
     torch.cuda.synchronize()
     if int(err.item()) != 0:
         raise RuntimeError(f"device error flag {int(err.item())}")
     ms = max_over_ranks(start.elapsed_time(end), world)
+    del graphs
     return {"value": replica_value(B, steps, world, ms), "unit": UNIT, "h2d_bytes_per_step": h2d / steps,
             "d2h_bytes_per_step": host_out.numel() * 4, "ms_per_step": ms / steps,
-            "copies_declared": True}
+            "copies_declared": True, "cuda_graph": not args.no_graph}
 
 
-# ---------------------------------------------------------------------------- our arm: config 3
 def run_long_bench(args, world, rank, local):
     """One 32K-token sequence, 32 layers (fp16, 4 GiB cache): a step is 32 x (append + decode + combine),
     captured once as a CUDA graph that reads its inputs from one staging buffer and replayed every step."""
