@@ -281,12 +281,17 @@ int kv_copy_pages(void* k_pages, void* v_pages, const int32_t* src_pages, const 
  *   num_splits: 1 = single pass; >1 = split each sequence's pages into that
  *   many contiguous ranges (split-KV) merged by a second combine kernel;
  *   0 = choose automatically from B, H_kv, max_blocks and the SM count;
- *   for bf16/fp16 K/V on the tensor-core kernel with more (sequence, KV
- *   head) rows than 4 x the SM count (and B <= 8192), a planned launch is
- *   used instead: a one-CTA plan kernel reads seq_lens and cuts every row
- *   into chunks of C pages chosen from the actual lengths (full chunks at
- *   the front of the grid, short tail chunks at the back), then the decode
- *   and combine kernels follow that plan (three launches).
+ *   for bf16/fp16 K/V on the warp-MMA kernel with more (sequence, KV head)
+ *   rows than 4 x the SM count (and B <= 8192), a planned launch is used
+ *   instead: a one-CTA plan kernel reads seq_lens and cuts every row into
+ *   chunks of C pages chosen from the actual lengths (full chunks at the
+ *   front of the grid, short tail chunks at the back), then the decode and
+ *   combine kernels follow that plan (three launches). On the tcgen05 kernel
+ *   (see paged_decode_set_kernel) num_splits = 0 with B > 1 (B <= 8192) is
+ *   always planned: the plan kernel lays the rows end to end, each counted
+ *   with one stage (128 keys) of extra cost, and gives each of the SM-count
+ *   persistent CTAs an equal range; rows cut between two CTAs leave
+ *   partials that a combine kernel merges (one CTA per range boundary).
  *   workspace / ws_bytes: device scratch for split partials, at least
  *   paged_decode_workspace_bytes(...) for the same arguments (NULL/0 is fine
  *   when no split is used); KV_ERR_WORKSPACE if too small. Calls sharing one
