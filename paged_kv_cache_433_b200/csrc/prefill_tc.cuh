@@ -393,7 +393,7 @@ __global__ void __launch_bounds__(384, 1)
             }
             float mx = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < kH; ++c) mx = fmaxf(mx, s[c]);
+            for (int c = 0; c < kH; c += 2) mx = fmax3(mx, s[c], s[c + 1]);
             mx = fmaxf(mx, meet(mx, okl));
             if (!okl) {
                 ok = false;  // both halves of every row of this pair stop here
@@ -430,19 +430,23 @@ __global__ void __launch_bounds__(384, 1)
             // probabilities -> P over this S buffer: hi pairs in columns 0..63, residual pairs in 64..127
             // (this thread's keys: hi columns 32 half .., lo columns 64 + 32 half ..)
             const float neg = (m_ref == -INFINITY) ? 0.f : -m_ref;
+            const float2 sl2v = make_float2(sl2, sl2), negv = make_float2(neg, neg);
+            float2 lsum = make_float2(0.f, 0.f);
 #pragma unroll
             for (int q2 = 0; q2 < 2; ++q2) {
                 uint32_t hi[16], lo[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const float p0 = exp2f(fmaf(s[q2 * 32 + 2 * i], sl2, neg));  // exp2(-inf) = 0 for masked keys
-                    const float p1 = exp2f(fmaf(s[q2 * 32 + 2 * i + 1], sl2, neg));
-                    l += p0 + p1;
+                    // two keys at a time: one packed multiply-add for the exponents, one packed add for the sums
+                    const float2 x = ffma2(make_float2(s[q2 * 32 + 2 * i], s[q2 * 32 + 2 * i + 1]), sl2v, negv);
+                    const float p0 = exp2f(x.x), p1 = exp2f(x.y);  // exp2(-inf) = 0 for masked keys
+                    lsum = fadd2(lsum, make_float2(p0, p1));
                     pack2_split_fast<kBF16>(p0, p1, hi[i], lo[i]);
                 }
                 tmem_st16(tmem + (j % 3) * C::kTP + lane_addr + half * 32 + q2 * 16, hi);
                 tmem_st16(tmem + (j % 3) * C::kTP + lane_addr + C::kTP / 2 + half * 32 + q2 * 16, lo);
             }
+            l += lsum.x + lsum.y;
             tmem_wait_st();
             // a key no row may see (past the tile, or on a page not loaded) may hold stale bytes: zero its V row
             // (this thread: box column `half` of V row r) once the V entry has landed; only warps with such a

@@ -28,12 +28,41 @@ namespace kvp {
 // hi = x truncated to bf16 (x - hi is then exact in fp32), lo = that residual
 // truncated to bf16. hi + lo carries x to ~2^-14 relative. fp16 pairs use the
 // rounding conversions above.
+// max(a, b, c) in one instruction (three-input form, sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// a + b and a - b on two fp32 lanes at once
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
 template <bool IS_BF16>
 __device__ __forceinline__ void pack2_split_fast(float x0, float x1, uint32_t& hi, uint32_t& lo) {
     if constexpr (IS_BF16) {
-        const uint32_t h0 = __float_as_uint(x0) & 0xffff0000u, h1 = __float_as_uint(x1) & 0xffff0000u;
-        hi = __byte_perm(h0, h1, 0x7632);
-        lo = __byte_perm(__float_as_uint(x0 - __uint_as_float(h0)), __float_as_uint(x1 - __uint_as_float(h1)), 0x7632);
+        hi = __byte_perm(__float_as_uint(x0), __float_as_uint(x1), 0x7632);  // upper halves: truncated pair
+        const float2 h = make_float2(__uint_as_float(__float_as_uint(x0) & 0xffff0000u),
+                                     __uint_as_float(__float_as_uint(x1) & 0xffff0000u));
+        const float2 r = fsub2(make_float2(x0, x1), h);  // exact residuals
+        lo = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x7632);
     } else {
         pack2_split<false>(x0, x1, hi, lo);
     }
