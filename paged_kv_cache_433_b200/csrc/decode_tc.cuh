@@ -87,13 +87,15 @@ struct TcCfg {
     static constexpr int kOffFlag = kOffRed + 2 * G * 4 * 4;  // 2 x 4 ints
     static constexpr int kMaxList = 96;          // work items of a CTA resolved once into shared memory
     static constexpr int kOffMask = kOffFlag + 32;            // ints: skipped-page mask per K entry, per S^T buffer
-    static constexpr int kOffStats = kOffMask + 32;           // 2 x [l, m][G] floats: an item's sums and maxima
-    static constexpr int kOffList = kOffStats + 2 * 2 * G * 4;  // int4 x 2 per item
+    static constexpr int kOBuf = 4;              // items in flight between the softmax and the epilogue
+    static constexpr int kOffStats = kOffMask + 32;           // kOBuf x [l, m][G] floats: an item's sums, maxima
+    static constexpr int kOffList = kOffStats + kOBuf * 2 * G * 4;  // int4 x 2 per item
     static constexpr int kOffStream = kOffList + kMaxList * 32;   // TcStream of a balanced plan (48 bytes)
     static constexpr int kOffBar = kOffStream + 48;
-    // full[R], empty[R], q_full[2], q_empty[2], s_full[2], s_empty[2], p_full[2], p_empty[2], o_full[2],
-    // o_empty[2], done (QK issuer), done (PV issuer), stats_full[2], stats_empty[2]
-    static constexpr int kNumBars = 2 * kRing + 4 + 4 + 4 + 4 + 2 + 4 + 2;  // + mask_full[2]
+    // full[R], empty[R], q_full[2], q_empty[2], s_full[2], s_empty[2], p_full[2], p_empty[2], done (QK
+    // issuer), done (PV issuer), mask_full[2], o_full[kOBuf], o_empty[kOBuf], stats_full[kOBuf],
+    // stats_empty[kOBuf]
+    static constexpr int kNumBars = 2 * kRing + 4 + 8 + 2 + 2 + 4 * kOBuf;
     static constexpr int kOffTmem = kOffBar + 8 * kNumBars;
     static constexpr int kSmem = 1024 + kOffTmem + 16;
     static constexpr int kThreads = 384;         // three warpgroups
@@ -105,7 +107,8 @@ struct TcCfg {
     // G scores per thread) and 2 (epilogue): 128 x their sum must fit in the launch's 384 x (registers per
     // thread), which the host checks before the first launch
     static constexpr uint32_t kRegsLow = 64, kRegsSoftmax = 248, kRegsEpi = 136;
-    static constexpr uint32_t kTmemCols = 4 * kN <= 64 ? 64 : 128;  // S^T x 2 + O^T x 2, N columns each
+    // S^T x 2 + O^T x kOBuf, N columns each, rounded up to a power of two
+    static constexpr uint32_t kTmemCols = (2 + kOBuf) * kN <= 64 ? 64 : ((2 + kOBuf) * kN <= 128 ? 128 : 256);
     static_assert((G == 4 || G == 8 || G == 16 || G == 32) && DH == 128, "instances: g in {4, 8, 16, 32}, Dh = 128");
     static_assert(kPPS * kBoxCols <= 32, "one TMA box per lane");
     static_assert(kSmem <= 227 * 1024, "shared memory");
@@ -420,16 +423,19 @@ __global__ void __launch_bounds__(384, 1)
     // P^T is double-buffered (stage J in buffer J & 1): the softmax of stage J writes while P.V(J - 1) runs
     auto p_full = [&](int i) { return bs0 + 32u + 8u * i; };
     auto p_empty = [&](int i) { return bs0 + 48u + 8u * i; };
-    auto o_full = [&](int i) { return bs0 + 64u + 8u * i; };
-    auto o_empty = [&](int i) { return bs0 + 80u + 8u * i; };
-    const uint32_t done_qk = bs0 + 96u;
-    const uint32_t done_pv = bs0 + 104u;
-    // an item's row sums and reference maxima, softmax -> epilogue warps (double-buffered by item parity)
-    auto stats_full = [&](int i) { return bs0 + 112u + 8u * i; };
-    auto stats_empty = [&](int i) { return bs0 + 128u + 8u * i; };
+    const uint32_t done_qk = bs0 + 64u;
+    const uint32_t done_pv = bs0 + 72u;
     // the skipped-page mask of a stage travels producer -> K entry word -> QK issuer -> S^T buffer word, the
     // last hop announced on mask_full (the softmax needs it before the V entry lands)
-    auto mask_full = [&](int i) { return bs0 + 144u + 8u * i; };
+    auto mask_full = [&](int i) { return bs0 + 80u + 8u * i; };
+    // O^T and the item's row sums and reference maxima (softmax -> epilogue warps) rotate over kOBuf items,
+    // so a run of short items does not wait for the epilogue of the one before last
+    const uint32_t bo0 = bs0 + 96u;
+    auto o_full = [&](int i) { return bo0 + 8u * (i % C::kOBuf); };
+    auto o_empty = [&](int i) { return bo0 + 8u * (C::kOBuf + i % C::kOBuf); };
+    auto stats_full = [&](int i) { return bo0 + 8u * (2 * C::kOBuf + i % C::kOBuf); };
+    auto stats_empty = [&](int i) { return bo0 + 8u * (3 * C::kOBuf + i % C::kOBuf); };
+    auto oph = [](int i) { return static_cast<uint32_t>((i / C::kOBuf) & 1); };  // phase of item i's slot
     volatile int* kmask = reinterpret_cast<volatile int*>(smem + C::kOffMask);      // [kKSlots]
     volatile int* smask = reinterpret_cast<volatile int*>(smem + C::kOffMask + 16);  // [2]
     float* stats = reinterpret_cast<float*>(smem + C::kOffStats);
@@ -443,8 +449,12 @@ __global__ void __launch_bounds__(384, 1)
         for (int i = 0; i < 2; ++i) {
             mbar_init(q_full(i), 1);
             mbar_init(q_empty(i), 1);
+        }
+        for (int i = 0; i < C::kOBuf; ++i) {
             mbar_init(o_full(i), 1);
             mbar_init(o_empty(i), 4);
+            mbar_init(stats_full(i), 4);
+            mbar_init(stats_empty(i), 4);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(s_full(i), 1);
@@ -456,11 +466,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         mbar_init(done_qk, 1);
         mbar_init(done_pv, 1);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(stats_full(i), 4);
-            mbar_init(stats_empty(i), 4);
-            mbar_init(mask_full(i), 1);
-        }
+        for (int i = 0; i < 2; ++i) mbar_init(mask_full(i), 1);
         fence_barrier_init();
     }
     int4* list_e = reinterpret_cast<int4*>(smem + C::kOffList);
@@ -490,7 +496,7 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t tS = tmem;           // S^T buffers: columns [0, 2N)
-    auto tO = [&](int i) { return tmem + 2 * N + i * N; };  // O^T of item parity i: columns [2N + iN, 3N + iN)
+    auto tO = [&](int i) { return tmem + 2 * N + (i % C::kOBuf) * N; };  // O^T of item i
     const uint32_t ring = sbase;
     auto sQ = [&](int i) { return sbase + C::kOffQ + i * C::kQB; };
     // P^T buffer b: hi tile at sP + 2b kPB, residual lo tile right after it
@@ -634,26 +640,26 @@ __global__ void __launch_bounds__(384, 1)
                         const int e = vslot(J);
                         if (!wait(full(e), vphase(J))) break;
                         if (!wait(p_full(J & 1), (J >> 1) & 1)) break;
-                        if (j == 0 && item_i > 1 && !wait(o_empty(item_i & 1), ((item_i >> 1) - 1) & 1)) break;
+                        if (j == 0 && item_i >= C::kOBuf && !wait(o_empty(item_i), oph(item_i) ^ 1u)) break;
                         tc_fence_after();
                         const uint32_t sV = ring + e * C::kEntry;
 #pragma unroll
                         for (int kk = 0; kk < C::kTP / 16; ++kk) {
                             const uint64_t a = smem_desc(sV + kk * 16 * 128, C::kBoxB, 1024, kSwz128);
-                            umma_ss(tO(item_i & 1), a, smem_desc(sPhi(J) + kk * 16 * C::kPRow, C::kPB, C::kPAtom, C::kPSwz),
+                            umma_ss(tO(item_i), a, smem_desc(sPhi(J) + kk * 16 * C::kPRow, C::kPB, C::kPAtom, C::kPSwz),
                                     kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
                         }
 #pragma unroll
                         for (int kk = 0; kk < C::kTP / 16; ++kk) {
                             const uint64_t a = smem_desc(sV + kk * 16 * 128, C::kBoxB, 1024, kSwz128);
-                            umma_ss(tO(item_i & 1), a,
+                            umma_ss(tO(item_i), a,
                                     smem_desc(sPhi(J) + C::kPB + kk * 16 * C::kPRow, C::kPB, C::kPAtom, C::kPSwz),
                                     kIdescPV, 1u);
                         }
                         umma_commit(empty(e));
                         umma_commit(p_empty(J & 1));
                     }
-                    if (ok) umma_commit(o_full(item_i & 1));
+                    if (ok) umma_commit(o_full(item_i));
                 }
                 ++item_i;
             }
@@ -770,11 +776,11 @@ __global__ void __launch_bounds__(384, 1)
                 if (rescale_o) {
                     tc_fence_after();
                     uint32_t a[N];
-                    tmem_ld_cols<N>(tO(item_i & 1) + lane_addr, a);
+                    tmem_ld_cols<N>(tO(item_i) + lane_addr, a);
                     tmem_wait_ld();
 #pragma unroll
                     for (int h = 0; h < G; ++h) a[h] = __float_as_uint(__uint_as_float(a[h]) * alpha[h]);
-                    tmem_st_cols<N>(tO(item_i & 1) + lane_addr, a);
+                    tmem_st_cols<N>(tO(item_i) + lane_addr, a);
                     tmem_wait_st();
                 }
                 // probabilities -> P^T row r (hi and residual lo; padding heads are zero), swizzled rows
@@ -824,18 +830,18 @@ __global__ void __launch_bounds__(384, 1)
             // ---- hand the item to the epilogue warps: row sums over the CTA and the reference maxima
             cta_heads_reduce<G, false>(lp, red, sw, lane, rbuf);
             bool oks = ok;
-            if (item_i >= 2) wait(oks, stats_empty(item_i & 1), ((item_i >> 1) - 1) & 1);
+            if (item_i >= C::kOBuf) wait(oks, stats_empty(item_i), oph(item_i) ^ 1u);
             if (exchange(oks ? 0 : 2) & 2) {
                 ok = false;
                 continue;
             }
             if (r == 0) {
-                float* stl = stats + (item_i & 1) * 2 * G;
+                float* stl = stats + (item_i % C::kOBuf) * 2 * G;
 #pragma unroll
                 for (int h = 0; h < G; ++h) stl[h] = lp[h], stl[G + h] = m_ref[h];
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(stats_full(item_i & 1));
+            if (lane == 0) mbar_arrive(stats_full(item_i));
             ++item_i;
         }
     } else {
@@ -872,8 +878,8 @@ __global__ void __launch_bounds__(384, 1)
                 continue;
             }
             bool okl = ok;
-            wait(okl, stats_full(item_i & 1), (item_i >> 1) & 1);
-            wait(okl, o_full(item_i & 1), (item_i >> 1) & 1);
+            wait(okl, stats_full(item_i), oph(item_i));
+            wait(okl, o_full(item_i), oph(item_i));
             if (!okl) {
                 ok = false;  // an earlier stage failed: this and the later rows are zeroed
                 zero_rows(wk);
@@ -883,22 +889,22 @@ __global__ void __launch_bounds__(384, 1)
             float o[G];
             {
                 uint32_t a[N];
-                tmem_ld_cols<N>(tO(item_i & 1) + lane_addr, a);
+                tmem_ld_cols<N>(tO(item_i) + lane_addr, a);
                 tmem_wait_ld();
 #pragma unroll
                 for (int h = 0; h < G; ++h) o[h] = __uint_as_float(a[h]);
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(o_empty(item_i & 1));
+            if (lane == 0) mbar_arrive(o_empty(item_i));
             float l[G], m[G];
             {
-                const float* stl = stats + (item_i & 1) * 2 * G;
+                const float* stl = stats + (item_i % C::kOBuf) * 2 * G;
 #pragma unroll
                 for (int h = 0; h < G; ++h) l[h] = stl[h], m[h] = stl[G + h];
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(stats_empty(item_i & 1));
+            if (lane == 0) mbar_arrive(stats_empty(item_i));
             ++item_i;
             const int64_t hq0 = (int64_t)wk.b * p.H_q + (int64_t)wk.kvh * G;
             if (!wk.split_mode) {
