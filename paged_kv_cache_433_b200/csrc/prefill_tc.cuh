@@ -70,8 +70,8 @@ struct PfCfg {
     static constexpr int kOffQ = kRing * kEntry;
     static constexpr int kOffX = kOffQ + kQB;   // row exchange: [2][2][128] floats + ints
     static constexpr int kOffBar = kOffX + 2 * 2 * 128 * 4 * 2;
-    // full[R], empty[R], q_full, s_full[3], p_full[2], p_empty[3], o_full, done (QK), done (PV)
-    static constexpr int kNumBars = 2 * kRing + 1 + 3 + 2 + 3 + 3;
+    // full[R], empty[R], q_full, s_full[3], p_full[3], p_empty[3], o_full, done (QK), done (PV)
+    static constexpr int kNumBars = 2 * kRing + 1 + 3 + 3 + 3 + 3;
     static constexpr int kOffTmem = kOffBar + 8 * kNumBars;
     static constexpr int kSmem = 1024 + kOffTmem + 16;
     static constexpr int kThreads = 384;
@@ -143,14 +143,17 @@ __global__ void __launch_bounds__(384, 1)
     auto vphase = [](int j) { return static_cast<uint32_t>((j / C::kVSlots) & 1); };
     const uint32_t q_full = bar0 + 8u * (2 * C::kRing);
     auto s_full = [&](int i) { return q_full + 8u + 8u * i; };
-    // P of stage j is announced on p_full(j & 1): the softmax of stage j + 1 may finish before the MMA
-    // thread has waited for stage j, so one barrier would run a whole phase ahead of its waiter
+    // P of stage j is announced on p_full(j % 3) by all eight softmax warps. The warps of different lane
+    // quarters do not wait for one another, and none waits for V, so one may arrive for stage j + 2 while
+    // another is still writing P(j): with two barriers that early arrival would complete stage j's phase.
+    // Stage j + 3 needs S(j + 3), hence QK(j + 3), hence P.V(j) done, hence every stage-j arrival: three
+    // barriers keep each phase's arrivals to its own stage.
     auto p_full = [&](int i) { return q_full + 32u + 8u * i; };
     // P.V(j) completion is announced on p_empty(j % 3), the barrier of the S columns it read
-    auto p_empty = [&](int i) { return q_full + 48u + 8u * i; };
-    const uint32_t o_full = q_full + 72;
-    const uint32_t done_qk = q_full + 80;
-    const uint32_t done_pv = q_full + 88;
+    auto p_empty = [&](int i) { return q_full + 56u + 8u * i; };
+    const uint32_t o_full = q_full + 80;
+    const uint32_t done_qk = q_full + 88;
+    const uint32_t done_pv = q_full + 96;
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::kOffTmem);
 
     if (threadIdx.x == 0) {
@@ -160,8 +163,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         mbar_init(q_full, C::kSoftmaxWarps);
         for (int i = 0; i < 3; ++i) mbar_init(s_full(i), 1);
-        mbar_init(p_full(0), C::kSoftmaxWarps);
-        mbar_init(p_full(1), C::kSoftmaxWarps);
+        for (int i = 0; i < 3; ++i) mbar_init(p_full(i), C::kSoftmaxWarps);
         for (int i = 0; i < 3; ++i) mbar_init(p_empty(i), 1);
         mbar_init(o_full, 1);
         mbar_init(done_qk, 1);
@@ -278,7 +280,7 @@ __global__ void __launch_bounds__(384, 1)
                 for (int j = 0; j < n_st; ++j) {
                     const int e = vslot(j);
                     if (!wait(full(e), vphase(j))) break;
-                    if (!wait(p_full(j & 1), (j >> 1) & 1)) break;
+                    if (!wait(p_full(j % 3), (j / 3) & 1)) break;
                     tc_fence_after();
                     const uint32_t sV = ring + e * C::kEntry;
                     const uint32_t tP = tmem + (j % 3) * C::kTP;
@@ -455,6 +457,13 @@ __global__ void __launch_bounds__(384, 1)
                 const int pgi = r / P;
                 const bool stale = kbase + r >= key_end || pgi >= np || ((bad >> pgi) & 1);
                 if (__any_sync(0xffffffffu, stale)) {
+                    // the entry's previous fill (stage j - kVSlots) must have been consumed first: its P.V done
+                    // means that fill landed, so the wait below cannot pass on that older phase's parity
+                    const int jp = j - C::kVSlots;
+                    if (jp >= 0 && !wait(okl, p_empty(jp % 3), (jp / 3) & 1)) {
+                        ok = false;  // the next meeting stops the pair
+                        continue;
+                    }
                     if (!wait(okl, full(ev), vphase(j))) {
                         ok = false;  // the next meeting stops the pair
                         continue;
@@ -469,7 +478,7 @@ __global__ void __launch_bounds__(384, 1)
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full(j & 1));
+            if (lane == 0) mbar_arrive(p_full(j % 3));
         }
         // ---- epilogue: O row / l (this thread: dims 64 half .. 64 half + 63)
         bool okl = ok;

@@ -94,6 +94,29 @@ def test_prefill_chunk_longer_than_sequence_sets_error():
     check_close(got[:5], ref, "bf16", "valid chunk next to an invalid one")
 
 
+@pytest.mark.parametrize("H_q,H_kv", [(8, 8), (32, 8)])
+def test_prefill_repeated_launches_identical(H_q, H_kv):
+    """The same launch repeated 40 times over a pool whose unused rows hold NaN: every run gives the same bits,
+    and the first matches the oracle. The softmax warps may run stages ahead of the V stream; the stale V rows
+    past the chunk must still be zeroed in the right fill of their ring entry, or a NaN row reaches P.V."""
+    cfg = W.DecodeConfig(f"prefill-repeat-{H_q}-{H_kv}", "bf16", B=5, H_q=H_q, H_kv=H_kv, Dh=128, page_size=16,
+                         seed=86)
+    totals = [700, 233, 95, 40, 1]
+    chunks = [100, 64, 95, 17, 1]
+    got, q, q_start, st, lens = _run(cfg, totals, chunks)
+    ref = R.paged_prefill(q, q_start, st.kp, st.vp, st.tab, lens, cfg.scale, "bf16")
+    check_close(got, ref, "bf16", cfg.name)
+    d_q = to_device(q, "bf16")
+    d_qs, d_tab, d_lens = torch.from_numpy(q_start).cuda(), torch.from_numpy(st.tab).cuda(), torch.from_numpy(lens).cuda()
+    out = torch.empty((int(q_start[-1]), H_q, 128), dtype=torch.float32, device="cuda")
+    first = torch.from_numpy(got).cuda()
+    for _ in range(40):
+        out.fill_(float("nan"))
+        K.paged_prefill_attention(out, d_q, d_qs, max(chunks), st.k_pages, st.v_pages, d_tab, d_lens, cfg.scale)
+        torch.cuda.synchronize()
+        assert torch.equal(out, first)
+
+
 def test_prefill_refuses_fp32():
     k = torch.zeros((2, 2, 16, 64), dtype=torch.float32, device="cuda")
     with pytest.raises(K.KvError):
