@@ -362,8 +362,12 @@ int kv_append_fp8(void* k_pages, void* v_pages, const void* k_new, const void* v
  *   K_t = code_t * k_scale[kv head], V_t = code_t * v_scale[kv head],
  * q of q_dtype (KV_DTYPE_BF16 or KV_DTYPE_F16; its values must lie within
  * fp16's range, +-65504, as the products run on the tensor cores in fp16 --
- * E4M3 values are exact in fp16). Tensor-core kernel only (H_q / H_kv <= 64,
- * Dh in {64, 128}, page_size in {16, 32}); num_splits, workspace (same size
+ * E4M3 values are exact in fp16). Tensor-core kernels only (H_q / H_kv <= 64,
+ * Dh in {64, 128}, page_size in {16, 32}): the warp-MMA kernel, or, when
+ * KV_DECODE_KERNEL_TCGEN05 is selected and H_q / H_kv is 4, 8 or 16 with
+ * Dh = 128, the tcgen05 kernel, which widens each stage's pages to fp16 on the
+ * SM (K into tensor memory, V into shared memory) and keeps the probabilities
+ * as one fp16 operand; num_splits, workspace (same size
  * as paged_decode_workspace_bytes), errors and output as
  * paged_decode_attention, except that the automatic split count
  * (num_splits = 0, B > 1) aims at half as many CTAs per SM, each moving half
@@ -391,9 +395,10 @@ int paged_decode_attention_fp8(float* out, const void* q, int32_t q_dtype, const
  *   KV_DECODE_KERNEL_SIMT  CUDA cores for every dtype (H_q / H_kv <= 32);
  *   KV_DECODE_KERNEL_MMA   warp MMA for every bf16/fp16 shape (never the
  *                          tcgen05 kernel; fp32 K/V still use CUDA cores);
- *   KV_DECODE_KERNEL_TCGEN05  the tcgen05 kernel wherever it applies: bf16/fp16
+ *   KV_DECODE_KERNEL_TCGEN05  the tcgen05 kernels wherever they apply: bf16/fp16
  *                          K/V, Dh = 128, H_q / H_kv in {4, 8, 16, 32}, no
- *                          fused rotation (else as AUTO).
+ *                          fused rotation; E4M3 K/V, Dh = 128, H_q / H_kv in
+ *                          {4, 8, 16} (else as AUTO).
  * All kernels compute the same function; this exists to compare them.
  * KV_ERR_ARG for an unknown kind. The multi-token query
  * (paged_prefill_attention) takes its tcgen05 kernel under AUTO and TCGEN05

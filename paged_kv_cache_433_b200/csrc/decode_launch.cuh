@@ -149,6 +149,10 @@ cudaError_t launch_tc(const DecodeParams& p, const CUtensorMap& tk, const CUtens
 // tcgen05 multi-token query kernel (prefill_tc.cu): Dh = 128, 128 % g == 0, bf16 / fp16 K/V.
 cudaError_t launch_prefill_tc(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int dtype, int P,
                               dim3 grid, cudaStream_t st);
+// tcgen05 kernel over E4M3 K/V (decode_tc_fp8.cu): g in {4, 8, 16}, Dh = 128, q of type q_dtype (bf16 or
+// fp16); n_work items over `grid` persistent CTAs.
+cudaError_t launch_tc_fp8(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int q_dtype, int P,
+                          int n_work, int grid, cudaStream_t st);
 // E4M3 K/V with q of type q_dtype (bf16 or fp16).
 cudaError_t launch_mma_fp8(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int q_dtype, int DH,
                            int P, dim3 grid, cudaStream_t st);

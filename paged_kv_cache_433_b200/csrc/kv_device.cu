@@ -275,8 +275,13 @@ bool use_mma(int32_t dtype, int32_t g) {
 // and 16 when the balanced plan has many rows to even out (B H_kv above four per SM): there it beats the
 // warp-MMA kernel's grid split (8B-shaped GQA, B = 256: 0.98 vs 0.91 of the copy peak); with fewer rows
 // (B = 64) the two are level and the warp-MMA kernel, which needs no plan, is kept.
+// E4M3 K/V (decode_tc_fp8.cuh: pages widened to fp16 on the SM) for groups of 4, 8 and 16 when selected
+// explicitly: its sixteen N = 16 MMAs per 128-token stage take ~0.8 us on the tensor pipe, longer than the
+// stage's 32 KB take from HBM, and the warp-MMA kernel stays faster (8B-shaped layer, B = 64: 68 vs 115 us).
 bool tc_ok(int32_t dtype, int32_t g, int32_t Dh, bool rope, int32_t B, int32_t H_kv, int32_t num_splits) {
     const int kind = g_kernel_kind.load(std::memory_order_relaxed);
+    if (dtype == KV_DTYPE_FP8_E4M3)
+        return kind == KV_DECODE_KERNEL_TCGEN05 && Dh == 128 && !rope && (g == 4 || g == 8 || g == 16);
     if ((dtype != KV_DTYPE_BF16 && dtype != KV_DTYPE_F16) || Dh != 128 || rope) return false;
     const bool shape = g == 4 || g == 8 || g == 16 || g == 32;
     if (kind == KV_DECODE_KERNEL_TCGEN05) return shape;
@@ -452,7 +457,8 @@ int paged_decode_workspace_bytes(int32_t B, int32_t H_q, int32_t H_kv, int32_t D
     size_t need = workspace_for(B, H_q, Dh, S);
     // the pool dtype is not known here: cover the tcgen05 kernel's balanced plan (16-bit pools) and the
     // chunked plan of the warp-MMA kernel (the other dtypes) wherever either may be chosen
-    const bool tc = H_q % H_kv == 0 && tc_ok(KV_DTYPE_BF16, H_q / H_kv, Dh, false, B, H_kv, num_splits);
+    const bool tc = H_q % H_kv == 0 && (tc_ok(KV_DTYPE_BF16, H_q / H_kv, Dh, false, B, H_kv, num_splits) ||
+                                        tc_ok(KV_DTYPE_FP8_E4M3, H_q / H_kv, Dh, false, B, H_kv, num_splits));
     if (tc && planned_tc(B, num_splits)) {
         const int sms = sm_count();
         if (sms <= 0) return KV_ERR_CUDA;
@@ -619,13 +625,17 @@ int decode_impl(float* out, const void* q, const void* k_new, const void* v_new,
         CUtensorMap tk, tv, tq;
         const int64_t rows = static_cast<int64_t>(num_pages) * H_kv * page_size;
         if (!make_pool_map(&tk, k_pages, dtype, rows, Dh, page_size) ||
-            !make_pool_map(&tv, v_pages, dtype, rows, Dh, page_size) ||
-            !make_q_map(&tq, q, dtype, static_cast<int64_t>(B) * H_q, Dh, g))
+            !make_pool_map(&tv, v_pages, dtype, rows, Dh, page_size))
             return KV_ERR_CUDA;
         const int64_t n_work = planned ? pgrid : static_cast<int64_t>(S) * H_kv * B;
         if (n_work > 0x7fffffffLL) return KV_ERR_UNSUPPORTED;
         const int tc_grid = static_cast<int>(std::min<int64_t>(n_work, sms_all));
-        e = launch_tc(p, tk, tv, tq, dtype, page_size, static_cast<int>(n_work), tc_grid, st);
+        if (dtype == KV_DTYPE_FP8_E4M3) {
+            e = launch_tc_fp8(p, tk, tv, q_dtype, page_size, static_cast<int>(n_work), tc_grid, st);
+        } else {
+            if (!make_q_map(&tq, q, dtype, static_cast<int64_t>(B) * H_q, Dh, g)) return KV_ERR_CUDA;
+            e = launch_tc(p, tk, tv, tq, dtype, page_size, static_cast<int>(n_work), tc_grid, st);
+        }
     } else if (mma) {
         CUtensorMap tk, tv;
         const int64_t rows = static_cast<int64_t>(num_pages) * H_kv * page_size;

@@ -29,7 +29,7 @@ STATUS_NAMES = {0: "OK", -1: "ARG", -2: "OOM", -3: "BAD_ID", -4: "DOUBLE_FREE", 
                 -7: "WORKSPACE", -8: "UNSUPPORTED"}
 
 KV_DTYPE_F32, KV_DTYPE_BF16, KV_DTYPE_F16, KV_DTYPE_FP8_E4M3 = 0, 1, 2, 3
-DTYPE_CODE = {"fp32": 0, "bf16": 1, "fp16": 2}
+DTYPE_CODE = {"fp32": 0, "bf16": 1, "fp16": 2, "e4m3": 3}  # K/V pool types (e4m3: launch queries only)
 
 KV_DEV_ERR_PAGE_RANGE = 1
 KV_DEV_ERR_SEQ_LEN = 2

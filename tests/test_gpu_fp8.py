@@ -158,6 +158,47 @@ def test_fp8_decode_against_oracle(q_dtype, Dh, P, H_q, H_kv, B, kind, splits):
     c.check_codes()
 
 
+TC_FP8_SHAPES = [
+    # q dtype, P, H_q, H_kv, B, lengths (g = 4, 8 and 16; the edge lengths include an empty row)
+    ("bf16", 16, 32, 8, 8, "llama"), ("fp16", 32, 32, 8, 6, "edge"), ("bf16", 32, 16, 2, 5, "llama"),
+    ("fp16", 16, 16, 2, 7, "edge"), ("bf16", 16, 64, 4, 4, "edge"), ("fp16", 32, 48, 3, 3, "llama"),
+]
+
+
+@pytest.mark.parametrize("q_dtype,P,H_q,H_kv,B,kind", TC_FP8_SHAPES)
+@pytest.mark.parametrize("splits", [1, 3, 0])
+def test_fp8_tcgen05_against_oracle(q_dtype, P, H_q, H_kv, B, kind, splits):
+    """The tcgen05 kernel over E4M3 pages (widened to fp16 on the SM), forced for every split mode."""
+    cfg = W.DecodeConfig(f"fp8-tc-{q_dtype}-{P}-{H_q}-{H_kv}", q_dtype, B=B, H_q=H_q, H_kv=H_kv, Dh=128, page_size=P,
+                         seed=65)
+    c = Fp8Cache(cfg, _lengths(kind, B, P, 65))
+    K.paged_decode_set_kernel(K.KV_DECODE_KERNEL_TCGEN05)
+    try:
+        _, kern = K.paged_decode_launch_info(B, H_q, H_kv, 128, c.max_blocks, P, "e4m3", splits)
+        assert kern == K.KV_DECODE_KERNEL_TCGEN05
+        for step in range(2):
+            out, ref, err = c.step(step, num_splits=splits)
+            assert err == 0
+            check_close(out, ref, "bf16", f"{cfg.name} splits={splits} step {step}")
+    finally:
+        K.paged_decode_set_kernel(K.KV_DECODE_KERNEL_AUTO)
+    c.check_codes()
+
+
+def test_fp8_kernel_choice():
+    # under AUTO, E4M3 pools stay on the warp-MMA kernel; TCGEN05 selects the tcgen05 kernel for groups of
+    # 4 / 8 / 16 at Dh = 128 and leaves the other shapes on the warp-MMA kernel
+    assert K.paged_decode_launch_info(64, 32, 8, 128, 300, 16, "e4m3", 0)[1] == K.KV_DECODE_KERNEL_MMA
+    K.paged_decode_set_kernel(K.KV_DECODE_KERNEL_TCGEN05)
+    try:
+        assert K.paged_decode_launch_info(64, 32, 8, 128, 300, 16, "e4m3", 0) == (0, K.KV_DECODE_KERNEL_TCGEN05)
+        assert K.paged_decode_launch_info(64, 32, 8, 128, 300, 16, "e4m3", 2)[1] == K.KV_DECODE_KERNEL_TCGEN05
+        assert K.paged_decode_launch_info(64, 32, 1, 128, 300, 16, "e4m3", 0)[1] == K.KV_DECODE_KERNEL_MMA
+        assert K.paged_decode_launch_info(64, 16, 4, 64, 300, 16, "e4m3", 0)[1] == K.KV_DECODE_KERNEL_MMA
+    finally:
+        K.paged_decode_set_kernel(K.KV_DECODE_KERNEL_AUTO)
+
+
 def test_fp8_long_context_split_and_planned_many_rows():
     # one 32K-token sequence (auto splits), then a batch past the planned-launch row threshold
     cfg = W.DecodeConfig("fp8-long", "fp16", B=1, H_q=32, H_kv=8, Dh=128, page_size=16, seed=62)
