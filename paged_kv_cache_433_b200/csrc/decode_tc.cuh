@@ -76,14 +76,21 @@ struct TcCfg {
     static constexpr int kKSlots = (kRing + 1) / 2, kVSlots = kRing / 2;
     static constexpr int kQRowsB = kN * 128;     // one box column of the Q tile
     static constexpr int kQB = kBoxCols * kQRowsB;
-    static constexpr int kPRow = kN * 2;         // bytes of one P^T row (token)
-    static constexpr int kPB = kTP * kPRow;      // one P^T tile (hi or lo); equals kPB0
+    // At g = 32 the P^T of a stage is one tile whose token rows hold the N hi probabilities, then their N
+    // residuals: the P.V MMA has 2N columns and accumulates hi into O^T columns [0, N) and lo into [N, 2N)
+    // (summed in the epilogue), 8 MMAs a stage instead of 16 (the tensor pipe's cost per small MMA bounds
+    // the MQA stage). Smaller groups, bound by HBM, keep separate hi and lo tiles.
+    static constexpr bool kStackP = G == 32;
+    static constexpr int kPRow = kN * (kStackP ? 4 : 2);  // bytes of one P^T row (token)
+    static constexpr int kPB = kTP * kPRow;      // one P^T tile (stacked, or hi or lo)
+    static constexpr int kPTiles = kStackP ? 2 : 4;  // P^T tiles of the two stage buffers
+    static constexpr int kPVN = kStackP ? 2 * kN : kN;  // columns of the P.V MMA and of an item's O^T
     // P^T rows of 32 / 64 bytes: MN-major with the 32- / 64-byte swizzle; 8-row atoms
-    static constexpr uint32_t kPSwz = kPRow == 32 ? kSwz32 : kSwz64;
+    static constexpr uint32_t kPSwz = kPRow == 32 ? kSwz32 : (kPRow == 64 ? kSwz64 : kSwz128);
     static constexpr int kPAtom = 8 * kPRow;
     static constexpr int kOffQ = kRing * kEntry;
     static constexpr int kOffP = kOffQ + 2 * kQB;  // two Q tiles (item parity)
-    static constexpr int kOffRed = kOffP + 4 * kPB;          // 2 x [G][4] floats (after 2 x (hi, lo) P^T)
+    static constexpr int kOffRed = kOffP + kPTiles * kPB;    // 2 x [G][4] floats (after the P^T tiles)
     static constexpr int kOffFlag = kOffRed + 2 * G * 4 * 4;  // 2 x 4 ints
     static constexpr int kMaxList = 96;          // work items of a CTA resolved once into shared memory
     static constexpr int kOffMask = kOffFlag + 32;            // ints: skipped-page mask per K entry, per S^T buffer
@@ -108,7 +115,9 @@ struct TcCfg {
     // thread), which the host checks before the first launch
     static constexpr uint32_t kRegsLow = 64, kRegsSoftmax = 248, kRegsEpi = 136;
     // S^T x 2 + O^T x kOBuf, N columns each, rounded up to a power of two
-    static constexpr uint32_t kTmemCols = (2 + kOBuf) * kN <= 64 ? 64 : ((2 + kOBuf) * kN <= 128 ? 128 : 256);
+    // S^T x 2 (N columns each) + O^T x kOBuf (kPVN each), rounded up to a power of two
+    static constexpr int kTmemNeed = 2 * kN + kOBuf * kPVN;
+    static constexpr uint32_t kTmemCols = kTmemNeed <= 64 ? 64 : (kTmemNeed <= 128 ? 128 : (kTmemNeed <= 256 ? 256 : 512));
     static_assert((G == 4 || G == 8 || G == 16 || G == 32) && DH == 128, "instances: g in {4, 8, 16, 32}, Dh = 128");
     static_assert(kPPS * kBoxCols <= 32, "one TMA box per lane");
     static_assert(kSmem <= 227 * 1024, "shared memory");
@@ -392,7 +401,7 @@ __global__ void __launch_bounds__(384, 1)
     constexpr bool kBF16 = KT == KV_DTYPE_BF16;
     constexpr int N = C::kN;
     constexpr uint32_t kIdescQK = idesc_f16(kBF16, 128, N, false, false);
-    constexpr uint32_t kIdescPV = idesc_f16(kBF16, 128, N, true, true);
+    constexpr uint32_t kIdescPV = idesc_f16(kBF16, 128, C::kPVN, true, true);
     extern __shared__ __align__(1024) unsigned char smem_raw[];
 
     const int warp = threadIdx.x >> 5;
@@ -496,12 +505,12 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t tS = tmem;           // S^T buffers: columns [0, 2N)
-    auto tO = [&](int i) { return tmem + 2 * N + (i % C::kOBuf) * N; };  // O^T of item i
+    auto tO = [&](int i) { return tmem + 2 * N + (i % C::kOBuf) * C::kPVN; };  // O^T of item i
     const uint32_t ring = sbase;
     auto sQ = [&](int i) { return sbase + C::kOffQ + i * C::kQB; };
-    // P^T buffer b: hi tile at sP + 2b kPB, residual lo tile right after it
     const uint32_t sP = sbase + C::kOffP;
-    auto sPhi = [&](uint32_t j) { return sP + (j & 1) * 2 * C::kPB; };
+    // P^T of stage j: the stacked tile, or the hi tile with the lo tile right after it
+    auto sPt = [&](uint32_t j) { return sP + (j & 1) * (C::kPTiles / 2) * C::kPB; };
 
     // the register split sits at the top of each warpgroup's branch, so every code path after it is
     // compiled for its own budget
@@ -646,15 +655,17 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
                         for (int kk = 0; kk < C::kTP / 16; ++kk) {
                             const uint64_t a = smem_desc(sV + kk * 16 * 128, C::kBoxB, 1024, kSwz128);
-                            umma_ss(tO(item_i), a, smem_desc(sPhi(J) + kk * 16 * C::kPRow, C::kPB, C::kPAtom, C::kPSwz),
+                            umma_ss(tO(item_i), a, smem_desc(sPt(J) + kk * 16 * C::kPRow, C::kPB, C::kPAtom, C::kPSwz),
                                     kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
                         }
+                        if constexpr (!C::kStackP) {
 #pragma unroll
-                        for (int kk = 0; kk < C::kTP / 16; ++kk) {
-                            const uint64_t a = smem_desc(sV + kk * 16 * 128, C::kBoxB, 1024, kSwz128);
-                            umma_ss(tO(item_i), a,
-                                    smem_desc(sPhi(J) + C::kPB + kk * 16 * C::kPRow, C::kPB, C::kPAtom, C::kPSwz),
-                                    kIdescPV, 1u);
+                            for (int kk = 0; kk < C::kTP / 16; ++kk) {
+                                const uint64_t a = smem_desc(sV + kk * 16 * 128, C::kBoxB, 1024, kSwz128);
+                                umma_ss(tO(item_i), a,
+                                        smem_desc(sPt(J) + C::kPB + kk * 16 * C::kPRow, C::kPB, C::kPAtom, C::kPSwz),
+                                        kIdescPV, 1u);
+                            }
                         }
                         umma_commit(empty(e));
                         umma_commit(p_empty(J & 1));
@@ -775,12 +786,15 @@ __global__ void __launch_bounds__(384, 1)
                 }
                 if (rescale_o) {
                     tc_fence_after();
-                    uint32_t a[N];
-                    tmem_ld_cols<N>(tO(item_i) + lane_addr, a);
-                    tmem_wait_ld();
 #pragma unroll
-                    for (int h = 0; h < G; ++h) a[h] = __float_as_uint(__uint_as_float(a[h]) * alpha[h]);
-                    tmem_st_cols<N>(tO(item_i) + lane_addr, a);
+                    for (int hf = 0; hf < C::kPVN / N; ++hf) {  // (stacked: the hi and the residual parts)
+                        uint32_t a[N];
+                        tmem_ld_cols<N>(tO(item_i) + hf * N + lane_addr, a);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int h = 0; h < G; ++h) a[h] = __float_as_uint(__uint_as_float(a[h]) * alpha[h]);
+                        tmem_st_cols<N>(tO(item_i) + hf * N + lane_addr, a);
+                    }
                     tmem_wait_st();
                 }
                 // probabilities -> P^T row r (hi and residual lo; padding heads are zero), swizzled rows
@@ -799,11 +813,14 @@ __global__ void __launch_bounds__(384, 1)
                 }
 #pragma unroll
                 for (int c = 0; c < N / 8; ++c) {
-                    // 16-byte chunk c of the row, placed as the MN-major swizzle of rows of kPRow bytes expects
-                    const uint32_t phys = C::kPRow == 32 ? (c ^ ((r >> 2) & 1)) : (c ^ ((r >> 1) & 3));
-                    const uint32_t off = r * C::kPRow + (phys << 4);
-                    sts128(sPhi(J) + off, hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
-                    sts128(sPhi(J) + C::kPB + off, lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
+                    // 16-byte chunks of the row (stacked: c hi, c + N / 8 lo; else chunk c of each tile),
+                    // placed as the MN-major swizzle of rows of kPRow bytes expects
+                    const uint32_t sw = C::kPRow == 32 ? ((r >> 2) & 1) : (C::kPRow == 64 ? ((r >> 1) & 3) : (r & 7));
+                    const uint32_t row = sPt(J) + r * C::kPRow;
+                    const uint32_t lo_at = C::kStackP ? row + ((((uint32_t)c + N / 8) ^ sw) << 4)
+                                                      : row + C::kPB + (((uint32_t)c ^ sw) << 4);
+                    sts128(row + (((uint32_t)c ^ sw) << 4), hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
+                    sts128(lo_at, lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
                 }
                 // a masked token's V row may hold stale bytes (even NaN): zero it before P.V, once the V entry
                 // has landed (only warps with such a row wait for it; the P.V issuer waits for every entry)
@@ -890,9 +907,17 @@ __global__ void __launch_bounds__(384, 1)
             {
                 uint32_t a[N];
                 tmem_ld_cols<N>(tO(item_i) + lane_addr, a);
-                tmem_wait_ld();
+                if constexpr (C::kStackP) {
+                    uint32_t b2[N];
+                    tmem_ld_cols<N>(tO(item_i) + N + lane_addr, b2);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int h = 0; h < G; ++h) o[h] = __uint_as_float(a[h]);
+                    for (int h = 0; h < G; ++h) o[h] = __uint_as_float(a[h]) + __uint_as_float(b2[h]);
+                } else {
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int h = 0; h < G; ++h) o[h] = __uint_as_float(a[h]);
+                }
             }
             tc_fence_before();
             __syncwarp();
