@@ -28,6 +28,8 @@ cudaError_t launch_tc_inst(const DecodeParams& p, const CUtensorMap& tk, const C
         if (need > pool) return cudaErrorInvalidConfiguration;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
         configured.fetch_or(bit, std::memory_order_acq_rel);
     }
     return launch_pdl(kern, dim3(grid), dim3(C::kThreads), C::kSmem, st, p, tk, tv, tq, n_work);

@@ -169,6 +169,29 @@ int sm_count() {
     return v;
 }
 
+// The plan and combine kernels run between decode kernels that use most of shared memory: they ask for
+// the same L1 / shared-memory split, so an SM need not reconfigure between them (once per device).
+int keep_shared_carveout() {
+    static std::atomic<uint64_t> done{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (done.load(std::memory_order_acquire) & bit) return 0;
+    const int c = cudaSharedmemCarveoutMaxShared;
+    const auto a = cudaFuncAttributePreferredSharedMemoryCarveout;
+    cudaError_t e = cudaFuncSetAttribute(paged_plan_stream_kernel, a, c);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(paged_plan_kernel, a, c);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(paged_combine_stream_kernel<128>, a, c);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(paged_combine_stream_kernel<64>, a, c);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(paged_combine_kernel<128, 1>, a, c);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(paged_combine_kernel<128, kCombineWarps>, a, c);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(paged_combine_kernel<64, 1>, a, c);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(paged_combine_kernel<64, kCombineWarps>, a, c);
+    if (e != cudaSuccess) return -1;
+    done.fetch_or(bit, std::memory_order_acq_rel);
+    return 0;
+}
+
 // Heads per consumer warp and consumer warps per CTA for a GQA group of g.
 bool plan_group(int32_t g, int* GW, int* HS, int* NW, int* WP) {
     int gw = (g % 4 == 0) ? 4 : (g % 2 == 0) ? 2 : 1;
@@ -569,7 +592,7 @@ int decode_impl(float* out, const void* q, const void* k_new, const void* v_new,
     cudaError_t e;
     int64_t pgrid = 0;
     const int sms_all = sm_count();
-    if (sms_all <= 0) return KV_ERR_CUDA;
+    if (sms_all <= 0 || keep_shared_carveout() != 0) return KV_ERR_CUDA;
     if (planned && tc) {
         // balanced plan: one persistent CTA per SM, each streaming the same number of pages
         pgrid = sms_all;
