@@ -57,6 +57,9 @@ def parse():
     ap.add_argument("--chunk", type=int, default=512, help="config 8: chunk tokens per sequence")
     ap.add_argument("--splits", type=int, default=0, help="num_splits passed to paged_decode_attention (0 = auto)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-parts", type=int, default=1,
+                    help="end-to-end steps: the batch goes through in this many contiguous parts, the copies of one "
+                         "part overlapping the decode of another (1: copy in, decode, copy out, one after another)")
     ap.add_argument("--no-sustained", action="store_true",
                     help="skip the >= 1 s repeats (median of 5) that follow the timed steps")
     ap.add_argument("--no-extra", action="store_true",
@@ -662,73 +665,109 @@ def peaks_tensor():
 
 
 def run_e2e(wl, cfg, warm, steps, args, world):
-    """Each step: one H2D copy of the step's inputs packed in a pinned staging buffer (q, k_new, v_new, slots,
-    lengths; the block table too when a page was added), kv_append + paged_decode_attention (fused by default),
-    D2H of the fp32 output, wait for it. Steps are serial, as in a decode loop whose next input depends on this
-    step's output; only the host slot bookkeeping of the next step (which does not depend on the output) is done
-    while the device runs this one. Unless --no-graph, each step's copies and launches are captured once as a
-    CUDA graph (as a serving loop captures its decode step) and replayed: the device then runs copy, kernels and
-    copy back to back instead of waiting on the host between them."""
+    """Each step: the step's inputs (q, k_new, v_new, slots, lengths and the block table, packed in a pinned
+    staging buffer) copied to the device, kv_append + paged_decode_attention (fused by default), the fp32
+    output copied back, then a wait for it. Steps are serial, as in a decode loop whose next input depends on
+    this step's output; only the host slot bookkeeping of the next step (which does not depend on the output)
+    is done while the device runs this one. With --e2e-parts > 1 the batch goes through in that many
+    contiguous parts, each one call of the public entry point on its rows, on three streams: the copy of part
+    k + 1's inputs runs while part k is decoded, and the copy of part k's output while part k + 1 is (8B-shaped
+    layer, B = 64: 182.7 us a step with two parts, 183.9 with one, 217.8 with four -- the smaller decodes cost
+    what the overlapped copies save, so one part is the default). Unless
+    --no-graph, each step's copies and launches are captured once as a CUDA graph (as a serving loop captures
+    its decode step) and replayed."""
     import torch
 
     K = wl.K
-    B, P = wl.B, cfg.page_size
+    B = wl.B
     dev = torch.device("cuda")
     n = warm + steps
     eb = cfg.elem_bytes
-    nq, nkv = B * cfg.H_q * cfg.Dh * eb, B * cfg.H_kv * cfg.Dh * eb
-    off_q, off_kn, off_vn = 0, nq, nq + nkv
-    off_slots = nq + 2 * nkv
-    off_lens = off_slots + 8 * B
-    off_tab = (off_lens + 4 * B + 15) // 16 * 16
-    tab_bytes = wl.tab.nbytes
-    total = off_tab + tab_bytes
+    nparts = max(1, min(args.e2e_parts, B))
+    bounds = [B * k // nparts for k in range(nparts + 1)]
+    mb = wl.tab.shape[1]
+
+    def a16(x):
+        return (x + 15) // 16 * 16
+
+    # staging layout: part k's rows [b0, b1) as q, k_new, v_new, slots, lengths, block table, one contiguous
+    # range per part
+    parts = []
+    off = 0
+    for k in range(nparts):
+        b0, b1 = bounds[k], bounds[k + 1]
+        nb = b1 - b0
+        o = {"b0": b0, "b1": b1, "nb": nb, "start": off, "nq": nb * cfg.H_q * cfg.Dh * eb,
+             "nkv": nb * cfg.H_kv * cfg.Dh * eb}
+        for name, size in (("q", o["nq"]), ("kn", o["nkv"]), ("vn", o["nkv"]), ("slots", 8 * nb), ("lens", 4 * nb),
+                           ("tab", 4 * nb * mb)):
+            o[name] = off
+            off = a16(off + size)
+        o["end"] = off
+        parts.append(o)
+    total = off
     host_in = [torch.empty(total, dtype=torch.uint8).pin_memory() for _ in range(n + 1)]
     gen = torch.Generator().manual_seed(cfg.seed + 77)
     for i in range(n):  # step inputs prepared before timing (q, k_new, v_new as the model would produce them)
         h = host_in[i]
-        h[off_q:off_q + nq].view(wl.dt).copy_(torch.randn(nq // eb, generator=gen).to(wl.dt))
-        h[off_kn:off_kn + 2 * nkv].view(wl.dt).copy_(torch.randn(2 * nkv // eb, generator=gen).to(wl.dt))
+        for o in parts:
+            for name, size in (("q", o["nq"]), ("kn", o["nkv"]), ("vn", o["nkv"])):
+                h[o[name]:o[name] + size].view(wl.dt).copy_(torch.randn(size // eb, generator=gen).to(wl.dt))
     host_out = torch.empty((B, cfg.H_q, cfg.Dh), dtype=torch.float32).pin_memory()
     d_in = torch.empty(total, dtype=torch.uint8, device=dev)
-    d_q = d_in[off_q:off_q + nq].view(wl.dt).view(B, cfg.H_q, cfg.Dh)
-    d_kn = d_in[off_kn:off_kn + nkv].view(wl.dt).view(B, cfg.H_kv, cfg.Dh)
-    d_vn = d_in[off_vn:off_vn + nkv].view(wl.dt).view(B, cfg.H_kv, cfg.Dh)
-    d_slots = d_in[off_slots:off_slots + 8 * B].view(torch.int64)
-    d_lens = d_in[off_lens:off_lens + 4 * B].view(torch.int32)
-    d_tab = d_in[off_tab:off_tab + tab_bytes].view(torch.int32).view(wl.tab.shape)
-    d_tab.copy_(torch.from_numpy(wl.tab))
+    views = []
+    for o in parts:
+        nb = o["nb"]
+        v = {"q": d_in[o["q"]:o["q"] + o["nq"]].view(wl.dt).view(nb, cfg.H_q, cfg.Dh),
+             "kn": d_in[o["kn"]:o["kn"] + o["nkv"]].view(wl.dt).view(nb, cfg.H_kv, cfg.Dh),
+             "vn": d_in[o["vn"]:o["vn"] + o["nkv"]].view(wl.dt).view(nb, cfg.H_kv, cfg.Dh),
+             "slots": d_in[o["slots"]:o["slots"] + 8 * nb].view(torch.int64),
+             "lens": d_in[o["lens"]:o["lens"] + 4 * nb].view(torch.int32),
+             "tab": d_in[o["tab"]:o["tab"] + 4 * nb * mb].view(torch.int32).view(nb, mb)}
+        v["tab"].copy_(torch.from_numpy(wl.tab[o["b0"]:o["b1"]]))
+        views.append(v)
     d_out = torch.empty((B, cfg.H_q, cfg.Dh), dtype=torch.float32, device=dev)
-    ws = wl.workspace()
+    # one workspace serves every part: their launches are ordered on one stream
+    nws = max(K.paged_decode_workspace_bytes(o["nb"], cfg.H_q, cfg.H_kv, cfg.Dh, mb, cfg.page_size, wl.splits)
+              for o in parts)
+    ws = torch.zeros(max(nws, 16), dtype=torch.uint8, device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
-    graphs_on = not args.no_graph
+    copy_in, copy_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in parts]
+    ev_done = [torch.cuda.Event() for _ in parts]
 
     def prep(i):
-        """Host step a1 for step i, packed into its staging buffer; True when the block table travels too."""
-        before = wl.lens.copy()
+        """Host step a1 for step i (slots, lengths, block table), packed into its staging buffer."""
         s, l = wl.bookkeeping()
         h = host_in[i].numpy()
-        h[off_slots:off_slots + 8 * B] = s.view(np.uint8)
-        h[off_lens:off_lens + 4 * B] = l.astype(np.int32).view(np.uint8)
-        if np.any(before % P == 0) or graphs_on:  # a page was added (or the graph copies the table anyway)
-            h[off_tab:off_tab + tab_bytes] = wl.tab.view(np.uint8).reshape(-1)
-            return True
-        return False
+        for o in parts:
+            b0, b1, nb = o["b0"], o["b1"], o["nb"]
+            h[o["slots"]:o["slots"] + 8 * nb] = s[b0:b1].view(np.uint8)
+            h[o["lens"]:o["lens"] + 4 * nb] = l[b0:b1].astype(np.int32).view(np.uint8)
+            h[o["tab"]:o["tab"] + 4 * nb * mb] = np.ascontiguousarray(wl.tab[b0:b1]).view(np.uint8).reshape(-1)
 
-    # the block table travels in the same copy whenever a page was added somewhere in the batch, which at
-    # B = 64 and P = 16 is nearly every step; the graphs copy it every step
-
-    def body(i, st, nb):
-        """Step i's copies (nb bytes of its staging buffer) and launches on stream st."""
-        with torch.cuda.stream(st):
-            d_in[:nb].copy_(host_in[i][:nb], non_blocking=True)
-            hot_path(K, args, cfg, wl.k_pages[0], wl.v_pages[0], d_kn, d_vn, d_slots, d_q, d_tab, d_lens, d_out, ws,
-                     err, st)
-            host_out.copy_(d_out, non_blocking=True)
+    def body(i, st):
+        """Step i's copies and launches: forked from st onto the copy streams and joined back into it."""
+        copy_in.wait_stream(st)
+        copy_out.wait_stream(st)
+        with torch.cuda.stream(copy_in):
+            for k, o in enumerate(parts):
+                d_in[o["start"]:o["end"]].copy_(host_in[i][o["start"]:o["end"]], non_blocking=True)
+                ev_in[k].record(copy_in)
+        for k, (o, v) in enumerate(zip(parts, views)):
+            st.wait_event(ev_in[k])
+            hot_path(K, args, cfg, wl.k_pages[0], wl.v_pages[0], v["kn"], v["vn"], v["slots"], v["q"], v["tab"],
+                     v["lens"], d_out[o["b0"]:o["b1"]], ws, err, st)
+            ev_done[k].record(st)
+            copy_out.wait_event(ev_done[k])
+            with torch.cuda.stream(copy_out):
+                host_out[o["b0"]:o["b1"]].copy_(d_out[o["b0"]:o["b1"]], non_blocking=True)
+        st.wait_stream(copy_in)
+        st.wait_stream(copy_out)
 
     graphs = None
-    if graphs_on:
+    if not args.no_graph:
         # one graph per step (each reads its own staging buffer); the host bookkeeping is not in them
         side = torch.cuda.Stream()
         side.wait_stream(stream)
@@ -736,40 +775,39 @@ def run_e2e(wl, cfg, warm, steps, args, world):
         for i in range(n):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=side):
-                body(i, torch.cuda.current_stream(), total)
+                body(i, torch.cuda.current_stream())
             graphs.append(g)
         stream.wait_stream(side)
         torch.cuda.synchronize()
 
-    def one(i, tab_too):
+    def one(i):
         if graphs is not None:
             graphs[i].replay()
         else:
-            body(i, stream, total if tab_too else off_tab)
-        nxt = prep(i + 1)  # overlaps the device work of step i
+            body(i, stream)
+        prep(i + 1)  # overlaps the device work of step i
         stream.synchronize()
-        return nxt
 
-    tab_too = prep(0)
+    prep(0)
     for i in range(warm):
-        tab_too = one(i, tab_too)
+        one(i)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
-    h2d = 0
     start.record(stream)
     for i in range(warm, n):
-        h2d += total if (tab_too or graphs is not None) else off_tab
-        tab_too = one(i, tab_too)
+        one(i)
     end.record(stream)
     torch.cuda.synchronize()
     if int(err.item()) != 0:
         raise RuntimeError(f"device error flag {int(err.item())}")
     ms = max_over_ranks(start.elapsed_time(end), world)
     del graphs
-    return {"value": replica_value(B, steps, world, ms), "unit": UNIT, "h2d_bytes_per_step": h2d / steps,
+    return {"value": replica_value(B, steps, world, ms), "unit": UNIT, "h2d_bytes_per_step": float(total),
             "d2h_bytes_per_step": host_out.numel() * 4, "ms_per_step": ms / steps,
-            "copies_declared": True, "cuda_graph": not args.no_graph}
+            "copies_declared": True, "cuda_graph": not args.no_graph, "parts": nparts,
+            "path": f"pinned staging -> device in {nparts} part(s), one public call per part, output back per part "
+                    f"(copies of one part overlap the other part's decode), wait every step"}
 
 
 def run_long_bench(args, world, rank, local):
