@@ -224,7 +224,12 @@ int resolve_splits(int32_t B, int32_t H_kv, int32_t max_blocks, int32_t num_spli
         const int64_t rows = static_cast<int64_t>(B) * H_kv;
         const int64_t slots = 2LL * sms;
         if (B == 1) {
-            S = static_cast<int32_t>(slots / rows > 1 ? slots / rows : 1);
+            // one wave, with an eighth of the slots left free: launched early, the CTAs of the previous step's
+            // combine still hold registers on some SMs when this launch starts, and a split that filled every
+            // slot would send its last CTAs to a second wave (32K context, 32 layers: 878.7 us a step at S = 32,
+            // 906.4 at S = 37 = all slots)
+            const int64_t free_slots = slots - slots / 8;
+            S = static_cast<int32_t>(free_slots / rows > 1 ? free_slots / rows : 1);
         } else {
             const int64_t per_slot = kv_bytes == 1 ? 3 : 6;
             S = static_cast<int32_t>((per_slot * slots + rows - 1) / rows);
