@@ -16,10 +16,10 @@ namespace kvp {
 // CTAs of kCombineWarps warps; WPR warps per (sequence, query head) row, so
 // a CTA covers kCombineWarps / WPR rows (WPR = 1 for few splits, 8 for
 // many). The kernel is latency-bound, so every load of a round is issued
-// before any is used: each warp of a row holds up to kPer of its splits in
-// registers while the lanes also fetch all m_s for m*; then weights, sums,
-// and (WPR > 1) a shared-memory sum over the row's warps, all relative to the
-// same m*.
+// before any is used (in a grid split the first round goes out together with
+// the row's length): each warp of a row holds up to kPer of its splits in
+// registers and folds them in relative to its own maximum m_w; with WPR > 1
+// the row's warps then meet in shared memory, each scaled by 2^{m_w - m*}.
 constexpr int kCombineWarps = 8;
 
 // Planned launches (plan != nullptr, WPR == 1 only): the row's chunk size and
@@ -36,7 +36,7 @@ __global__ void __launch_bounds__(32 * kCombineWarps) paged_combine_kernel(
     constexpr int kRound = WPR * kPer;
     constexpr int kRows = kCombineWarps / WPR;
     __shared__ float red_u[kCombineWarps][DH];
-    __shared__ float red_l[kCombineWarps];
+    __shared__ float red_l[kCombineWarps], red_m[kCombineWarps];
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int rw = warp % WPR;  // warp within its row
@@ -44,35 +44,38 @@ __global__ void __launch_bounds__(32 * kCombineWarps) paged_combine_kernel(
     grid_dependency_wait();  // the decode kernel's partials
     if (threadIdx.x == 0) grid_launch_dependents();
     bool live = item < (int64_t)B * H_q;
-    int ns = 0;
+    // grid split: partial s of the row sits at (row, s) whatever the row's length, so the loads of the first
+    // round go out together with that of the length, and splits past the row's last page are masked after
+    int len = 0;
+    if (live) len = seq_lens[item / H_q];
+    int ns = plan != nullptr ? 0 : S;  // splits loaded; the row's own count is known once `len` has arrived
     int64_t base = item * S, stride = 1;
-    if (live) {
+    if (live && plan != nullptr) {
         const int b = static_cast<int>(item / H_q);
-        int len = seq_lens[b];
         if (len < 0 || len > max_blocks * P) len = 0;
         const int n_pages = (len + P - 1) / P;
-        if (plan != nullptr) {
-            const int C = plan[0];
-            const int items_b = (n_pages + C - 1) / C;
-            const int g = H_q / H_kv;
-            const int hq = static_cast<int>(item % H_q);
-            if (items_b == 1) live = false;  // the decode kernel wrote this row
-            ns = items_b > 1 ? items_b : 0;
-            const int64_t t0 = (int64_t)H_kv * plan[kPlanHdr + b] + (int64_t)(hq / g) * items_b;
-            base = t0 * g + hq % g;
-            stride = g;
-        } else {
-            ns = min(S, (n_pages + pages_per_split - 1) / pages_per_split);
-        }
+        const int C = plan[0];
+        const int items_b = (n_pages + C - 1) / C;
+        const int g = H_q / H_kv;
+        const int hq = static_cast<int>(item % H_q);
+        if (items_b == 1) live = false;  // the decode kernel wrote this row
+        ns = items_b > 1 ? items_b : 0;
+        const int64_t t0 = (int64_t)H_kv * plan[kPlanHdr + b] + (int64_t)(hq / g) * items_b;
+        base = t0 * g + hq % g;
+        stride = g;
     }
+    if (!live) ns = 0;
     const float2* ml = part_ml + base;
     const float* pu = part_u + base * DH + lane * kD;
 
+    // this warp's splits folded in with their own reference maximum m_w (moved per round as needed); the
+    // warps of a row then meet relative to the largest m_w
     float acc[kD];
 #pragma unroll
     for (int i = 0; i < kD; ++i) acc[i] = 0.f;
     float L = 0.f;
-    float mstar = -INFINITY;
+    float mw = -INFINITY;
+    int nrow = ns;  // the row's splits
     for (int r0 = 0; r0 < ns; r0 += kRound) {
         float2 st[kPer];
         float v[kPer][kD];
@@ -95,16 +98,29 @@ __global__ void __launch_bounds__(32 * kCombineWarps) paged_combine_kernel(
                 for (int i = 0; i < kD; ++i) v[j][i] = 0.f;
             }
         }
-        if (r0 == 0) {
-            for (int s = lane; s < ns; s += 32) mstar = fmaxf(mstar, ml[s * stride].x);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mstar = fmaxf(mstar, __shfl_xor_sync(0xffffffffu, mstar, o));
+        if (plan == nullptr && r0 == 0) {
+            if (len < 0 || len > max_blocks * P) len = 0;
+            const int n_pages = (len + P - 1) / P;
+            nrow = min(S, (n_pages + pages_per_split - 1) / pages_per_split);
         }
-        if (mstar != -INFINITY) {
+        float mr = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < kPer; ++j)
+            if (r0 + rw + j * WPR >= nrow) st[j].x = -INFINITY;  // a split with no pages of this row
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) mr = fmaxf(mr, st[j].x);
+        if (mr > mw) {
+            const float a = mw == -INFINITY ? 0.f : exp2f(mw - mr);
+            L *= a;
+#pragma unroll
+            for (int i = 0; i < kD; ++i) acc[i] *= a;
+            mw = mr;
+        }
+        if (mw != -INFINITY) {
 #pragma unroll
             for (int j = 0; j < kPer; ++j) {
                 if (st[j].x == -INFINITY) continue;
-                const float w = exp2f(st[j].x - mstar);
+                const float w = exp2f(st[j].x - mw);
                 L += w * st[j].y;
 #pragma unroll
                 for (int i = 0; i < kD; ++i) acc[i] += w * v[j][i];
@@ -125,17 +141,24 @@ __global__ void __launch_bounds__(32 * kCombineWarps) paged_combine_kernel(
     } else {
 #pragma unroll
         for (int i = 0; i < kD; ++i) red_u[warp][lane * kD + i] = acc[i];
-        if (lane == 0) red_l[warp] = L;
+        if (lane == 0) red_l[warp] = L, red_m[warp] = mw;
         __syncthreads();
         const int row_w0 = (warp / WPR) * WPR;
         if (live && rw == 0) {
-            for (int d = lane; d < DH; d += 32) {
-                float U = 0.f, Lt = 0.f;
+            float ms = -INFINITY;
 #pragma unroll
-                for (int w = 0; w < WPR; ++w) {
-                    U += red_u[row_w0 + w][d];
-                    Lt += red_l[row_w0 + w];
-                }
+            for (int w = 0; w < WPR; ++w) ms = fmaxf(ms, red_m[row_w0 + w]);
+            float sc[WPR];
+            float Lt = 0.f;
+#pragma unroll
+            for (int w = 0; w < WPR; ++w) {
+                sc[w] = red_m[row_w0 + w] == -INFINITY ? 0.f : exp2f(red_m[row_w0 + w] - ms);
+                Lt += sc[w] * red_l[row_w0 + w];
+            }
+            for (int d = lane; d < DH; d += 32) {
+                float U = 0.f;
+#pragma unroll
+                for (int w = 0; w < WPR; ++w) U += sc[w] * red_u[row_w0 + w][d];
                 out[item * DH + d] = (Lt > 0.f) ? U / Lt : 0.f;
             }
         }
