@@ -389,7 +389,8 @@ int paged_decode_attention_fp8(float* out, const void* q, int32_t q_dtype, const
  *                          in tensor memory; persistent, one CTA per SM; with
  *                          num_splits = 0 and B > 1 a device plan gives every
  *                          CTA the same share of the batch's pages, each work
- *                          item counted one stage extra). Other bf16/fp16 shapes with
+ *                          item counted one stage extra, three at g = 32).
+ *                          Other bf16/fp16 shapes with
  *                          H_q / H_kv <= 64: warp MMA on TMA-staged swizzled
  *                          tiles. fp32 K/V: CUDA cores (packed f32x2 FMA);
  *   KV_DECODE_KERNEL_SIMT  CUDA cores for every dtype (H_q / H_kv <= 32);

@@ -611,10 +611,13 @@ int decode_impl(float* out, const void* q, const void* k_new, const void* v_new,
         p.part_u = reinterpret_cast<float*>(w + L.u_off);
         p.part_ml = reinterpret_cast<float2*>(w + L.ml_off);
         p.num_splits = 0;
-        // at least two stages of 128 keys per CTA; a work item's fixed cost counted as one stage of pages
+        // at least two stages of 128 keys per CTA; a work item's fixed cost counted as one stage of pages, three
+        // at g = 32, whose items pay CTA-wide reductions over 32 heads (log-normal batch, B = 256: MQA 68.4 vs
+        // 72.2 us at P = 16, 69.2 vs 74.1 at P = 32; GQA best at one stage: 8B-shaped B = 64 108.0 vs 110.9 us)
         const int32_t stage_pages = std::max<int32_t>(1, 128 / page_size);
+        const int32_t item_pages = stage_pages * (H_q / H_kv >= 32 ? 3 : 1);
         e = launch_pdl(paged_plan_stream_kernel, dim3(1), dim3(kPlanThreads), 0, st, seq_lens, B, H_kv, page_size,
-                       max_blocks, static_cast<int32_t>(pgrid), 2 * stage_pages, stage_pages, plan, out, H_q, Dh,
+                       max_blocks, static_cast<int32_t>(pgrid), 2 * stage_pages, item_pages, plan, out, H_q, Dh,
                        err_flag);
         if (e != cudaSuccess) return KV_ERR_CUDA;
     } else if (planned) {
