@@ -243,3 +243,29 @@ def test_fp8_llama8b_full_size():
     out, ref, err = c.step(0)
     assert err == 0
     check_close(out, ref, "bf16", "fp8 8B full")
+
+
+def test_fp8_tcgen05_repeated_launches_identical():
+    """The tcgen05 E4M3 kernel repeated 30 times over a pool whose unused slots hold NaN codes: every launch
+    gives the bits of the first (converters, issuers and softmax warps meet on the right barrier phases)."""
+    cfg = W.DecodeConfig("fp8-tc-repeat", "bf16", B=12, H_q=32, H_kv=8, Dh=128, page_size=16, seed=66)
+    c = Fp8Cache(cfg, _lengths("llama", 12, 16, 66))
+    K.paged_decode_set_kernel(K.KV_DECODE_KERNEL_TCGEN05)
+    try:
+        out, ref, err = c.step(0, num_splits=0)
+        assert err == 0
+        check_close(out, ref, "bf16", cfg.name)
+        q = to_device(W.queries(cfg, 0, 0)[:12], "bf16")
+        tab, lens = torch.from_numpy(c.tab).cuda(), torch.from_numpy(c.lens.astype(np.int32)).cuda()
+        ws = torch.zeros(max(16, K.paged_decode_workspace_bytes(12, 32, 8, 128, c.max_blocks, 16, 0)),
+                         dtype=torch.uint8, device="cuda")
+        first = torch.from_numpy(out).cuda()
+        got = torch.empty_like(first)
+        for _ in range(30):
+            got.fill_(float("nan"))
+            K.paged_decode_attention_fp8(got, q, c.k_pages, c.v_pages, c.dks, c.dvs, tab, lens, cfg.scale,
+                                         num_splits=0, workspace=ws)
+            torch.cuda.synchronize()
+            assert torch.equal(got, first)
+    finally:
+        K.paged_decode_set_kernel(K.KV_DECODE_KERNEL_AUTO)

@@ -215,3 +215,32 @@ def test_tc_matches_warp_mma_kernel():
     finally:
         K.paged_decode_set_kernel(K.KV_DECODE_KERNEL_TCGEN05)
     check_close(out.cpu().numpy(), ref, "bf16", "warp mma")
+
+
+@pytest.mark.parametrize("H_q,H_kv,splits", [(32, 1, 0), (32, 8, 0), (32, 1, 3)])
+def test_tc_repeated_launches_identical(H_q, H_kv, splits):
+    """The same decode repeated 30 times over a pool whose unused slots hold NaN: every launch gives the bits
+    of the first, which matches the oracle. A barrier wait passing on an older phase, or a stale V row reaching
+    P.V, would show as a changed or non-finite element in some launch."""
+    cfg = W.DecodeConfig(f"tc-repeat-{H_q}-{H_kv}-{splits}", "bf16", B=24, H_q=H_q, H_kv=H_kv, Dh=128, page_size=16,
+                         seed=48)
+    lens = W.generator(48, W.S_LENGTHS, 24).integers(1, 700, 24)
+    lens[::5] = [1, 15, 16, 17, 128][: len(lens[::5])]
+    st = build_cache(cfg, lens, extra_blocks=1, slack_pages=32)
+    S = _assert_tc(cfg, st.max_blocks, splits)
+    assert (S == 0) == (splits == 0)
+    got, ref, err = append_and_decode(st, step=0, num_splits=splits, fused=False, check_pools=False)
+    assert err == 0
+    check_close(got, ref, "bf16", cfg.name)
+    B = len(st.lens)
+    q = to_device(W.queries(cfg, 0, 0)[:B], "bf16")
+    tab, lens32 = torch.from_numpy(st.tab).cuda(), torch.from_numpy(st.lens.astype(np.int32)).cuda()
+    ws = torch.zeros(max(16, K.paged_decode_workspace_bytes(B, H_q, H_kv, 128, st.max_blocks, 16, splits)),
+                     dtype=torch.uint8, device="cuda")
+    first = torch.from_numpy(got).cuda()
+    out = torch.empty_like(first)
+    for _ in range(30):
+        out.fill_(float("nan"))
+        K.paged_decode_attention(out, q, st.k_pages, st.v_pages, tab, lens32, cfg.scale, num_splits=splits, workspace=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(out, first)
