@@ -183,41 +183,72 @@ __global__ void __launch_bounds__(32 * kCombineStreamWarps) paged_combine_stream
     constexpr int kRound = 4;  // pieces whose dims are loaded together
     const int h = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const int g = H_q / H_kv;
+    const int c = blockIdx.x;
+    // The row this CTA merges comes from the plan alone. The plan kernel completed before the decode kernel
+    // this one follows let it launch (that kernel waits for the plan before it triggers), so the row is found
+    // before the wait for the partials; the plan is read from L2 (ld.global.cg), never from a line an
+    // earlier kernel left in this SM's L1.
+    int ns = 0, b = 0, kvh = 0;
+    if (h < g) {
+        const int32_t w1 = __ldcg(plan + 1);
+        const int G = w1 & 0xffff, v = static_cast<int>(static_cast<uint32_t>(w1) >> 16);
+        const long long T = static_cast<long long>(static_cast<uint32_t>(__ldcg(plan + 2))) |
+                            (static_cast<long long>(__ldcg(plan + 3)) << 32);
+        if (c + 1 < G) {  // the last range ends the line
+            const long long lo = T * c / G, hi = T * (c + 1) / G;
+            // the row whose span holds position hi: its sequence starts CTA c + 1's range
+            const int bb = __ldcg(plan + kPlanHdr + 2 * (B + 1) + c + 1);
+            const long long* pre = reinterpret_cast<const long long*>(plan + kPlanHdr);
+            const long long s0 = __ldcg(pre + bb), d = __ldcg(pre + bb + 1) - s0;
+            if (d > 0) {
+                const int kv = static_cast<int>((hi - (long long)H_kv * s0) / d);
+                const long long r0 = (long long)H_kv * s0 + (long long)kv * d + v, n = d - v;  // its real pages
+                // cut at this boundary when its real pages start inside this range (they then run past hi)
+                if (r0 < hi && r0 >= lo) {
+                    ns = plan_stream_cta(r0 + n - 1, T, G) - c + 1;
+                    b = bb;
+                    kvh = kv;
+                }
+            }
+        }
+    }
     grid_dependency_wait();  // the decode kernel's partials
     if (threadIdx.x == 0) grid_launch_dependents();
-    const int g = H_q / H_kv;
-    if (h >= g) return;
-    const int G = plan_stream_G(plan), v = plan_stream_v(plan);
-    const int c = blockIdx.x;
-    if (c + 1 >= G) return;  // the last range ends the line
-    const long long T = plan_stream_T(plan);
-    const int64_t* pre = plan_stream_prefix(plan);
-    const long long lo = T * c / G, hi = T * (c + 1) / G;
-    // the row whose span holds position hi: its sequence starts CTA c + 1's range
-    const int b = plan[kPlanHdr + 2 * (B + 1) + c + 1];
-    const long long s0 = pre[b], d = pre[b + 1] - s0;
-    if (d <= 0) return;
-    const int kvh = static_cast<int>((hi - (long long)H_kv * s0) / d);
-    const long long r0 = (long long)H_kv * s0 + (long long)kvh * d + v, n = d - v;  // the row's real pages
-    // cut at this boundary when its real pages start inside this range (they then run past hi)
-    if (r0 >= hi || r0 < lo) return;
-    const int ns = plan_stream_cta(r0 + n - 1, T, G) - c + 1;
+    if (ns <= 0) return;
     auto slot = [&](int s) { return (s == 0 ? 2LL * c + 1 : 2LL * (c + s)) * g + h; };
+    // first round: piece `lane`'s (m, l) and the dims of the first kRound pieces go out together
+    float2 st0 = make_float2(-INFINITY, 0.f);
+    if (lane < ns) st0 = part_ml[slot(lane)];
+    float v0[kRound][kD];
+#pragma unroll
+    for (int q = 0; q < kRound; ++q) {
+        if (q < ns) {
+            const float* src = part_u + slot(q) * DH + lane * kD;
+#pragma unroll
+            for (int i = 0; i < kD; ++i) v0[q][i] = src[i];
+        } else {
+#pragma unroll
+            for (int i = 0; i < kD; ++i) v0[q][i] = 0.f;
+        }
+    }
+    float mstar = st0.x;
+    for (int s = lane + 32; s < ns; s += 32) mstar = fmaxf(mstar, part_ml[slot(s)].x);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mstar = fmaxf(mstar, __shfl_xor_sync(0xffffffffu, mstar, o));
     float acc[kD];
 #pragma unroll
     for (int i = 0; i < kD; ++i) acc[i] = 0.f;
     float L = 0.f;
-    // the maximum over all pieces, then passes of 32 pieces (lane s: piece base + s's weight)
-    float mstar = -INFINITY;
-    for (int s = lane; s < ns; s += 32) mstar = fmaxf(mstar, part_ml[slot(s)].x);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mstar = fmaxf(mstar, __shfl_xor_sync(0xffffffffu, mstar, o));
+    // passes of 32 pieces (lane s: piece base + s's weight); a piece of weight 0 contributes 0, whatever its
+    // dims hold
     for (int base = 0; base < ns && mstar != -INFINITY; base += 32) {
         const int s_l = base + lane;
+        float2 st = st0;
+        if (base > 0) st = s_l < ns ? part_ml[slot(s_l)] : make_float2(-INFINITY, 0.f);
         float w = 0.f;
-        if (s_l < ns) {
-            const float2 st = part_ml[slot(s_l)];
-            if (st.x != -INFINITY) w = exp2f(st.x - mstar);
+        if (s_l < ns && st.x != -INFINITY) {
+            w = exp2f(st.x - mstar);
             L += w * st.y;
         }
         const int cnt = min(32, ns - base);
@@ -227,7 +258,10 @@ __global__ void __launch_bounds__(32 * kCombineStreamWarps) paged_combine_stream
 #pragma unroll
             for (int q = 0; q < kRound; ++q) {
                 ws[q] = __shfl_sync(0xffffffffu, w, (s + q) & 31);
-                if (s + q < cnt && ws[q] != 0.f) {
+                if (base == 0 && s == 0) {
+#pragma unroll
+                    for (int i = 0; i < kD; ++i) v[q][i] = v0[q][i];
+                } else if (s + q < cnt) {
                     const float* src = part_u + slot(base + s + q) * DH + lane * kD;
 #pragma unroll
                     for (int i = 0; i < kD; ++i) v[q][i] = src[i];
@@ -239,7 +273,7 @@ __global__ void __launch_bounds__(32 * kCombineStreamWarps) paged_combine_stream
 #pragma unroll
             for (int q = 0; q < kRound; ++q)
 #pragma unroll
-                for (int i = 0; i < kD; ++i) acc[i] += ws[q] * v[q][i];
+                for (int i = 0; i < kD; ++i) acc[i] += ws[q] != 0.f ? ws[q] * v[q][i] : 0.f;
         }
     }
 #pragma unroll
