@@ -41,29 +41,30 @@ __global__ void __launch_bounds__(32 * kCombineWarps) paged_combine_kernel(
     const int lane = threadIdx.x & 31;
     const int rw = warp % WPR;  // warp within its row
     const int64_t item = (int64_t)blockIdx.x * kRows + warp / WPR;
-    grid_dependency_wait();  // the decode kernel's partials
-    if (threadIdx.x == 0) grid_launch_dependents();
     bool live = item < (int64_t)B * H_q;
-    // grid split: partial s of the row sits at (row, s) whatever the row's length, so the loads of the first
-    // round go out together with that of the length, and splits past the row's last page are masked after
+    // The lengths and a plan were written before the decode kernel this one follows could start (it waits for
+    // its predecessors before it lets this one launch, and writes neither), so they are read before the wait
+    // for the partials, from L2 (ld.global.cg), never from a line an earlier kernel left in this SM's L1.
     int len = 0;
-    if (live) len = seq_lens[item / H_q];
-    int ns = plan != nullptr ? 0 : S;  // splits loaded; the row's own count is known once `len` has arrived
+    if (live) len = __ldcg(seq_lens + item / H_q);
+    int ns = plan != nullptr ? 0 : S;  // splits loaded (grid split: the row's own count masks them after)
     int64_t base = item * S, stride = 1;
     if (live && plan != nullptr) {
         const int b = static_cast<int>(item / H_q);
         if (len < 0 || len > max_blocks * P) len = 0;
         const int n_pages = (len + P - 1) / P;
-        const int C = plan[0];
+        const int C = __ldcg(plan);
         const int items_b = (n_pages + C - 1) / C;
         const int g = H_q / H_kv;
         const int hq = static_cast<int>(item % H_q);
         if (items_b == 1) live = false;  // the decode kernel wrote this row
         ns = items_b > 1 ? items_b : 0;
-        const int64_t t0 = (int64_t)H_kv * plan[kPlanHdr + b] + (int64_t)(hq / g) * items_b;
+        const int64_t t0 = (int64_t)H_kv * __ldcg(plan + kPlanHdr + b) + (int64_t)(hq / g) * items_b;
         base = t0 * g + hq % g;
         stride = g;
     }
+    grid_dependency_wait();  // the decode kernel's partials
+    if (threadIdx.x == 0) grid_launch_dependents();
     if (!live) ns = 0;
     const float2* ml = part_ml + base;
     const float* pu = part_u + base * DH + lane * kD;
